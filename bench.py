@@ -1,0 +1,526 @@
+"""Benchmark of the routed-expert MoE layer with decoupled top-k1/top-k2
+renormalisation on B200.
+
+Default workload ("decode_b1"): 48 layers, each with its own weights,
+d=2048, E=128 experts, I=768, bf16, T=1 token per layer per step, no router
+bias; headline condition k1=4, k2=16 (half the trained k of 8, reference
+mass of 16 experts), with the other five (k1, k2) conditions of the sweep
+reported beside it.  A step is one token through all 48 layers, each layer's
+router -> softmax -> top-k -> Eq. 2 weights -> expert FFN -> combine, the
+layers chained in one stream (each layer's kernels wait for the previous
+layer's) and replayed from one CUDA graph.  value = tokens/s of the 48-layer
+stack (T / step time, summed over ranks); us_per_layer = step time / 48.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl native|reference]
+                    [--workload decode_b1|decode_small_batch|prefill|large]
+                    [--k1 K1 --k2 K2] [--T T] [--layers L]
+
+N > 1: launched by torch.distributed.run, one rank per GPU, each rank an
+independent replica decoding its own tokens (weak scaling, no collective on
+the data path; one all-reduce of the elapsed time after the timed region).
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "MoE-layer tokens/s and achieved HBM GB/s (decode) / TFLOP/s (prefill) vs k1,k2"
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_PATH = os.path.join(ROOT, "profiles", "traffic.json")
+
+WORKLOADS = {
+    "decode_b1": dict(T=1, d=2048, E=128, I=768, layers=48, bias=None,
+                      sweep=[(4, 16), (8, 8), (8, 16), (8, 128), (4, 4), (4, 128)]),
+    "decode_small_batch": dict(T=8, d=2048, E=128, I=768, layers=48, bias="normal",
+                               sweep=[(4, 16), (8, 8)]),
+    "prefill": dict(T=4096, d=2048, E=128, I=768, layers=4, bias="zipf", sweep=[(8, 16), (4, 16)]),
+    "large": dict(T=1, d=4096, E=512, I=1024, layers=8, bias=None, sweep=[(5, 20), (10, 10)]),
+}
+
+
+# ---------------------------------------------------------------------- helpers
+def load_peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def kernel_source_digest():
+    import hashlib
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "routed_expert_layer_route_b200", "csrc")
+    for name in sorted(os.listdir(d)):
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload, k1):
+    """ncu DRAM bytes per launch of the streaming kernel, if recorded for the
+    current kernel source (null once the source has changed)."""
+    try:
+        with open(TRAFFIC_PATH) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("source_digest") != kernel_source_digest():
+        return None
+    return rec.get("k_stream", {}).get("%s_k1_%d" % (workload, k1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def smi_index(local):
+    """nvidia-smi's id for this process's CUDA device."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local < len(ids):
+            return ids[local]
+    return str(local)
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def allreduce_max(v, world):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------------- model
+class Stack:
+    """L layers of seeded synthetic weights and per-layer tokens on the GPU."""
+
+    def __init__(self, wl, seed, device):
+        from routed_expert_layer_route_b200 import synth
+        self.wl = wl
+        self.layers = []
+        for l in range(wl["layers"]):
+            self.layers.append(synth.make_layer(wl["T"], wl["d"], wl["E"], wl["I"], seed=seed,
+                                               layer=l, device=device, bias=wl["bias"]))
+        torch.cuda.synchronize()
+
+
+def build_graph(stack, k1, k2, ws_list, ys, stream):
+    """Capture one step (every layer's moe_layer) into a CUDA graph."""
+    from routed_expert_layer_route_b200 import moe
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        # one eager pass first (module attribute set-up happens outside capture)
+        for L, ws, y in zip(stack.layers, ws_list, ys):
+            moe.moe_layer(L.x, L.w_router, L.bias, L.w_gate, L.w_up, L.w_down, k1, k2, y, ws,
+                          stream=stream)
+        stream.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            for L, ws, y in zip(stack.layers, ws_list, ys):
+                moe.moe_layer(L.x, L.w_router, L.bias, L.w_gate, L.w_up, L.w_down, k1, k2, y, ws,
+                              stream=stream)
+    return g
+
+
+def unique_experts(stack, k1, k2, ws_list, ys, stream):
+    """Activated experts per layer, read back from the routing outputs."""
+    from routed_expert_layer_route_b200 import moe
+    us = []
+    wl = stack.wl
+    for L, ws, y in zip(stack.layers, ws_list, ys):
+        idx = torch.empty(wl["T"], k1, dtype=torch.int32, device=L.x.device)
+        moe.moe_layer(L.x, L.w_router, L.bias, L.w_gate, L.w_up, L.w_down, k1, k2, y, ws,
+                      topk_idx_out=idx, stream=stream)
+        stream.synchronize()
+        us.append(int(torch.unique(idx).numel()))
+    return us
+
+
+def time_dominant_kernel(stack, k1, ws_list, ys, stream, reps):
+    """Average duration of the expert-streaming kernel launched alone (CUDA
+    events on its stream), cycling through the layers so weights come from
+    HBM, not L2."""
+    from routed_expert_layer_route_b200 import moe
+    starts, ends = [], []
+    with torch.cuda.stream(stream):
+        for r in range(reps):
+            for L, ws, y in zip(stack.layers, ws_list, ys):
+                s = torch.cuda.Event(enable_timing=True)
+                e = torch.cuda.Event(enable_timing=True)
+                s.record(stream)
+                moe.moe_test_expert_stream(L.x, L.w_gate, L.w_up, L.w_down, k1, y, ws, stream=stream)
+                e.record(stream)
+                starts.append(s)
+                ends.append(e)
+    stream.synchronize()
+    ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    return statistics.mean(ms[len(stack.layers):] or ms)  # first pass is warm-up
+
+
+def e2e_tokens_per_s(stack, k1, k2, ws_list, steps, warmup, stream):
+    """Through the public API with host buffers: per step, pinned-host ->
+    device copy of every layer's tokens, every layer's moe_layer call, and a
+    device -> pinned-host copy of every layer's output."""
+    from routed_expert_layer_route_b200 import moe
+    wl = stack.wl
+    T, d, L_ = wl["T"], wl["d"], wl["layers"]
+    host_x = torch.stack([L.x for L in stack.layers]).cpu().pin_memory()
+    host_y = torch.empty(L_, T, d, dtype=torch.bfloat16).pin_memory()
+    dev_x = torch.empty(L_, T, d, dtype=torch.bfloat16, device="cuda")
+    dev_y = torch.empty(L_, T, d, dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        dev_x.copy_(host_x, non_blocking=True)
+        for l, (L, ws) in enumerate(zip(stack.layers, ws_list)):
+            moe.moe_layer(dev_x[l], L.w_router, L.bias, L.w_gate, L.w_up, L.w_down, k1, k2,
+                          dev_y[l], ws, stream=stream)
+        host_y.copy_(dev_y, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            step()
+        stream.synchronize()
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(steps):
+            step()
+        e.record(stream)
+        e.synchronize()
+    ms = s.elapsed_time(e) / steps
+    return T * 1000.0 / ms, host_x[0].numel() * 2 * L_, host_y[0].numel() * 2 * L_
+
+
+# ---------------------------------------------------------------------- CPU oracle
+def cpu_oracle_rate(stack, k1, k2, budget_s=12.0):
+    """The oracle as it stands, on the host cores: router logits, routing,
+    the k1 experts and the combine, layer after layer until the time budget
+    is spent.  Returns (tokens/s for the whole stack, layers run, threads)."""
+    import oracle
+    from routed_expert_layer_route_b200 import synth
+    wl = stack.wl
+    T = wl["T"]
+    prepared = []
+    # fetch only what the sample needs (router, bias, the routed experts)
+    for L in stack.layers:
+        x = synth.to_numpy(L.x)
+        wr = synth.to_numpy(L.w_router)
+        b = synth.to_numpy(L.bias)
+        z = oracle.logits(x, wr, b)
+        idx, _ = oracle.route_f32(z, k1, k2)
+        experts = {int(e): (synth.to_numpy(L.w_gate[int(e)]), synth.to_numpy(L.w_up[int(e)]),
+                            synth.to_numpy(L.w_down[int(e)])) for e in np.unique(idx)}
+        prepared.append((x, wr, b, experts))
+        if len(prepared) >= 6:
+            break
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        x, wr, b, experts = prepared[n % len(prepared)]
+        z = oracle.logits(x, wr, b)
+        oracle.layer_tokens(x, z, lambda e: experts[e], k1, k2)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or n >= 4 * wl["layers"]:
+            break
+    per_layer = el / n
+    return T / (per_layer * wl["layers"]), n, oracle.num_threads(), el
+
+
+# ---------------------------------------------------------------------- main
+def run_native(args, world, rank):
+    from routed_expert_layer_route_b200 import build as pkg_build
+    from routed_expert_layer_route_b200 import moe
+    pkg_build.build()
+    wl = dict(WORKLOADS[args.workload])
+    if args.T:
+        wl["T"] = args.T
+    if args.layers:
+        wl["layers"] = args.layers
+    sweep = list(wl["sweep"])
+    if args.k1:
+        sweep = [(args.k1, args.k2 or args.k1)]
+    head = sweep[0]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.Stream()
+    hbm_peak, bf16_peak, peak_kind = load_peaks()
+
+    stack = Stack(wl, seed=rank, device=dev)
+    T, d, E, I, Ln = wl["T"], wl["d"], wl["E"], wl["I"], wl["layers"]
+    results = []
+    graphs = {}
+    for (k1, k2) in sweep:
+        ws_list = [moe.workspace(T, d, E, I, k1, device=dev) for _ in range(Ln)]
+        ys = [torch.empty(T, d, dtype=torch.bfloat16, device=dev) for _ in range(Ln)]
+        g = build_graph(stack, k1, k2, ws_list, ys, stream)
+        graphs[(k1, k2)] = (g, ws_list, ys)
+
+    def timed(k1, k2, steps, warmup, clocks=None):
+        g = graphs[(k1, k2)][0]
+        with torch.cuda.stream(stream):
+            for _ in range(warmup):
+                g.replay()
+        stream.synchronize()
+        barrier(world)
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        if clocks:
+            clocks.start()
+        s.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(steps):
+                g.replay()
+        e.record(stream)
+        e.synchronize()
+        if clocks:
+            c = clocks.stop()
+        else:
+            c = None
+        barrier(world)
+        ms = s.elapsed_time(e)
+        return allreduce_max(ms, world) / steps, c
+
+    # headline: the timed region of the contract
+    clocks = ClockSampler(smi_index(torch.cuda.current_device()))
+    ms_step, clk = timed(*head, args.steps, args.warmup, clocks)
+    value = world * T * 1000.0 / ms_step
+
+    # every (k1, k2) condition of the sweep, same protocol, outside the headline region
+    for (k1, k2) in sweep:
+        ms = ms_step if (k1, k2) == head else timed(k1, k2, args.steps, args.warmup)[0]
+        _, ws_list, ys = graphs[(k1, k2)]
+        us = unique_experts(stack, k1, k2, ws_list, ys, stream)
+        U = statistics.mean(us)
+        bytes_layer = U * 3 * d * I * 2
+        results.append({"k1": k1, "k2": k2, "ms_per_step": ms, "us_per_layer": ms * 1000 / Ln,
+                        "tokens_per_s": world * T * 1000.0 / ms, "unique_experts_per_layer": U,
+                        "expert_GBps": bytes_layer / (ms / Ln * 1e-3) / 1e9})
+
+    # dominant kernel alone, events on its own stream
+    k1h, k2h = head
+    _, ws_list, ys = graphs[head]
+    kern_ms = time_dominant_kernel(stack, k1h, ws_list, ys, stream, reps=3)
+    U_head = results[0]["unique_experts_per_layer"]
+    alg_bytes = U_head * 3 * d * I * 2
+    achieved = alg_bytes / (kern_ms * 1e-3) / 1e9
+    traffic = recorded_traffic(args.workload, k1h)
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
+                "kernel": "moe::k_stream", "kernel_us": round(kern_ms * 1000, 2),
+                "algorithmic_bytes_per_launch": int(alg_bytes),
+                "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
+                if peak_kind == "measured" else "fallback 6650 GB/s"}
+
+    # end to end through the public API with host buffers
+    e2e_val, h2d, d2h = e2e_tokens_per_s(stack, k1h, k2h, ws_list, max(3, args.steps // 4),
+                                         args.warmup, stream)
+    e2e_val = world * T * 1000.0 / allreduce_max(T * 1000.0 / e2e_val, world)
+
+    # ratio of k1=4 to k1=8 layer time (same k2 where possible)
+    by = {(r["k1"], r["k2"]): r for r in results}
+    ratio = None
+    if (4, 16) in by and (8, 16) in by:
+        ratio = by[(4, 16)]["us_per_layer"] / by[(8, 16)]["us_per_layer"]
+    elif (4, 4) in by and (8, 8) in by:
+        ratio = by[(4, 4)]["us_per_layer"] / by[(8, 8)]["us_per_layer"]
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, nl, thr, el = cpu_oracle_rate(stack, k1h, k2h)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+               "sample": "%d single-token layers of this workload (k1=%d, k2=%d) in %.1f s, "
+                         "per-layer time scaled to the %d-layer stack" % (nl, k1h, k2h, el, Ln)}
+
+    per_step_launches = 2 if T == 1 else 3
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,0.02) weights, RMS-normalised N(0,1) tokens)",
+        "config": {"workload": "%s: %d layers, d=%d, E=%d, I=%d, T=%d per rank, k1=%d, k2=%d"
+                               % (args.workload, Ln, d, E, I, T, k1h, k2h),
+                   "layers": Ln, "d": d, "E": E, "I": I, "T": T, "k1": k1h, "k2": k2h,
+                   "bias": wl["bias"], "us_per_layer": round(ms_step * 1000 / Ln, 3),
+                   "l2": "inputs larger than L2: every step reads the routed experts of all "
+                         "%d layers (%.2f GB) from HBM" % (Ln, alg_bytes * Ln / 1e9),
+                   "timing": "CUDA graph of the %d-layer step, CUDA events, max over ranks" % Ln,
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_val, 3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "path": "moe_layer C-ABI per layer from Python, pinned host x in, y out"},
+        "gpu_launches": per_step_launches * Ln * args.steps,
+        "clocks": clk,
+        "sweep": results,
+        "k1_4_over_k1_8_time_ratio": None if ratio is None else round(ratio, 4),
+    }
+    for g, _, _ in graphs.values():
+        del g
+    graphs.clear()
+    return line
+
+
+def run_reference(args, world, rank):
+    """The oracle as it stands on the host cores, on the same workload."""
+    if rank != 0:
+        return None
+    wl = dict(WORKLOADS[args.workload])
+    if args.T:
+        wl["T"] = args.T
+    if args.layers:
+        wl["layers"] = args.layers
+    k1, k2 = (args.k1, args.k2 or args.k1) if args.k1 else wl["sweep"][0]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    small = dict(wl)
+    small["layers"] = min(6, wl["layers"])
+    stack = Stack(small, seed=0, device=dev)
+    rates = []
+    for _ in range(args.warmup):
+        cpu_oracle_rate(stack, k1, k2, budget_s=1.0)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        r, nl, thr, el = cpu_oracle_rate(stack, k1, k2, budget_s=3.0)
+        rates.append(r)
+    total = time.perf_counter() - t0
+    # each rate is already the per-layer time scaled to the full stack
+    r_stack = statistics.mean(rates)
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(r_stack, 4), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1000.0 * wl["T"] / r_stack, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32 (bf16 inputs widened)",
+        "data": "synthetic", "config": {"workload": "%s: %d layers, d=%d, E=%d, I=%d, T=%d, k1=%d, "
+                                                    "k2=%d" % (args.workload, wl["layers"], wl["d"],
+                                                               wl["E"], wl["I"], wl["T"], k1, k2)},
+        "cpu_baseline": {"value": round(r_stack, 4), "unit": "tokens/s", "cores": thr,
+                         "kind": "oracle", "sample": "each step: single-token layers for 3 s, "
+                                                     "per-layer time scaled to the %d-layer stack"
+                                                     % wl["layers"]},
+        "e2e": {"value": round(r_stack, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "wall_s": round(total, 2),
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode_b1")
+    ap.add_argument("--k1", type=int, default=0)
+    ap.add_argument("--k2", type=int, default=0)
+    ap.add_argument("--T", type=int, default=0)
+    ap.add_argument("--layers", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, world, rank)
+        else:
+            line = run_native(args, world, rank)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

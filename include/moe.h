@@ -1,0 +1,165 @@
+/*
+ * moe.h -- C ABI of libmoe.so: a routed-expert Mixture-of-Experts layer with
+ * decoupled top-k1 / top-k2 renormalisation, for NVIDIA B200 (sm_100a).
+ *
+ * The method ("Paper of the Week #3 -- Half the FLOPs Is Not Half the Time",
+ * sotaaz.com, section "The Receipt", Eq. 2):
+ *
+ *     z = x W_r^T (+ b)                         router logits
+ *     p = softmax(z)  in float32                over the E experts
+ *     w_i = p_i / sum_{j in Top-k2} p_j         for i in Top-k1
+ *           (k2 = k1: standard renormalisation; k2 >= E: no renormalisation)
+ *     y = sum_{i in Top-k1} w_i * FFN_i(x)      FFN_i a SwiGLU gated MLP
+ *
+ * Each routed expert is a gated MLP whose channel c owns gate row c, up row c
+ * and down column c ("Channel Selection for Mixture-of-Experts Decoding Needs
+ * No Calibration Data", paperlayer.ai, section 2 "Background"):
+ *     h_c = silu(W_gate[c,:] . x) * (W_up[c,:] . x),  o = W_down h.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Pointers named *_bf16 point to bfloat16 data, *_f32/float* to float32,
+ *    int32_t* to 32-bit integers.  All tensors are dense row-major.
+ *  - All data pointers are DEVICE pointers, owned by the caller, 16-byte
+ *    aligned; they must stay valid until the work queued on `stream` ends.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Every call only enqueues work: none synchronises, none
+ *    allocates or frees device memory (moe_read_device_status is the one
+ *    call that synchronises).
+ *  - Shapes: T tokens (T >= 0; T = 0 is a no-op), hidden size d, E experts,
+ *    expert intermediate size I (channels), k1 experts run per token, k2
+ *    experts in the reference mass.  Requirements: 1 <= k1 <= k2,
+ *    k1 <= min(E, 32), 1 <= E <= 1024, d % 64 == 0, I % 16 == 0,
+ *    64 <= d <= 16384, 16 <= I <= 16384.  k2 > E is accepted and means
+ *    k2 = E (no renormalisation), as the page's min(k2, E) does.
+ *  - Routing is deterministic: probabilities are ranked by (p descending,
+ *    expert index ascending); the float32 softmax and the top-k2 mass follow
+ *    one fixed sequence of float32 operations, so indices and weights are
+ *    bit-identical to the CPU oracle that follows the same sequence.
+ *  - Weight layouts (per expert e): w_gate, w_up [E x I x d] (row c of
+ *    expert e = channel c), w_down [E x d x I] (column c = channel c),
+ *    w_router [E x d], bias [E] float32 (nullable).
+ *  - Return value: MOE_OK or a negative moe_status.  Argument checks happen
+ *    on the host before anything is enqueued; on an error nothing is
+ *    enqueued.  MOE_ERR_CUDA means a launch failed (the CUDA error is left
+ *    for cudaGetLastError).  Problems found on the device (a bounded wait
+ *    that gave up, an index out of range) are recorded in the workspace's
+ *    status word; read it with moe_read_device_status.
+ *  - Workspace: `ws` is caller-owned device memory of at least
+ *    moe_workspace_size(...) bytes, 256-byte aligned, initialised once with
+ *    moe_workspace_init before its first use.  Calls leave it initialised.
+ *    Calls that share one workspace must be ordered on one stream.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1,         /* null pointer, k1/k2 out of range, misaligned pointer   */
+    MOE_ERR_UNSUPPORTED_SHAPE = -2,   /* d, I, E, T outside the supported limits                */
+    MOE_ERR_WORKSPACE_TOO_SMALL = -3, /* ws_bytes < moe_workspace_size(...)                     */
+    MOE_ERR_CUDA = -4,                /* a CUDA runtime call failed                             */
+    MOE_ERR_TIMEOUT = -5,             /* device status: a bounded wait gave up                  */
+    MOE_ERR_DEVICE_CHECK = -6         /* device status: an index check failed on the device     */
+} moe_status;
+
+/* Output element types for moe_combine / moe_layer. */
+#define MOE_DTYPE_F32 0
+#define MOE_DTYPE_BF16 1
+
+/* moe_layer / moe_expert_ffn flags: which expert-FFN path runs.
+ * AUTO picks by the expected number of tokens per activated expert. */
+#define MOE_PATH_AUTO 0
+#define MOE_PATH_STREAM 1  /* weight-streaming path (small batches)        */
+#define MOE_PATH_GROUPED 2 /* tcgen05 grouped GEMM path (large batches)    */
+
+/* Human-readable text for a moe_status value.  Never NULL. */
+const char *moe_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int moe_version(void);
+
+/* Bytes of workspace the calls below need for these shapes (the maximum over
+ * moe_route, moe_permute, moe_expert_ffn and moe_layer, on either path).
+ * Returns 0 when the shapes are invalid. */
+size_t moe_workspace_size(int T, int d, int E, int I, int k1);
+
+/* Zero the workspace's header (status word and the counters the kernels use
+ * for cross-block hand-off).  Enqueued on `stream`. */
+int moe_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/* Copy the workspace's device status word into *status_out (MOE_OK or a
+ * device-side moe_status) and clear it.  Synchronises `stream`. */
+int moe_read_device_status(void *ws, int *status_out, void *stream);
+
+/* Router: logits, float32 softmax, top-k1 of the ranking, Eq. 2 weights.
+ * ("Paper of the Week #3", sections "The Receipt" (Eq. 2) and "Ship It /
+ * Code of the Week": logits = linear(x, W_r); probs = softmax in float32;
+ * topk(probs, min(k2, E)); first k1; divided by the sum of all min(k2, E)
+ * taken probabilities unless k2 >= E.)
+ *
+ *  x_bf16 == NULL : `logits` is an INPUT [T x E] float32; w_router_bf16 and
+ *                   bias are ignored (this is the entry that routes given
+ *                   logits, used for bit-exact comparison).
+ *  x_bf16 != NULL : x [T x d] bf16, w_router [E x d] bf16, bias [E] float32
+ *                   or NULL; `logits` (nullable) receives x W_r^T + b as
+ *                   float32 [T x E] (float32 accumulation).
+ *  topk_idx [T x k1] int32: expert ids in rank order.
+ *  topk_w   [T x k1] float32: Eq. 2 weights aligned with topk_idx.
+ *  ws: workspace (needed only when x_bf16 != NULL and logits == NULL; may be
+ *      NULL otherwise). */
+int moe_route(const void *x_bf16, const void *w_router_bf16, const float *bias, float *logits,
+              int T, int d, int E, int k1, int k2, int32_t *topk_idx, float *topk_w, void *ws,
+              size_t ws_bytes, void *stream);
+
+/* Stable counting sort of the T*k1 routed slots by expert (slot i = t*k1+s,
+ * the s-th expert of token t).  The grouping the expert FFN needs: every
+ * expert's tokens become one contiguous run.
+ *  expert_offsets [E+1]: exclusive scan of the per-expert slot counts;
+ *  sorted_slot [T*k1]: slots ordered by (expert, slot index);
+ *  slot_pos    [T*k1]: inverse, sorted_slot[slot_pos[i]] == i.
+ *  An expert id outside [0, E) sets MOE_ERR_DEVICE_CHECK in the device status
+ *  word when ws is given (the slot is then dropped).  ws may be NULL. */
+int moe_permute(const int32_t *topk_idx, int T, int k1, int E, int32_t *expert_offsets,
+                int32_t *sorted_slot, int32_t *slot_pos, void *ws, size_t ws_bytes, void *stream);
+
+/* Expert FFN for every routed slot (unweighted):
+ *  out[p, :] = W_down[e] (silu(W_gate[e] x_t) * (W_up[e] x_t))  (float32)
+ * for sorted position p in [expert_offsets[e], expert_offsets[e+1]), where
+ * t = sorted_slot[p] / k1.  out is [T*k1 x d] float32 in sorted order.
+ * ("Channel Selection ...", section 2: channel c = gate row c, up row c,
+ * down column c.)  Accumulation is float32; x and the weights are bf16.
+ * flags: MOE_PATH_*.  ws: workspace. */
+int moe_expert_ffn(const void *x_bf16, const int32_t *expert_offsets, const int32_t *sorted_slot,
+                   const void *w_gate_bf16, const void *w_up_bf16, const void *w_down_bf16, int T,
+                   int d, int E, int I, int k1, float *out, int flags, void *ws, size_t ws_bytes,
+                   void *stream);
+
+/* Weighted combine (Eq. 2 weights):
+ *  y[t, :] = sum_{s=0}^{k1-1} topk_w[t, s] * expert_out[slot_pos[t*k1+s], :]
+ * summed in s order in float32; y is [T x d] of y_dtype (MOE_DTYPE_*). */
+int moe_combine(const float *expert_out, const int32_t *slot_pos, const float *topk_w, int T,
+                int d, int k1, void *y, int y_dtype, void *stream);
+
+/* The whole layer: router (as moe_route), permutation, expert FFN and
+ * combine.  y [T x d] of y_dtype.  Optional outputs (each nullable):
+ * topk_idx_out / topk_w_out [T x k1], logits_out [T x E] float32.
+ * flags: MOE_PATH_*.  ws: workspace. */
+int moe_layer(const void *x_bf16, const void *w_router_bf16, const float *bias,
+              const void *w_gate_bf16, const void *w_up_bf16, const void *w_down_bf16, int T, int d,
+              int E, int I, int k1, int k2, void *y, int y_dtype, int32_t *topk_idx_out,
+              float *topk_w_out, float *logits_out, int flags, void *ws, size_t ws_bytes,
+              void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */

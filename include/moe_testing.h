@@ -1,0 +1,39 @@
+/*
+ * moe_testing.h -- test hooks of libmoe.so.  Not part of the layer's API;
+ * they expose internal device functions so tests can check them alone.
+ */
+#ifndef MOE_TESTING_H
+#define MOE_TESTING_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* y[i] = the routing softmax's float32 exponential of x[i], computed by the
+ * device function the router kernels use (Cody-Waite reduction, degree-7
+ * Taylor polynomial in Horner form with fused multiply-adds, exact 2^n
+ * scaling; +0 below -87).  x, y: device float32 arrays of n elements.
+ * Returns a moe_status. */
+int moe_test_exp_c(const float *x, float *y, int64_t n, void *stream);
+
+/* Number of SMs the library sizes its persistent grids for on the current
+ * device (0 if no device). */
+int moe_test_num_sms(void);
+
+/* Re-run only the expert-streaming kernel (expert FFN + combine into y) of
+ * the last moe_layer call made with this workspace and these shapes, reusing
+ * the routing that call left in the workspace.  Launched without
+ * programmatic dependent launch, so events recorded around it on `stream`
+ * bracket this one kernel.  Used to time the dominant kernel alone.
+ * Arguments as for moe_layer.  Returns a moe_status. */
+int moe_test_expert_stream(const void *x_bf16, const void *w_gate_bf16, const void *w_up_bf16,
+                           const void *w_down_bf16, int T, int d, int E, int I, int k1, void *y,
+                           int y_dtype, void *ws, size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_TESTING_H */

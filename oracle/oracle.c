@@ -142,6 +142,7 @@ float oracle_exp_c(float x)
 
 void oracle_exp_c_array(const float *x, float *y, int64_t n)
 {
+#pragma omp parallel for schedule(static) if (n > 100000)
     for (int64_t i = 0; i < n; ++i)
         y[i] = oracle_exp_c(x[i]);
 }

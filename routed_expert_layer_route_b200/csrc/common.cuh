@@ -1,0 +1,178 @@
+// common.cuh -- small device helpers shared by the kernels of libmoe.so:
+// bf16 unpacking, mbarrier / bulk-copy / programmatic-dependent-launch PTX
+// wrappers, bounded waits and the workspace header.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+#define MOE_DEVINL __device__ __forceinline__
+
+// ---------------------------------------------------------------------------
+// Workspace header: the first 256 bytes of every workspace.
+struct WsHeader {
+    int status;              // device status word (moe_status), 0 = OK
+    unsigned route_arrive;   // last-block hand-off counter of the router kernel
+    unsigned bar_count;      // grid barrier of the streaming kernel: arrivals
+    unsigned bar_gen;        // grid barrier generation
+    unsigned pad[60];
+};
+static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
+
+// Bounded waits give up after this many nanoseconds (globaltimer) and record
+// MOE_ERR_TIMEOUT; no correct launch comes anywhere near it.
+#define MOE_WAIT_LIMIT_NS 2000000000ull
+
+MOE_DEVINL uint64_t global_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+MOE_DEVINL void set_status(int *status, int code)
+{
+    if (status)
+        atomicCAS(status, 0, code);
+}
+
+// ---------------------------------------------------------------------------
+// bf16 helpers: a bf16 value is the upper half of a float32.
+MOE_DEVINL float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
+MOE_DEVINL float bf16hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+MOE_DEVINL uint16_t f32_to_bf16_rn(float f)
+{
+    uint32_t u = __float_as_uint(f);
+    if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x7fffffu))  // NaN stays NaN
+        return (uint16_t)((u >> 16) | 0x40u);
+    uint32_t r = u + 0x7fffu + ((u >> 16) & 1u);
+    return (uint16_t)(r >> 16);
+}
+
+// 8 bf16 (one 16-byte vector) times 8 floats, accumulated into acc.
+MOE_DEVINL float dot8_bf16(const uint4 w, const float *x, float acc)
+{
+    acc = fmaf(bf16lo(w.x), x[0], acc);
+    acc = fmaf(bf16hi(w.x), x[1], acc);
+    acc = fmaf(bf16lo(w.y), x[2], acc);
+    acc = fmaf(bf16hi(w.y), x[3], acc);
+    acc = fmaf(bf16lo(w.z), x[4], acc);
+    acc = fmaf(bf16hi(w.z), x[5], acc);
+    acc = fmaf(bf16lo(w.w), x[6], acc);
+    acc = fmaf(bf16hi(w.w), x[7], acc);
+    return acc;
+}
+
+MOE_DEVINL float warp_sum(float v)
+{
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch.  griddepcontrol.wait returns once every
+// grid this one depends on has completed and its memory is visible; it is a
+// no-op when the kernel was launched without the attribute.
+MOE_DEVINL void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+MOE_DEVINL void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
+// Shared-memory mbarriers and bulk asynchronous copies (no multicast).
+MOE_DEVINL uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+MOE_DEVINL void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+
+MOE_DEVINL void fence_mbar_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+MOE_DEVINL void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+MOE_DEVINL void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+MOE_DEVINL bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase of `bar` with the given parity to complete.  Gives up
+// after MOE_WAIT_LIMIT_NS, records MOE_ERR_TIMEOUT and returns false.
+MOE_DEVINL bool mbar_wait(uint64_t *bar, uint32_t parity, int *status)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_ns() - t0 > MOE_WAIT_LIMIT_NS) {
+            set_status(status, MOE_ERR_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+// L2 policy for weights streamed exactly once: evict first.
+MOE_DEVINL uint64_t l2_evict_first_policy()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// Global -> shared bulk copy of `bytes` (multiple of 16, both addresses
+// 16-byte aligned); completion is counted on `bar` as transaction bytes.
+MOE_DEVINL void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar, uint64_t pol)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(pol)
+        : "memory");
+}
+
+MOE_DEVINL void named_bar_sync(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+MOE_DEVINL unsigned ld_acquire_u32(const unsigned *p)
+{
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+MOE_DEVINL uint4 ld_nc_v4(const void *p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}

@@ -1,0 +1,503 @@
+// moe_api.cu -- the C ABI of libmoe.so (declared in include/moe.h): argument
+// checks, workspace layout and kernel launches.  All work is enqueued on the
+// caller's stream; consecutive kernels are chained with programmatic
+// dependent launch so each kernel's prologue (and the router's weight
+// prefetch) overlaps the tail of the previous one.  Every kernel waits
+// (griddepcontrol.wait) before it touches data written by earlier work.
+#include <cuda_runtime.h>
+
+#include <mutex>
+#include <utility>
+
+#include "../../include/moe.h"
+#include "../../include/moe_testing.h"
+#include "combine.cuh"
+#include "route.cuh"
+#include "stream.cuh"
+
+namespace moe {
+
+// ------------------------------------------------------------------ limits
+constexpr int kMaxE = 1024;
+constexpr int kMaxK1 = 32;
+constexpr int kMinD = 64, kMaxD = 8192;
+constexpr int kMinI = 16, kMaxI = 8192;
+constexpr int kMaxT = 1 << 20;
+
+static inline size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+struct WsLayout {
+    size_t logits, idx, w, offsets, sorted_slot, slot_pos, uniq_count, uniq_list, h, out, total;
+};
+
+static WsLayout ws_layout(int T, int d, int E, int I, int k1)
+{
+    WsLayout L;
+    size_t o = sizeof(WsHeader);
+    const size_t n = (size_t)T * k1;
+    L.logits = o;      o = align256(o + sizeof(float) * (size_t)T * E);
+    L.idx = o;         o = align256(o + sizeof(int32_t) * n);
+    L.w = o;           o = align256(o + sizeof(float) * n);
+    L.offsets = o;     o = align256(o + sizeof(int32_t) * (size_t)(E + 1));
+    L.sorted_slot = o; o = align256(o + sizeof(int32_t) * n);
+    L.slot_pos = o;    o = align256(o + sizeof(int32_t) * n);
+    L.uniq_count = o;  o = align256(o + sizeof(int32_t));
+    L.uniq_list = o;   o = align256(o + sizeof(int32_t) * (size_t)E);
+    L.h = o;           o = align256(o + sizeof(float) * n * (size_t)I);
+    L.out = o;         o = align256(o + sizeof(float) * n * (size_t)d);
+    L.total = o;
+    return L;
+}
+
+template <typename P>
+static inline P *at(void *ws, size_t off)
+{
+    return reinterpret_cast<P *>(reinterpret_cast<char *>(ws) + off);
+}
+
+static inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+static int check_shape(int T, int d, int E, int I, int k1)
+{
+    if (T < 0 || T > kMaxT)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (E < 1 || E > kMaxE)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (d < kMinD || d > kMaxD || d % 64)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (I < kMinI || I > kMaxI || I % 16)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (k1 < 1 || k1 > kMaxK1 || k1 > E)
+        return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+static int check_route(int E, int k1, int k2)
+{
+    if (E < 1 || E > kMaxE)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (k1 < 1 || k1 > kMaxK1 || k1 > E || k2 < k1)
+        return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+// ------------------------------------------------------------------ device info
+struct DevInfo {
+    bool ready = false;
+    int num_sms = 0;
+};
+static DevInfo g_dev[64];
+static std::mutex g_dev_mu;
+
+static int device_info(DevInfo *&out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    DevInfo &di = g_dev[dev];
+    if (!di.ready) {
+        if (cudaDeviceGetAttribute(&di.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        const int stream_smem = 227 * 1024;
+        if (cudaFuncSetAttribute(k_stream, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 stream_smem) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        const int small = 96 * 1024;
+        if (cudaFuncSetAttribute(k_logits, cudaFuncAttributeMaxDynamicSharedMemorySize, small) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(k_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, small) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(k_permute, cudaFuncAttributeMaxDynamicSharedMemorySize, small) !=
+                cudaSuccess)
+            return MOE_ERR_CUDA;
+        di.ready = true;
+    }
+    out = &di;
+    return MOE_OK;
+}
+
+// ------------------------------------------------------------------ launch
+template <typename... KArgs, typename... Args>
+static int launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                  bool pdl, Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+    return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+static int topk_threads(int E)
+{
+    int t = ((E + 31) / 32) * 32;
+    if (t < 128)
+        t = 128;
+    if (t > 1024)
+        t = 1024;
+    return t;
+}
+
+// logits for T tokens (no routing tail)
+static int enqueue_logits(const void *x, const void *wr, const float *bias, float *z, float *z_copy,
+                          int T, int d, int E, cudaStream_t s)
+{
+    LogitsArgs a = {};
+    a.x = static_cast<const uint16_t *>(x);
+    a.wr = static_cast<const uint16_t *>(wr);
+    a.bias = bias;
+    a.z = z;
+    a.z_copy = z_copy;
+    a.T = T;
+    a.d = d;
+    a.E = E;
+    a.tail = 0;
+    const int items = E * ((T + kLogitsTok - 1) / kLogitsTok);
+    const int grid = (items + kLogitsWarps - 1) / kLogitsWarps;
+    return launch(k_logits, dim3(grid), dim3(kLogitsWarps * 32), 0, s, true, a);
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+// ========================================================================== ABI
+extern "C" {
+
+const char *moe_status_string(int status)
+{
+    switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_DEVICE_CHECK: return "device-side check failed";
+    default: return "unknown status";
+    }
+}
+
+int moe_version(void) { return 10000; }
+
+size_t moe_workspace_size(int T, int d, int E, int I, int k1)
+{
+    if (check_shape(T, d, E, I, k1) != MOE_OK)
+        return 0;
+    return ws_layout(T, d, E, I, k1).total;
+}
+
+int moe_workspace_init(void *ws, size_t ws_bytes, void *stream)
+{
+    if (!ws || ws_bytes < sizeof(WsHeader) || (reinterpret_cast<uintptr_t>(ws) & 255))
+        return MOE_ERR_INVALID_ARG;
+    return cudaMemsetAsync(ws, 0, sizeof(WsHeader), static_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
+int moe_read_device_status(void *ws, int *status_out, void *stream)
+{
+    if (!ws || !status_out)
+        return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int v = 0;
+    if (cudaMemcpyAsync(&v, ws, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, sizeof(int), s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    *status_out = v;
+    return MOE_OK;
+}
+
+int moe_route(const void *x_bf16, const void *w_router_bf16, const float *bias, float *logits,
+              int T, int d, int E, int k1, int k2, int32_t *topk_idx, float *topk_w, void *ws,
+              size_t ws_bytes, void *stream)
+{
+    int rc = check_route(E, k1, k2);
+    if (rc != MOE_OK)
+        return rc;
+    if (T < 0 || T > kMaxT)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!topk_idx || !topk_w)
+        return MOE_ERR_INVALID_ARG;
+    if (!x_bf16 && !logits)
+        return MOE_ERR_INVALID_ARG;
+    if (x_bf16) {
+        if (!w_router_bf16)
+            return MOE_ERR_INVALID_ARG;
+        if (d < kMinD || d > kMaxD || d % 64)
+            return MOE_ERR_UNSUPPORTED_SHAPE;
+        if (!aligned16(x_bf16) || !aligned16(w_router_bf16))
+            return MOE_ERR_INVALID_ARG;
+        if (!logits) {
+            if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255))
+                return MOE_ERR_INVALID_ARG;
+            const size_t need = sizeof(WsHeader) + align256(sizeof(float) * (size_t)T * E);
+            if (ws_bytes < need)
+                return MOE_ERR_WORKSPACE_TOO_SMALL;
+        }
+    }
+    if (ws && ws_bytes < sizeof(WsHeader))
+        return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (T == 0)
+        return MOE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    DevInfo *di;
+    if ((rc = device_info(di)) != MOE_OK)
+        return rc;
+    const float *z = logits;
+    if (x_bf16) {
+        float *zbuf = logits ? logits : at<float>(ws, sizeof(WsHeader));
+        if ((rc = enqueue_logits(x_bf16, w_router_bf16, bias, zbuf, nullptr, T, d, E, s)) != MOE_OK)
+            return rc;
+        z = zbuf;
+    }
+    PermOut none = {};
+    return launch(k_topk, dim3(T), dim3(topk_threads(E)), 0, s, true, z, T, E, k1, k2, topk_idx,
+                  topk_w, (int32_t *)nullptr, (float *)nullptr, none,
+                  ws ? static_cast<WsHeader *>(ws) : (WsHeader *)nullptr);
+}
+
+int moe_permute(const int32_t *topk_idx, int T, int k1, int E, int32_t *expert_offsets,
+                int32_t *sorted_slot, int32_t *slot_pos, void *ws, size_t ws_bytes, void *stream)
+{
+    if (E < 1 || E > kMaxE)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (k1 < 1 || k1 > kMaxK1 || k1 > E)
+        return MOE_ERR_INVALID_ARG;
+    if (T < 0 || T > kMaxT)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!expert_offsets || (T > 0 && (!topk_idx || !sorted_slot || !slot_pos)))
+        return MOE_ERR_INVALID_ARG;
+    if (ws && ws_bytes < sizeof(WsHeader))
+        return MOE_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    DevInfo *di;
+    int rc;
+    if ((rc = device_info(di)) != MOE_OK)
+        return rc;
+    PermOut po = {expert_offsets, sorted_slot, slot_pos, nullptr, nullptr};
+    int *status = ws ? &static_cast<WsHeader *>(ws)->status : nullptr;
+    return launch(k_permute, dim3(1), dim3(1024), permute_smem_bytes(E, T), s, true, topk_idx, T,
+                  k1, E, po, status);
+}
+
+static int expert_ffn_stream(const void *x, const int32_t *offsets, const int32_t *sorted_slot,
+                             const int32_t *uniq_count, const int32_t *uniq_list, const void *wg,
+                             const void *wu, const void *wd, int T, int d, int E, int I, int k1,
+                             float *h, float *out, void *y, int y_dtype, const float *topk_w,
+                             const int32_t *slot_pos, WsHeader *hdr, cudaStream_t s,
+                             bool pdl = true)
+{
+    DevInfo *di;
+    int rc;
+    if ((rc = device_info(di)) != MOE_OK)
+        return rc;
+    StreamArgs a = {};
+    a.x = static_cast<const uint16_t *>(x);
+    a.wg = static_cast<const uint16_t *>(wg);
+    a.wu = static_cast<const uint16_t *>(wu);
+    a.wd = static_cast<const uint16_t *>(wd);
+    a.T = T;
+    a.d = d;
+    a.E = E;
+    a.I = I;
+    a.k1 = k1;
+    a.offsets = offsets;
+    a.sorted_slot = sorted_slot;
+    a.uniq_count = uniq_count;
+    a.uniq_list = uniq_list;
+    a.h = h;
+    a.out = out;
+    a.y = y;
+    a.y_dtype = y_dtype;
+    a.topk_w = topk_w;
+    a.slot_pos = slot_pos;
+    a.hdr = hdr;
+    return launch(k_stream, dim3(di->num_sms), dim3(kSThreads), stream_smem_bytes(d, I), s, pdl,
+                  a);
+}
+
+int moe_expert_ffn(const void *x_bf16, const int32_t *expert_offsets, const int32_t *sorted_slot,
+                   const void *w_gate_bf16, const void *w_up_bf16, const void *w_down_bf16, int T,
+                   int d, int E, int I, int k1, float *out, int flags, void *ws, size_t ws_bytes,
+                   void *stream)
+{
+    int rc = check_shape(T, d, E, I, k1);
+    if (rc != MOE_OK)
+        return rc;
+    if (flags < MOE_PATH_AUTO || flags > MOE_PATH_GROUPED)
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0)
+        return MOE_OK;
+    if (!x_bf16 || !expert_offsets || !sorted_slot || !w_gate_bf16 || !w_up_bf16 ||
+        !w_down_bf16 || !out || !ws)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x_bf16) || !aligned16(w_gate_bf16) || !aligned16(w_up_bf16) ||
+        !aligned16(w_down_bf16) || !aligned16(out) || (reinterpret_cast<uintptr_t>(ws) & 255))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(T, d, E, I, k1);
+    if (ws_bytes < L.total)
+        return MOE_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    DevInfo *di;
+    if ((rc = device_info(di)) != MOE_OK)
+        return rc;
+    if ((rc = launch(k_uniq_from_offsets, dim3(1), dim3(1024), 0, s, true, expert_offsets, E,
+                     at<int32_t>(ws, L.uniq_count), at<int32_t>(ws, L.uniq_list))) != MOE_OK)
+        return rc;
+    return expert_ffn_stream(x_bf16, expert_offsets, sorted_slot, at<int32_t>(ws, L.uniq_count),
+                             at<int32_t>(ws, L.uniq_list), w_gate_bf16, w_up_bf16, w_down_bf16, T,
+                             d, E, I, k1, at<float>(ws, L.h), out, nullptr, 0, nullptr, nullptr,
+                             static_cast<WsHeader *>(ws), s);
+}
+
+int moe_combine(const float *expert_out, const int32_t *slot_pos, const float *topk_w, int T,
+                int d, int k1, void *y, int y_dtype, void *stream)
+{
+    if (T < 0 || T > kMaxT || d < kMinD || d > kMaxD || d % 64)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (k1 < 1 || k1 > kMaxK1 || (y_dtype != MOE_DTYPE_F32 && y_dtype != MOE_DTYPE_BF16))
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0)
+        return MOE_OK;
+    if (!expert_out || !slot_pos || !topk_w || !y || !aligned16(expert_out) || !aligned16(y))
+        return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int per_block = 4 * kCombineThreads;
+    return launch(k_combine, dim3((d + per_block - 1) / per_block, T), dim3(kCombineThreads), 0, s,
+                  true, expert_out, slot_pos, topk_w, T, d, k1, y, y_dtype, (int *)nullptr);
+}
+
+int moe_layer(const void *x_bf16, const void *w_router_bf16, const float *bias,
+              const void *w_gate_bf16, const void *w_up_bf16, const void *w_down_bf16, int T, int d,
+              int E, int I, int k1, int k2, void *y, int y_dtype, int32_t *topk_idx_out,
+              float *topk_w_out, float *logits_out, int flags, void *ws, size_t ws_bytes,
+              void *stream)
+{
+    int rc = check_shape(T, d, E, I, k1);
+    if (rc != MOE_OK)
+        return rc;
+    if ((rc = check_route(E, k1, k2)) != MOE_OK)
+        return rc;
+    if (flags < MOE_PATH_AUTO || flags > MOE_PATH_GROUPED)
+        return MOE_ERR_INVALID_ARG;
+    if (y_dtype != MOE_DTYPE_F32 && y_dtype != MOE_DTYPE_BF16)
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0)
+        return MOE_OK;
+    if (!x_bf16 || !w_router_bf16 || !w_gate_bf16 || !w_up_bf16 || !w_down_bf16 || !y || !ws)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x_bf16) || !aligned16(w_router_bf16) || !aligned16(w_gate_bf16) ||
+        !aligned16(w_up_bf16) || !aligned16(w_down_bf16) || (reinterpret_cast<uintptr_t>(ws) & 255))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(T, d, E, I, k1);
+    if (ws_bytes < L.total)
+        return MOE_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    DevInfo *di;
+    if ((rc = device_info(di)) != MOE_OK)
+        return rc;
+    WsHeader *hdr = static_cast<WsHeader *>(ws);
+    float *z = at<float>(ws, L.logits);
+    int32_t *idx = at<int32_t>(ws, L.idx);
+    float *w = at<float>(ws, L.w);
+    PermOut po = {at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.sorted_slot),
+                  at<int32_t>(ws, L.slot_pos), at<int32_t>(ws, L.uniq_count),
+                  at<int32_t>(ws, L.uniq_list)};
+
+    if (T == 1) {
+        // router + last-block routing and permutation in one kernel
+        LogitsArgs a = {};
+        a.x = static_cast<const uint16_t *>(x_bf16);
+        a.wr = static_cast<const uint16_t *>(w_router_bf16);
+        a.bias = bias;
+        a.z = z;
+        a.z_copy = logits_out;
+        a.T = 1;
+        a.d = d;
+        a.E = E;
+        a.tail = 1;
+        a.k1 = k1;
+        a.k2 = k2;
+        a.idx = idx;
+        a.w = w;
+        a.idx_copy = topk_idx_out;
+        a.w_copy = topk_w_out;
+        a.perm = po;
+        a.hdr = hdr;
+        const int grid = (E + kLogitsWarps - 1) / kLogitsWarps;
+        if ((rc = launch(k_logits, dim3(grid), dim3(kLogitsWarps * 32), permute_smem_bytes(E, 1),
+                         s, true, a)) != MOE_OK)
+            return rc;
+    } else {
+        if ((rc = enqueue_logits(x_bf16, w_router_bf16, bias, z, logits_out, T, d, E, s)) != MOE_OK)
+            return rc;
+        if ((rc = launch(k_topk, dim3(T), dim3(topk_threads(E)), permute_smem_bytes(E, T), s, true,
+                         (const float *)z, T, E, k1, k2, idx, w, topk_idx_out, topk_w_out, po,
+                         hdr)) != MOE_OK)
+            return rc;
+    }
+    return expert_ffn_stream(x_bf16, po.offsets, po.sorted_slot, po.uniq_count, po.uniq_list,
+                             w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I, k1, at<float>(ws, L.h),
+                             at<float>(ws, L.out), y, y_dtype, w, po.slot_pos, hdr, s);
+}
+
+int moe_test_exp_c(const float *x, float *y, int64_t n, void *stream)
+{
+    if (n < 0 || (n > 0 && (!x || !y)))
+        return MOE_ERR_INVALID_ARG;
+    if (n == 0)
+        return MOE_OK;
+    int64_t blocks = (n + 255) / 256;
+    if (blocks > 65535 * 16)
+        blocks = 65535 * 16;
+    return launch(k_test_expc, dim3((unsigned)blocks), dim3(256), 0,
+                  static_cast<cudaStream_t>(stream), false, x, y, n);
+}
+
+int moe_test_expert_stream(const void *x_bf16, const void *w_gate_bf16, const void *w_up_bf16,
+                           const void *w_down_bf16, int T, int d, int E, int I, int k1, void *y,
+                           int y_dtype, void *ws, size_t ws_bytes, void *stream)
+{
+    int rc = check_shape(T, d, E, I, k1);
+    if (rc != MOE_OK)
+        return rc;
+    if (T == 0)
+        return MOE_OK;
+    if (!x_bf16 || !w_gate_bf16 || !w_up_bf16 || !w_down_bf16 || !y || !ws)
+        return MOE_ERR_INVALID_ARG;
+    if (y_dtype != MOE_DTYPE_F32 && y_dtype != MOE_DTYPE_BF16)
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(T, d, E, I, k1);
+    if (ws_bytes < L.total)
+        return MOE_ERR_WORKSPACE_TOO_SMALL;
+    return expert_ffn_stream(x_bf16, at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.sorted_slot),
+                             at<int32_t>(ws, L.uniq_count), at<int32_t>(ws, L.uniq_list),
+                             w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I, k1, at<float>(ws, L.h),
+                             at<float>(ws, L.out), y, y_dtype, at<float>(ws, L.w),
+                             at<int32_t>(ws, L.slot_pos), static_cast<WsHeader *>(ws),
+                             static_cast<cudaStream_t>(stream), false);
+}
+
+int moe_test_num_sms(void)
+{
+    DevInfo *di;
+    if (device_info(di) != MOE_OK)
+        return 0;
+    return di->num_sms;
+}
+
+}  // extern "C"

@@ -1,0 +1,534 @@
+// route.cuh -- router logits, float32 softmax, top-k1/top-k2 selection with
+// the decoupled renormalisation of Eq. 2, and the stable counting sort that
+// groups routed slots by expert.
+//
+// Eq. 2 ("Paper of the Week #3 -- Half the FLOPs Is Not Half the Time",
+// section "The Receipt"): w_i = p_i / sum_{j in Top-k2} p_j, i in Top-k1;
+// k2 >= E means no division.  Order of operations ("Code of the Week"
+// section of the same page): float32 softmax, top min(k2, E) in descending
+// order, first k1 kept, divided by the sum of all min(k2, E) taken values.
+//
+// The float32 softmax and the top-k2 mass follow one fixed sequence of
+// IEEE-754 binary32 operations so the result is reproducible bit for bit:
+//   m   = max_j z_j
+//   e_j = expc(z_j - m)                       (expc: see below)
+//   Z   : 32 partial sums, partial q adds e_q, e_{q+32}, ... in order from +0;
+//         then five butterfly rounds P[q] <- P[q] + P[q ^ o], o = 16..1
+//   p_j = e_j / Z                             (round-to-nearest division)
+//   rank by (p descending, j ascending); K = min(k2, E)
+//   S   = (((p_(0) + p_(1)) + ...) + p_(K-1)) in rank order (k2 < E only)
+//   w_s = p_(s) / S   (k2 < E)   or   p_(s)   (k2 >= E),   s < k1.
+// Every float operation below that takes part in this sequence is written
+// with an explicit round-to-nearest intrinsic so the compiler cannot fuse or
+// reorder it.
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// expc: float32 exponential for x <= 88, from Cody & Waite's two-constant
+// argument reduction (W. J. Cody, W. Waite, "Software Manual for the
+// Elementary Functions", 1980) and the Taylor series of e^r up to r^7 in
+// Horner form with fused multiply-adds; 2^n applied through exponent bits.
+// ln2 split: the high part is ln 2 cut to 12 significant bits (n * hi is
+// exact for |n| < 2^12), the low part is float32(ln 2 - hi).  Below -87 (and
+// for NaN) the result is +0, so results are never subnormal.
+__device__ __forceinline__ float expc(float x)
+{
+    const float kLog2e = 0x1.715476p+0f;
+    const float kLn2Hi = 0x1.62ep-1f;
+    const float kLn2Lo = 0x1.0bfbe8p-15f;
+    if (!(x >= -87.0f))
+        return 0.0f;
+    if (x > 88.0f)
+        return __int_as_float(0x7f800000);
+    const float n = rintf(__fmul_rn(x, kLog2e));
+    float r = __fmaf_rn(-n, kLn2Hi, x);
+    r = __fmaf_rn(-n, kLn2Lo, r);
+    float p = 0x1.a01a02p-13f;             // 1/7!
+    p = __fmaf_rn(p, r, 0x1.6c16c2p-10f);  // 1/6!
+    p = __fmaf_rn(p, r, 0x1.111112p-7f);   // 1/5!
+    p = __fmaf_rn(p, r, 0x1.555556p-5f);   // 1/4!
+    p = __fmaf_rn(p, r, 0x1.555556p-3f);   // 1/3!
+    p = __fmaf_rn(p, r, 0x1p-1f);          // 1/2!
+    p = __fmaf_rn(p, r, 1.0f);
+    p = __fmaf_rn(p, r, 1.0f);
+    const int ni = (int)n;
+    return __fmul_rn(p, __int_as_float((ni + 127) << 23));
+}
+
+__global__ void k_test_expc(const float *x, float *y, int64_t n)
+{
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x)
+        y[i] = expc(x[i]);
+}
+
+// ---------------------------------------------------------------------------
+// One CTA routes one token whose E logits sit in shared memory.
+// Shared scratch (caller-provided): ps[E], sel_p[E], sel_j[E], red[64].
+// Writes idx_out[s], w_out[s] for s < k1 (global).  All threads of the CTA
+// must call it.
+struct __align__(16) RouteSmem {
+    float ps[1024];
+    float sel_p[1024];
+    int sel_j[1024];
+    float red[64];
+};
+
+__device__ void route_token_block(const float *zs, int E, int k1, int k2, RouteSmem &sm,
+                                  int32_t *idx_out, float *w_out, int32_t *idx_copy,
+                                  float *w_copy)
+{
+    const int tid = threadIdx.x, nt = blockDim.x;
+    const int lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
+    const int K = k2 < E ? k2 : E;
+    const bool renorm = k2 < E;
+    const int Kneed = renorm ? K : k1;
+
+    // m = max_j z_j (exact in any order)
+    float m = -__int_as_float(0x7f800000);
+    for (int j = tid; j < E; j += nt)
+        m = fmaxf(m, zs[j]);
+    for (int o = 16; o >= 1; o >>= 1)
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0)
+        sm.red[warp] = m;
+    __syncthreads();
+    if (warp == 0) {
+        float v = lane < nw ? sm.red[lane] : -__int_as_float(0x7f800000);
+        for (int o = 16; o >= 1; o >>= 1)
+            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+        if (lane == 0)
+            sm.red[32] = v;
+    }
+    __syncthreads();
+    m = sm.red[32];
+
+    for (int j = tid; j < E; j += nt)
+        sm.ps[j] = expc(__fsub_rn(zs[j], m));
+    __syncthreads();
+
+    // Z in the canonical 32-partial order, then the butterfly
+    if (warp == 0) {
+        float acc = 0.0f;
+        for (int j = lane; j < E; j += 32)
+            acc = __fadd_rn(acc, sm.ps[j]);
+        for (int o = 16; o >= 1; o >>= 1)
+            acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o));
+        if (lane == 0)
+            sm.red[33] = acc;
+    }
+    __syncthreads();
+    const float Z = sm.red[33];
+    for (int j = tid; j < E; j += nt)
+        sm.ps[j] = __fdiv_rn(sm.ps[j], Z);
+    __syncthreads();
+
+    // rank_j = #{i : p_i > p_j} + #{i < j : p_i == p_j}; keep rank < Kneed
+    for (int j = tid; j < E; j += nt) {
+        const float pj = sm.ps[j];
+        int r = 0;
+        int i = 0;
+        for (; i + 4 <= E; i += 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(&sm.ps[i]);
+            r += (v.x > pj) | ((v.x == pj) & (i + 0 < j));
+            r += (v.y > pj) | ((v.y == pj) & (i + 1 < j));
+            r += (v.z > pj) | ((v.z == pj) & (i + 2 < j));
+            r += (v.w > pj) | ((v.w == pj) & (i + 3 < j));
+        }
+        for (; i < E; ++i) {
+            const float v = sm.ps[i];
+            r += (v > pj) | ((v == pj) & (i < j));
+        }
+        if (r < Kneed) {
+            sm.sel_p[r] = pj;
+            sm.sel_j[r] = j;
+        }
+    }
+    __syncthreads();
+    if (renorm && tid == 0) {
+        float S = 0.0f;
+        for (int r = 0; r < K; ++r)
+            S = __fadd_rn(S, sm.sel_p[r]);
+        sm.red[34] = S;
+    }
+    __syncthreads();
+    if (tid < k1) {
+        const float p = sm.sel_p[tid];
+        const int j = sm.sel_j[tid];
+        const float wv = renorm ? __fdiv_rn(p, sm.red[34]) : p;
+        idx_out[tid] = j;
+        w_out[tid] = wv;
+        if (idx_copy)
+            idx_copy[tid] = j;
+        if (w_copy)
+            w_copy[tid] = wv;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Block-wide exclusive scan of n ints (in place in smem), returns the total.
+// scratch: >= 33 ints.
+__device__ int block_exclusive_scan(int *v, int n, int *scratch)
+{
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
+    const int per = (n + nt - 1) / nt;
+    const int b = tid * per, e = min(n, b + per);
+    int local = 0;
+    for (int i = b; i < e; ++i)
+        local += v[i];
+    int incl = local;
+    for (int o = 1; o < 32; o <<= 1) {
+        int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o)
+            incl += t;
+    }
+    if (lane == 31)
+        scratch[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int nw = nt >> 5;
+        int t = lane < nw ? scratch[lane] : 0;
+        int s = t;
+        for (int o = 1; o < 32; o <<= 1) {
+            int u = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o)
+                s += u;
+        }
+        scratch[lane] = s - t;  // exclusive prefix of warp totals
+        if (lane == 31)
+            scratch[32] = s;
+    }
+    __syncthreads();
+    int run = scratch[warp] + incl - local;
+    for (int i = b; i < e; ++i) {
+        const int t = v[i];
+        v[i] = run;
+        run += t;
+    }
+    const int total = scratch[32];
+    __syncthreads();
+    return total;
+}
+
+// ---------------------------------------------------------------------------
+// Stable counting sort of the n = T*k1 slots by expert, one CTA.
+// Token chunks of 32*WC tokens are marked in a per-expert bitmap (bit l of
+// word w of expert e = token t0 + 32w + l routes to e); the stable position
+// of slot (t, s) is offsets[e] + (#tokens before t routed to e), counted with
+// popc over the bitmap rows.
+// smem (dynamic, ints): cnt[E+1] | run[E] | bits[E*WC] | pref[E*WC] | scan[40]
+// Outputs: expert_offsets[E+1], sorted_slot[n], slot_pos[n],
+// uniq_count[1], uniq_list[U] (activated experts, ascending).
+struct PermOut {
+    int32_t *offsets;
+    int32_t *sorted_slot;
+    int32_t *slot_pos;
+    int32_t *uniq_count;  // nullable
+    int32_t *uniq_list;   // nullable
+};
+
+// 32-token words of the bitmap handled per chunk: bounded by 32, by a 4096-word
+// bitmap, and by the tokens there are.
+__host__ __device__ inline int permute_words_per_chunk(int E, int T)
+{
+    int wc = 4096 / (E > 0 ? E : 1);
+    const int need = (T + 31) / 32;
+    if (wc > 32)
+        wc = 32;
+    if (wc > need)
+        wc = need;
+    return wc < 1 ? 1 : wc;
+}
+
+__device__ void permute_block(const int32_t *idx, int T, int k1, int E, PermOut out, int *smem,
+                              int *status)
+{
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
+    const int WC = permute_words_per_chunk(E, T);
+    int *cnt = smem;
+    int *run = cnt + (E + 1);
+    unsigned *bits = reinterpret_cast<unsigned *>(run + E);
+    int *pref = reinterpret_cast<int *>(bits + E * WC);
+    int *scan = pref + E * WC;
+    const int n = T * k1;
+
+    for (int e = tid; e <= E; e += nt)
+        cnt[e] = 0;
+    __syncthreads();
+    // pass 1: per-expert counts, warp-aggregated
+    for (int base = warp * 32; base < n; base += nt) {
+        const int i = base + lane;
+        int e = i < n ? __ldcg(&idx[i]) : -1;
+        const bool valid = (e >= 0) & (e < E);
+        if (i < n && !valid)
+            set_status(status, MOE_ERR_DEVICE_CHECK);
+        const int key = valid ? e : -1;
+        const unsigned grp = __match_any_sync(0xffffffffu, key);
+        if (valid && lane == __ffs(grp) - 1)
+            atomicAdd(&cnt[e], __popc(grp));
+    }
+    __syncthreads();
+    // uniq list from the counts (before the scan overwrites them)
+    for (int e = tid; e < E; e += nt)
+        run[e] = cnt[e] > 0 ? 1 : 0;
+    __syncthreads();
+    const int U = block_exclusive_scan(run, E, scan);
+    if (out.uniq_list)
+        for (int e = tid; e < E; e += nt)
+            if (cnt[e] > 0)
+                out.uniq_list[run[e]] = e;
+    if (out.uniq_count && tid == 0)
+        *out.uniq_count = U;
+    __syncthreads();
+    block_exclusive_scan(cnt, E + 1, scan);  // cnt[e] = offsets[e], cnt[E] = n
+    for (int e = tid; e <= E; e += nt)
+        out.offsets[e] = cnt[e];
+    for (int e = tid; e < E; e += nt)
+        run[e] = 0;
+    __syncthreads();
+
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int t0 = 0; t0 < T; t0 += 32 * WC) {
+        for (int i = tid; i < E * WC; i += nt)
+            bits[i] = 0u;
+        __syncthreads();
+        for (int w = warp; w < WC; w += nw) {
+            const int t = t0 + 32 * w + lane;
+            for (int s = 0; s < k1; ++s) {
+                int e = t < T ? __ldcg(&idx[t * k1 + s]) : -1;
+                const bool valid = (e >= 0) & (e < E);
+                const int key = valid ? e : -1;
+                const unsigned grp = __match_any_sync(0xffffffffu, key);
+                if (valid && lane == __ffs(grp) - 1) {
+                    if (bits[e * WC + w] & grp)
+                        set_status(status, MOE_ERR_DEVICE_CHECK);  // repeated expert in a token
+                    bits[e * WC + w] |= grp;
+                }
+                __syncwarp();
+            }
+        }
+        __syncthreads();
+        for (int e = tid; e < E; e += nt) {
+            int acc = run[e];
+            for (int w = 0; w < WC; ++w) {
+                pref[e * WC + w] = acc;
+                acc += __popc(bits[e * WC + w]);
+            }
+            run[e] = acc;
+        }
+        __syncthreads();
+        for (int w = warp; w < WC; w += nw) {
+            const int t = t0 + 32 * w + lane;
+            if (t < T) {
+                for (int s = 0; s < k1; ++s) {
+                    const int e = __ldcg(&idx[t * k1 + s]);
+                    if (e < 0 || e >= E)
+                        continue;
+                    const int pos = cnt[e] + pref[e * WC + w] + __popc(bits[e * WC + w] & lt_mask);
+                    out.sorted_slot[pos] = t * k1 + s;
+                    out.slot_pos[t * k1 + s] = pos;
+                }
+            }
+        }
+        __syncthreads();
+    }
+}
+
+__host__ __device__ inline size_t permute_smem_bytes(int E, int T)
+{
+    const int WC = permute_words_per_chunk(E, T);
+    return sizeof(int) * ((size_t)(E + 1) + E + 2 * (size_t)E * WC + 40);
+}
+
+// ---------------------------------------------------------------------------
+// k_permute: standalone permutation (one CTA).
+__global__ void __launch_bounds__(1024) k_permute(const int32_t *idx, int T, int k1, int E,
+                                                  PermOut out, int *status)
+{
+    extern __shared__ int dsm[];
+    pdl_wait();
+    pdl_trigger();
+    permute_block(idx, T, k1, E, out, dsm, status);
+}
+
+// ---------------------------------------------------------------------------
+// k_topk: one CTA per token routes from float32 logits [T x E].  With
+// `perm.offsets` non-null, the last CTA to finish also runs the permutation
+// of all T*k1 slots (last-block hand-off through hdr->route_arrive).
+__global__ void __launch_bounds__(1024) k_topk(const float *logits, int T, int E, int k1, int k2,
+                                               int32_t *idx, float *w, int32_t *idx_copy,
+                                               float *w_copy, PermOut perm, WsHeader *hdr)
+{
+    __shared__ RouteSmem sm;
+    __shared__ float zs[1024];
+    __shared__ int is_last;
+    extern __shared__ int dsm[];
+    pdl_wait();
+    pdl_trigger();
+    int *status = hdr ? &hdr->status : nullptr;
+    for (int t = blockIdx.x; t < T; t += gridDim.x) {
+        for (int j = threadIdx.x; j < E; j += blockDim.x)
+            zs[j] = logits[(size_t)t * E + j];
+        __syncthreads();
+        route_token_block(zs, E, k1, k2, sm, idx + (size_t)t * k1, w + (size_t)t * k1,
+                          idx_copy ? idx_copy + (size_t)t * k1 : nullptr,
+                          w_copy ? w_copy + (size_t)t * k1 : nullptr);
+        __syncthreads();
+    }
+    if (perm.offsets == nullptr)
+        return;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned prev = atomicAdd(&hdr->route_arrive, 1u);
+        is_last = (prev == gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!is_last)
+        return;
+    if (threadIdx.x == 0)
+        hdr->route_arrive = 0u;
+    __threadfence();
+    permute_block(idx, T, k1, E, perm, dsm, status);
+}
+
+// ---------------------------------------------------------------------------
+// k_logits: z[t, e] = sum_k x[t, k] W_r[e, k] (+ b[e]) with float32
+// accumulation.  One warp per (expert, chunk of up to 8 tokens).  The warp's
+// W_r row is loaded into registers before the programmatic-launch wait (the
+// router weights never depend on earlier kernels), so its HBM latency
+// overlaps the previous kernel.  With `tail` set (T == 1), the last CTA to
+// finish routes the token and builds the permutation.
+constexpr int kLogitsWarps = 8;
+constexpr int kLogitsTok = 8;
+constexpr int kLogitsMaxVec = 16;  // register prefetch covers d <= 4096
+
+struct LogitsArgs {
+    const uint16_t *x;
+    const uint16_t *wr;
+    const float *bias;
+    float *z;          // [T x E] output (workspace or caller)
+    float *z_copy;     // nullable second copy (caller's logits_out)
+    int T, d, E;
+    // tail (T == 1): route + permute by the last CTA
+    int tail;
+    int k1, k2;
+    int32_t *idx;
+    float *w;
+    int32_t *idx_copy;
+    float *w_copy;
+    PermOut perm;
+    WsHeader *hdr;
+};
+
+__global__ void __launch_bounds__(kLogitsWarps * 32) k_logits(LogitsArgs a)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nchunk = (a.T + kLogitsTok - 1) / kLogitsTok;
+    const int item = blockIdx.x * kLogitsWarps + warp;
+    const int nitems = a.E * nchunk;
+    const int nvec = a.d >> 3;  // 16-byte vectors per row
+    const bool has_item = item < nitems;
+    const int e = has_item ? item % a.E : 0;
+    const int chunk = has_item ? item / a.E : 0;
+
+    uint4 wv[kLogitsMaxVec];
+    const bool prefetch = nvec <= 32 * kLogitsMaxVec;
+    if (has_item && prefetch) {
+        const uint4 *row = reinterpret_cast<const uint4 *>(a.wr + (size_t)e * a.d);
+#pragma unroll
+        for (int i = 0; i < kLogitsMaxVec; ++i) {
+            const int v = lane + 32 * i;
+            wv[i] = v < nvec ? ld_nc_v4(row + v) : make_uint4(0, 0, 0, 0);
+        }
+    }
+    pdl_wait();
+    pdl_trigger();
+
+    if (has_item) {
+        const uint4 *row = reinterpret_cast<const uint4 *>(a.wr + (size_t)e * a.d);
+        const int t0 = chunk * kLogitsTok;
+        const int nt = min(kLogitsTok, a.T - t0);
+        float acc[kLogitsTok];
+#pragma unroll
+        for (int t = 0; t < kLogitsTok; ++t)
+            acc[t] = 0.0f;
+        if (prefetch) {
+#pragma unroll
+            for (int i = 0; i < kLogitsMaxVec; ++i) {
+                const int v = lane + 32 * i;
+                if (v < nvec) {
+#pragma unroll
+                    for (int t = 0; t < kLogitsTok; ++t) {
+                        if (t < nt) {
+                            const uint4 xv = *(reinterpret_cast<const uint4 *>(
+                                                   a.x + (size_t)(t0 + t) * a.d) +
+                                               v);
+                            float xf[8] = {bf16lo(xv.x), bf16hi(xv.x), bf16lo(xv.y), bf16hi(xv.y),
+                                           bf16lo(xv.z), bf16hi(xv.z), bf16lo(xv.w), bf16hi(xv.w)};
+                            acc[t] = dot8_bf16(wv[i], xf, acc[t]);
+                        }
+                    }
+                }
+            }
+        } else {
+            for (int v = lane; v < nvec; v += 32) {
+                const uint4 wq = ld_nc_v4(row + v);
+#pragma unroll
+                for (int t = 0; t < kLogitsTok; ++t) {
+                    if (t < nt) {
+                        const uint4 xv =
+                            *(reinterpret_cast<const uint4 *>(a.x + (size_t)(t0 + t) * a.d) + v);
+                        float xf[8] = {bf16lo(xv.x), bf16hi(xv.x), bf16lo(xv.y), bf16hi(xv.y),
+                                       bf16lo(xv.z), bf16hi(xv.z), bf16lo(xv.w), bf16hi(xv.w)};
+                        acc[t] = dot8_bf16(wq, xf, acc[t]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < kLogitsTok; ++t) {
+            if (t < nt) {
+                float s = warp_sum(acc[t]);
+                if (lane == 0) {
+                    if (a.bias)
+                        s = s + a.bias[e];
+                    a.z[(size_t)(t0 + t) * a.E + e] = s;
+                    if (a.z_copy)
+                        a.z_copy[(size_t)(t0 + t) * a.E + e] = s;
+                }
+            }
+        }
+    }
+    if (!a.tail)
+        return;
+
+    // last-block hand-off: the final CTA routes the single token
+    __shared__ int is_last;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned prev = atomicAdd(&a.hdr->route_arrive, 1u);
+        is_last = (prev == gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!is_last)
+        return;
+    if (threadIdx.x == 0)
+        a.hdr->route_arrive = 0u;
+    __threadfence();
+    __shared__ RouteSmem sm;
+    __shared__ float zs[1024];
+    for (int j = threadIdx.x; j < a.E; j += blockDim.x)
+        zs[j] = __ldcg(&a.z[j]);
+    __syncthreads();
+    route_token_block(zs, a.E, a.k1, a.k2, sm, a.idx, a.w, a.idx_copy, a.w_copy);
+    __syncthreads();
+    extern __shared__ int dsm[];
+    permute_block(a.idx, 1, a.k1, a.E, a.perm, dsm, &a.hdr->status);
+}
+
+}  // namespace moe

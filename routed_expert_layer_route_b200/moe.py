@@ -1,0 +1,206 @@
+"""ctypes binding of libmoe.so.  Argument marshalling only: every step of the
+layer runs in the library's CUDA kernels.  The call names are those of
+include/moe.h; arguments are torch tensors on the current CUDA device (or
+None where the C call takes NULL).  A non-OK status raises MoeError.
+
+There is no fallback: if libmoe.so is missing or fails to load, every call
+raises.
+"""
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoe.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = -1
+MOE_ERR_UNSUPPORTED_SHAPE = -2
+MOE_ERR_WORKSPACE_TOO_SMALL = -3
+MOE_ERR_CUDA = -4
+MOE_ERR_TIMEOUT = -5
+MOE_ERR_DEVICE_CHECK = -6
+
+MOE_DTYPE_F32 = 0
+MOE_DTYPE_BF16 = 1
+
+MOE_PATH_AUTO = 0
+MOE_PATH_STREAM = 1
+MOE_PATH_GROUPED = 2
+
+# every symbol include/*.h declares, with (restype, argtypes)
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_sz = ctypes.c_size_t
+SIGNATURES = {
+    "moe_status_string": (ctypes.c_char_p, [_i]),
+    "moe_version": (_i, []),
+    "moe_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
+    "moe_workspace_init": (_i, [_vp, _sz, _vp]),
+    "moe_read_device_status": (_i, [_vp, ctypes.POINTER(_i), _vp]),
+    "moe_route": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp]),
+    "moe_permute": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_expert_ffn": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _sz,
+                            _vp]),
+    "moe_combine": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _i, _vp]),
+    "moe_layer": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp,
+                       _vp, _i, _vp, _sz, _vp]),
+    "moe_test_exp_c": (_i, [_vp, _vp, ctypes.c_int64, _vp]),
+    "moe_test_num_sms": (_i, []),
+    "moe_test_expert_stream": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _sz,
+                                    _vp]),
+}
+
+_lib = None
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__("%s failed: %s (%d)" % (where, status_string(status), status))
+
+
+def lib():
+    """Load libmoe.so (raises if it is missing: there is no CPU fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libmoe.so not built (%s); run python -m "
+                               "routed_expert_layer_route_b200.build" % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(status):
+    return lib().moe_status_string(int(status)).decode()
+
+
+def _p(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc, where):
+    if rc != MOE_OK:
+        raise MoeError(rc, where)
+
+
+def moe_version():
+    return lib().moe_version()
+
+
+def moe_workspace_size(T, d, E, I, k1):
+    return lib().moe_workspace_size(T, d, E, I, k1)
+
+
+def moe_workspace_init(ws, stream=None):
+    _check(lib().moe_workspace_init(_p(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "moe_workspace_init")
+
+
+def moe_read_device_status(ws, stream=None):
+    v = ctypes.c_int(0)
+    _check(lib().moe_read_device_status(_p(ws), ctypes.byref(v), _stream(stream)),
+           "moe_read_device_status")
+    return v.value
+
+
+def workspace(T, d, E, I, k1, device=None):
+    """Allocate (torch) and initialise a workspace for these shapes."""
+    n = moe_workspace_size(T, d, E, I, k1)
+    if n == 0:
+        raise MoeError(MOE_ERR_UNSUPPORTED_SHAPE, "moe_workspace_size")
+    ws = torch.empty(n, dtype=torch.uint8, device=device or torch.device("cuda"))
+    moe_workspace_init(ws)
+    return ws
+
+
+def _ws_args(ws):
+    if ws is None:
+        return None, 0
+    return _p(ws), ws.numel() * ws.element_size()
+
+
+def moe_route(x, w_router, bias, logits, k1, k2, topk_idx, topk_w, ws=None, stream=None, T=None,
+              d=None, E=None):
+    """x None: route the given float32 logits [T x E]; else compute them."""
+    if x is not None:
+        T, d = x.shape
+        E = w_router.shape[0]
+    else:
+        T, E = logits.shape
+        d = d or 0
+    wsp, wsn = _ws_args(ws)
+    _check(lib().moe_route(_p(x), _p(w_router), _p(bias), _p(logits), T, d, E, k1, k2,
+                           _p(topk_idx), _p(topk_w), wsp, wsn, _stream(stream)), "moe_route")
+
+
+def moe_permute(topk_idx, E, expert_offsets, sorted_slot, slot_pos, ws=None, stream=None):
+    T, k1 = topk_idx.shape
+    wsp, wsn = _ws_args(ws)
+    _check(lib().moe_permute(_p(topk_idx), T, k1, E, _p(expert_offsets), _p(sorted_slot),
+                             _p(slot_pos), wsp, wsn, _stream(stream)), "moe_permute")
+
+
+def moe_expert_ffn(x, expert_offsets, sorted_slot, w_gate, w_up, w_down, k1, out, ws,
+                   flags=MOE_PATH_AUTO, stream=None):
+    T, d = x.shape
+    E, I, _ = w_gate.shape
+    wsp, wsn = _ws_args(ws)
+    _check(lib().moe_expert_ffn(_p(x), _p(expert_offsets), _p(sorted_slot), _p(w_gate), _p(w_up),
+                                _p(w_down), T, d, E, I, k1, _p(out), flags, wsp, wsn,
+                                _stream(stream)), "moe_expert_ffn")
+
+
+def moe_combine(expert_out, slot_pos, topk_w, y, stream=None):
+    T, k1 = topk_w.shape
+    d = y.shape[1]
+    y_dtype = MOE_DTYPE_BF16 if y.dtype == torch.bfloat16 else MOE_DTYPE_F32
+    _check(lib().moe_combine(_p(expert_out), _p(slot_pos), _p(topk_w), T, d, k1, _p(y), y_dtype,
+                             _stream(stream)), "moe_combine")
+
+
+def moe_layer(x, w_router, bias, w_gate, w_up, w_down, k1, k2, y, ws, topk_idx_out=None,
+              topk_w_out=None, logits_out=None, flags=MOE_PATH_AUTO, stream=None):
+    T, d = x.shape
+    E, I, _ = w_gate.shape
+    y_dtype = MOE_DTYPE_BF16 if y.dtype == torch.bfloat16 else MOE_DTYPE_F32
+    wsp, wsn = _ws_args(ws)
+    _check(lib().moe_layer(_p(x), _p(w_router), _p(bias), _p(w_gate), _p(w_up), _p(w_down), T, d,
+                           E, I, k1, k2, _p(y), y_dtype, _p(topk_idx_out), _p(topk_w_out),
+                           _p(logits_out), flags, wsp, wsn, _stream(stream)), "moe_layer")
+
+
+def moe_test_exp_c(x, y, stream=None):
+    _check(lib().moe_test_exp_c(_p(x), _p(y), x.numel(), _stream(stream)), "moe_test_exp_c")
+
+
+def moe_test_num_sms():
+    return lib().moe_test_num_sms()
+
+
+def moe_test_expert_stream(x, w_gate, w_up, w_down, k1, y, ws, stream=None):
+    T, d = x.shape
+    E, I, _ = w_gate.shape
+    y_dtype = MOE_DTYPE_BF16 if y.dtype == torch.bfloat16 else MOE_DTYPE_F32
+    wsp, wsn = _ws_args(ws)
+    _check(lib().moe_test_expert_stream(_p(x), _p(w_gate), _p(w_up), _p(w_down), T, d, E, I, k1,
+                                        _p(y), y_dtype, wsp, wsn, _stream(stream)),
+           "moe_test_expert_stream")

@@ -1,0 +1,95 @@
+"""Helpers shared by the GPU parity tests: run the C-ABI path on seeded
+inputs and compare with the CPU oracle.
+
+Tolerances (layer output, float32 accumulation on bf16-rounded inputs):
+max-abs error 2e-2 and relative L2 error 5e-3 against the oracle.  Routing
+indices and weights are compared bit for bit, the oracle routing the GPU's
+own float32 logits (so a near-tie at the k1 boundary cannot turn a
+last-bit logit difference into an O(1) output difference); the logits
+themselves are checked separately against the oracle's.
+"""
+import numpy as np
+import torch
+
+import oracle
+from routed_expert_layer_route_b200 import moe, synth
+
+MAX_ABS = 2e-2
+REL_L2 = 5e-3
+
+
+def rel_l2(a, b):
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+
+
+def assert_close_layer(y_gpu, y_ref, what=""):
+    err = float(np.abs(y_gpu - y_ref).max()) if y_ref.size else 0.0
+    rel = rel_l2(y_gpu, y_ref) if y_ref.size else 0.0
+    assert err <= MAX_ABS and rel <= REL_L2, "%s max-abs %.3g rel-L2 %.3g" % (what, err, rel)
+    return err, rel
+
+
+def logits_bound(x, w):
+    d = x.shape[-1]
+    return 1e-4 * np.sqrt(d) * float(x.abs().max()) * float(w.abs().max())
+
+
+def run_layer(L, k1, k2, y_dtype=torch.float32, flags=moe.MOE_PATH_AUTO, ws=None):
+    T, d = L.x.shape
+    E, I, _ = L.w_gate.shape
+    dev = L.x.device
+    if ws is None:
+        ws = moe.workspace(T, d, E, I, k1, device=dev)
+    y = torch.empty(T, d, device=dev, dtype=y_dtype)
+    idx = torch.empty(T, k1, device=dev, dtype=torch.int32)
+    w = torch.empty(T, k1, device=dev, dtype=torch.float32)
+    z = torch.empty(T, E, device=dev, dtype=torch.float32)
+    moe.moe_layer(L.x, L.w_router, L.bias, L.w_gate, L.w_up, L.w_down, k1, k2, y, ws,
+                  topk_idx_out=idx, topk_w_out=w, logits_out=z, flags=flags)
+    torch.cuda.synchronize()
+    status = moe.moe_read_device_status(ws)
+    assert status == 0, moe.status_string(status)
+    return y, idx, w, z
+
+
+def check_layer_full(L, k1, k2, flags=moe.MOE_PATH_AUTO, tight=True):
+    """Whole-layer parity against oracle.layer (all tokens, all weights on host)."""
+    y, idx, w, z = run_layer(L, k1, k2, flags=flags)
+    zn = z.cpu().numpy()
+    # logits against the oracle's own
+    z_or = oracle.logits(synth.to_numpy(L.x), synth.to_numpy(L.w_router), synth.to_numpy(L.bias))
+    assert np.abs(zn - z_or).max() <= logits_bound(L.x, L.w_router)
+    ref = oracle.layer(synth.to_numpy(L.x), synth.to_numpy(L.w_router), synth.to_numpy(L.bias),
+                       synth.to_numpy(L.w_gate), synth.to_numpy(L.w_up), synth.to_numpy(L.w_down),
+                       k1, k2, logits_in=zn)
+    assert np.array_equal(idx.cpu().numpy(), ref["idx"])
+    assert np.array_equal(w.cpu().numpy(), ref["w"])
+    yy = y.cpu().numpy()
+    err, rel = assert_close_layer(yy, ref["y"], "layer")
+    if tight:
+        # float32 output: only summation order differs from the oracle
+        assert rel <= 1e-4, rel
+    return yy, ref
+
+
+def check_layer_sampled(L, k1, k2, tokens, flags=moe.MOE_PATH_AUTO):
+    """Parity on sampled tokens; expert weights are fetched to the host only
+    for the experts those tokens use."""
+    y, idx, w, z = run_layer(L, k1, k2, flags=flags)
+    tokens = np.asarray(tokens)
+    zn = z.cpu().numpy()[tokens]
+    xs = synth.to_numpy(L.x[torch.as_tensor(tokens, device=L.x.device)])
+    # logits of the sampled tokens against the oracle's own
+    z_or = oracle.logits(xs, synth.to_numpy(L.w_router), synth.to_numpy(L.bias))
+    assert np.abs(zn - z_or).max() <= logits_bound(L.x, L.w_router)
+
+    def fetch(e):
+        return (synth.to_numpy(L.w_gate[e]), synth.to_numpy(L.w_up[e]), synth.to_numpy(L.w_down[e]))
+
+    ref = oracle.layer_tokens(xs, zn, fetch, k1, k2)
+    assert np.array_equal(idx.cpu().numpy()[tokens], ref["idx"])
+    assert np.array_equal(w.cpu().numpy()[tokens], ref["w"])
+    yy = y.cpu().numpy()[tokens]
+    err, rel = assert_close_layer(yy, ref["y"], "sampled layer")
+    assert rel <= 1e-4, rel
+    return idx.cpu().numpy()

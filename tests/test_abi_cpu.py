@@ -1,0 +1,111 @@
+"""Host-side checks of the C-ABI library that need no GPU: it loads, it
+exports every function include/*.h declares, and argument checking returns
+the documented status codes before anything is enqueued."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from routed_expert_layer_route_b200 import build as pkg_build
+from routed_expert_layer_route_b200 import moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 1 << 40  # 256-byte aligned non-null pointer value; never dereferenced here
+
+
+@pytest.fixture(scope="module")
+def L():
+    pkg_build.build()
+    return moe.lib()
+
+
+def declared_functions():
+    names = set()
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not h.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", h)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"\b(moe_[a-z0-9_]+)\s*\(", text):
+            names.add(m.group(1))
+    return names
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert {"moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer"} <= names
+    for n in names:
+        assert hasattr(L, n), n
+    assert names == set(moe.SIGNATURES), names ^ set(moe.SIGNATURES)
+
+
+def test_status_strings(L):
+    for code in range(0, -7, -1):
+        s = moe.status_string(code)
+        assert s and s != "unknown status"
+    assert moe.status_string(-99) == "unknown status"
+    assert moe.moe_version() >= 10000
+
+
+def test_workspace_size(L):
+    n1 = moe.moe_workspace_size(1, 2048, 128, 768, 8)
+    n2 = moe.moe_workspace_size(64, 2048, 128, 768, 8)
+    assert n1 >= 256 and n2 > n1 and n1 % 256 == 0
+    assert moe.moe_workspace_size(1, 100, 128, 768, 8) == 0      # d % 64
+    assert moe.moe_workspace_size(1, 2048, 2000, 768, 8) == 0    # E > 1024
+    assert moe.moe_workspace_size(1, 2048, 128, 770, 8) == 0     # I % 16
+    assert moe.moe_workspace_size(1, 2048, 128, 768, 0) == 0     # k1 < 1
+    assert moe.moe_workspace_size(1, 2048, 8, 768, 9) == 0       # k1 > E
+
+
+def layer(L, T=1, d=2048, E=128, I=768, k1=8, k2=8, y=FAKE, ws=FAKE, ws_bytes=1 << 40,
+          ptr=FAKE, y_dtype=1, flags=0):
+    return L.moe_layer(ptr, ptr, None, ptr, ptr, ptr, T, d, E, I, k1, k2, y, y_dtype, None, None,
+                       None, flags, ws, ws_bytes, None)
+
+
+def test_layer_argument_checks(L):
+    assert layer(L, k1=8, k2=4) == moe.MOE_ERR_INVALID_ARG           # k2 < k1
+    assert layer(L, k1=0, k2=4) == moe.MOE_ERR_INVALID_ARG
+    assert layer(L, E=4, k1=8, k2=8) == moe.MOE_ERR_INVALID_ARG      # k1 > E
+    assert layer(L, k1=33, k2=40) == moe.MOE_ERR_INVALID_ARG          # k1 > 32
+    assert layer(L, d=100) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert layer(L, I=8) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert layer(L, E=1025, k1=8) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert layer(L, y=None) == moe.MOE_ERR_INVALID_ARG
+    assert layer(L, ws=None) == moe.MOE_ERR_INVALID_ARG
+    assert layer(L, ws=FAKE + 16) == moe.MOE_ERR_INVALID_ARG          # ws not 256-aligned
+    assert layer(L, ptr=FAKE + 8) == moe.MOE_ERR_INVALID_ARG          # misaligned tensor
+    assert layer(L, y_dtype=7) == moe.MOE_ERR_INVALID_ARG
+    assert layer(L, flags=9) == moe.MOE_ERR_INVALID_ARG
+    assert layer(L, ws_bytes=1024) == moe.MOE_ERR_WORKSPACE_TOO_SMALL
+    assert layer(L, T=0) == moe.MOE_OK                                 # no-op, nothing enqueued
+    assert layer(L, T=0, k2=9) == moe.MOE_OK                           # k2 > E-independent, valid
+
+
+def test_other_calls_argument_checks(L):
+    r = L.moe_route(FAKE, FAKE, None, None, 4, 2048, 128, 8, 4, FAKE, FAKE, None, 0, None)
+    assert r == moe.MOE_ERR_INVALID_ARG                                # k2 < k1
+    r = L.moe_route(None, None, None, None, 4, 0, 128, 8, 16, FAKE, FAKE, None, 0, None)
+    assert r == moe.MOE_ERR_INVALID_ARG                                # no logits given
+    r = L.moe_route(None, None, None, FAKE, 0, 0, 128, 8, 16, FAKE, FAKE, None, 0, None)
+    assert r == moe.MOE_OK                                             # T = 0
+    assert L.moe_permute(FAKE, 4, 8, 2000, FAKE, FAKE, FAKE, None, 0, None) == \
+        moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert L.moe_permute(FAKE, 4, 8, 128, None, FAKE, FAKE, None, 0, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_expert_ffn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2048, 128, 768, 8, FAKE, 0,
+                            FAKE, 1024, None) == moe.MOE_ERR_WORKSPACE_TOO_SMALL
+    assert L.moe_combine(FAKE, FAKE, FAKE, 4, 2048, 8, FAKE, 3, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_combine(FAKE, FAKE, FAKE, 4, 100, 8, FAKE, 1, None) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert L.moe_workspace_init(None, 4096, None) == moe.MOE_ERR_INVALID_ARG
+    v = ctypes.c_int(0)
+    assert L.moe_read_device_status(None, ctypes.byref(v), None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_test_exp_c(None, None, 0, None) == moe.MOE_OK
+
+
+def test_binding_raises_without_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(moe, "_lib", None)
+    monkeypatch.setattr(moe, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError):
+        moe.lib()

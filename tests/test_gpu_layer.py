@@ -1,0 +1,151 @@
+"""GPU parity of the whole layer and of its expert-FFN / combine steps
+against the CPU oracle, at small sizes (every token checked) and at the
+method's full workload sizes (sampled tokens).
+
+Expert structure: "Channel Selection for Mixture-of-Experts Decoding Needs No
+Calibration Data", section 2 "Background"; weights: Eq. 2 of "Paper of the
+Week #3", section "The Receipt".
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from routed_expert_layer_route_b200 import moe, synth
+
+from parity import (assert_close_layer, check_layer_full, check_layer_sampled, run_layer)
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda:0")
+
+
+@pytest.fixture(autouse=True)
+def _free():
+    yield
+    torch.cuda.empty_cache()
+
+
+SMALL = [
+    # T, d, E, I, k1, k2, bias
+    (1, 64, 16, 32, 2, 2, None),
+    (4, 64, 16, 32, 2, 4, None),
+    (4, 64, 16, 32, 2, 16, None),
+    (1, 256, 16, 64, 2, 4, None),
+    (2, 256, 64, 96, 8, 16, "normal"),
+    (7, 512, 64, 256, 4, 16, "normal"),
+    (33, 256, 32, 80, 3, 5, None),
+    (64, 1024, 64, 128, 8, 64, "zipf"),
+    (5, 128, 1, 48, 1, 1, None),
+    (3, 192, 20, 32, 20, 20, None),      # k1 = E: every expert runs
+    (17, 320, 40, 112, 6, 1000, None),   # k2 > E: no renormalisation
+]
+
+
+@pytest.mark.parametrize("T,d,E,I,k1,k2,bias", SMALL)
+def test_layer_small_all_tokens(T, d, E, I, k1, k2, bias):
+    L = synth.make_layer(T, d, E, I, seed=T + d + E, device=DEV, bias=bias)
+    check_layer_full(L, k1, k2)
+
+
+def test_layer_bf16_output_is_rounded_f32_output():
+    L = synth.make_layer(9, 512, 32, 64, seed=2, device=DEV)
+    y32, *_ = run_layer(L, 4, 8, y_dtype=torch.float32)
+    y16, *_ = run_layer(L, 4, 8, y_dtype=torch.bfloat16)
+    assert torch.equal(y32.to(torch.bfloat16), y16)
+
+
+def test_layer_deterministic_and_workspace_reuse():
+    L = synth.make_layer(8, 512, 32, 64, seed=3, device=DEV, bias="normal")
+    big = moe.workspace(64, 2048, 128, 768, 8, device=DEV)   # larger than needed
+    a, ia, wa, _ = run_layer(L, 4, 16, ws=big)
+    b, ib, wb, _ = run_layer(L, 4, 16, ws=big)
+    c, ic, wc, _ = run_layer(L, 4, 16)
+    assert torch.equal(a, b) and torch.equal(a, c)
+    assert torch.equal(ia, ic) and torch.equal(wa, wc)
+
+
+def test_indices_do_not_depend_on_k2():
+    L = synth.make_layer(16, 256, 64, 32, seed=4, device=DEV)
+    base = run_layer(L, 4, 4)[1]
+    for k2 in (8, 16, 64, 500):
+        assert torch.equal(run_layer(L, 4, k2)[1], base)
+
+
+def test_expert_ffn_and_combine_steps():
+    T, d, E, I, k1, k2 = 12, 384, 24, 96, 3, 6
+    L = synth.make_layer(T, d, E, I, seed=5, device=DEV, bias="normal")
+    ws = moe.workspace(T, d, E, I, k1, device=DEV)
+    z = torch.empty(T, E, dtype=torch.float32, device=DEV)
+    idx = torch.empty(T, k1, dtype=torch.int32, device=DEV)
+    w = torch.empty(T, k1, dtype=torch.float32, device=DEV)
+    moe.moe_route(L.x, L.w_router, L.bias, z, k1, k2, idx, w)
+    off = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    ss = torch.empty(T * k1, dtype=torch.int32, device=DEV)
+    sp = torch.empty(T * k1, dtype=torch.int32, device=DEV)
+    moe.moe_permute(idx, E, off, ss, sp)
+    out = torch.empty(T * k1, d, dtype=torch.float32, device=DEV)
+    moe.moe_expert_ffn(L.x, off, ss, L.w_gate, L.w_up, L.w_down, k1, out, ws)
+    y = torch.empty(T, d, dtype=torch.float32, device=DEV)
+    moe.moe_combine(out, sp, w, y)
+    torch.cuda.synchronize()
+    assert moe.moe_read_device_status(ws) == 0
+    # per-slot expert outputs against the oracle expert
+    ssn, idxn, on = ss.cpu().numpy(), idx.cpu().numpy(), out.cpu().numpy()
+    xn = synth.to_numpy(L.x)
+    xf = (xn.astype(np.uint32) << 16).view(np.float32)
+    for p in range(T * k1):
+        slot = int(ssn[p])
+        t, e = slot // k1, int(idxn.ravel()[slot])
+        _, o = oracle.expert(xf[t], synth.to_numpy(L.w_gate[e]), synth.to_numpy(L.w_up[e]),
+                             synth.to_numpy(L.w_down[e]))
+        assert_close_layer(on[p], o, "slot %d" % p)
+        assert np.abs(on[p] - o).max() <= 1e-4 * max(1.0, np.abs(o).max())
+    # combine against the oracle combine of the GPU's own expert outputs
+    spn, wn = sp.cpu().numpy(), w.cpu().numpy()
+    for t in range(T):
+        ref = oracle.combine(on[spn[t * k1:(t + 1) * k1]], wn[t])
+        assert np.allclose(y[t].cpu().numpy(), ref, rtol=0, atol=1e-6)
+    # and the whole layer gives the same y
+    y2, *_ = run_layer(L, k1, k2)
+    assert torch.allclose(y, y2, rtol=0, atol=1e-6)
+
+
+def test_zero_tokens_is_a_noop():
+    L = synth.make_layer(0, 256, 16, 32, seed=6, device=DEV)
+    ws = moe.workspace(1, 256, 16, 32, 2, device=DEV)
+    y = torch.empty(0, 256, device=DEV)
+    moe.moe_layer(L.x, L.w_router, None, L.w_gate, L.w_up, L.w_down, 2, 4, y, ws)
+    torch.cuda.synchronize()
+
+
+# ------------------------------------------------------------------ full sizes
+# the method's workloads: d=2048, E=128, I=768 (decode / prefill) and
+# d=4096, E=512, I=1024 (large), bf16, launched exactly as the benchmark does
+@pytest.mark.parametrize("k1,k2", [(8, 8), (8, 16), (8, 128), (4, 4), (4, 16), (4, 128)])
+def test_decode_b1_full_size(k1, k2):
+    for layer in range(2):
+        L = synth.make_layer(1, 2048, 128, 768, seed=0, layer=layer, device=DEV)
+        check_layer_sampled(L, k1, k2, [0])
+
+
+@pytest.mark.parametrize("T", [8, 32])
+@pytest.mark.parametrize("k1,k2", [(8, 8), (4, 16)])
+def test_decode_small_batch_full_size(T, k1, k2):
+    L = synth.make_layer(T, 2048, 128, 768, seed=0, layer=1, device=DEV, bias="normal")
+    check_layer_sampled(L, k1, k2, list(range(T)) if T == 8 else [0, 5, 17, 31])
+
+
+@pytest.mark.parametrize("T", [1, 64])
+@pytest.mark.parametrize("k1,k2", [(10, 10), (5, 20)])
+def test_large_full_size(T, k1, k2):
+    L = synth.make_layer(T, 4096, 512, 1024, seed=0, layer=0, device=DEV)
+    check_layer_sampled(L, k1, k2, [0] if T == 1 else [0, 9, 40, 63])
+
+
+@pytest.mark.parametrize("k1,k2", [(8, 16), (4, 16)])
+def test_prefill_full_size_sampled(k1, k2):
+    L = synth.make_layer(4096, 2048, 128, 768, seed=0, layer=0, device=DEV, bias="zipf")
+    idx = check_layer_sampled(L, k1, k2, [0, 1, 777, 2048, 4000, 4095])
+    # Zipf bias: the most popular expert gets many more tokens than the least
+    counts = np.bincount(idx.ravel(), minlength=128)
+    assert counts.max() > 4 * max(1, np.median(counts))
