@@ -83,36 +83,50 @@ def recorded_traffic(workload, k1):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clocks and throttle reasons, sampled from before the timed
+    region to after it; samples are kept with their host time so the ones
+    inside a window can be picked out."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
+    def __init__(self, gpu_id):
+        self.gpu = gpu_id
         self.proc = None
-        self.lines = []
+        self.samples = []  # (host time, sm MHz, max MHz, set of active reasons)
         self.thread = None
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
             return
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
+        t0 = time.time()
+        while not self.samples and time.time() - t0 < 5.0:  # let the sampler come up
+            time.sleep(0.05)
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            parts = [p.strip() for p in line.strip().split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm, mx = float(parts[0]), float(parts[1])
+            except ValueError:
+                continue
+            reasons = {n for n, v in zip(self.NAMES, parts[4:8]) if v.lower() == "active"}
+            self.samples.append((time.time(), sm, mx, reasons))
 
     def stop(self):
         if self.proc is None:
-            return None
+            return
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -120,24 +134,18 @@ class ClockSampler:
             self.proc.kill()
         if self.thread:
             self.thread.join(timeout=2)
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
-                "reasons": sorted(reasons)}
+
+    def summary(self, t0, t1, min_samples=3):
+        sel = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed region"
+        if len(sel) < min_samples:
+            return None, window
+        reasons = set()
+        for s in sel:
+            reasons |= s[3]
+        return {"sm_mhz": statistics.median(s[1] for s in sel),
+                "sm_max_mhz": max(s[2] for s in sel), "samples": len(sel),
+                "reasons": sorted(reasons), "window": window}, window
 
 
 def smi_index(local):
@@ -345,7 +353,7 @@ def run_native(args, world, rank):
         g = build_graph(stack, k1, k2, ws_list, ys, stream)
         graphs[(k1, k2)] = (g, ws_list, ys)
 
-    def timed(k1, k2, steps, warmup, clocks=None):
+    def timed(k1, k2, steps, warmup):
         g = graphs[(k1, k2)][0]
         with torch.cuda.stream(stream):
             for _ in range(warmup):
@@ -354,30 +362,29 @@ def run_native(args, world, rank):
         barrier(world)
         s = torch.cuda.Event(enable_timing=True)
         e = torch.cuda.Event(enable_timing=True)
-        if clocks:
-            clocks.start()
+        h0 = time.time()
         s.record(stream)
         with torch.cuda.stream(stream):
             for _ in range(steps):
                 g.replay()
         e.record(stream)
         e.synchronize()
-        if clocks:
-            c = clocks.stop()
-        else:
-            c = None
+        h1 = time.time()
         barrier(world)
         ms = s.elapsed_time(e)
-        return allreduce_max(ms, world) / steps, c
+        return allreduce_max(ms, world) / steps, (h0, h1)
 
-    # headline: the timed region of the contract
+    # headline: the timed region of the contract (clocks sampled around it)
     clocks = ClockSampler(smi_index(torch.cuda.current_device()))
-    ms_step, clk = timed(*head, args.steps, args.warmup, clocks)
+    clocks.start()
+    ms_step, head_win = timed(*head, args.steps, args.warmup)
     value = world * T * 1000.0 / ms_step
+    sweep_t0 = head_win[0]
 
     # every (k1, k2) condition of the sweep, same protocol, outside the headline region
     for (k1, k2) in sweep:
         ms = ms_step if (k1, k2) == head else timed(k1, k2, args.steps, args.warmup)[0]
+        sweep_t1 = time.time()
         _, ws_list, ys = graphs[(k1, k2)]
         us = unique_experts(stack, k1, k2, ws_list, ys, stream)
         U = statistics.mean(us)
@@ -385,6 +392,13 @@ def run_native(args, world, rank):
         results.append({"k1": k1, "k2": k2, "ms_per_step": ms, "us_per_layer": ms * 1000 / Ln,
                         "tokens_per_s": world * T * 1000.0 / ms, "unique_experts_per_layer": U,
                         "expert_GBps": bytes_layer / (ms / Ln * 1e-3) / 1e9})
+
+    clocks.stop()
+    clk, _ = clocks.summary(*head_win)
+    if clk is None:  # timed region shorter than the sampling period: use the sweep's
+        clk, _ = clocks.summary(sweep_t0, sweep_t1)
+        if clk is not None:
+            clk["window"] = "headline and sweep timed regions"
 
     # dominant kernel alone, events on its own stream
     k1h, k2h = head
@@ -496,7 +510,7 @@ def run_reference(args, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode_b1")
