@@ -67,7 +67,8 @@ typedef enum {
     MOE_ERR_WORKSPACE_TOO_SMALL = -3, /* ws_bytes < moe_workspace_size(...)                     */
     MOE_ERR_CUDA = -4,                /* a CUDA runtime call failed                             */
     MOE_ERR_TIMEOUT = -5,             /* device status: a bounded wait gave up                  */
-    MOE_ERR_DEVICE_CHECK = -6         /* device status: an index check failed on the device     */
+    MOE_ERR_DEVICE_CHECK = -6,        /* device status: an index check failed on the device     */
+    MOE_ERR_SCRATCH_LIMIT = -7        /* moe_expert_ffn_noalloc: shapes exceed its fixed scratch */
 } moe_status;
 
 /* Output element types for moe_combine / moe_layer. */
@@ -157,6 +158,34 @@ int moe_layer(const void *x_bf16, const void *w_router_bf16, const float *bias,
               int E, int I, int k1, int k2, void *y, int y_dtype, int32_t *topk_idx_out,
               float *topk_w_out, float *logits_out, int flags, void *ws, size_t ws_bytes,
               void *stream);
+
+/* moe_expert_ffn without a caller workspace.  The paper has no counterpart;
+ * this entry exists for callers that cannot hand the library device memory
+ * for scratch: plugins running inside an engine that owns the whole device
+ * memory pool, services that fix their memory footprint at start-up and treat
+ * any later allocation as a fault, and bindings that can pass pointers they
+ * were given but have no way to allocate device memory themselves.
+ *
+ * Same inputs, output and result as moe_expert_ffn (flags are not taken: it
+ * always uses the weight-streaming path).  Its scratch is a fixed array
+ * compiled into libmoe.so (4 MiB per GPU that loads the library, held until
+ * the process exits); the call itself allocates and frees nothing.
+ *  - Limit: T * k1 * I <= 1047424 (the float32 channel activations of all
+ *    routed slots must fit the array), and the usual shape limits; larger
+ *    shapes return MOE_ERR_SCRATCH_LIMIT and enqueue nothing.
+ *  - The first call on a device looks up the array's device address (once
+ *    per device, with that device current); make that first call outside any
+ *    stream capture.
+ *  - Every call on a device shares the one array, and each call clears the
+ *    part that must start at zero.  Calls whose work overlaps on the GPU
+ *    (e.g. on two streams at once) race on the array; order them on one
+ *    stream.
+ *  - Device-side problems (bounded waits, index checks) cannot be read back
+ *    through a workspace; they leave out unspecified. */
+int moe_expert_ffn_noalloc(const void *x_bf16, const int32_t *expert_offsets,
+                           const int32_t *sorted_slot, const void *w_gate_bf16,
+                           const void *w_up_bf16, const void *w_down_bf16, int T, int d, int E,
+                           int I, int k1, float *out, void *stream);
 
 #ifdef __cplusplus
 }

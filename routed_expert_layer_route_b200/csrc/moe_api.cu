@@ -182,6 +182,8 @@ const char *moe_status_string(int status)
     case MOE_ERR_CUDA: return "CUDA error";
     case MOE_ERR_TIMEOUT: return "device wait timed out";
     case MOE_ERR_DEVICE_CHECK: return "device-side check failed";
+    case MOE_ERR_SCRATCH_LIMIT:
+        return "shapes exceed the fixed scratch of moe_expert_ffn_noalloc (T*k1*I > 1047424)";
     default: return "unknown status";
     }
 }
@@ -501,3 +503,77 @@ int moe_test_num_sms(void)
 }
 
 }  // extern "C"
+
+// ====================================================================== no-alloc
+// Scratch for moe_expert_ffn_noalloc: a fixed array in the library image, so
+// callers that cannot give the library device memory can still run the
+// expert FFN.  Layout: header (grid-barrier counters, status) | activated
+// expert count | activated expert list (E <= 1024) | float32 channel
+// activations of every routed slot [T*k1 x I].
+namespace moe {
+constexpr size_t kNoAllocBytes = 4u << 20;
+constexpr size_t kNoAllocHOffset = 256 + 256 + sizeof(int32_t) * 1024;
+constexpr size_t kNoAllocMaxH = (kNoAllocBytes - kNoAllocHOffset) / sizeof(float);  // 1047424
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+// Device address of g_noalloc_scratch per device (the host-side name is only
+// a stand-in, so kernels get this address instead).
+static void *g_noalloc_ptr[64];
+static std::mutex g_noalloc_mu;
+
+static int noalloc_scratch(void *&out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
+            return MOE_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    out = g_noalloc_ptr[dev];
+    return MOE_OK;
+}
+}  // namespace moe
+
+extern "C" int moe_expert_ffn_noalloc(const void *x_bf16, const int32_t *expert_offsets,
+                                      const int32_t *sorted_slot, const void *w_gate_bf16,
+                                      const void *w_up_bf16, const void *w_down_bf16, int T, int d,
+                                      int E, int I, int k1, float *out, void *stream)
+{
+    int rc = check_shape(T, d, E, I, k1);
+    if (rc != MOE_OK)
+        return rc;
+    if ((size_t)T * (size_t)k1 * (size_t)I > kNoAllocMaxH)
+        return MOE_ERR_SCRATCH_LIMIT;
+    if (T == 0)
+        return MOE_OK;
+    if (!x_bf16 || !expert_offsets || !sorted_slot || !w_gate_bf16 || !w_up_bf16 ||
+        !w_down_bf16 || !out)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x_bf16) || !aligned16(w_gate_bf16) || !aligned16(w_up_bf16) ||
+        !aligned16(w_down_bf16) || !aligned16(out))
+        return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    DevInfo *di;
+    if ((rc = device_info(di)) != MOE_OK)
+        return rc;
+    void *scratch = nullptr;
+    if ((rc = noalloc_scratch(scratch)) != MOE_OK)
+        return rc;
+    // the grid-barrier counters and the status word must start at zero
+    if (cudaMemsetAsync(scratch, 0, sizeof(WsHeader), s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    int32_t *uniq_count = at<int32_t>(scratch, 256);
+    int32_t *uniq_list = at<int32_t>(scratch, 512);
+    float *h = at<float>(scratch, kNoAllocHOffset);
+    if ((rc = launch(k_uniq_from_offsets, dim3(1), dim3(1024), 0, s, true, expert_offsets, E,
+                     uniq_count, uniq_list)) != MOE_OK)
+        return rc;
+    return expert_ffn_stream(x_bf16, expert_offsets, sorted_slot, uniq_count, uniq_list,
+                             w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I, k1, h, out, nullptr,
+                             0, nullptr, nullptr, static_cast<WsHeader *>(scratch), s);
+}

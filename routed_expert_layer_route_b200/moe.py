@@ -21,6 +21,7 @@ MOE_ERR_WORKSPACE_TOO_SMALL = -3
 MOE_ERR_CUDA = -4
 MOE_ERR_TIMEOUT = -5
 MOE_ERR_DEVICE_CHECK = -6
+MOE_ERR_SCRATCH_LIMIT = -7
 
 MOE_DTYPE_F32 = 0
 MOE_DTYPE_BF16 = 1
@@ -46,6 +47,7 @@ SIGNATURES = {
     "moe_combine": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _i, _vp]),
     "moe_layer": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp,
                        _vp, _i, _vp, _sz, _vp]),
+    "moe_expert_ffn_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
     "moe_test_exp_c": (_i, [_vp, _vp, ctypes.c_int64, _vp]),
     "moe_test_num_sms": (_i, []),
     "moe_test_expert_stream": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _sz,
@@ -167,6 +169,19 @@ def moe_expert_ffn(x, expert_offsets, sorted_slot, w_gate, w_up, w_down, k1, out
     _check(lib().moe_expert_ffn(_p(x), _p(expert_offsets), _p(sorted_slot), _p(w_gate), _p(w_up),
                                 _p(w_down), T, d, E, I, k1, _p(out), flags, wsp, wsn,
                                 _stream(stream)), "moe_expert_ffn")
+
+
+def moe_expert_ffn_noalloc(x, expert_offsets, sorted_slot, w_gate, w_up, w_down, k1, out,
+                           stream=None):
+    """moe_expert_ffn for callers that cannot provide device scratch memory:
+    the library uses a fixed array of its own instead of a workspace (limit
+    T * k1 * I <= 1047424; calls that overlap on the GPU share that array and
+    race, so keep them on one stream)."""
+    T, d = x.shape
+    E, I, _ = w_gate.shape
+    _check(lib().moe_expert_ffn_noalloc(_p(x), _p(expert_offsets), _p(sorted_slot), _p(w_gate),
+                                        _p(w_up), _p(w_down), T, d, E, I, k1, _p(out),
+                                        _stream(stream)), "moe_expert_ffn_noalloc")
 
 
 def moe_combine(expert_out, slot_pos, topk_w, y, stream=None):

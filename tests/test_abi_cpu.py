@@ -41,7 +41,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_status_strings(L):
-    for code in range(0, -7, -1):
+    for code in range(0, -8, -1):
         s = moe.status_string(code)
         assert s and s != "unknown status"
     assert moe.status_string(-99) == "unknown status"
@@ -102,6 +102,13 @@ def test_other_calls_argument_checks(L):
     v = ctypes.c_int(0)
     assert L.moe_read_device_status(None, ctypes.byref(v), None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_test_exp_c(None, None, 0, None) == moe.MOE_OK
+    # the no-alloc expert FFN refuses shapes beyond its fixed scratch before touching CUDA
+    assert L.moe_expert_ffn_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 128, 512, 64, 1024, 8, FAKE,
+                                    None) == moe.MOE_ERR_SCRATCH_LIMIT
+    assert L.moe_expert_ffn_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 512, 64, 1024, 8, FAKE,
+                                    None) == moe.MOE_OK
+    assert L.moe_expert_ffn_noalloc(FAKE, None, FAKE, FAKE, FAKE, FAKE, 4, 512, 64, 1024, 8, FAKE,
+                                    None) == moe.MOE_ERR_INVALID_ARG
 
 
 def test_binding_raises_without_library(tmp_path, monkeypatch):
