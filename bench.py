@@ -234,7 +234,7 @@ def unique_experts(stack, k1, k2, ws_list, ys, stream):
     return us
 
 
-def time_dominant_kernel(stack, k1, ws_list, ys, stream, reps):
+def time_dominant_kernel(stack, k1, k2, ws_list, ys, stream, reps):
     """Average duration of the expert-streaming kernel launched alone (CUDA
     events on its stream), cycling through the layers so weights come from
     HBM, not L2."""
@@ -246,7 +246,8 @@ def time_dominant_kernel(stack, k1, ws_list, ys, stream, reps):
                 s = torch.cuda.Event(enable_timing=True)
                 e = torch.cuda.Event(enable_timing=True)
                 s.record(stream)
-                moe.moe_test_expert_stream(L.x, L.w_gate, L.w_up, L.w_down, k1, y, ws, stream=stream)
+                moe.moe_test_expert_stream(L.x, L.w_gate, L.w_up, L.w_down, k1, k2, y, ws,
+                                           stream=stream)
                 e.record(stream)
                 starts.append(s)
                 ends.append(e)
@@ -403,7 +404,7 @@ def run_native(args, world, rank):
     # dominant kernel alone, events on its own stream
     k1h, k2h = head
     _, ws_list, ys = graphs[head]
-    kern_ms = time_dominant_kernel(stack, k1h, ws_list, ys, stream, reps=3)
+    kern_ms = time_dominant_kernel(stack, k1h, k2h, ws_list, ys, stream, reps=3)
     U_head = results[0]["unique_experts_per_layer"]
     alg_bytes = U_head * 3 * d * I * 2
     achieved = alg_bytes / (kern_ms * 1e-3) / 1e9

@@ -24,13 +24,14 @@ int moe_test_num_sms(void);
 
 /* Re-run only the expert-streaming kernel (expert FFN + combine into y) of
  * the last moe_layer call made with this workspace and these shapes, reusing
- * the routing that call left in the workspace.  Launched without
+ * the logits (T == 1, where the kernel routes the token itself) or the
+ * routing tables (T > 1) that call left in the workspace.  Launched without
  * programmatic dependent launch, so events recorded around it on `stream`
  * bracket this one kernel.  Used to time the dominant kernel alone.
  * Arguments as for moe_layer.  Returns a moe_status. */
 int moe_test_expert_stream(const void *x_bf16, const void *w_gate_bf16, const void *w_up_bf16,
-                           const void *w_down_bf16, int T, int d, int E, int I, int k1, void *y,
-                           int y_dtype, void *ws, size_t ws_bytes, void *stream);
+                           const void *w_down_bf16, int T, int d, int E, int I, int k1, int k2,
+                           void *y, int y_dtype, void *ws, size_t ws_bytes, void *stream);
 
 #ifdef __cplusplus
 }

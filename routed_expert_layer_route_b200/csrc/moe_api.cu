@@ -99,7 +99,7 @@ static int device_info(DevInfo *&out)
     if (!di.ready) {
         if (cudaDeviceGetAttribute(&di.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return MOE_ERR_CUDA;
-        const int stream_smem = 227 * 1024;
+        const int stream_smem = (int)stream_smem_bytes();
         if (cudaFuncSetAttribute(k_stream, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  stream_smem) != cudaSuccess)
             return MOE_ERR_CUDA;
@@ -159,7 +159,6 @@ static int enqueue_logits(const void *x, const void *wr, const float *bias, floa
     a.T = T;
     a.d = d;
     a.E = E;
-    a.tail = 0;
     const int items = E * ((T + kLogitsTok - 1) / kLogitsTok);
     const int grid = (items + kLogitsWarps - 1) / kLogitsWarps;
     return launch(k_logits, dim3(grid), dim3(kLogitsWarps * 32), 0, s, true, a);
@@ -296,40 +295,92 @@ int moe_permute(const int32_t *topk_idx, int T, int k1, int E, int32_t *expert_o
                   k1, E, po, status);
 }
 
-static int expert_ffn_stream(const void *x, const int32_t *offsets, const int32_t *sorted_slot,
-                             const int32_t *uniq_count, const int32_t *uniq_list, const void *wg,
-                             const void *wu, const void *wd, int T, int d, int E, int I, int k1,
-                             float *h, float *out, void *y, int y_dtype, const float *topk_w,
-                             const int32_t *slot_pos, WsHeader *hdr, cudaStream_t s,
-                             bool pdl = true)
+struct StreamCall {
+    const void *x, *wg, *wu, *wd;
+    int T, d, E, I, k1, k2;
+    int route_in_kernel;
+    const float *logits;
+    int32_t *topk_idx;
+    float *topk_w;
+    int32_t *idx_copy;
+    float *w_copy;
+    int32_t *offsets, *sorted_slot, *slot_pos, *uniq_count, *uniq_list;
+    float *h, *out;
+    void *y;
+    int y_dtype;
+    WsHeader *hdr;
+};
+
+static int enqueue_stream(const StreamCall &c, cudaStream_t s, bool pdl = true)
 {
     DevInfo *di;
     int rc;
     if ((rc = device_info(di)) != MOE_OK)
         return rc;
     StreamArgs a = {};
-    a.x = static_cast<const uint16_t *>(x);
-    a.wg = static_cast<const uint16_t *>(wg);
-    a.wu = static_cast<const uint16_t *>(wu);
-    a.wd = static_cast<const uint16_t *>(wd);
-    a.T = T;
-    a.d = d;
-    a.E = E;
-    a.I = I;
-    a.k1 = k1;
-    a.offsets = offsets;
-    a.sorted_slot = sorted_slot;
-    a.uniq_count = uniq_count;
-    a.uniq_list = uniq_list;
-    a.h = h;
-    a.out = out;
-    a.y = y;
-    a.y_dtype = y_dtype;
-    a.topk_w = topk_w;
-    a.slot_pos = slot_pos;
-    a.hdr = hdr;
-    return launch(k_stream, dim3(di->num_sms), dim3(kSThreads), stream_smem_bytes(d, I), s, pdl,
-                  a);
+    a.x = static_cast<const uint16_t *>(c.x);
+    a.wg = static_cast<const uint16_t *>(c.wg);
+    a.wu = static_cast<const uint16_t *>(c.wu);
+    a.wd = static_cast<const uint16_t *>(c.wd);
+    a.T = c.T;
+    a.d = c.d;
+    a.E = c.E;
+    a.I = c.I;
+    a.k1 = c.k1;
+    a.k2 = c.k2;
+    a.route_in_kernel = c.route_in_kernel;
+    a.logits = c.logits;
+    a.topk_idx = c.topk_idx;
+    a.topk_w = c.topk_w;
+    a.idx_copy = c.idx_copy;
+    a.w_copy = c.w_copy;
+    a.offsets = c.offsets;
+    a.sorted_slot = c.sorted_slot;
+    a.slot_pos = c.slot_pos;
+    a.uniq_count = c.uniq_count;
+    a.uniq_list = c.uniq_list;
+    a.h = c.h;
+    a.out = c.out;
+    a.y = c.y;
+    a.y_dtype = c.y_dtype;
+    a.hdr = c.hdr;
+    return launch(k_stream, dim3(di->num_sms), dim3(kSThreads), stream_smem_bytes(), s, pdl, a);
+}
+
+// The streaming call of a moe_layer on workspace ws (routing tables there).
+static StreamCall layer_stream_call(const void *x, const void *wg, const void *wu, const void *wd,
+                                    int T, int d, int E, int I, int k1, int k2, void *y,
+                                    int y_dtype, int32_t *idx_copy, float *w_copy, void *ws)
+{
+    const WsLayout L = ws_layout(T, d, E, I, k1);
+    StreamCall c = {};
+    c.x = x;
+    c.wg = wg;
+    c.wu = wu;
+    c.wd = wd;
+    c.T = T;
+    c.d = d;
+    c.E = E;
+    c.I = I;
+    c.k1 = k1;
+    c.k2 = k2;
+    c.route_in_kernel = T == 1;
+    c.logits = at<float>(ws, L.logits);
+    c.topk_idx = at<int32_t>(ws, L.idx);
+    c.topk_w = at<float>(ws, L.w);
+    c.idx_copy = idx_copy;
+    c.w_copy = w_copy;
+    c.offsets = at<int32_t>(ws, L.offsets);
+    c.sorted_slot = at<int32_t>(ws, L.sorted_slot);
+    c.slot_pos = at<int32_t>(ws, L.slot_pos);
+    c.uniq_count = at<int32_t>(ws, L.uniq_count);
+    c.uniq_list = at<int32_t>(ws, L.uniq_list);
+    c.h = at<float>(ws, L.h);
+    c.out = at<float>(ws, L.out);
+    c.y = y;
+    c.y_dtype = y_dtype;
+    c.hdr = static_cast<WsHeader *>(ws);
+    return c;
 }
 
 int moe_expert_ffn(const void *x_bf16, const int32_t *expert_offsets, const int32_t *sorted_slot,
@@ -360,10 +411,25 @@ int moe_expert_ffn(const void *x_bf16, const int32_t *expert_offsets, const int3
     if ((rc = launch(k_uniq_from_offsets, dim3(1), dim3(1024), 0, s, true, expert_offsets, E,
                      at<int32_t>(ws, L.uniq_count), at<int32_t>(ws, L.uniq_list))) != MOE_OK)
         return rc;
-    return expert_ffn_stream(x_bf16, expert_offsets, sorted_slot, at<int32_t>(ws, L.uniq_count),
-                             at<int32_t>(ws, L.uniq_list), w_gate_bf16, w_up_bf16, w_down_bf16, T,
-                             d, E, I, k1, at<float>(ws, L.h), out, nullptr, 0, nullptr, nullptr,
-                             static_cast<WsHeader *>(ws), s);
+    StreamCall c = {};
+    c.x = x_bf16;
+    c.wg = w_gate_bf16;
+    c.wu = w_up_bf16;
+    c.wd = w_down_bf16;
+    c.T = T;
+    c.d = d;
+    c.E = E;
+    c.I = I;
+    c.k1 = k1;
+    c.k2 = k1;
+    c.offsets = const_cast<int32_t *>(expert_offsets);
+    c.sorted_slot = const_cast<int32_t *>(sorted_slot);
+    c.uniq_count = at<int32_t>(ws, L.uniq_count);
+    c.uniq_list = at<int32_t>(ws, L.uniq_list);
+    c.h = at<float>(ws, L.h);
+    c.out = out;
+    c.hdr = static_cast<WsHeader *>(ws);
+    return enqueue_stream(c, s);
 }
 
 int moe_combine(const float *expert_out, const int32_t *slot_pos, const float *topk_w, int T,
@@ -420,41 +486,20 @@ int moe_layer(const void *x_bf16, const void *w_router_bf16, const float *bias,
                   at<int32_t>(ws, L.slot_pos), at<int32_t>(ws, L.uniq_count),
                   at<int32_t>(ws, L.uniq_list)};
 
-    if (T == 1) {
-        // router + last-block routing and permutation in one kernel
-        LogitsArgs a = {};
-        a.x = static_cast<const uint16_t *>(x_bf16);
-        a.wr = static_cast<const uint16_t *>(w_router_bf16);
-        a.bias = bias;
-        a.z = z;
-        a.z_copy = logits_out;
-        a.T = 1;
-        a.d = d;
-        a.E = E;
-        a.tail = 1;
-        a.k1 = k1;
-        a.k2 = k2;
-        a.idx = idx;
-        a.w = w;
-        a.idx_copy = topk_idx_out;
-        a.w_copy = topk_w_out;
-        a.perm = po;
-        a.hdr = hdr;
-        const int grid = (E + kLogitsWarps - 1) / kLogitsWarps;
-        if ((rc = launch(k_logits, dim3(grid), dim3(kLogitsWarps * 32), permute_smem_bytes(E, 1),
-                         s, true, a)) != MOE_OK)
-            return rc;
-    } else {
-        if ((rc = enqueue_logits(x_bf16, w_router_bf16, bias, z, logits_out, T, d, E, s)) != MOE_OK)
-            return rc;
+    if ((rc = enqueue_logits(x_bf16, w_router_bf16, bias, z, logits_out, T, d, E, s)) != MOE_OK)
+        return rc;
+    if (T > 1) {
+        // one CTA per token ranks its probabilities; the last one to finish
+        // builds the permutation tables
         if ((rc = launch(k_topk, dim3(T), dim3(topk_threads(E)), permute_smem_bytes(E, T), s, true,
                          (const float *)z, T, E, k1, k2, idx, w, topk_idx_out, topk_w_out, po,
                          hdr)) != MOE_OK)
             return rc;
     }
-    return expert_ffn_stream(x_bf16, po.offsets, po.sorted_slot, po.uniq_count, po.uniq_list,
-                             w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I, k1, at<float>(ws, L.h),
-                             at<float>(ws, L.out), y, y_dtype, w, po.slot_pos, hdr, s);
+    // T == 1: the streaming kernel routes the token itself
+    return enqueue_stream(layer_stream_call(x_bf16, w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I,
+                                            k1, k2, y, y_dtype, topk_idx_out, topk_w_out, ws),
+                          s);
 }
 
 int moe_test_exp_c(const float *x, float *y, int64_t n, void *stream)
@@ -471,11 +516,13 @@ int moe_test_exp_c(const float *x, float *y, int64_t n, void *stream)
 }
 
 int moe_test_expert_stream(const void *x_bf16, const void *w_gate_bf16, const void *w_up_bf16,
-                           const void *w_down_bf16, int T, int d, int E, int I, int k1, void *y,
-                           int y_dtype, void *ws, size_t ws_bytes, void *stream)
+                           const void *w_down_bf16, int T, int d, int E, int I, int k1, int k2,
+                           void *y, int y_dtype, void *ws, size_t ws_bytes, void *stream)
 {
     int rc = check_shape(T, d, E, I, k1);
     if (rc != MOE_OK)
+        return rc;
+    if ((rc = check_route(E, k1, k2)) != MOE_OK)
         return rc;
     if (T == 0)
         return MOE_OK;
@@ -486,12 +533,9 @@ int moe_test_expert_stream(const void *x_bf16, const void *w_gate_bf16, const vo
     const WsLayout L = ws_layout(T, d, E, I, k1);
     if (ws_bytes < L.total)
         return MOE_ERR_WORKSPACE_TOO_SMALL;
-    return expert_ffn_stream(x_bf16, at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.sorted_slot),
-                             at<int32_t>(ws, L.uniq_count), at<int32_t>(ws, L.uniq_list),
-                             w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I, k1, at<float>(ws, L.h),
-                             at<float>(ws, L.out), y, y_dtype, at<float>(ws, L.w),
-                             at<int32_t>(ws, L.slot_pos), static_cast<WsHeader *>(ws),
-                             static_cast<cudaStream_t>(stream), false);
+    return enqueue_stream(layer_stream_call(x_bf16, w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I,
+                                            k1, k2, y, y_dtype, nullptr, nullptr, ws),
+                          static_cast<cudaStream_t>(stream), false);
 }
 
 int moe_test_num_sms(void)
@@ -573,7 +617,23 @@ extern "C" int moe_expert_ffn_noalloc(const void *x_bf16, const int32_t *expert_
     if ((rc = launch(k_uniq_from_offsets, dim3(1), dim3(1024), 0, s, true, expert_offsets, E,
                      uniq_count, uniq_list)) != MOE_OK)
         return rc;
-    return expert_ffn_stream(x_bf16, expert_offsets, sorted_slot, uniq_count, uniq_list,
-                             w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I, k1, h, out, nullptr,
-                             0, nullptr, nullptr, static_cast<WsHeader *>(scratch), s);
+    StreamCall c = {};
+    c.x = x_bf16;
+    c.wg = w_gate_bf16;
+    c.wu = w_up_bf16;
+    c.wd = w_down_bf16;
+    c.T = T;
+    c.d = d;
+    c.E = E;
+    c.I = I;
+    c.k1 = k1;
+    c.k2 = k1;
+    c.offsets = const_cast<int32_t *>(expert_offsets);
+    c.sorted_slot = const_cast<int32_t *>(sorted_slot);
+    c.uniq_count = uniq_count;
+    c.uniq_list = uniq_list;
+    c.h = h;
+    c.out = out;
+    c.hdr = static_cast<WsHeader *>(scratch);
+    return enqueue_stream(c, s);
 }

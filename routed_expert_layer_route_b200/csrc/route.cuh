@@ -68,13 +68,17 @@ __global__ void k_test_expc(const float *x, float *y, int64_t n)
 // ---------------------------------------------------------------------------
 // One CTA routes one token whose E logits sit in shared memory.
 // Shared scratch (caller-provided): ps[E], sel_p[E], sel_j[E], red[64].
-// Writes idx_out[s], w_out[s] for s < k1 (global).  All threads of the CTA
-// must call it.
+// Leaves the k1 selected experts and weights in sm.out_j / sm.out_w and
+// writes them to idx_out / w_out and the optional copies (each pointer
+// nullable).  All threads of the CTA must call it; blockDim.x is a multiple
+// of 32 and at least 32 * 2.
 struct __align__(16) RouteSmem {
     float ps[1024];
     float sel_p[1024];
     int sel_j[1024];
     float red[64];
+    int out_j[32];    // the k1 selected experts, rank order
+    float out_w[32];  // their Eq. 2 weights
 };
 
 __device__ void route_token_block(const float *zs, int E, int k1, int k2, RouteSmem &sm,
@@ -159,8 +163,12 @@ __device__ void route_token_block(const float *zs, int E, int k1, int k2, RouteS
         const float p = sm.sel_p[tid];
         const int j = sm.sel_j[tid];
         const float wv = renorm ? __fdiv_rn(p, sm.red[34]) : p;
-        idx_out[tid] = j;
-        w_out[tid] = wv;
+        sm.out_j[tid] = j;
+        sm.out_w[tid] = wv;
+        if (idx_out)
+            idx_out[tid] = j;
+        if (w_out)
+            w_out[tid] = wv;
         if (idx_copy)
             idx_copy[tid] = j;
         if (w_copy)
@@ -400,8 +408,7 @@ __global__ void __launch_bounds__(1024) k_topk(const float *logits, int T, int E
 // accumulation.  One warp per (expert, chunk of up to 8 tokens).  The warp's
 // W_r row is loaded into registers before the programmatic-launch wait (the
 // router weights never depend on earlier kernels), so its HBM latency
-// overlaps the previous kernel.  With `tail` set (T == 1), the last CTA to
-// finish routes the token and builds the permutation.
+// overlaps the previous kernel.
 constexpr int kLogitsWarps = 8;
 constexpr int kLogitsTok = 8;
 constexpr int kLogitsMaxVec = 16;  // register prefetch covers d <= 4096
@@ -410,18 +417,9 @@ struct LogitsArgs {
     const uint16_t *x;
     const uint16_t *wr;
     const float *bias;
-    float *z;          // [T x E] output (workspace or caller)
-    float *z_copy;     // nullable second copy (caller's logits_out)
+    float *z;       // [T x E] output (workspace or caller)
+    float *z_copy;  // nullable second copy (caller's logits_out)
     int T, d, E;
-    // tail (T == 1): route + permute by the last CTA
-    int tail;
-    int k1, k2;
-    int32_t *idx;
-    float *w;
-    int32_t *idx_copy;
-    float *w_copy;
-    PermOut perm;
-    WsHeader *hdr;
 };
 
 __global__ void __launch_bounds__(kLogitsWarps * 32) k_logits(LogitsArgs a)
@@ -447,88 +445,65 @@ __global__ void __launch_bounds__(kLogitsWarps * 32) k_logits(LogitsArgs a)
     }
     pdl_wait();
     pdl_trigger();
+    if (!has_item)
+        return;
 
-    if (has_item) {
-        const uint4 *row = reinterpret_cast<const uint4 *>(a.wr + (size_t)e * a.d);
-        const int t0 = chunk * kLogitsTok;
-        const int nt = min(kLogitsTok, a.T - t0);
-        float acc[kLogitsTok];
+    const uint4 *row = reinterpret_cast<const uint4 *>(a.wr + (size_t)e * a.d);
+    const int t0 = chunk * kLogitsTok;
+    const int nt = min(kLogitsTok, a.T - t0);
+    float acc[kLogitsTok];
 #pragma unroll
-        for (int t = 0; t < kLogitsTok; ++t)
-            acc[t] = 0.0f;
-        if (prefetch) {
-#pragma unroll
-            for (int i = 0; i < kLogitsMaxVec; ++i) {
-                const int v = lane + 32 * i;
-                if (v < nvec) {
-#pragma unroll
-                    for (int t = 0; t < kLogitsTok; ++t) {
-                        if (t < nt) {
-                            const uint4 xv = *(reinterpret_cast<const uint4 *>(
-                                                   a.x + (size_t)(t0 + t) * a.d) +
-                                               v);
-                            float xf[8] = {bf16lo(xv.x), bf16hi(xv.x), bf16lo(xv.y), bf16hi(xv.y),
-                                           bf16lo(xv.z), bf16hi(xv.z), bf16lo(xv.w), bf16hi(xv.w)};
-                            acc[t] = dot8_bf16(wv[i], xf, acc[t]);
-                        }
-                    }
-                }
-            }
-        } else {
-            for (int v = lane; v < nvec; v += 32) {
-                const uint4 wq = ld_nc_v4(row + v);
-#pragma unroll
-                for (int t = 0; t < kLogitsTok; ++t) {
-                    if (t < nt) {
-                        const uint4 xv =
-                            *(reinterpret_cast<const uint4 *>(a.x + (size_t)(t0 + t) * a.d) + v);
-                        float xf[8] = {bf16lo(xv.x), bf16hi(xv.x), bf16lo(xv.y), bf16hi(xv.y),
-                                       bf16lo(xv.z), bf16hi(xv.z), bf16lo(xv.w), bf16hi(xv.w)};
-                        acc[t] = dot8_bf16(wq, xf, acc[t]);
-                    }
-                }
-            }
-        }
+    for (int t = 0; t < kLogitsTok; ++t)
+        acc[t] = 0.0f;
+    if (prefetch) {
+        // all x vectors of this lane first (independent loads), then the math
+        uint4 xv[kLogitsMaxVec];
 #pragma unroll
         for (int t = 0; t < kLogitsTok; ++t) {
             if (t < nt) {
-                float s = warp_sum(acc[t]);
-                if (lane == 0) {
-                    if (a.bias)
-                        s = s + a.bias[e];
-                    a.z[(size_t)(t0 + t) * a.E + e] = s;
-                    if (a.z_copy)
-                        a.z_copy[(size_t)(t0 + t) * a.E + e] = s;
+                const uint4 *xr = reinterpret_cast<const uint4 *>(a.x + (size_t)(t0 + t) * a.d);
+#pragma unroll
+                for (int i = 0; i < kLogitsMaxVec; ++i) {
+                    const int v = lane + 32 * i;
+                    xv[i] = v < nvec ? xr[v] : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int i = 0; i < kLogitsMaxVec; ++i) {
+                    float xf[8] = {bf16lo(xv[i].x), bf16hi(xv[i].x), bf16lo(xv[i].y),
+                                   bf16hi(xv[i].y), bf16lo(xv[i].z), bf16hi(xv[i].z),
+                                   bf16lo(xv[i].w), bf16hi(xv[i].w)};
+                    acc[t] = dot8_bf16(wv[i], xf, acc[t]);
+                }
+            }
+        }
+    } else {
+        for (int v = lane; v < nvec; v += 32) {
+            const uint4 wq = ld_nc_v4(row + v);
+#pragma unroll
+            for (int t = 0; t < kLogitsTok; ++t) {
+                if (t < nt) {
+                    const uint4 xq =
+                        *(reinterpret_cast<const uint4 *>(a.x + (size_t)(t0 + t) * a.d) + v);
+                    float xf[8] = {bf16lo(xq.x), bf16hi(xq.x), bf16lo(xq.y), bf16hi(xq.y),
+                                   bf16lo(xq.z), bf16hi(xq.z), bf16lo(xq.w), bf16hi(xq.w)};
+                    acc[t] = dot8_bf16(wq, xf, acc[t]);
                 }
             }
         }
     }
-    if (!a.tail)
-        return;
-
-    // last-block hand-off: the final CTA routes the single token
-    __shared__ int is_last;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        const unsigned prev = atomicAdd(&a.hdr->route_arrive, 1u);
-        is_last = (prev == gridDim.x - 1);
+#pragma unroll
+    for (int t = 0; t < kLogitsTok; ++t) {
+        if (t < nt) {
+            float s = warp_sum(acc[t]);
+            if (lane == 0) {
+                if (a.bias)
+                    s = s + a.bias[e];
+                a.z[(size_t)(t0 + t) * a.E + e] = s;
+                if (a.z_copy)
+                    a.z_copy[(size_t)(t0 + t) * a.E + e] = s;
+            }
+        }
     }
-    __syncthreads();
-    if (!is_last)
-        return;
-    if (threadIdx.x == 0)
-        a.hdr->route_arrive = 0u;
-    __threadfence();
-    __shared__ RouteSmem sm;
-    __shared__ float zs[1024];
-    for (int j = threadIdx.x; j < a.E; j += blockDim.x)
-        zs[j] = __ldcg(&a.z[j]);
-    __syncthreads();
-    route_token_block(zs, a.E, a.k1, a.k2, sm, a.idx, a.w, a.idx_copy, a.w_copy);
-    __syncthreads();
-    extern __shared__ int dsm[];
-    permute_block(a.idx, 1, a.k1, a.E, a.perm, dsm, &a.hdr->status);
 }
 
 }  // namespace moe

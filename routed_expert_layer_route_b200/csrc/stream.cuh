@@ -7,63 +7,84 @@
 //     h_c = silu(W_gate[c,:] . x) * (W_up[c,:] . x),   o = W_down h.
 //
 // Design (one persistent CTA per SM, grid = number of SMs):
+//  * routing state first: either the CTA routes the single token itself from
+//    its float32 logits (T == 1, every CTA redundantly, with the same fixed
+//    float32 operation sequence as the router kernels), or it loads the
+//    routing tables written by the permutation kernel -- in both cases in one
+//    round of independent loads, into shared memory, together with the
+//    tokens' x rows when they fit;
 //  * the U activated experts (ascending ids) are laid end to end as U*I
 //    channels; CTA b owns the contiguous channel range
 //    [b*U*I/G, (b+1)*U*I/G), so every CTA streams the same number of gate/up
 //    bytes (within one channel) whatever k1, U or the batch;
-//  * phase 1: gate and up rows of the CTA's channels (contiguous in HBM) are
-//    moved by bulk asynchronous copies (cp.async.bulk, no multicast) into a
-//    ring of shared-memory stages by one producer thread; 16 consumer warps
-//    form the dot products with the expert's tokens (staged in shared
-//    memory) and write h (float32) for their channels;
+//  * one producer thread moves the CTA's weights with bulk asynchronous
+//    copies (cp.async.bulk, no multicast) into a ring of kStages shared-memory
+//    stages; stage s lands in slot s % kStages and is consumed by the
+//    consumer warps bound to that slot, each warp owning whole work units
+//    (one channel = its gate row and up row; or one down row), so no stage
+//    needs a cross-warp reduction or barrier;
+//  * phase 1: gate/up rows of the CTA's channels -> h (float32) for them;
 //  * one grid-wide barrier (bounded spin) makes every h visible;
 //  * phase 2: CTA b owns the output rows [b*d/G, (b+1)*d/G) of every
-//    activated expert; its W_down rows (contiguous, I elements each) stream
+//    activated expert; its W_down rows (contiguous, I elements each) go
 //    through the same ring -- the producer issues them before the barrier
-//    completes, so the barrier hides under copies in flight -- and the
-//    consumers write o = W_down h for the expert's tokens;
-//  * the combine of Eq. 2's weights runs on the CTA's own rows: y[t, r] =
+//    completes, so the barrier hides under copies in flight;
+//  * the combine with Eq. 2's weights runs on the CTA's own rows: y[t, r] =
 //    sum_s w[t, s] o[slot(t, s), r] in slot order, float32, no atomics, so
 //    the output is deterministic.
 #pragma once
 #include "common.cuh"
+#include "route.cuh"
 
 namespace moe {
 
-constexpr int kSC = 16;                      // consumer warps
-constexpr int kSThreads = (kSC + 1) * 32;    // + one producer warp
-constexpr int kStages = 5;
+constexpr int kSC = 12;                    // consumer warps (13 warps in all: <= 4 per SM
+                                           // sub-partition, so up to 128 registers each)
+constexpr int kSThreads = (kSC + 1) * 32;  // + one producer warp
+constexpr int kStages = 4;
+constexpr int kWPS = kSC / kStages;        // consumer warps bound to each ring slot
 constexpr int kStageBytes = 32 * 1024;
-constexpr int kTokChunk = 8;                 // most tokens staged in shared memory at once
-constexpr int kTokBytes = 32 * 1024;         // staging area for one token chunk
-constexpr int kMaxRows = 128;                // rows of one stage
-constexpr int kPartItems = 128;              // (row, slice) items of one stage
-constexpr int kConsumerBar = 1;              // named barrier id of the consumer warps
+constexpr int kTokChunk = 4;               // most tokens per dot-product pass
+constexpr int kAreaBytes = 48 * 1024;      // x rows (phase 1) or h rows (phase 2)
+constexpr int kMaxRows = 128;              // rows of one stage
+constexpr int kMetaU = 1024;               // activated experts kept in shared memory
+constexpr int kSlotMax = 1024;             // routed slots kept in shared memory
+constexpr int kObufFloats = 4096;          // per-slot down outputs of this CTA's rows
+constexpr int kConsumerBar = 1;            // named barrier id of the consumer warps
+
+static_assert(kSC % kStages == 0, "consumer warps split evenly over the ring slots");
 
 struct StreamArgs {
     const uint16_t *x;   // [T x d]
     const uint16_t *wg;  // [E x I x d]
     const uint16_t *wu;  // [E x I x d]
     const uint16_t *wd;  // [E x d x I]
-    int T, d, E, I, k1;
-    const int32_t *offsets;      // [E+1]
-    const int32_t *sorted_slot;  // [T*k1]
-    const int32_t *uniq_count;   // [1]
-    const int32_t *uniq_list;    // [E]
-    float *h;                    // [T*k1 x I] scratch
-    float *out;                  // [T*k1 x d] per-slot outputs, sorted order
-    void *y;                     // nullable: combine into y [T x d]
+    int T, d, E, I, k1, k2;
+    // route_in_kernel (T == 1): route from logits[0..E) and write the routing
+    // tables below (CTA 0); otherwise the tables are inputs.
+    int route_in_kernel;
+    const float *logits;
+    int32_t *topk_idx;     // [T x k1]  (route mode: output)
+    float *topk_w;         // [T x k1]  (route mode: output; combine: input)
+    int32_t *idx_copy;     // nullable user copies (route mode)
+    float *w_copy;
+    int32_t *offsets;      // [E+1]
+    int32_t *sorted_slot;  // [T*k1]
+    int32_t *slot_pos;     // [T*k1]
+    int32_t *uniq_count;   // [1]
+    int32_t *uniq_list;    // [E]
+    float *h;              // [T*k1 x I] scratch
+    float *out;            // [T*k1 x d] per-slot outputs, sorted order (nullable when y is set)
+    void *y;               // nullable: combine into y [T x d]
     int y_dtype;
-    const float *topk_w;         // [T x k1]
-    const int32_t *slot_pos;     // [T*k1]
     WsHeader *hdr;
 };
 
-// The ordered list of stages a CTA works through; the producer and the
-// consumers walk it independently and identically.
+// The ordered list of stages a CTA works through; the producer and every
+// consumer warp walk it independently and identically.
 struct Stage {
     int phase;  // 1: gate/up rows of channels [c, c+n); 2: W_down rows [r, r+n)
-    int u;      // index into uniq_list
+    int u;      // index into the activated-expert list
     int c;      // first channel (phase 1) or first row (phase 2)
     int n;      // channels (phase 1) or rows (phase 2)
 };
@@ -84,7 +105,11 @@ struct StageIter {
         c_hi = tot * (b + 1) / G;
         r_lo = (int)((int64_t)d * b / G);
         r_hi = (int)((int64_t)d * (b + 1) / G);
+        // channels per stage: a multiple of the warps serving a slot when the
+        // stage holds that many, so each warp owns the same number of units
         nch = max(1, min(kMaxRows / 2, kStageBytes / (4 * d)));
+        if (nch >= kWPS)
+            nch -= nch % kWPS;
         nrows = max(1, min(kMaxRows, kStageBytes / (2 * I)));
         u2 = 0;
         r2 = r_lo;
@@ -128,34 +153,109 @@ struct StageIter {
     }
 };
 
-__device__ __forceinline__ int floor_pow2(int v)
-{
-    int p = 1;
-    while (p * 2 <= v)
-        p *= 2;
-    return p;
-}
-
-struct __align__(16) ConsumerSmem {
-    float part[2][kPartItems * kTokChunk];
-    int tok_pos0;  // first sorted position of the staged expert
-    int tok_cnt;   // tokens of the staged expert
+// Shared memory besides the ring (dynamic, right after the ring's barriers).
+struct __align__(16) StreamSmem {
+    float obuf[kObufFloats];  // o[p][r - r_lo] when it fits
+    int ue[kMetaU];           // activated experts, ascending
+    int up0[kMetaU];          // first sorted position of each
+    int uM[kMetaU];           // tokens of each
+    int stok[kSlotMax];       // token of each sorted position
+    float sw[kSlotMax];       // Eq. 2 weight of each slot t*k1+s
+    int spos[kSlotMax];       // sorted position of each slot
+    int U;
     int abort;
-    int issued;    // stages issued by the producer
+    int issued;  // stages issued by the producer
+    int pad;
 };
 
 __device__ __forceinline__ void consumer_sync() { named_bar_sync(kConsumerBar, kSC * 32); }
 
-// tokens per staged chunk: as many rows of x (bf16, d) or h (float32, I) as
-// fit the staging area, at most kTokChunk
-__host__ __device__ __forceinline__ int tok_chunk(int d, int I)
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+
+__device__ __forceinline__ void bf16x8(const uint4 v, float f[8])
 {
-    const int row = 2 * d > 4 * I ? 2 * d : 4 * I;
-    const int n = kTokBytes / row;
-    return n < 1 ? 1 : (n > kTokChunk ? kTokChunk : n);
+    f[0] = bf16lo(v.x);
+    f[1] = bf16hi(v.x);
+    f[2] = bf16lo(v.y);
+    f[3] = bf16hi(v.y);
+    f[4] = bf16lo(v.z);
+    f[5] = bf16hi(v.z);
+    f[6] = bf16lo(v.w);
+    f[7] = bf16hi(v.w);
 }
 
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+// Row pointers of up to kTokChunk tokens, passed by value so they stay in
+// registers.
+struct XRows {
+    const uint4 *r[kTokChunk];
+};
+struct HRows {
+    const float4 *r[kTokChunk];
+};
+
+// One channel: g_t = W_gate[c,:] . x_t and u_t = W_up[c,:] . x_t for NT
+// tokens (rows xr.r[t], bf16), reduced over the warp (every lane gets the sums).
+template <int NT>
+__device__ __forceinline__ void unit_gate_up(const uint4 *grow, const uint4 *urow, const XRows xr,
+                                             int nvec, int lane, float (&g)[kTokChunk],
+                                             float (&u)[kTokChunk])
+{
+    float ag[NT], au[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+        ag[t] = au[t] = 0.0f;
+    for (int v = lane; v < nvec; v += 32) {
+        const uint4 wg = grow[v], wu = urow[v];
+        float fg[8], fu[8];
+        bf16x8(wg, fg);
+        bf16x8(wu, fu);
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            float xf[8];
+            bf16x8(xr.r[t][v], xf);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                ag[t] = fmaf(fg[k], xf[k], ag[t]);
+                au[t] = fmaf(fu[k], xf[k], au[t]);
+            }
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+        g[t] = warp_sum(ag[t]);
+        u[t] = warp_sum(au[t]);
+    }
+}
+
+// One down row: o_t = W_down[r,:] . h_t for NT tokens (rows hr.r[t], float32).
+template <int NT>
+__device__ __forceinline__ void unit_down(const uint4 *wrow, const HRows hr, int nvec, int lane,
+                                          float (&o)[kTokChunk])
+{
+    float acc[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+        acc[t] = 0.0f;
+    for (int v = lane; v < nvec; v += 32) {
+        float fw[8];
+        bf16x8(wrow[v], fw);
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            const float4 h0 = hr.r[t][2 * v], h1 = hr.r[t][2 * v + 1];
+            acc[t] = fmaf(fw[0], h0.x, acc[t]);
+            acc[t] = fmaf(fw[1], h0.y, acc[t]);
+            acc[t] = fmaf(fw[2], h0.z, acc[t]);
+            acc[t] = fmaf(fw[3], h0.w, acc[t]);
+            acc[t] = fmaf(fw[4], h1.x, acc[t]);
+            acc[t] = fmaf(fw[5], h1.y, acc[t]);
+            acc[t] = fmaf(fw[6], h1.z, acc[t]);
+            acc[t] = fmaf(fw[7], h1.w, acc[t]);
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+        o[t] = warp_sum(acc[t]);
+}
 
 __global__ void __launch_bounds__(kSThreads, 1) k_stream(StreamArgs a)
 {
@@ -163,22 +263,25 @@ __global__ void __launch_bounds__(kSThreads, 1) k_stream(StreamArgs a)
     uint8_t *ring = smem;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes);
     uint64_t *empty = full + kStages;
-    ConsumerSmem *cs = reinterpret_cast<ConsumerSmem *>(empty + kStages);
-    // staging area for one token chunk: x rows (bf16, phase 1) or h rows
-    // (float32, phase 2); 16-byte aligned
-    uint8_t *tok_area = reinterpret_cast<uint8_t *>(cs + 1);
+    StreamSmem *ss = reinterpret_cast<StreamSmem *>(empty + kStages);
+    uint8_t *area = reinterpret_cast<uint8_t *>(ss + 1);  // kAreaBytes, 16-byte aligned
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = gridDim.x, b = blockIdx.x;
     int *status = &a.hdr->status;
+    const int T = a.T, d = a.d, E = a.E, I = a.I, k1 = a.k1;
+    const int nslots = T * k1;
+    const bool slots_in_smem = nslots <= kSlotMax;
+    const bool x_in_smem = (size_t)T * d * 2 <= (size_t)kAreaBytes;
+    const bool h_in_smem = (size_t)nslots * I * 4 <= (size_t)kAreaBytes;
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kSC);
+            mbar_init(&empty[s], kWPS);
         }
-        cs->abort = 0;
-        cs->issued = 0;
+        ss->abort = 0;
+        ss->issued = 0;
         fence_mbar_init();
     }
     __syncthreads();
@@ -186,15 +289,112 @@ __global__ void __launch_bounds__(kSThreads, 1) k_stream(StreamArgs a)
     pdl_wait();
     pdl_trigger();
 
-    const int nslots = a.T * a.k1;
-    int U = __ldcg(a.uniq_count);
-    if (U < 0 || U > a.E) {
-        if (tid == 0)
-            set_status(status, MOE_ERR_DEVICE_CHECK);
-        U = 0;
+    // ------------------------------------------------------------ routing state
+    // the tokens' x rows (independent of routing) go out in the same round
+    if (x_in_smem) {
+        const int nv = T * (d >> 3);
+        for (int i = tid; i < nv; i += kSThreads)
+            reinterpret_cast<uint4 *>(area)[i] = reinterpret_cast<const uint4 *>(a.x)[i];
     }
-    const int d = a.d, I = a.I, k1 = a.k1;
-    const int mtc = tok_chunk(d, I);
+    if (a.route_in_kernel) {
+        // T == 1: every CTA ranks the E probabilities itself (the ring is idle
+        // until routing is known, so the routing scratch lives there)
+        RouteSmem &rs = *reinterpret_cast<RouteSmem *>(ring);
+        float *zs = reinterpret_cast<float *>(ring + sizeof(RouteSmem));
+        for (int j = tid; j < E; j += kSThreads)
+            zs[j] = __ldcg(&a.logits[j]);
+        __syncthreads();
+        route_token_block(zs, E, k1, a.k2, rs, b == 0 ? a.topk_idx : nullptr,
+                          b == 0 ? a.topk_w : nullptr, b == 0 ? a.idx_copy : nullptr,
+                          b == 0 ? a.w_copy : nullptr);
+        __syncthreads();
+        if (tid < k1) {
+            const int e = rs.out_j[tid];
+            int p = 0;
+            for (int s = 0; s < k1; ++s)
+                p += rs.out_j[s] < e;
+            ss->ue[p] = e;
+            ss->up0[p] = p;
+            ss->uM[p] = 1;
+            ss->stok[p] = 0;
+            ss->sw[tid] = rs.out_w[tid];
+            ss->spos[tid] = p;
+            if (b == 0) {
+                a.uniq_list[p] = e;
+                a.sorted_slot[p] = tid;
+                a.slot_pos[tid] = p;
+            }
+        }
+        if (tid == 0) {
+            ss->U = k1;
+            if (b == 0)
+                *a.uniq_count = k1;
+        }
+        if (b == 0) {
+            for (int e = tid; e <= E; e += kSThreads) {
+                int c = 0;
+                for (int s = 0; s < k1; ++s)
+                    c += rs.out_j[s] < e;
+                a.offsets[e] = c;
+            }
+        }
+        __syncthreads();
+    } else {
+        // tables written by the permutation kernel: one round of loads
+        int *t_uniq = reinterpret_cast<int *>(ring);  // [E]
+        int *t_off = t_uniq + 1024;                   // [E+1]
+        for (int i = tid; i < E; i += kSThreads)
+            t_uniq[i] = __ldcg(&a.uniq_list[i]);
+        for (int i = tid; i <= E; i += kSThreads)
+            t_off[i] = __ldcg(&a.offsets[i]);
+        if (slots_in_smem) {
+            for (int i = tid; i < nslots; i += kSThreads) {
+                const int sl = __ldcg(&a.sorted_slot[i]);
+                int t = sl / k1;
+                if (sl < 0 || t >= T) {
+                    set_status(status, MOE_ERR_DEVICE_CHECK);
+                    t = 0;
+                }
+                ss->stok[i] = t;
+                if (a.y) {
+                    ss->sw[i] = __ldcg(&a.topk_w[i]);
+                    int p = __ldcg(&a.slot_pos[i]);
+                    if (p < 0 || p >= nslots) {
+                        set_status(status, MOE_ERR_DEVICE_CHECK);
+                        p = 0;
+                    }
+                    ss->spos[i] = p;
+                }
+            }
+        }
+        if (tid == 0) {
+            int U = __ldcg(a.uniq_count);
+            if (U < 0 || U > E || U > kMetaU) {
+                set_status(status, MOE_ERR_DEVICE_CHECK);
+                U = 0;
+            }
+            ss->U = U;
+        }
+        __syncthreads();
+        const int U = ss->U;
+        for (int u = tid; u < U; u += kSThreads) {
+            const int e = min(max(t_uniq[u], 0), E - 1);
+            int p0 = t_off[e], M = t_off[e + 1] - p0;
+            if (p0 < 0 || M < 0 || p0 + M > nslots) {  // inconsistent routing state
+                set_status(status, MOE_ERR_DEVICE_CHECK);
+                p0 = 0;
+                M = 0;
+            }
+            ss->ue[u] = e;
+            ss->up0[u] = p0;
+            ss->uM[u] = M;
+        }
+        __syncthreads();
+    }
+    const int U = ss->U;
+    const int r_lo = (int)((int64_t)d * b / G), r_hi = (int)((int64_t)d * (b + 1) / G);
+    const int nr = r_hi - r_lo;
+    const bool obuf_ok = a.y && (size_t)nslots * nr <= (size_t)kObufFloats;
 
     if (warp == kSC) {
         // ------------------------------------------------------------ producer
@@ -206,14 +406,14 @@ __global__ void __launch_bounds__(kSThreads, 1) k_stream(StreamArgs a)
             uint32_t ph = 0;
             int issued = 0;
             while (it.valid()) {
-                if (*(volatile int *)&cs->abort)
+                if (*(volatile int *)&ss->abort)
                     break;
                 if (!mbar_wait(&empty[slot], ph ^ 1u, status)) {
-                    cs->abort = 1;
+                    ss->abort = 1;
                     break;
                 }
                 const Stage st = it.get();
-                const int e = min(max(__ldcg(&a.uniq_list[st.u]), 0), a.E - 1);
+                const int e = ss->ue[st.u];
                 uint8_t *dst = ring + (size_t)slot * kStageBytes;
                 if (st.phase == 1) {
                     const uint32_t bytes = (uint32_t)st.n * d * 2;
@@ -233,220 +433,175 @@ __global__ void __launch_bounds__(kSThreads, 1) k_stream(StreamArgs a)
                     ph ^= 1u;
                 }
             }
-            cs->issued = issued;
+            ss->issued = issued;
         }
         __syncwarp();
     } else {
         // ------------------------------------------------------------ consumers
+        const int group = warp / kWPS;  // the ring slot this warp serves
+        const int gl = warp % kWPS;     // this warp's index inside its group
         StageIter it;
         it.init(U, I, d, b, G);
-        int slot = 0;
-        uint32_t ph = 0;
-        int iter = 0;       // part[] double-buffer parity
-        int staged_u = -1;  // expert whose token chunk sits in tok_area
-        int staged_m0 = -1;
-        int staged_phase = 0;
+        int sidx = 0;  // global stage index
         bool arrived = false;
 
-        auto do_grid_barrier = [&]() {
-            __threadfence();  // this thread's h stores are visible device-wide
-            consumer_sync();
-            if (tid == 0) {
-                unsigned gen0 = ld_acquire_u32(&a.hdr->bar_gen);
-                // the generation read above was taken before this CTA
-                // arrives, so it cannot have advanced yet
-                __threadfence();
-                const unsigned prev = atomicAdd(&a.hdr->bar_count, 1u);
-                if (prev == (unsigned)G - 1) {
-                    atomicExch(&a.hdr->bar_count, 0u);
-                    __threadfence();
-                    atomicAdd(&a.hdr->bar_gen, 1u);
-                } else {
-                    const uint64_t t0 = global_ns();
-                    while (ld_acquire_u32(&a.hdr->bar_gen) == gen0) {
-                        if (global_ns() - t0 > MOE_WAIT_LIMIT_NS) {
-                            set_status(status, MOE_ERR_TIMEOUT);
-                            cs->abort = 1;
-                            break;
-                        }
-                        __nanosleep(64);
-                    }
-                }
-                __threadfence();
+        auto x_row = [&](int p) -> const uint4 * {
+            int t;
+            if (slots_in_smem) {
+                t = ss->stok[p];
+            } else {
+                const int sl = __ldcg(&a.sorted_slot[p]);
+                t = sl / k1;
+                if (sl < 0 || t >= T)
+                    t = 0;
             }
-            consumer_sync();
+            return x_in_smem ? reinterpret_cast<const uint4 *>(area + (size_t)t * d * 2)
+                             : reinterpret_cast<const uint4 *>(a.x + (size_t)t * d);
+        };
+        auto h_row = [&](int p) -> const float4 * {
+            return h_in_smem ? reinterpret_cast<const float4 *>(area + (size_t)p * I * 4)
+                             : reinterpret_cast<const float4 *>(a.h + (size_t)p * I);
         };
 
         while (true) {
             const bool have = it.valid();
             const Stage st = have ? it.get() : Stage{0, 0, 0, 0};
             if (!arrived && (!have || st.phase == 2)) {
-                do_grid_barrier();
+                // grid barrier: every CTA's h is written before any is read
+                __threadfence();
+                consumer_sync();
+                if (tid == 0) {
+                    const unsigned gen0 = ld_acquire_u32(&a.hdr->bar_gen);
+                    // read before this CTA arrives, so it cannot have advanced yet
+                    __threadfence();
+                    const unsigned prev = atomicAdd(&a.hdr->bar_count, 1u);
+                    if (prev == (unsigned)G - 1) {
+                        atomicExch(&a.hdr->bar_count, 0u);
+                        __threadfence();
+                        atomicAdd(&a.hdr->bar_gen, 1u);
+                    } else {
+                        const uint64_t t0 = global_ns();
+                        while (ld_acquire_u32(&a.hdr->bar_gen) == gen0) {
+                            if (global_ns() - t0 > MOE_WAIT_LIMIT_NS) {
+                                set_status(status, MOE_ERR_TIMEOUT);
+                                ss->abort = 1;
+                                break;
+                            }
+                        }
+                    }
+                    __threadfence();
+                }
+                consumer_sync();
+                if (h_in_smem && have) {
+                    const int n4 = nslots * (I >> 2);
+                    for (int i = tid; i < n4; i += kSC * 32)
+                        reinterpret_cast<float4 *>(area)[i] =
+                            __ldcg(reinterpret_cast<const float4 *>(a.h) + i);
+                    consumer_sync();
+                }
                 arrived = true;
-                staged_u = -1;
             }
             if (!have)
                 break;
 
-            const int e = min(max(__ldcg(&a.uniq_list[st.u]), 0), a.E - 1);
-            int p0 = __ldcg(&a.offsets[e]);
-            int M = __ldcg(&a.offsets[e + 1]) - p0;
-            if (p0 < 0 || M < 0 || p0 + M > nslots) {  // inconsistent routing state
-                if (tid == 0)
-                    set_status(status, MOE_ERR_DEVICE_CHECK);
-                p0 = 0;
-                M = 0;
-            }
-
-            const bool ok = !*(volatile int *)&cs->abort && mbar_wait(&full[slot], ph, status);
-            if (!ok)
-                cs->abort = 1;
-
-            const int rows = st.phase == 1 ? 2 * st.n : st.n;
-            const int rowlen = st.phase == 1 ? d : I;  // elements per row
-            const int nvec = rowlen >> 3;
-            int S = floor_pow2(max(1, kSC / rows));
-            S = min(S, max(1, nvec / 32));
-            const int items = rows * S;
-            const int vper = (nvec + S - 1) / S;  // vectors per slice
-            const uint8_t *stg = ring + (size_t)slot * kStageBytes;
-
-            for (int m0 = 0; m0 < M; m0 += mtc) {
-                const int mt = min(mtc, M - m0);
-                // stage this expert's token chunk (x for phase 1, h for phase 2)
-                if (staged_u != st.u || staged_m0 != m0 || staged_phase != st.phase) {
-                    consumer_sync();  // nobody still reads tok_area
-                    if (st.phase == 1) {
-                        const int vpr = d >> 3;
-                        for (int i = tid; i < mt * vpr; i += kSC * 32) {
-                            const int m = i / vpr, v = i % vpr;
-                            const int slotid = __ldcg(&a.sorted_slot[p0 + m0 + m]);
-                            int t = slotid / k1;
-                            if (slotid < 0 || t >= a.T) {
-                                set_status(status, MOE_ERR_DEVICE_CHECK);
-                                t = 0;
-                            }
-                            reinterpret_cast<uint4 *>(tok_area)[m * vpr + v] =
-                                reinterpret_cast<const uint4 *>(a.x + (size_t)t * d)[v];
-                        }
-                    } else {
-                        const int vpr = I >> 2;  // float4 per h row
-                        for (int i = tid; i < mt * vpr; i += kSC * 32) {
-                            const int m = i / vpr, v = i % vpr;
-                            reinterpret_cast<float4 *>(tok_area)[m * vpr + v] = __ldcg(
-                                reinterpret_cast<const float4 *>(a.h + (size_t)(p0 + m0 + m) * I) + v);
-                        }
-                    }
-                    consumer_sync();
-                    staged_u = st.u;
-                    staged_m0 = m0;
-                    staged_phase = st.phase;
-                }
-                float *part = cs->part[iter & 1];
+            if (sidx % kStages == group) {
+                const int slot = group;
+                const uint32_t parity = (uint32_t)((sidx / kStages) & 1);
+                const bool ok =
+                    !*(volatile int *)&ss->abort && mbar_wait(&full[slot], parity, status);
+                if (!ok)
+                    ss->abort = 1;
                 if (ok) {
-                    for (int item = warp; item < items; item += kSC) {
-                        const int r = item / S, sl = item % S;
-                        const uint4 *wrow =
-                            reinterpret_cast<const uint4 *>(stg + (size_t)r * rowlen * 2);
-                        float acc[kTokChunk];
-#pragma unroll
-                        for (int m = 0; m < kTokChunk; ++m)
-                            acc[m] = 0.0f;
-                        const int vb = sl * vper, ve = min(nvec, vb + vper);
-                        for (int v = vb + lane; v < ve; v += 32) {
-                            const uint4 wv = wrow[v];
+                    const int p0 = ss->up0[st.u];
+                    const int M = ss->uM[st.u];
+                    const uint8_t *stg = ring + (size_t)slot * kStageBytes;
+                    for (int unit = gl; unit < st.n; unit += kWPS) {
+                        for (int m0 = 0; m0 < M; m0 += kTokChunk) {
+                            const int mt = min(kTokChunk, M - m0);
+                            float r0[kTokChunk], r1[kTokChunk];
                             if (st.phase == 1) {
+                                const uint4 *grow =
+                                    reinterpret_cast<const uint4 *>(stg + (size_t)unit * d * 2);
+                                const uint4 *urow = reinterpret_cast<const uint4 *>(
+                                    stg + (size_t)(st.n + unit) * d * 2);
+                                XRows xr;
 #pragma unroll
-                                for (int m = 0; m < kTokChunk; ++m) {
-                                    if (m < mt) {
-                                        const uint4 xv =
-                                            reinterpret_cast<const uint4 *>(tok_area)[m * nvec + v];
-                                        float xf[8] = {bf16lo(xv.x), bf16hi(xv.x), bf16lo(xv.y),
-                                                       bf16hi(xv.y), bf16lo(xv.z), bf16hi(xv.z),
-                                                       bf16lo(xv.w), bf16hi(xv.w)};
-                                        acc[m] = dot8_bf16(wv, xf, acc[m]);
-                                    }
-                                }
+                                for (int t = 0; t < kTokChunk; ++t)
+                                    xr.r[t] = x_row(p0 + m0 + min(t, mt - 1));
+                                const int nvec = d >> 3;
+                                if (mt == 1)
+                                    unit_gate_up<1>(grow, urow, xr, nvec, lane, r0, r1);
+                                else if (mt == 2)
+                                    unit_gate_up<2>(grow, urow, xr, nvec, lane, r0, r1);
+                                else
+                                    unit_gate_up<4>(grow, urow, xr, nvec, lane, r0, r1);
+#pragma unroll
+                                for (int t = 0; t < kTokChunk; ++t)
+                                    if (lane == t && t < mt)
+                                        a.h[(size_t)(p0 + m0 + t) * I + st.c + unit] =
+                                            silu_mul(r0[t], r1[t]);
                             } else {
+                                const uint4 *wrow =
+                                    reinterpret_cast<const uint4 *>(stg + (size_t)unit * I * 2);
+                                HRows hr;
 #pragma unroll
-                                for (int m = 0; m < kTokChunk; ++m) {
-                                    if (m < mt) {
-                                        const float4 *hp = reinterpret_cast<const float4 *>(
-                                            tok_area + ((size_t)m * I + (size_t)v * 8) * 4);
-                                        const float4 h0 = hp[0], h1 = hp[1];
-                                        float hf[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-                                        acc[m] = dot8_bf16(wv, hf, acc[m]);
+                                for (int t = 0; t < kTokChunk; ++t)
+                                    hr.r[t] = h_row(p0 + m0 + min(t, mt - 1));
+                                const int nvec = I >> 3;
+                                if (mt == 1)
+                                    unit_down<1>(wrow, hr, nvec, lane, r0);
+                                else if (mt == 2)
+                                    unit_down<2>(wrow, hr, nvec, lane, r0);
+                                else
+                                    unit_down<4>(wrow, hr, nvec, lane, r0);
+                                const int row = st.c + unit;
+#pragma unroll
+                                for (int t = 0; t < kTokChunk; ++t) {
+                                    if (lane == t && t < mt) {
+                                        const int p = p0 + m0 + t;
+                                        if (obuf_ok)
+                                            ss->obuf[p * nr + (row - r_lo)] = r0[t];
+                                        else
+                                            a.out[(size_t)p * d + row] = r0[t];
                                     }
                                 }
                             }
                         }
-#pragma unroll
-                        for (int m = 0; m < kTokChunk; ++m) {
-                            if (m < mt) {
-                                const float s = warp_sum(acc[m]);
-                                if (lane == 0)
-                                    part[item * kTokChunk + m] = s;
-                            }
-                        }
                     }
                 }
-                if (m0 + mtc >= M) {
-                    // last read of this stage's weights: hand the slot back
-                    __syncwarp();
-                    if (lane == 0)
-                        mbar_arrive(&empty[slot]);
-                }
-                consumer_sync();
-                if (ok) {
-                    if (st.phase == 1) {
-                        for (int i = tid; i < st.n * mt; i += kSC * 32) {
-                            const int ch = i / mt, m = i % mt;
-                            float g = 0.0f, u = 0.0f;
-                            for (int sl = 0; sl < S; ++sl) {
-                                g += part[((ch)*S + sl) * kTokChunk + m];
-                                u += part[((st.n + ch) * S + sl) * kTokChunk + m];
-                            }
-                            a.h[(size_t)(p0 + m0 + m) * I + st.c + ch] = silu_mul(g, u);
-                        }
-                    } else {
-                        for (int i = tid; i < st.n * mt; i += kSC * 32) {
-                            const int r = i / mt, m = i % mt;
-                            float o = 0.0f;
-                            for (int sl = 0; sl < S; ++sl)
-                                o += part[(r * S + sl) * kTokChunk + m];
-                            a.out[(size_t)(p0 + m0 + m) * d + st.c + r] = o;
-                        }
-                    }
-                }
-                ++iter;
-            }
-            if (M == 0) {  // cannot happen for an activated expert; keep the ring moving
+                // this warp is done with the stage's weights: hand the slot back
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(&empty[slot]);
             }
+            ++sidx;
             it.next();
-            if (++slot == kStages) {
-                slot = 0;
-                ph ^= 1u;
-            }
         }
 
         // ------------------------------------------------------------ combine
         if (a.y) {
-            consumer_sync();  // every out[] row of this CTA is written
-            const int r_lo = (int)((int64_t)d * b / G), r_hi = (int)((int64_t)d * (b + 1) / G);
-            const int nr = r_hi - r_lo;
-            for (int i = tid; i < a.T * nr; i += kSC * 32) {
+            consumer_sync();  // every o of this CTA's rows is written
+            for (int i = tid; i < T * nr; i += kSC * 32) {
                 const int t = i / nr, r = r_lo + i % nr;
                 float acc = 0.0f;
                 for (int s = 0; s < k1; ++s) {
-                    const int pos = __ldcg(&a.slot_pos[t * k1 + s]);
-                    if (pos < 0 || pos >= nslots) {
-                        set_status(status, MOE_ERR_DEVICE_CHECK);
-                        continue;
+                    const int sl = t * k1 + s;
+                    int pos;
+                    float w;
+                    if (slots_in_smem) {
+                        pos = ss->spos[sl];
+                        w = ss->sw[sl];
+                    } else {
+                        pos = __ldcg(&a.slot_pos[sl]);
+                        w = __ldcg(&a.topk_w[sl]);
+                        if (pos < 0 || pos >= nslots) {
+                            set_status(status, MOE_ERR_DEVICE_CHECK);
+                            continue;
+                        }
                     }
-                    const float prod = __ldcg(&a.topk_w[t * k1 + s]) * a.out[(size_t)pos * d + r];
+                    const float o = obuf_ok ? ss->obuf[pos * nr + (r - r_lo)]
+                                            : a.out[(size_t)pos * d + r];
+                    const float prod = w * o;
                     acc = acc + prod;
                 }
                 if (a.y_dtype == MOE_DTYPE_BF16)
@@ -460,8 +615,8 @@ __global__ void __launch_bounds__(kSThreads, 1) k_stream(StreamArgs a)
     __syncthreads();
     // After an abort, wait (bounded) for copies that may still be in flight
     // before the CTA's shared memory is released.
-    if (tid == 0 && cs->abort) {
-        const int issued = cs->issued;
+    if (tid == 0 && ss->abort) {
+        const int issued = ss->issued;
         for (int s = 0; s < kStages && s < issued; ++s) {
             const int last = issued - 1 - ((issued - 1 - s) % kStages);  // last stage on slot s
             const uint32_t parity = (uint32_t)((last / kStages) & 1);
@@ -470,11 +625,10 @@ __global__ void __launch_bounds__(kSThreads, 1) k_stream(StreamArgs a)
     }
 }
 
-size_t stream_smem_bytes(int d, int I)
+inline size_t stream_smem_bytes()
 {
-    const size_t tok = (size_t)tok_chunk(d, I) * (size_t)(d * 2 > I * 4 ? d * 2 : I * 4);
-    return (size_t)kStages * kStageBytes + 2 * kStages * sizeof(uint64_t) + sizeof(ConsumerSmem) +
-           16 + tok;
+    return (size_t)kStages * kStageBytes + 2 * kStages * sizeof(uint64_t) + sizeof(StreamSmem) +
+           kAreaBytes;
 }
 
 }  // namespace moe

@@ -50,8 +50,8 @@ SIGNATURES = {
     "moe_expert_ffn_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
     "moe_test_exp_c": (_i, [_vp, _vp, ctypes.c_int64, _vp]),
     "moe_test_num_sms": (_i, []),
-    "moe_test_expert_stream": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _sz,
-                                    _vp]),
+    "moe_test_expert_stream": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _vp,
+                                    _sz, _vp]),
 }
 
 _lib = None
@@ -211,11 +211,11 @@ def moe_test_num_sms():
     return lib().moe_test_num_sms()
 
 
-def moe_test_expert_stream(x, w_gate, w_up, w_down, k1, y, ws, stream=None):
+def moe_test_expert_stream(x, w_gate, w_up, w_down, k1, k2, y, ws, stream=None):
     T, d = x.shape
     E, I, _ = w_gate.shape
     y_dtype = MOE_DTYPE_BF16 if y.dtype == torch.bfloat16 else MOE_DTYPE_F32
     wsp, wsn = _ws_args(ws)
     _check(lib().moe_test_expert_stream(_p(x), _p(w_gate), _p(w_up), _p(w_down), T, d, E, I, k1,
-                                        _p(y), y_dtype, wsp, wsn, _stream(stream)),
+                                        k2, _p(y), y_dtype, wsp, wsn, _stream(stream)),
            "moe_test_expert_stream")
