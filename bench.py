@@ -69,8 +69,8 @@ def kernel_source_digest():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload, k1):
-    """ncu DRAM bytes per launch of the streaming kernel, if recorded for the
+def recorded_traffic(workload, k1, kernel):
+    """ncu DRAM bytes per launch of the dominant kernel, if recorded for the
     current kernel source (null once the source has changed)."""
     try:
         with open(TRAFFIC_PATH) as f:
@@ -79,7 +79,7 @@ def recorded_traffic(workload, k1):
         return None
     if rec.get("source_digest") != kernel_source_digest():
         return None
-    return rec.get("k_stream", {}).get("%s_k1_%d" % (workload, k1))
+    return rec.get(kernel, {}).get("%s_k1_%d" % (workload, k1))
 
 
 class ClockSampler:
@@ -191,16 +191,30 @@ def barrier(world):
 
 # ---------------------------------------------------------------------- model
 class Stack:
-    """L layers of seeded synthetic weights and per-layer tokens on the GPU."""
+    """L layers of seeded synthetic weights and per-layer tokens on the GPU.
+    For one-token workloads the down matrices are packed channel-major once,
+    at set-up (moe_pack_w_down; the original layout is then freed), and the
+    layers run the single-pass decode path."""
 
     def __init__(self, wl, seed, device):
-        from routed_expert_layer_route_b200 import synth
+        from routed_expert_layer_route_b200 import moe, synth
         self.wl = wl
         self.layers = []
+        self.channel_major = wl["T"] == 1
+        self.flags = moe.MOE_WDOWN_CHANNEL_MAJOR if self.channel_major else moe.MOE_PATH_AUTO
         for l in range(wl["layers"]):
-            self.layers.append(synth.make_layer(wl["T"], wl["d"], wl["E"], wl["I"], seed=seed,
-                                               layer=l, device=device, bias=wl["bias"]))
+            L = synth.make_layer(wl["T"], wl["d"], wl["E"], wl["I"], seed=seed, layer=l,
+                                 device=device, bias=wl["bias"])
+            if self.channel_major:
+                L.w_down = moe.moe_pack_w_down(L.w_down)
+            self.layers.append(L)
         torch.cuda.synchronize()
+
+    def down_hf(self, L, e):
+        """Expert e's down matrix in the [d x I] layout (host copy for the oracle)."""
+        from routed_expert_layer_route_b200 import synth
+        wd = L.w_down[e].t() if self.channel_major else L.w_down[e]
+        return synth.to_numpy(wd.contiguous())
 
 
 def build_graph(stack, k1, k2, ws_list, ys, stream):
@@ -211,12 +225,12 @@ def build_graph(stack, k1, k2, ws_list, ys, stream):
         # one eager pass first (module attribute set-up happens outside capture)
         for L, ws, y in zip(stack.layers, ws_list, ys):
             moe.moe_layer(L.x, L.w_router, L.bias, L.w_gate, L.w_up, L.w_down, k1, k2, y, ws,
-                          stream=stream)
+                          flags=stack.flags, stream=stream)
         stream.synchronize()
         with torch.cuda.graph(g, stream=stream):
             for L, ws, y in zip(stack.layers, ws_list, ys):
                 moe.moe_layer(L.x, L.w_router, L.bias, L.w_gate, L.w_up, L.w_down, k1, k2, y, ws,
-                              stream=stream)
+                              flags=stack.flags, stream=stream)
     return g
 
 
@@ -228,7 +242,7 @@ def unique_experts(stack, k1, k2, ws_list, ys, stream):
     for L, ws, y in zip(stack.layers, ws_list, ys):
         idx = torch.empty(wl["T"], k1, dtype=torch.int32, device=L.x.device)
         moe.moe_layer(L.x, L.w_router, L.bias, L.w_gate, L.w_up, L.w_down, k1, k2, y, ws,
-                      topk_idx_out=idx, stream=stream)
+                      topk_idx_out=idx, flags=stack.flags, stream=stream)
         stream.synchronize()
         us.append(int(torch.unique(idx).numel()))
     return us
@@ -247,7 +261,7 @@ def time_dominant_kernel(stack, k1, k2, ws_list, ys, stream, reps):
                 e = torch.cuda.Event(enable_timing=True)
                 s.record(stream)
                 moe.moe_test_expert_stream(L.x, L.w_gate, L.w_up, L.w_down, k1, k2, y, ws,
-                                           stream=stream)
+                                           flags=stack.flags, stream=stream)
                 e.record(stream)
                 starts.append(s)
                 ends.append(e)
@@ -272,7 +286,7 @@ def e2e_tokens_per_s(stack, k1, k2, ws_list, steps, warmup, stream):
         dev_x.copy_(host_x, non_blocking=True)
         for l, (L, ws) in enumerate(zip(stack.layers, ws_list)):
             moe.moe_layer(dev_x[l], L.w_router, L.bias, L.w_gate, L.w_up, L.w_down, k1, k2,
-                          dev_y[l], ws, stream=stream)
+                          dev_y[l], ws, flags=stack.flags, stream=stream)
         host_y.copy_(dev_y, non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -308,7 +322,7 @@ def cpu_oracle_rate(stack, k1, k2, budget_s=12.0):
         z = oracle.logits(x, wr, b)
         idx, _ = oracle.route_f32(z, k1, k2)
         experts = {int(e): (synth.to_numpy(L.w_gate[int(e)]), synth.to_numpy(L.w_up[int(e)]),
-                            synth.to_numpy(L.w_down[int(e)])) for e in np.unique(idx)}
+                            stack.down_hf(L, int(e))) for e in np.unique(idx)}
         prepared.append((x, wr, b, experts))
         if len(prepared) >= 6:
             break
@@ -408,10 +422,12 @@ def run_native(args, world, rank):
     U_head = results[0]["unique_experts_per_layer"]
     alg_bytes = U_head * 3 * d * I * 2
     achieved = alg_bytes / (kern_ms * 1e-3) / 1e9
-    traffic = recorded_traffic(args.workload, k1h)
+    kname = "k_decode" if stack.channel_major else "k_stream"
+    traffic = recorded_traffic(args.workload, k1h, kname)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
-                "kernel": "moe::k_stream", "kernel_us": round(kern_ms * 1000, 2),
+                "kernel": "moe::" + kname,
+                "kernel_us": round(kern_ms * 1000, 2),
                 "algorithmic_bytes_per_launch": int(alg_bytes),
                 "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
                 if peak_kind == "measured" else "fallback 6650 GB/s"}
@@ -436,7 +452,7 @@ def run_native(args, world, rank):
                "sample": "%d single-token layers of this workload (k1=%d, k2=%d) in %.1f s, "
                          "per-layer time scaled to the %d-layer stack" % (nl, k1h, k2h, el, Ln)}
 
-    per_step_launches = 2 if T == 1 else 3
+    per_step_launches = 3  # router, expert kernel, finalize (T == 1) / router, top-k, expert
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
@@ -449,6 +465,8 @@ def run_native(args, world, rank):
                    "l2": "inputs larger than L2: every step reads the routed experts of all "
                          "%d layers (%.2f GB) from HBM" % (Ln, alg_bytes * Ln / 1e9),
                    "timing": "CUDA graph of the %d-layer step, CUDA events, max over ranks" % Ln,
+                   "w_down_layout": "channel-major [E x I x d], packed once at set-up"
+                   if stack.channel_major else "[E x d x I]",
                    "parallelism": "replicas" if world > 1 else "single GPU"},
         "roofline": roofline,
         "cpu_baseline": cpu,

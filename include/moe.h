@@ -76,10 +76,18 @@ typedef enum {
 #define MOE_DTYPE_BF16 1
 
 /* moe_layer / moe_expert_ffn flags: which expert-FFN path runs.
- * AUTO picks by the expected number of tokens per activated expert. */
+ * AUTO picks by batch size and shapes. */
 #define MOE_PATH_AUTO 0
-#define MOE_PATH_STREAM 1  /* weight-streaming path (small batches)        */
-#define MOE_PATH_GROUPED 2 /* tcgen05 grouped GEMM path (large batches)    */
+#define MOE_PATH_STREAM 1  /* two-phase weight streaming, deterministic output        */
+#define MOE_PATH_GROUPED 2 /* tcgen05 grouped GEMM path (large batches)               */
+#define MOE_PATH_DECODE 3  /* one token: a single pass over the routed experts with the
+                              down matrix channel-major (needs MOE_WDOWN_CHANNEL_MAJOR);
+                              the float32 sum into y runs in a timing-dependent order,
+                              so y may differ between runs in the last bits           */
+#define MOE_PATH_MASK 0xff
+/* moe_layer flag bit: w_down points to the channel-major copy [E x I x d] made
+ * by moe_pack_w_down (down column c of expert e is then contiguous). */
+#define MOE_WDOWN_CHANNEL_MAJOR 0x100
 
 /* Human-readable text for a moe_status value.  Never NULL. */
 const char *moe_status_string(int status);
@@ -92,8 +100,9 @@ int moe_version(void);
  * Returns 0 when the shapes are invalid. */
 size_t moe_workspace_size(int T, int d, int E, int I, int k1);
 
-/* Zero the workspace's header (status word and the counters the kernels use
- * for cross-block hand-off).  Enqueued on `stream`. */
+/* Zero the workspace's header (status word and the counters and flags the
+ * kernels use for cross-block hand-off).  Enqueued on `stream`.  Call it once
+ * before the first use, and again after a call recorded MOE_ERR_TIMEOUT. */
 int moe_workspace_init(void *ws, size_t ws_bytes, void *stream);
 
 /* Copy the workspace's device status word into *status_out (MOE_OK or a
@@ -152,12 +161,26 @@ int moe_combine(const float *expert_out, const int32_t *slot_pos, const float *t
 /* The whole layer: router (as moe_route), permutation, expert FFN and
  * combine.  y [T x d] of y_dtype.  Optional outputs (each nullable):
  * topk_idx_out / topk_w_out [T x k1], logits_out [T x E] float32.
- * flags: MOE_PATH_*.  ws: workspace. */
+ * flags: MOE_PATH_* | MOE_WDOWN_CHANNEL_MAJOR.  With the HF down layout
+ * [E x d x I] the two-phase streaming path runs (deterministic).  With
+ * MOE_WDOWN_CHANNEL_MAJOR (w_down from moe_pack_w_down) and T == 1 the
+ * single-pass decode path runs; other T return MOE_ERR_UNSUPPORTED_SHAPE.
+ * ws: workspace. */
 int moe_layer(const void *x_bf16, const void *w_router_bf16, const float *bias,
               const void *w_gate_bf16, const void *w_up_bf16, const void *w_down_bf16, int T, int d,
               int E, int I, int k1, int k2, void *y, int y_dtype, int32_t *topk_idx_out,
               float *topk_w_out, float *logits_out, int flags, void *ws, size_t ws_bytes,
               void *stream);
+
+/* Channel-major copy of a down matrix, made once when the weights are
+ * loaded: w_down_cm[e][c][r] = w_down[e][r][c] (w_down [E x d x I] bf16 ->
+ * w_down_cm [E x I x d] bf16, separate buffers).  The channel decomposition
+ * of a routed expert ("Channel Selection for Mixture-of-Experts Decoding
+ * Needs No Calibration Data", section 2: channel c owns down column c) then
+ * reads each channel's down column as one contiguous row.  Enqueued on
+ * `stream`. */
+int moe_pack_w_down(const void *w_down_bf16, void *w_down_cm_bf16, int E, int d, int I,
+                    void *stream);
 
 /* moe_expert_ffn without a caller workspace.  The paper has no counterpart;
  * this entry exists for callers that cannot hand the library device memory
@@ -168,8 +191,8 @@ int moe_layer(const void *x_bf16, const void *w_router_bf16, const float *bias,
  *
  * Same inputs, output and result as moe_expert_ffn (flags are not taken: it
  * always uses the weight-streaming path).  Its scratch is a fixed array
- * compiled into libmoe.so (4 MiB per GPU that loads the library, held until
- * the process exits); the call itself allocates and frees nothing.
+ * compiled into libmoe.so (a little over 4 MiB per GPU that loads the library,
+ * held until the process exits); the call itself allocates and frees nothing.
  *  - Limit: T * k1 * I <= 1047424 (the float32 channel activations of all
  *    routed slots must fit the array), and the usual shape limits; larger
  *    shapes return MOE_ERR_SCRATCH_LIMIT and enqueue nothing.

@@ -22,16 +22,19 @@ int moe_test_exp_c(const float *x, float *y, int64_t n, void *stream);
  * device (0 if no device). */
 int moe_test_num_sms(void);
 
-/* Re-run only the expert-streaming kernel (expert FFN + combine into y) of
- * the last moe_layer call made with this workspace and these shapes, reusing
- * the logits (T == 1, where the kernel routes the token itself) or the
- * routing tables (T > 1) that call left in the workspace.  Launched without
- * programmatic dependent launch, so events recorded around it on `stream`
- * bracket this one kernel.  Used to time the dominant kernel alone.
+/* Re-run only the expert kernel of the last moe_layer call made with this
+ * workspace, these shapes and these flags, reusing the logits (T == 1, where
+ * the kernel routes the token itself) or the routing tables (T > 1) that call
+ * left in the workspace: the single-pass decode kernel when flags carry
+ * MOE_WDOWN_CHANNEL_MAJOR (its output accumulator is left as it ends; y is
+ * not written), else the two-phase streaming kernel (writes y).  Launched
+ * without programmatic dependent launch, so events recorded around it on
+ * `stream` bracket this one kernel.  Used to time the dominant kernel alone.
  * Arguments as for moe_layer.  Returns a moe_status. */
 int moe_test_expert_stream(const void *x_bf16, const void *w_gate_bf16, const void *w_up_bf16,
                            const void *w_down_bf16, int T, int d, int E, int I, int k1, int k2,
-                           void *y, int y_dtype, void *ws, size_t ws_bytes, void *stream);
+                           void *y, int y_dtype, int flags, void *ws, size_t ws_bytes,
+                           void *stream);
 
 #ifdef __cplusplus
 }

@@ -11,15 +11,17 @@
 #define MOE_DEVINL __device__ __forceinline__
 
 // ---------------------------------------------------------------------------
-// Workspace header: the first 256 bytes of every workspace.
+// Workspace header: the first 4 KiB of every workspace.
+constexpr int kMaxGridCtas = 960;  // most CTAs a grid barrier can serve
 struct WsHeader {
-    int status;              // device status word (moe_status), 0 = OK
-    unsigned route_arrive;   // last-block hand-off counter of the router kernel
-    unsigned bar_count;      // grid barrier of the streaming kernel: arrivals
-    unsigned bar_gen;        // grid barrier generation
-    unsigned pad[60];
+    int status;             // device status word (moe_status), 0 = OK
+    unsigned route_arrive;  // last-block hand-off counter of the top-k kernel
+    unsigned pad0[30];
+    unsigned bar_go;        // grid barrier: generation released so far (own 128-byte line)
+    unsigned pad1[31];
+    unsigned bar_flag[kMaxGridCtas];  // grid barrier: generation each CTA has reached
 };
-static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
+static_assert(sizeof(WsHeader) == 4096, "header is 4 KiB");
 
 // Bounded waits give up after this many nanoseconds (globaltimer) and record
 // MOE_ERR_TIMEOUT; no correct launch comes anywhere near it.
@@ -166,6 +168,48 @@ MOE_DEVINL unsigned ld_acquire_u32(const unsigned *p)
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+
+MOE_DEVINL unsigned ld_relaxed_u32(const unsigned *p)
+{
+    unsigned v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+MOE_DEVINL void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
+// Release store: a gpu-scope acq_rel fence, then a relaxed store.
+MOE_DEVINL void st_release_u32(unsigned *p, unsigned v)
+{
+    fence_acq_rel_gpu();
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Spin (bounded) on relaxed loads until *p == want, then one acq_rel fence
+// (acquire).  Records MOE_ERR_TIMEOUT and returns false when
+// MOE_WAIT_LIMIT_NS passes first.
+MOE_DEVINL bool wait_flag_eq(const unsigned *p, unsigned want, int *status)
+{
+    if (ld_relaxed_u32(p) != want) {
+        const uint64_t t0 = global_ns();
+        while (ld_relaxed_u32(p) != want) {
+            if (global_ns() - t0 > MOE_WAIT_LIMIT_NS) {
+                set_status(status, MOE_ERR_TIMEOUT);
+                return false;
+            }
+            __nanosleep(20);
+        }
+    }
+    fence_acq_rel_gpu();
+    return true;
+}
+
+// Balanced split of n items over G parts: part b gets [split_lo(n,G,b), split_lo(n,G,b+1)).
+MOE_DEVINL unsigned split_lo(unsigned n, unsigned G, unsigned b)
+{
+    const unsigned q = n / G, r = n % G;
+    return q * b + (b < r ? b : r);
 }
 
 MOE_DEVINL uint4 ld_nc_v4(const void *p)

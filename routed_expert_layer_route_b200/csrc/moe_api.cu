@@ -12,6 +12,7 @@
 #include "../../include/moe.h"
 #include "../../include/moe_testing.h"
 #include "combine.cuh"
+#include "decode.cuh"
 #include "route.cuh"
 #include "stream.cuh"
 
@@ -27,7 +28,8 @@ constexpr int kMaxT = 1 << 20;
 static inline size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct WsLayout {
-    size_t logits, idx, w, offsets, sorted_slot, slot_pos, uniq_count, uniq_list, h, out, total;
+    size_t logits, idx, w, offsets, sorted_slot, slot_pos, uniq_count, uniq_list, h, out, y_acc,
+        total;
 };
 
 static WsLayout ws_layout(int T, int d, int E, int I, int k1)
@@ -45,6 +47,7 @@ static WsLayout ws_layout(int T, int d, int E, int I, int k1)
     L.uniq_list = o;   o = align256(o + sizeof(int32_t) * (size_t)E);
     L.h = o;           o = align256(o + sizeof(float) * n * (size_t)I);
     L.out = o;         o = align256(o + sizeof(float) * n * (size_t)d);
+    L.y_acc = o;       o = align256(o + sizeof(float) * (size_t)T * d);
     L.total = o;
     return L;
 }
@@ -100,8 +103,20 @@ static int device_info(DevInfo *&out)
         if (cudaDeviceGetAttribute(&di.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return MOE_ERR_CUDA;
         const int stream_smem = (int)stream_smem_bytes();
-        if (cudaFuncSetAttribute(k_stream, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(k_stream<0, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 stream_smem) != cudaSuccess ||
+            cudaFuncSetAttribute(k_stream<8, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 stream_smem) != cudaSuccess ||
+            cudaFuncSetAttribute(k_stream<16, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  stream_smem) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        const int decode_smem = 227 * 1024;
+        if (cudaFuncSetAttribute(k_decode<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 decode_smem) != cudaSuccess ||
+            cudaFuncSetAttribute(k_decode<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 decode_smem) != cudaSuccess ||
+            cudaFuncSetAttribute(k_decode<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 decode_smem) != cudaSuccess)
             return MOE_ERR_CUDA;
         const int small = 96 * 1024;
         if (cudaFuncSetAttribute(k_logits, cudaFuncAttributeMaxDynamicSharedMemorySize, small) !=
@@ -148,7 +163,8 @@ static int topk_threads(int E)
 
 // logits for T tokens (no routing tail)
 static int enqueue_logits(const void *x, const void *wr, const float *bias, float *z, float *z_copy,
-                          int T, int d, int E, cudaStream_t s)
+                          int T, int d, int E, cudaStream_t s, float4 *zero = nullptr,
+                          int zero_n4 = 0)
 {
     LogitsArgs a = {};
     a.x = static_cast<const uint16_t *>(x);
@@ -159,9 +175,56 @@ static int enqueue_logits(const void *x, const void *wr, const float *bias, floa
     a.T = T;
     a.d = d;
     a.E = E;
+    a.zero = zero;
+    a.zero_n4 = zero_n4;
     const int items = E * ((T + kLogitsTok - 1) / kLogitsTok);
     const int grid = (items + kLogitsWarps - 1) / kLogitsWarps;
     return launch(k_logits, dim3(grid), dim3(kLogitsWarps * 32), 0, s, true, a);
+}
+
+// The single-pass decode path of moe_layer after the router (T == 1, down
+// matrix channel-major): the decode kernel (routing, gate/up, down partials
+// into y_acc) and the finalize kernel (y_acc -> y).  y_acc was cleared by the
+// router kernel.
+static int enqueue_decode(const void *x, const void *wg, const void *wu, const void *wdt, int d,
+                          int E, int I, int k1, int k2, void *y, int y_dtype, int32_t *idx_copy,
+                          float *w_copy, void *ws, int G, cudaStream_t s)
+{
+    const WsLayout L = ws_layout(1, d, E, I, k1);
+    DecodeArgs a = {};
+    a.x = static_cast<const uint16_t *>(x);
+    a.wg = static_cast<const uint16_t *>(wg);
+    a.wu = static_cast<const uint16_t *>(wu);
+    a.wdt = static_cast<const uint16_t *>(wdt);
+    a.d = d;
+    a.E = E;
+    a.I = I;
+    a.k1 = k1;
+    a.k2 = k2;
+    a.logits = at<float>(ws, L.logits);
+    a.topk_idx = at<int32_t>(ws, L.idx);
+    a.topk_w = at<float>(ws, L.w);
+    a.idx_copy = idx_copy;
+    a.w_copy = w_copy;
+    a.offsets = at<int32_t>(ws, L.offsets);
+    a.sorted_slot = at<int32_t>(ws, L.sorted_slot);
+    a.slot_pos = at<int32_t>(ws, L.slot_pos);
+    a.uniq_count = at<int32_t>(ws, L.uniq_count);
+    a.uniq_list = at<int32_t>(ws, L.uniq_list);
+    a.y_acc = at<float>(ws, L.y_acc);
+    a.hdr = static_cast<WsHeader *>(ws);
+    const size_t smem = decode_smem_bytes(d);
+    int rc;
+    if (d == 2048)
+        rc = launch(k_decode<8>, dim3(G), dim3(kSThreads), smem, s, true, a);
+    else if (d == 4096)
+        rc = launch(k_decode<16>, dim3(G), dim3(kSThreads), smem, s, true, a);
+    else
+        rc = launch(k_decode<0>, dim3(G), dim3(kSThreads), smem, s, true, a);
+    if (rc != MOE_OK)
+        return rc;
+    return launch(k_finalize, dim3((d / 4 + 255) / 256), dim3(256), 0, s, true,
+                  (const float *)at<float>(ws, L.y_acc), d, y, y_dtype);
 }
 
 }  // namespace moe
@@ -344,7 +407,18 @@ static int enqueue_stream(const StreamCall &c, cudaStream_t s, bool pdl = true)
     a.y = c.y;
     a.y_dtype = c.y_dtype;
     a.hdr = c.hdr;
-    return launch(k_stream, dim3(di->num_sms), dim3(kSThreads), stream_smem_bytes(), s, pdl, a);
+    const unsigned grid = (unsigned)(di->num_sms < kMaxGridCtas ? di->num_sms : kMaxGridCtas);
+    switch (stream_variant(c.T, c.d, c.I, c.k1)) {
+    case 1:
+        return launch(k_stream<8, 3>, dim3(grid), dim3(kSThreads), stream_smem_bytes(), s,
+                      pdl, a);
+    case 2:
+        return launch(k_stream<16, 4>, dim3(grid), dim3(kSThreads), stream_smem_bytes(), s,
+                      pdl, a);
+    default:
+        return launch(k_stream<0, 0>, dim3(grid), dim3(kSThreads), stream_smem_bytes(), s,
+                      pdl, a);
+    }
 }
 
 // The streaming call of a moe_layer on workspace ws (routing tables there).
@@ -460,7 +534,13 @@ int moe_layer(const void *x_bf16, const void *w_router_bf16, const float *bias,
         return rc;
     if ((rc = check_route(E, k1, k2)) != MOE_OK)
         return rc;
-    if (flags < MOE_PATH_AUTO || flags > MOE_PATH_GROUPED)
+    const int path = flags & MOE_PATH_MASK;
+    const bool down_cm = (flags & MOE_WDOWN_CHANNEL_MAJOR) != 0;
+    if (path > MOE_PATH_DECODE || (flags & ~(MOE_PATH_MASK | MOE_WDOWN_CHANNEL_MAJOR)))
+        return MOE_ERR_INVALID_ARG;
+    if (path == MOE_PATH_DECODE && !down_cm)
+        return MOE_ERR_INVALID_ARG;  // the decode kernel reads the channel-major down matrix
+    if (down_cm && path != MOE_PATH_AUTO && path != MOE_PATH_DECODE)
         return MOE_ERR_INVALID_ARG;
     if (y_dtype != MOE_DTYPE_F32 && y_dtype != MOE_DTYPE_BF16)
         return MOE_ERR_INVALID_ARG;
@@ -486,8 +566,17 @@ int moe_layer(const void *x_bf16, const void *w_router_bf16, const float *bias,
                   at<int32_t>(ws, L.slot_pos), at<int32_t>(ws, L.uniq_count),
                   at<int32_t>(ws, L.uniq_list)};
 
-    if ((rc = enqueue_logits(x_bf16, w_router_bf16, bias, z, logits_out, T, d, E, s)) != MOE_OK)
+    const int G = di->num_sms;
+    const bool decode = down_cm && decode_fits(T, d, E, I, k1, G);
+    if (down_cm && !decode)
+        return MOE_ERR_UNSUPPORTED_SHAPE;  // channel-major down matrix: one-token calls only
+    float4 *y_acc = decode ? at<float4>(ws, L.y_acc) : nullptr;
+    if ((rc = enqueue_logits(x_bf16, w_router_bf16, bias, z, logits_out, T, d, E, s, y_acc,
+                             T * d / 4)) != MOE_OK)
         return rc;
+    if (decode)
+        return enqueue_decode(x_bf16, w_gate_bf16, w_up_bf16, w_down_bf16, d, E, I, k1, k2, y,
+                              y_dtype, topk_idx_out, topk_w_out, ws, G, s);
     if (T > 1) {
         // one CTA per token ranks its probabilities; the last one to finish
         // builds the permutation tables
@@ -500,6 +589,19 @@ int moe_layer(const void *x_bf16, const void *w_router_bf16, const float *bias,
     return enqueue_stream(layer_stream_call(x_bf16, w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I,
                                             k1, k2, y, y_dtype, topk_idx_out, topk_w_out, ws),
                           s);
+}
+
+int moe_pack_w_down(const void *w_down_bf16, void *w_down_cm_bf16, int E, int d, int I,
+                    void *stream)
+{
+    if (E < 1 || E > kMaxE || d < kMinD || d > kMaxD || d % 64 || I < kMinI || I > kMaxI || I % 16)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!w_down_bf16 || !w_down_cm_bf16 || w_down_bf16 == w_down_cm_bf16)
+        return MOE_ERR_INVALID_ARG;
+    return launch(k_pack_w_down, dim3((I + 63) / 64, (d + 63) / 64, E), dim3(256), 0,
+                  static_cast<cudaStream_t>(stream), true,
+                  static_cast<const uint16_t *>(w_down_bf16), static_cast<uint16_t *>(w_down_cm_bf16),
+                  d, I);
 }
 
 int moe_test_exp_c(const float *x, float *y, int64_t n, void *stream)
@@ -517,7 +619,8 @@ int moe_test_exp_c(const float *x, float *y, int64_t n, void *stream)
 
 int moe_test_expert_stream(const void *x_bf16, const void *w_gate_bf16, const void *w_up_bf16,
                            const void *w_down_bf16, int T, int d, int E, int I, int k1, int k2,
-                           void *y, int y_dtype, void *ws, size_t ws_bytes, void *stream)
+                           void *y, int y_dtype, int flags, void *ws, size_t ws_bytes,
+                           void *stream)
 {
     int rc = check_shape(T, d, E, I, k1);
     if (rc != MOE_OK)
@@ -533,9 +636,43 @@ int moe_test_expert_stream(const void *x_bf16, const void *w_gate_bf16, const vo
     const WsLayout L = ws_layout(T, d, E, I, k1);
     if (ws_bytes < L.total)
         return MOE_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    DevInfo *di;
+    if ((rc = device_info(di)) != MOE_OK)
+        return rc;
+    if (flags & MOE_WDOWN_CHANNEL_MAJOR) {
+        if (!decode_fits(T, d, E, I, k1, di->num_sms))
+            return MOE_ERR_UNSUPPORTED_SHAPE;
+        DecodeArgs a = {};
+        a.x = static_cast<const uint16_t *>(x_bf16);
+        a.wg = static_cast<const uint16_t *>(w_gate_bf16);
+        a.wu = static_cast<const uint16_t *>(w_up_bf16);
+        a.wdt = static_cast<const uint16_t *>(w_down_bf16);
+        a.d = d;
+        a.E = E;
+        a.I = I;
+        a.k1 = k1;
+        a.k2 = k2;
+        a.logits = at<float>(ws, L.logits);
+        a.topk_idx = at<int32_t>(ws, L.idx);
+        a.topk_w = at<float>(ws, L.w);
+        a.offsets = at<int32_t>(ws, L.offsets);
+        a.sorted_slot = at<int32_t>(ws, L.sorted_slot);
+        a.slot_pos = at<int32_t>(ws, L.slot_pos);
+        a.uniq_count = at<int32_t>(ws, L.uniq_count);
+        a.uniq_list = at<int32_t>(ws, L.uniq_list);
+        a.y_acc = at<float>(ws, L.y_acc);
+        a.hdr = static_cast<WsHeader *>(ws);
+        const size_t smem = decode_smem_bytes(d);
+        if (d == 2048)
+            return launch(k_decode<8>, dim3(di->num_sms), dim3(kSThreads), smem, s, false, a);
+        if (d == 4096)
+            return launch(k_decode<16>, dim3(di->num_sms), dim3(kSThreads), smem, s, false, a);
+        return launch(k_decode<0>, dim3(di->num_sms), dim3(kSThreads), smem, s, false, a);
+    }
     return enqueue_stream(layer_stream_call(x_bf16, w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I,
                                             k1, k2, y, y_dtype, nullptr, nullptr, ws),
-                          static_cast<cudaStream_t>(stream), false);
+                          s, false);
 }
 
 int moe_test_num_sms(void)
@@ -551,13 +688,14 @@ int moe_test_num_sms(void)
 // ====================================================================== no-alloc
 // Scratch for moe_expert_ffn_noalloc: a fixed array in the library image, so
 // callers that cannot give the library device memory can still run the
-// expert FFN.  Layout: header (grid-barrier counters, status) | activated
+// expert FFN.  Layout: header (grid-barrier flags, status) | activated
 // expert count | activated expert list (E <= 1024) | float32 channel
 // activations of every routed slot [T*k1 x I].
 namespace moe {
-constexpr size_t kNoAllocBytes = 4u << 20;
-constexpr size_t kNoAllocHOffset = 256 + 256 + sizeof(int32_t) * 1024;
-constexpr size_t kNoAllocMaxH = (kNoAllocBytes - kNoAllocHOffset) / sizeof(float);  // 1047424
+constexpr size_t kNoAllocMaxH = 1047424;  // float32 channel activations that fit
+constexpr size_t kNoAllocUOffset = sizeof(WsHeader);
+constexpr size_t kNoAllocHOffset = kNoAllocUOffset + 256 + sizeof(int32_t) * 1024;
+constexpr size_t kNoAllocBytes = kNoAllocHOffset + sizeof(float) * kNoAllocMaxH;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
@@ -611,8 +749,8 @@ extern "C" int moe_expert_ffn_noalloc(const void *x_bf16, const int32_t *expert_
     // the grid-barrier counters and the status word must start at zero
     if (cudaMemsetAsync(scratch, 0, sizeof(WsHeader), s) != cudaSuccess)
         return MOE_ERR_CUDA;
-    int32_t *uniq_count = at<int32_t>(scratch, 256);
-    int32_t *uniq_list = at<int32_t>(scratch, 512);
+    int32_t *uniq_count = at<int32_t>(scratch, kNoAllocUOffset);
+    int32_t *uniq_list = at<int32_t>(scratch, kNoAllocUOffset + 256);
     float *h = at<float>(scratch, kNoAllocHOffset);
     if ((rc = launch(k_uniq_from_offsets, dim3(1), dim3(1024), 0, s, true, expert_offsets, E,
                      uniq_count, uniq_list)) != MOE_OK)

@@ -66,21 +66,22 @@ __global__ void k_test_expc(const float *x, float *y, int64_t n)
 }
 
 // ---------------------------------------------------------------------------
-// One CTA routes one token whose E logits sit in shared memory.
-// Shared scratch (caller-provided): ps[E], sel_p[E], sel_j[E], red[64].
+struct __align__(16) RouteSmem {
+    float ps[1024];    // e_j = expc(z_j - m)
+    float pp[1024];    // p_j = e_j / Z
+    float sel_p[1024]; // probabilities in rank order (ranks < Kneed)
+    int sel_j[1024];   // their expert ids
+    float red[64];
+    int out_j[32];     // the k1 selected experts, rank order
+    float out_w[32];   // their Eq. 2 weights
+};
+
+// One CTA routes one token whose E logits sit in shared memory (E <= 1024).
 // Leaves the k1 selected experts and weights in sm.out_j / sm.out_w and
 // writes them to idx_out / w_out and the optional copies (each pointer
 // nullable).  All threads of the CTA must call it; blockDim.x is a multiple
-// of 32 and at least 32 * 2.
-struct __align__(16) RouteSmem {
-    float ps[1024];
-    float sel_p[1024];
-    int sel_j[1024];
-    float red[64];
-    int out_j[32];    // the k1 selected experts, rank order
-    float out_w[32];  // their Eq. 2 weights
-};
-
+// of 32.  Five block barriers: the normaliser Z is formed by every warp
+// redundantly, in the same fixed order, so no barrier is needed after it.
 __device__ void route_token_block(const float *zs, int E, int k1, int k2, RouteSmem &sm,
                                   int32_t *idx_out, float *w_out, int32_t *idx_copy,
                                   float *w_copy)
@@ -99,51 +100,39 @@ __device__ void route_token_block(const float *zs, int E, int k1, int k2, RouteS
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if (lane == 0)
         sm.red[warp] = m;
-    __syncthreads();
-    if (warp == 0) {
-        float v = lane < nw ? sm.red[lane] : -__int_as_float(0x7f800000);
-        for (int o = 16; o >= 1; o >>= 1)
-            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-        if (lane == 0)
-            sm.red[32] = v;
-    }
-    __syncthreads();
-    m = sm.red[32];
+    __syncthreads();  // 1
+    m = sm.red[0];
+    for (int w = 1; w < nw; ++w)
+        m = fmaxf(m, sm.red[w]);
 
     for (int j = tid; j < E; j += nt)
         sm.ps[j] = expc(__fsub_rn(zs[j], m));
-    __syncthreads();
+    __syncthreads();  // 2
 
-    // Z in the canonical 32-partial order, then the butterfly
-    if (warp == 0) {
-        float acc = 0.0f;
-        for (int j = lane; j < E; j += 32)
-            acc = __fadd_rn(acc, sm.ps[j]);
-        for (int o = 16; o >= 1; o >>= 1)
-            acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o));
-        if (lane == 0)
-            sm.red[33] = acc;
-    }
-    __syncthreads();
-    const float Z = sm.red[33];
+    // Z in the canonical 32-partial order, then the butterfly (every warp)
+    float Z = 0.0f;
+    for (int j = lane; j < E; j += 32)
+        Z = __fadd_rn(Z, sm.ps[j]);
+    for (int o = 16; o >= 1; o >>= 1)
+        Z = __fadd_rn(Z, __shfl_xor_sync(0xffffffffu, Z, o));
     for (int j = tid; j < E; j += nt)
-        sm.ps[j] = __fdiv_rn(sm.ps[j], Z);
-    __syncthreads();
+        sm.pp[j] = __fdiv_rn(sm.ps[j], Z);
+    __syncthreads();  // 3
 
     // rank_j = #{i : p_i > p_j} + #{i < j : p_i == p_j}; keep rank < Kneed
     for (int j = tid; j < E; j += nt) {
-        const float pj = sm.ps[j];
+        const float pj = sm.pp[j];
         int r = 0;
         int i = 0;
         for (; i + 4 <= E; i += 4) {
-            const float4 v = *reinterpret_cast<const float4 *>(&sm.ps[i]);
+            const float4 v = *reinterpret_cast<const float4 *>(&sm.pp[i]);
             r += (v.x > pj) | ((v.x == pj) & (i + 0 < j));
             r += (v.y > pj) | ((v.y == pj) & (i + 1 < j));
             r += (v.z > pj) | ((v.z == pj) & (i + 2 < j));
             r += (v.w > pj) | ((v.w == pj) & (i + 3 < j));
         }
         for (; i < E; ++i) {
-            const float v = sm.ps[i];
+            const float v = sm.pp[i];
             r += (v > pj) | ((v == pj) & (i < j));
         }
         if (r < Kneed) {
@@ -151,20 +140,24 @@ __device__ void route_token_block(const float *zs, int E, int k1, int k2, RouteS
             sm.sel_j[r] = j;
         }
     }
-    __syncthreads();
-    if (renorm && tid == 0) {
+    __syncthreads();  // 4
+
+    // S = (((p_(0) + p_(1)) + ...) + p_(K-1)) in rank order; Eq. 2 weights
+    if (tid == 0) {
         float S = 0.0f;
-        for (int r = 0; r < K; ++r)
-            S = __fadd_rn(S, sm.sel_p[r]);
-        sm.red[34] = S;
+        if (renorm)
+            for (int r = 0; r < K; ++r)
+                S = __fadd_rn(S, sm.sel_p[r]);
+        for (int s = 0; s < k1; ++s) {
+            const float p = sm.sel_p[s];
+            sm.out_j[s] = sm.sel_j[s];
+            sm.out_w[s] = renorm ? __fdiv_rn(p, S) : p;
+        }
     }
-    __syncthreads();
+    __syncthreads();  // 5
     if (tid < k1) {
-        const float p = sm.sel_p[tid];
-        const int j = sm.sel_j[tid];
-        const float wv = renorm ? __fdiv_rn(p, sm.red[34]) : p;
-        sm.out_j[tid] = j;
-        sm.out_w[tid] = wv;
+        const int j = sm.out_j[tid];
+        const float wv = sm.out_w[tid];
         if (idx_out)
             idx_out[tid] = j;
         if (w_out)
@@ -420,6 +413,8 @@ struct LogitsArgs {
     float *z;       // [T x E] output (workspace or caller)
     float *z_copy;  // nullable second copy (caller's logits_out)
     int T, d, E;
+    float4 *zero;   // nullable: float4 buffer the grid clears (the layer's y accumulator)
+    int zero_n4;
 };
 
 __global__ void __launch_bounds__(kLogitsWarps * 32) k_logits(LogitsArgs a)
@@ -445,63 +440,50 @@ __global__ void __launch_bounds__(kLogitsWarps * 32) k_logits(LogitsArgs a)
     }
     pdl_wait();
     pdl_trigger();
+    if (a.zero) {
+        for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < a.zero_n4; i += gridDim.x * blockDim.x)
+            a.zero[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     if (!has_item)
         return;
 
     const uint4 *row = reinterpret_cast<const uint4 *>(a.wr + (size_t)e * a.d);
     const int t0 = chunk * kLogitsTok;
     const int nt = min(kLogitsTok, a.T - t0);
-    float acc[kLogitsTok];
+#pragma unroll 1
+    for (int t = 0; t < nt; ++t) {
+        const uint4 *xr = reinterpret_cast<const uint4 *>(a.x + (size_t)(t0 + t) * a.d);
+        float acc = 0.0f;
+        if (prefetch) {
+            // all x vectors of this lane first (independent loads), then the math
+            uint4 xv[kLogitsMaxVec];
 #pragma unroll
-    for (int t = 0; t < kLogitsTok; ++t)
-        acc[t] = 0.0f;
-    if (prefetch) {
-        // all x vectors of this lane first (independent loads), then the math
-        uint4 xv[kLogitsMaxVec];
+            for (int i = 0; i < kLogitsMaxVec; ++i) {
+                const int v = lane + 32 * i;
+                xv[i] = v < nvec ? xr[v] : make_uint4(0, 0, 0, 0);
+            }
 #pragma unroll
-        for (int t = 0; t < kLogitsTok; ++t) {
-            if (t < nt) {
-                const uint4 *xr = reinterpret_cast<const uint4 *>(a.x + (size_t)(t0 + t) * a.d);
-#pragma unroll
-                for (int i = 0; i < kLogitsMaxVec; ++i) {
-                    const int v = lane + 32 * i;
-                    xv[i] = v < nvec ? xr[v] : make_uint4(0, 0, 0, 0);
-                }
-#pragma unroll
-                for (int i = 0; i < kLogitsMaxVec; ++i) {
-                    float xf[8] = {bf16lo(xv[i].x), bf16hi(xv[i].x), bf16lo(xv[i].y),
-                                   bf16hi(xv[i].y), bf16lo(xv[i].z), bf16hi(xv[i].z),
-                                   bf16lo(xv[i].w), bf16hi(xv[i].w)};
-                    acc[t] = dot8_bf16(wv[i], xf, acc[t]);
-                }
+            for (int i = 0; i < kLogitsMaxVec; ++i) {
+                float xf[8] = {bf16lo(xv[i].x), bf16hi(xv[i].x), bf16lo(xv[i].y), bf16hi(xv[i].y),
+                               bf16lo(xv[i].z), bf16hi(xv[i].z), bf16lo(xv[i].w), bf16hi(xv[i].w)};
+                acc = dot8_bf16(wv[i], xf, acc);
+            }
+        } else {
+            for (int v = lane; v < nvec; v += 32) {
+                const uint4 wq = ld_nc_v4(row + v);
+                const uint4 xq = xr[v];
+                float xf[8] = {bf16lo(xq.x), bf16hi(xq.x), bf16lo(xq.y), bf16hi(xq.y),
+                               bf16lo(xq.z), bf16hi(xq.z), bf16lo(xq.w), bf16hi(xq.w)};
+                acc = dot8_bf16(wq, xf, acc);
             }
         }
-    } else {
-        for (int v = lane; v < nvec; v += 32) {
-            const uint4 wq = ld_nc_v4(row + v);
-#pragma unroll
-            for (int t = 0; t < kLogitsTok; ++t) {
-                if (t < nt) {
-                    const uint4 xq =
-                        *(reinterpret_cast<const uint4 *>(a.x + (size_t)(t0 + t) * a.d) + v);
-                    float xf[8] = {bf16lo(xq.x), bf16hi(xq.x), bf16lo(xq.y), bf16hi(xq.y),
-                                   bf16lo(xq.z), bf16hi(xq.z), bf16lo(xq.w), bf16hi(xq.w)};
-                    acc[t] = dot8_bf16(wq, xf, acc[t]);
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int t = 0; t < kLogitsTok; ++t) {
-        if (t < nt) {
-            float s = warp_sum(acc[t]);
-            if (lane == 0) {
-                if (a.bias)
-                    s = s + a.bias[e];
-                a.z[(size_t)(t0 + t) * a.E + e] = s;
-                if (a.z_copy)
-                    a.z_copy[(size_t)(t0 + t) * a.E + e] = s;
-            }
+        float sum = warp_sum(acc);
+        if (lane == 0) {
+            if (a.bias)
+                sum = sum + a.bias[e];
+            a.z[(size_t)(t0 + t) * a.E + e] = sum;
+            if (a.z_copy)
+                a.z_copy[(size_t)(t0 + t) * a.E + e] = sum;
         }
     }
 }

@@ -14,9 +14,9 @@
 //    round of independent loads, into shared memory, together with the
 //    tokens' x rows when they fit;
 //  * the U activated experts (ascending ids) are laid end to end as U*I
-//    channels; CTA b owns the contiguous channel range
-//    [b*U*I/G, (b+1)*U*I/G), so every CTA streams the same number of gate/up
-//    bytes (within one channel) whatever k1, U or the batch;
+//    channels; CTA b owns a contiguous channel range of floor(U*I/G) or one
+//    more channels, so every CTA streams the same number of gate/up bytes
+//    (within one channel) whatever k1, U or the batch;
 //  * one producer thread moves the CTA's weights with bulk asynchronous
 //    copies (cp.async.bulk, no multicast) into a ring of kStages shared-memory
 //    stages; stage s lands in slot s % kStages and is consumed by the
@@ -24,8 +24,10 @@
 //    (one channel = its gate row and up row; or one down row), so no stage
 //    needs a cross-warp reduction or barrier;
 //  * phase 1: gate/up rows of the CTA's channels -> h (float32) for them;
-//  * one grid-wide barrier (bounded spin) makes every h visible;
-//  * phase 2: CTA b owns the output rows [b*d/G, (b+1)*d/G) of every
+//  * one grid-wide barrier (bounded spins on per-CTA generation flags that
+//    CTA 0 gathers, then one release flag; no same-address atomics) makes
+//    every h visible;
+//  * phase 2: CTA b owns a contiguous range of about d/G output rows of every
 //    activated expert; its W_down rows (contiguous, I elements each) go
 //    through the same ring -- the producer issues them before the barrier
 //    completes, so the barrier hides under copies in flight;
@@ -90,9 +92,9 @@ struct Stage {
 };
 
 struct StageIter {
-    int64_t c_cur, c_hi;  // phase-1 channel cursor over [0, U*I)
-    int r_lo, r_hi;       // phase-2 rows of this CTA
-    int u2, r2;           // phase-2 cursor
+    unsigned c_cur, c_hi;  // phase-1 channel cursor over [0, U*I)
+    int r_lo, r_hi;        // phase-2 rows of this CTA
+    int u2, r2;            // phase-2 cursor
     int U, I, nch, nrows;
     int phase;
 
@@ -100,11 +102,11 @@ struct StageIter {
     {
         U = U_;
         I = I_;
-        const int64_t tot = (int64_t)U * I;
-        c_cur = tot * b / G;
-        c_hi = tot * (b + 1) / G;
-        r_lo = (int)((int64_t)d * b / G);
-        r_hi = (int)((int64_t)d * (b + 1) / G);
+        const unsigned tot = (unsigned)U * (unsigned)I;
+        c_cur = split_lo(tot, G, b);
+        c_hi = split_lo(tot, G, b + 1);
+        r_lo = (int)split_lo(d, G, b);
+        r_hi = (int)split_lo(d, G, b + 1);
         // channels per stage: a multiple of the warps serving a slot when the
         // stage holds that many, so each warp owns the same number of units
         nch = max(1, min(kMaxRows / 2, kStageBytes / (4 * d)));
@@ -123,10 +125,10 @@ struct StageIter {
         Stage s;
         if (phase == 1) {
             s.phase = 1;
-            s.u = (int)(c_cur / I);
-            s.c = (int)(c_cur % I);
-            int64_t lim = min((int64_t)(I - s.c), c_hi - c_cur);
-            s.n = (int)min((int64_t)nch, lim);
+            s.u = (int)(c_cur / (unsigned)I);
+            s.c = (int)(c_cur % (unsigned)I);
+            const unsigned lim = min((unsigned)(I - s.c), c_hi - c_cur);
+            s.n = (int)min((unsigned)nch, lim);
         } else {
             s.phase = 2;
             s.u = u2;
@@ -164,8 +166,8 @@ struct __align__(16) StreamSmem {
     int spos[kSlotMax];       // sorted position of each slot
     int U;
     int abort;
-    int issued;  // stages issued by the producer
-    int pad;
+    int issued;    // stages issued by the producer
+    unsigned gen;  // grid-barrier generation of this launch
 };
 
 __device__ __forceinline__ void consumer_sync() { named_bar_sync(kConsumerBar, kSC * 32); }
@@ -257,6 +259,89 @@ __device__ __forceinline__ void unit_down(const uint4 *wrow, const HRows hr, int
         o[t] = warp_sum(acc[t]);
 }
 
+// ---------------------------------------------------------------------------
+// Single-token fast path (T == 1, d = 256*VPL, I = 256*VPLI): lane l always
+// handles the 16-byte vectors l, l+32, ... of a row, so the token's x (phase
+// 1) and the expert's h (phase 2) stay in registers and each warp's units run
+// as long independent load/FMA streams with interleaved warp reductions.
+
+// x of the single token: in registers for d <= 2048, else read from shared
+// memory inside the loop (register budget).
+constexpr int kXRegMax = 8;
+
+// One channel: h = silu(W_gate[c,:] . x) * (W_up[c,:] . x), both rows at once.
+template <int VPL>
+__device__ __forceinline__ float fast_channel(const uint4 *grow, const uint4 *urow,
+                                              const uint4 (&xv)[VPL <= kXRegMax ? VPL : 1],
+                                              const uint4 *xs, int lane)
+{
+    float g0 = 0.f, g1 = 0.f, u0 = 0.f, u1 = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+        const uint4 wg = grow[lane + 32 * i];
+        const uint4 wu = urow[lane + 32 * i];
+        float xf[8], fg[8], fu[8];
+        if constexpr (VPL <= kXRegMax)
+            bf16x8(xv[i], xf);
+        else
+            bf16x8(xs[lane + 32 * i], xf);
+        bf16x8(wg, fg);
+        bf16x8(wu, fu);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            if (i & 1) {
+                g1 = fmaf(fg[k], xf[k], g1);
+                u1 = fmaf(fu[k], xf[k], u1);
+            } else {
+                g0 = fmaf(fg[k], xf[k], g0);
+                u0 = fmaf(fu[k], xf[k], u0);
+            }
+        }
+    }
+    float g = g0 + g1, u = u0 + u1;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        g += __shfl_xor_sync(0xffffffffu, g, o);
+        u += __shfl_xor_sync(0xffffffffu, u, o);
+    }
+    return silu_mul(g, u);
+}
+
+// Up to four down rows of one warp at once: o_r = W_down[row_r,:] . h.
+template <int VPLI>
+__device__ __forceinline__ void fast_rows(const uint8_t *stg, int I, int u0, int n,
+                                          const float (&hv)[VPLI][8], int lane, float (&o)[4])
+{
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+        o[r] = 0.f;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int unit = u0 + r * kWPS;
+        if (unit < n) {
+            const uint4 *wrow = reinterpret_cast<const uint4 *>(stg + (size_t)unit * I * 2);
+#pragma unroll
+            for (int i = 0; i < VPLI; ++i) {
+                float fw[8];
+                bf16x8(wrow[lane + 32 * i], fw);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    o[r] = fmaf(fw[k], hv[i][k], o[r]);
+            }
+        }
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+            o[r] += __shfl_xor_sync(0xffffffffu, o[r], off);
+    }
+}
+
+// The streaming kernel.  VPL/VPLI > 0 selects the single-token fast path for
+// d = 256*VPL and I = 256*VPLI (x and h held in registers); VPL = VPLI = 0 is
+// the general path (any T, d, I).
+template <int VPL, int VPLI>
 __global__ void __launch_bounds__(kSThreads, 1) k_stream(StreamArgs a)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -288,6 +373,8 @@ __global__ void __launch_bounds__(kSThreads, 1) k_stream(StreamArgs a)
 
     pdl_wait();
     pdl_trigger();
+    if (tid == 0)
+        ss->gen = ld_relaxed_u32(&a.hdr->bar_go);  // cannot advance before this CTA arrives
 
     // ------------------------------------------------------------ routing state
     // the tokens' x rows (independent of routing) go out in the same round
@@ -307,7 +394,6 @@ __global__ void __launch_bounds__(kSThreads, 1) k_stream(StreamArgs a)
         route_token_block(zs, E, k1, a.k2, rs, b == 0 ? a.topk_idx : nullptr,
                           b == 0 ? a.topk_w : nullptr, b == 0 ? a.idx_copy : nullptr,
                           b == 0 ? a.w_copy : nullptr);
-        __syncthreads();
         if (tid < k1) {
             const int e = rs.out_j[tid];
             int p = 0;
@@ -392,7 +478,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_stream(StreamArgs a)
         __syncthreads();
     }
     const int U = ss->U;
-    const int r_lo = (int)((int64_t)d * b / G), r_hi = (int)((int64_t)d * (b + 1) / G);
+    const int r_lo = (int)split_lo(d, G, b), r_hi = (int)split_lo(d, G, b + 1);
     const int nr = r_hi - r_lo;
     const bool obuf_ok = a.y && (size_t)nslots * nr <= (size_t)kObufFloats;
 
@@ -443,8 +529,27 @@ __global__ void __launch_bounds__(kSThreads, 1) k_stream(StreamArgs a)
         StageIter it;
         it.init(U, I, d, b, G);
         int sidx = 0;  // global stage index
-        bool arrived = false;
 
+        // Wait for stage sidx if this warp serves its slot; returns the stage
+        // buffer, or nullptr when this warp skips the stage (not its slot) or
+        // the launch aborted.  Every served stage is handed back with release().
+        auto acquire = [&](bool &mine) -> const uint8_t * {
+            mine = (sidx % kStages) == group;
+            if (!mine)
+                return nullptr;
+            const uint32_t parity = (uint32_t)((sidx / kStages) & 1);
+            const bool ok = !*(volatile int *)&ss->abort && mbar_wait(&full[group], parity, status);
+            if (!ok) {
+                ss->abort = 1;
+                return nullptr;
+            }
+            return ring + (size_t)group * kStageBytes;
+        };
+        auto release = [&]() {
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&empty[group]);
+        };
         auto x_row = [&](int p) -> const uint4 * {
             int t;
             if (slots_in_smem) {
@@ -463,67 +568,34 @@ __global__ void __launch_bounds__(kSThreads, 1) k_stream(StreamArgs a)
                              : reinterpret_cast<const float4 *>(a.h + (size_t)p * I);
         };
 
-        while (true) {
-            const bool have = it.valid();
-            const Stage st = have ? it.get() : Stage{0, 0, 0, 0};
-            if (!arrived && (!have || st.phase == 2)) {
-                // grid barrier: every CTA's h is written before any is read
-                __threadfence();
-                consumer_sync();
-                if (tid == 0) {
-                    const unsigned gen0 = ld_acquire_u32(&a.hdr->bar_gen);
-                    // read before this CTA arrives, so it cannot have advanced yet
-                    __threadfence();
-                    const unsigned prev = atomicAdd(&a.hdr->bar_count, 1u);
-                    if (prev == (unsigned)G - 1) {
-                        atomicExch(&a.hdr->bar_count, 0u);
-                        __threadfence();
-                        atomicAdd(&a.hdr->bar_gen, 1u);
-                    } else {
-                        const uint64_t t0 = global_ns();
-                        while (ld_acquire_u32(&a.hdr->bar_gen) == gen0) {
-                            if (global_ns() - t0 > MOE_WAIT_LIMIT_NS) {
-                                set_status(status, MOE_ERR_TIMEOUT);
-                                ss->abort = 1;
-                                break;
-                            }
-                        }
-                    }
-                    __threadfence();
-                }
-                consumer_sync();
-                if (h_in_smem && have) {
-                    const int n4 = nslots * (I >> 2);
-                    for (int i = tid; i < n4; i += kSC * 32)
-                        reinterpret_cast<float4 *>(area)[i] =
-                            __ldcg(reinterpret_cast<const float4 *>(a.h) + i);
-                    consumer_sync();
-                }
-                arrived = true;
+        // ---------------------------------------------------- phase 1: h
+        {
+            uint4 xv[VPL > 0 && VPL <= kXRegMax ? VPL : 1];
+            const uint4 *xs = reinterpret_cast<const uint4 *>(area);
+            if constexpr (VPL > 0 && VPL <= kXRegMax) {
+#pragma unroll
+                for (int i = 0; i < VPL; ++i)
+                    xv[i] = xs[lane + 32 * i];
             }
-            if (!have)
-                break;
-
-            if (sidx % kStages == group) {
-                const int slot = group;
-                const uint32_t parity = (uint32_t)((sidx / kStages) & 1);
-                const bool ok =
-                    !*(volatile int *)&ss->abort && mbar_wait(&full[slot], parity, status);
-                if (!ok)
-                    ss->abort = 1;
-                if (ok) {
+            while (it.valid() && it.phase == 1) {
+                const Stage st = it.get();
+                bool mine;
+                const uint8_t *stg = acquire(mine);
+                if (stg) {
                     const int p0 = ss->up0[st.u];
                     const int M = ss->uM[st.u];
-                    const uint8_t *stg = ring + (size_t)slot * kStageBytes;
                     for (int unit = gl; unit < st.n; unit += kWPS) {
-                        for (int m0 = 0; m0 < M; m0 += kTokChunk) {
-                            const int mt = min(kTokChunk, M - m0);
-                            float r0[kTokChunk], r1[kTokChunk];
-                            if (st.phase == 1) {
-                                const uint4 *grow =
-                                    reinterpret_cast<const uint4 *>(stg + (size_t)unit * d * 2);
-                                const uint4 *urow = reinterpret_cast<const uint4 *>(
-                                    stg + (size_t)(st.n + unit) * d * 2);
+                        const uint4 *grow = reinterpret_cast<const uint4 *>(stg + (size_t)unit * d * 2);
+                        const uint4 *urow =
+                            reinterpret_cast<const uint4 *>(stg + (size_t)(st.n + unit) * d * 2);
+                        if constexpr (VPL > 0) {
+                            const float hval = fast_channel<VPL>(grow, urow, xv, xs, lane);
+                            if (lane == 0)
+                                a.h[(size_t)p0 * I + st.c + unit] = hval;
+                        } else {
+                            for (int m0 = 0; m0 < M; m0 += kTokChunk) {
+                                const int mt = min(kTokChunk, M - m0);
+                                float r0[kTokChunk], r1[kTokChunk];
                                 XRows xr;
 #pragma unroll
                                 for (int t = 0; t < kTokChunk; ++t)
@@ -540,9 +612,95 @@ __global__ void __launch_bounds__(kSThreads, 1) k_stream(StreamArgs a)
                                     if (lane == t && t < mt)
                                         a.h[(size_t)(p0 + m0 + t) * I + st.c + unit] =
                                             silu_mul(r0[t], r1[t]);
-                            } else {
-                                const uint4 *wrow =
-                                    reinterpret_cast<const uint4 *>(stg + (size_t)unit * I * 2);
+                            }
+                        }
+                    }
+                }
+                if (mine)
+                    release();
+                ++sidx;
+                it.next();
+            }
+        }
+
+        // ---------------------------------------------------- grid barrier
+        // every CTA's h is written before any is read
+        consumer_sync();
+        {
+            const unsigned target = ss->gen + 1u;
+            if (tid == 0)
+                st_release_u32(&a.hdr->bar_flag[b], target);
+            if (b == 0) {
+                // CTA 0 gathers every CTA's arrival flag, then releases all
+                for (int i = tid; i < G; i += kSC * 32)
+                    if (!wait_flag_eq(&a.hdr->bar_flag[i], target, status))
+                        ss->abort = 1;
+                consumer_sync();
+                if (tid == 0)
+                    st_release_u32(&a.hdr->bar_go, target);
+            }
+            if (tid == 0 && !wait_flag_eq(&a.hdr->bar_go, target, status))
+                ss->abort = 1;
+        }
+        consumer_sync();
+        if (h_in_smem && it.valid()) {
+            const int n4 = nslots * (I >> 2);
+            for (int i = tid; i < n4; i += kSC * 32)
+                reinterpret_cast<float4 *>(area)[i] = __ldcg(reinterpret_cast<const float4 *>(a.h) + i);
+            consumer_sync();
+        }
+
+        // ---------------------------------------------------- phase 2: o
+        {
+            float hv[VPLI > 0 ? VPLI : 1][8];
+            int hv_pos = -1;
+            while (it.valid()) {
+                const Stage st = it.get();
+                bool mine;
+                const uint8_t *stg = acquire(mine);
+                if (stg) {
+                    const int p0 = ss->up0[st.u];
+                    const int M = ss->uM[st.u];
+                    if constexpr (VPLI > 0) {
+                        if (hv_pos != p0) {  // this expert's h into registers
+                            const float4 *hs = reinterpret_cast<const float4 *>(area + (size_t)p0 * I * 4);
+#pragma unroll
+                            for (int i = 0; i < VPLI; ++i) {
+                                const float4 q0 = hs[2 * (lane + 32 * i)];
+                                const float4 q1 = hs[2 * (lane + 32 * i) + 1];
+                                hv[i][0] = q0.x;
+                                hv[i][1] = q0.y;
+                                hv[i][2] = q0.z;
+                                hv[i][3] = q0.w;
+                                hv[i][4] = q1.x;
+                                hv[i][5] = q1.y;
+                                hv[i][6] = q1.z;
+                                hv[i][7] = q1.w;
+                            }
+                            hv_pos = p0;
+                        }
+                        for (int u0 = gl; u0 < st.n; u0 += 4 * kWPS) {
+                            float o[4];
+                            fast_rows<VPLI>(stg, I, u0, st.n, hv, lane, o);
+#pragma unroll
+                            for (int r = 0; r < 4; ++r) {
+                                const int unit = u0 + r * kWPS;
+                                if (lane == r && unit < st.n) {
+                                    const int row = st.c + unit;
+                                    if (obuf_ok)
+                                        ss->obuf[p0 * nr + (row - r_lo)] = o[r];
+                                    else
+                                        a.out[(size_t)p0 * d + row] = o[r];
+                                }
+                            }
+                        }
+                    } else {
+                        for (int unit = gl; unit < st.n; unit += kWPS) {
+                            const uint4 *wrow = reinterpret_cast<const uint4 *>(stg + (size_t)unit * I * 2);
+                            const int row = st.c + unit;
+                            for (int m0 = 0; m0 < M; m0 += kTokChunk) {
+                                const int mt = min(kTokChunk, M - m0);
+                                float r0[kTokChunk];
                                 HRows hr;
 #pragma unroll
                                 for (int t = 0; t < kTokChunk; ++t)
@@ -554,7 +712,6 @@ __global__ void __launch_bounds__(kSThreads, 1) k_stream(StreamArgs a)
                                     unit_down<2>(wrow, hr, nvec, lane, r0);
                                 else
                                     unit_down<4>(wrow, hr, nvec, lane, r0);
-                                const int row = st.c + unit;
 #pragma unroll
                                 for (int t = 0; t < kTokChunk; ++t) {
                                     if (lane == t && t < mt) {
@@ -569,13 +726,11 @@ __global__ void __launch_bounds__(kSThreads, 1) k_stream(StreamArgs a)
                         }
                     }
                 }
-                // this warp is done with the stage's weights: hand the slot back
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&empty[slot]);
+                if (mine)
+                    release();
+                ++sidx;
+                it.next();
             }
-            ++sidx;
-            it.next();
         }
 
         // ------------------------------------------------------------ combine
@@ -599,8 +754,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_stream(StreamArgs a)
                             continue;
                         }
                     }
-                    const float o = obuf_ok ? ss->obuf[pos * nr + (r - r_lo)]
-                                            : a.out[(size_t)pos * d + r];
+                    const float o = obuf_ok ? ss->obuf[pos * nr + (r - r_lo)] : a.out[(size_t)pos * d + r];
                     const float prod = w * o;
                     acc = acc + prod;
                 }
@@ -623,6 +777,19 @@ __global__ void __launch_bounds__(kSThreads, 1) k_stream(StreamArgs a)
             mbar_wait(&full[s], parity, status);
         }
     }
+}
+
+// Which instantiation serves these shapes: the single-token fast path when x
+// and every routed slot's h fit the shared-memory staging area.
+inline int stream_variant(int T, int d, int I, int k1)
+{
+    if (T != 1 || (size_t)d * 2 > (size_t)kAreaBytes || (size_t)k1 * I * 4 > (size_t)kAreaBytes)
+        return 0;
+    if (d == 2048 && I == 768)
+        return 1;
+    if (d == 4096 && I == 1024)
+        return 2;
+    return 0;
 }
 
 inline size_t stream_smem_bytes()

@@ -29,6 +29,9 @@ MOE_DTYPE_BF16 = 1
 MOE_PATH_AUTO = 0
 MOE_PATH_STREAM = 1
 MOE_PATH_GROUPED = 2
+MOE_PATH_DECODE = 3
+MOE_PATH_MASK = 0xFF
+MOE_WDOWN_CHANNEL_MAJOR = 0x100
 
 # every symbol include/*.h declares, with (restype, argtypes)
 _vp = ctypes.c_void_p
@@ -48,9 +51,10 @@ SIGNATURES = {
     "moe_layer": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp,
                        _vp, _i, _vp, _sz, _vp]),
     "moe_expert_ffn_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
+    "moe_pack_w_down": (_i, [_vp, _vp, _i, _i, _i, _vp]),
     "moe_test_exp_c": (_i, [_vp, _vp, ctypes.c_int64, _vp]),
     "moe_test_num_sms": (_i, []),
-    "moe_test_expert_stream": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _vp,
+    "moe_test_expert_stream": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _i, _vp,
                                     _sz, _vp]),
 }
 
@@ -184,6 +188,16 @@ def moe_expert_ffn_noalloc(x, expert_offsets, sorted_slot, w_gate, w_up, w_down,
                                         _stream(stream)), "moe_expert_ffn_noalloc")
 
 
+def moe_pack_w_down(w_down, w_down_cm=None, stream=None):
+    """Channel-major copy [E x I x d] of a down matrix [E x d x I] (bf16)."""
+    E, d, I = w_down.shape
+    if w_down_cm is None:
+        w_down_cm = torch.empty((E, I, d), dtype=w_down.dtype, device=w_down.device)
+    _check(lib().moe_pack_w_down(_p(w_down), _p(w_down_cm), E, d, I, _stream(stream)),
+           "moe_pack_w_down")
+    return w_down_cm
+
+
 def moe_combine(expert_out, slot_pos, topk_w, y, stream=None):
     T, k1 = topk_w.shape
     d = y.shape[1]
@@ -194,6 +208,8 @@ def moe_combine(expert_out, slot_pos, topk_w, y, stream=None):
 
 def moe_layer(x, w_router, bias, w_gate, w_up, w_down, k1, k2, y, ws, topk_idx_out=None,
               topk_w_out=None, logits_out=None, flags=MOE_PATH_AUTO, stream=None):
+    """w_down: [E x d x I], or the channel-major [E x I x d] copy from
+    moe_pack_w_down together with flags | MOE_WDOWN_CHANNEL_MAJOR."""
     T, d = x.shape
     E, I, _ = w_gate.shape
     y_dtype = MOE_DTYPE_BF16 if y.dtype == torch.bfloat16 else MOE_DTYPE_F32
@@ -211,11 +227,12 @@ def moe_test_num_sms():
     return lib().moe_test_num_sms()
 
 
-def moe_test_expert_stream(x, w_gate, w_up, w_down, k1, k2, y, ws, stream=None):
+def moe_test_expert_stream(x, w_gate, w_up, w_down, k1, k2, y, ws, flags=MOE_PATH_AUTO,
+                           stream=None):
     T, d = x.shape
     E, I, _ = w_gate.shape
     y_dtype = MOE_DTYPE_BF16 if y.dtype == torch.bfloat16 else MOE_DTYPE_F32
     wsp, wsn = _ws_args(ws)
     _check(lib().moe_test_expert_stream(_p(x), _p(w_gate), _p(w_up), _p(w_down), T, d, E, I, k1,
-                                        k2, _p(y), y_dtype, wsp, wsn, _stream(stream)),
+                                        k2, _p(y), y_dtype, flags, wsp, wsn, _stream(stream)),
            "moe_test_expert_stream")

@@ -34,7 +34,9 @@ def logits_bound(x, w):
     return 1e-4 * np.sqrt(d) * float(x.abs().max()) * float(w.abs().max())
 
 
-def run_layer(L, k1, k2, y_dtype=torch.float32, flags=moe.MOE_PATH_AUTO, ws=None):
+def run_layer(L, k1, k2, y_dtype=torch.float32, flags=moe.MOE_PATH_AUTO, ws=None, w_down=None):
+    """moe_layer on the GPU; w_down overrides L.w_down (e.g. the channel-major
+    copy, with flags | MOE_WDOWN_CHANNEL_MAJOR)."""
     T, d = L.x.shape
     E, I, _ = L.w_gate.shape
     dev = L.x.device
@@ -44,7 +46,8 @@ def run_layer(L, k1, k2, y_dtype=torch.float32, flags=moe.MOE_PATH_AUTO, ws=None
     idx = torch.empty(T, k1, device=dev, dtype=torch.int32)
     w = torch.empty(T, k1, device=dev, dtype=torch.float32)
     z = torch.empty(T, E, device=dev, dtype=torch.float32)
-    moe.moe_layer(L.x, L.w_router, L.bias, L.w_gate, L.w_up, L.w_down, k1, k2, y, ws,
+    moe.moe_layer(L.x, L.w_router, L.bias, L.w_gate, L.w_up,
+                  L.w_down if w_down is None else w_down, k1, k2, y, ws,
                   topk_idx_out=idx, topk_w_out=w, logits_out=z, flags=flags)
     torch.cuda.synchronize()
     status = moe.moe_read_device_status(ws)
@@ -52,9 +55,9 @@ def run_layer(L, k1, k2, y_dtype=torch.float32, flags=moe.MOE_PATH_AUTO, ws=None
     return y, idx, w, z
 
 
-def check_layer_full(L, k1, k2, flags=moe.MOE_PATH_AUTO, tight=True):
+def check_layer_full(L, k1, k2, flags=moe.MOE_PATH_AUTO, tight=True, w_down=None):
     """Whole-layer parity against oracle.layer (all tokens, all weights on host)."""
-    y, idx, w, z = run_layer(L, k1, k2, flags=flags)
+    y, idx, w, z = run_layer(L, k1, k2, flags=flags, w_down=w_down)
     zn = z.cpu().numpy()
     # logits against the oracle's own
     z_or = oracle.logits(synth.to_numpy(L.x), synth.to_numpy(L.w_router), synth.to_numpy(L.bias))
@@ -72,10 +75,10 @@ def check_layer_full(L, k1, k2, flags=moe.MOE_PATH_AUTO, tight=True):
     return yy, ref
 
 
-def check_layer_sampled(L, k1, k2, tokens, flags=moe.MOE_PATH_AUTO):
+def check_layer_sampled(L, k1, k2, tokens, flags=moe.MOE_PATH_AUTO, w_down=None):
     """Parity on sampled tokens; expert weights are fetched to the host only
     for the experts those tokens use."""
-    y, idx, w, z = run_layer(L, k1, k2, flags=flags)
+    y, idx, w, z = run_layer(L, k1, k2, flags=flags, w_down=w_down)
     tokens = np.asarray(tokens)
     zn = z.cpu().numpy()[tokens]
     xs = synth.to_numpy(L.x[torch.as_tensor(tokens, device=L.x.device)])

@@ -79,6 +79,9 @@ def test_layer_argument_checks(L):
     assert layer(L, ptr=FAKE + 8) == moe.MOE_ERR_INVALID_ARG          # misaligned tensor
     assert layer(L, y_dtype=7) == moe.MOE_ERR_INVALID_ARG
     assert layer(L, flags=9) == moe.MOE_ERR_INVALID_ARG
+    assert layer(L, flags=moe.MOE_PATH_DECODE) == moe.MOE_ERR_INVALID_ARG        # needs channel-major
+    assert layer(L, flags=moe.MOE_PATH_STREAM | moe.MOE_WDOWN_CHANNEL_MAJOR) == moe.MOE_ERR_INVALID_ARG
+    assert layer(L, flags=0x200) == moe.MOE_ERR_INVALID_ARG
     assert layer(L, ws_bytes=1024) == moe.MOE_ERR_WORKSPACE_TOO_SMALL
     assert layer(L, T=0) == moe.MOE_OK                                 # no-op, nothing enqueued
     assert layer(L, T=0, k2=9) == moe.MOE_OK                           # k2 > E-independent, valid
@@ -99,6 +102,8 @@ def test_other_calls_argument_checks(L):
     assert L.moe_combine(FAKE, FAKE, FAKE, 4, 2048, 8, FAKE, 3, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_combine(FAKE, FAKE, FAKE, 4, 100, 8, FAKE, 1, None) == moe.MOE_ERR_UNSUPPORTED_SHAPE
     assert L.moe_workspace_init(None, 4096, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_pack_w_down(FAKE, FAKE, 4, 100, 32, None) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert L.moe_pack_w_down(FAKE, FAKE, 4, 128, 32, None) == moe.MOE_ERR_INVALID_ARG  # in place
     v = ctypes.c_int(0)
     assert L.moe_read_device_status(None, ctypes.byref(v), None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_test_exp_c(None, None, 0, None) == moe.MOE_OK

@@ -41,27 +41,75 @@ SMALL = [
 ]
 
 
+CM = moe.MOE_WDOWN_CHANNEL_MAJOR
+
+
 @pytest.mark.parametrize("T,d,E,I,k1,k2,bias", SMALL)
 def test_layer_small_all_tokens(T, d, E, I, k1, k2, bias):
     L = synth.make_layer(T, d, E, I, seed=T + d + E, device=DEV, bias=bias)
     check_layer_full(L, k1, k2)
+    if T == 1:  # the single-pass decode path on the channel-major down matrix
+        wdc = moe.moe_pack_w_down(L.w_down)
+        check_layer_full(L, k1, k2, flags=CM, w_down=wdc)
+        check_layer_full(L, k1, k2, flags=moe.MOE_PATH_DECODE | CM, w_down=wdc)
 
 
-def test_layer_bf16_output_is_rounded_f32_output():
-    L = synth.make_layer(9, 512, 32, 64, seed=2, device=DEV)
-    y32, *_ = run_layer(L, 4, 8, y_dtype=torch.float32)
-    y16, *_ = run_layer(L, 4, 8, y_dtype=torch.bfloat16)
-    assert torch.equal(y32.to(torch.bfloat16), y16)
+@pytest.mark.parametrize("E,d,I", [(16, 64, 32), (3, 2048, 768), (2, 320, 112), (1, 4096, 1024)])
+def test_pack_w_down_is_the_transpose(E, d, I):
+    wd = synth.normal((E, d, I), 1.0, synth.make_generator(DEV, 5), DEV, torch.bfloat16)
+    wdc = moe.moe_pack_w_down(wd)
+    torch.cuda.synchronize()
+    assert torch.equal(wdc, wd.transpose(1, 2).contiguous())
+
+
+@pytest.mark.parametrize("d,E,I,k1,k2", [(64, 16, 32, 2, 4), (256, 64, 96, 8, 16),
+                                          (1024, 40, 112, 6, 1000), (192, 20, 32, 20, 20),
+                                          (512, 128, 256, 32, 64)])
+def test_decode_path_single_token(d, E, I, k1, k2):
+    L = synth.make_layer(1, d, E, I, seed=d + E + k1, device=DEV, bias="normal")
+    wdc = moe.moe_pack_w_down(L.w_down)
+    check_layer_full(L, k1, k2, flags=CM, w_down=wdc)
+
+
+def test_channel_major_down_needs_one_token():
+    L = synth.make_layer(2, 256, 16, 32, seed=7, device=DEV)
+    wdc = moe.moe_pack_w_down(L.w_down)
+    with pytest.raises(moe.MoeError) as ei:
+        run_layer(L, 2, 4, flags=CM, w_down=wdc)
+    assert ei.value.status == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    with pytest.raises(moe.MoeError) as ei:  # the decode path needs the channel-major matrix
+        run_layer(L, 2, 4, flags=moe.MOE_PATH_DECODE)
+    assert ei.value.status == moe.MOE_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("packed", [False, True], ids=["stream", "decode"])
+def test_layer_bf16_output_is_rounded_f32_output(packed):
+    T = 1 if packed else 9
+    L = synth.make_layer(T, 512, 32, 64, seed=2, device=DEV)
+    kw = dict(flags=CM, w_down=moe.moe_pack_w_down(L.w_down)) if packed else {}
+    y32, *_ = run_layer(L, 4, 8, y_dtype=torch.float32, **kw)
+    y16, *_ = run_layer(L, 4, 8, y_dtype=torch.bfloat16, **kw)
+    if not packed:  # deterministic path: exactly the rounded float32 output
+        assert torch.equal(y32.to(torch.bfloat16), y16)
+    else:  # float32 sums in a timing-dependent order: equal up to one bf16 rounding step
+        assert torch.allclose(y32.to(torch.bfloat16).float(), y16.float(), rtol=2 ** -7, atol=1e-6)
 
 
 def test_layer_deterministic_and_workspace_reuse():
     L = synth.make_layer(8, 512, 32, 64, seed=3, device=DEV, bias="normal")
     big = moe.workspace(64, 2048, 128, 768, 8, device=DEV)   # larger than needed
-    a, ia, wa, _ = run_layer(L, 4, 16, ws=big)
-    b, ib, wb, _ = run_layer(L, 4, 16, ws=big)
-    c, ic, wc, _ = run_layer(L, 4, 16)
+    st = moe.MOE_PATH_STREAM
+    a, ia, wa, _ = run_layer(L, 4, 16, ws=big, flags=st)
+    b, ib, wb, _ = run_layer(L, 4, 16, ws=big, flags=st)
+    c, ic, wc, _ = run_layer(L, 4, 16, flags=st)
     assert torch.equal(a, b) and torch.equal(a, c)
     assert torch.equal(ia, ic) and torch.equal(wa, wc)
+    # the one-token decode path routes identically and agrees to float32 rounding
+    L1 = synth.make_layer(1, 512, 32, 64, seed=3, device=DEV, bias="normal")
+    s_y, s_i, s_w, _ = run_layer(L1, 4, 16, ws=big, flags=st)
+    d_y, d_i, d_w, _ = run_layer(L1, 4, 16, ws=big, flags=CM, w_down=moe.moe_pack_w_down(L1.w_down))
+    assert torch.equal(d_i, s_i) and torch.equal(d_w, s_w)
+    assert torch.allclose(d_y, s_y, rtol=1e-5, atol=1e-6)
 
 
 def test_indices_do_not_depend_on_k2():
@@ -126,6 +174,7 @@ def test_decode_b1_full_size(k1, k2):
     for layer in range(2):
         L = synth.make_layer(1, 2048, 128, 768, seed=0, layer=layer, device=DEV)
         check_layer_sampled(L, k1, k2, [0])
+        check_layer_sampled(L, k1, k2, [0], flags=CM, w_down=moe.moe_pack_w_down(L.w_down))
 
 
 @pytest.mark.parametrize("T", [8, 32])
@@ -140,6 +189,8 @@ def test_decode_small_batch_full_size(T, k1, k2):
 def test_large_full_size(T, k1, k2):
     L = synth.make_layer(T, 4096, 512, 1024, seed=0, layer=0, device=DEV)
     check_layer_sampled(L, k1, k2, [0] if T == 1 else [0, 9, 40, 63])
+    if T == 1:
+        check_layer_sampled(L, k1, k2, [0], flags=CM, w_down=moe.moe_pack_w_down(L.w_down))
 
 
 @pytest.mark.parametrize("k1,k2", [(8, 16), (4, 16)])
