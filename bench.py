@@ -173,20 +173,29 @@ def dist_setup(args):
     return world, rank, local
 
 
-def allreduce_max(v, world):
+def allreduce_max(v, world, device="cuda"):
+    """Max of v over the ranks (the job's time is its slowest rank's)."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def barrier(world):
+def barrier(world, cuda=True):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if cuda:
+        torch.cuda.synchronize()
+
+
+def job_rate(units_per_rank, ms_per_rank, world, device="cuda"):
+    """Whole-job throughput: the units all ranks processed over the slowest
+    rank's time (weak scaling: every rank processes the same units)."""
+    ms = allreduce_max(ms_per_rank, world, device)
+    return world * units_per_rank * 1000.0 / ms, ms
 
 
 # ---------------------------------------------------------------------- model
@@ -387,7 +396,7 @@ def run_native(args, world, rank):
         h1 = time.time()
         barrier(world)
         ms = s.elapsed_time(e)
-        return allreduce_max(ms, world) / steps, (h0, h1)
+        return job_rate(T * steps, ms, world)[1] / steps, (h0, h1)
 
     # headline: the timed region of the contract (clocks sampled around it)
     clocks = ClockSampler(smi_index(torch.cuda.current_device()))

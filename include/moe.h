@@ -30,7 +30,7 @@
  *    expert intermediate size I (channels), k1 experts run per token, k2
  *    experts in the reference mass.  Requirements: 1 <= k1 <= k2,
  *    k1 <= min(E, 32), 1 <= E <= 1024, d % 64 == 0, I % 16 == 0,
- *    64 <= d <= 16384, 16 <= I <= 16384.  k2 > E is accepted and means
+ *    64 <= d <= 8192, 16 <= I <= 8192.  k2 > E is accepted and means
  *    k2 = E (no renormalisation), as the page's min(k2, E) does.
  *  - Routing is deterministic: probabilities are ranked by (p descending,
  *    expert index ascending); the float32 softmax and the top-k2 mass follow

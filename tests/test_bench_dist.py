@@ -1,0 +1,69 @@
+"""Host logic of bench.py's multi-rank (replica) mode on CPU: two gloo ranks
+in child processes, the max-over-ranks time, the whole-job rate and the
+reference arm's rank-0-only rule."""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, q):
+    import datetime
+
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        import bench
+        bench.barrier(world, cuda=False)
+        ms = 2.0 + 3.0 * rank  # rank 1 is the slow one
+        rate, ms_max = bench.job_rate(1, ms, world, device="cpu")
+
+        class A:
+            pass
+        args = A()
+        ref = bench.run_reference(args, world, rank) if rank != 0 else "skipped"
+        q.put((rank, rate, ms_max, ref))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_take_max_time_and_sum_units():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = {}
+    for _ in range(world):
+        r, rate, ms_max, ref = q.get(timeout=120)
+        out[r] = (rate, ms_max, ref)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    # every rank sees the slowest rank's time; the rate counts both ranks' units
+    assert out[0][1] == out[1][1] == pytest.approx(5.0)
+    assert out[0][0] == out[1][0] == pytest.approx(2 * 1000.0 / 5.0)
+    # only rank 0 runs the reference arm
+    assert out[1][2] is None
+
+
+def test_single_rank_rate_needs_no_process_group():
+    sys.path.insert(0, ROOT)
+    import bench
+    rate, ms = bench.job_rate(4, 2.0, 1)
+    assert ms == 2.0 and rate == pytest.approx(2000.0)
