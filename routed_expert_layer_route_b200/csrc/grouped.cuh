@@ -1,0 +1,616 @@
+// grouped.cuh -- the large-batch expert FFN as two grouped GEMMs on the
+// fifth-generation tensor cores (tcgen05.mma, accumulators in tensor memory).
+//
+// Expert structure ("Channel Selection for Mixture-of-Experts Decoding Needs
+// No Calibration Data", section 2 "Background"): a gated MLP; with the
+// routed slots grouped by expert (the counting sort of route.cuh), expert
+// e's n_e token rows X_e form two dense contractions:
+//     GEMM 1:  G = W_gate[e] X_e^T,  U = W_up[e] X_e^T   ([I x n_e], K = d)
+//              H = silu(G) * U, stored bf16 as rows of the slot-ordered H
+//     GEMM 2:  O = W_down[e] H_e^T                         ([d x n_e], K = I)
+//              y[t] += w[t, s] * O[:, slot]   (Eq. 2 weight, "Paper of the
+//              Week #3", section "The Receipt"), or O stored per slot.
+// The weight matrix is the MMA's M side (128 rows per tile) and the tokens
+// its N side (up to 256 per tile, padded to 16), so an expert with few tokens
+// costs little padding.  Both operands are K-major bf16 tiles of 64 K values
+// (one 128-byte row) in the 128-byte swizzled shared-memory layout.
+//
+// One persistent CTA per SM walks the work items (expert, weight-row tile,
+// token tile; token tile fastest, so CTAs that run at the same time share
+// weight tiles and token rows through L2).  Warp roles:
+//   warps 0-3   epilogue: tensor memory -> registers (tcgen05.ld), SwiGLU or
+//               the weighted combine, global stores / float32 red.add;
+//   warp 4      TMA producer (weight tiles; for GEMM 2 also H tiles), no
+//               multicast;
+//   warp 5      allocates tensor memory and issues the MMAs (one thread);
+//   warps 6-9   (GEMM 1 only) gather the routed tokens' x rows with cp.async
+//               into the swizzled layout.
+// Every wait is bounded: a wait that gives up records MOE_ERR_TIMEOUT and the
+// CTA drains what it issued and leaves.
+#pragma once
+#include <cuda.h>
+
+#include "common.cuh"
+#include "route.cuh"
+#include "stream.cuh"
+
+namespace moe {
+
+constexpr int kGBM = 128;                 // weight rows per tile (MMA M)
+constexpr int kGBK = 64;                  // K values per stage (one 128-byte row)
+constexpr int kGBN = 256;                 // most tokens per tile (MMA N)
+constexpr int kGTileA = kGBM * kGBK * 2;  // 16 KB
+constexpr int kGTileB = kGBN * kGBK * 2;  // 32 KB
+constexpr int kG1Stages = 3;              // A_gate + A_up + B = 64 KB per stage
+constexpr int kG2Stages = 4;              // A_down + B = 48 KB per stage
+constexpr int kG1Stage = 2 * kGTileA + kGTileB;
+constexpr int kG2Stage = kGTileA + kGTileB;
+constexpr int kGEpiThreads = 128;
+constexpr int kGGatherThreads = 128;
+constexpr int kG1Threads = kGEpiThreads + 64 + kGGatherThreads;  // 320
+constexpr int kG2Threads = kGEpiThreads + 64;                    // 192
+constexpr int kGMaxE = 1024;
+constexpr int kGWarpTma = 4, kGWarpMma = 5;
+
+// ---------------------------------------------------------------------------
+// tcgen05 / TMA wrappers
+MOE_DEVINL void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+MOE_DEVINL void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+MOE_DEVINL void tmem_alloc(uint32_t *dst, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(dst)),
+                 "r"(ncols)
+                 : "memory");
+}
+MOE_DEVINL void tmem_relinquish()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+MOE_DEVINL void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand in the 128-byte swizzled
+// layout (rows of 128 bytes, 8-row groups 1024 bytes apart), tile base
+// 1024-byte aligned; the K step inside a row advances the start address.
+MOE_DEVINL uint64_t umma_desc_sw128(uint32_t saddr)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu)     // start address
+           | ((uint64_t)1 << 16)                  // leading byte offset (unused here), 16 B
+           | ((uint64_t)(1024 >> 4) << 32)        // stride byte offset: 8 rows x 128 B
+           | ((uint64_t)1 << 46)                  // descriptor version of this architecture
+           | ((uint64_t)2 << 61);                 // 128-byte swizzle
+}
+
+// Instruction descriptor of kind::f16: bf16 A and B, float32 accumulator,
+// both K-major, M x N.
+MOE_DEVINL uint32_t umma_idesc_bf16(int M, int N)
+{
+    return (1u << 4)                        // D float32
+           | (1u << 7)                      // A bf16
+           | (1u << 10)                     // B bf16
+           | ((uint32_t)(N >> 3) << 17)     // N / 8
+           | ((uint32_t)(M >> 4) << 24);    // M / 16
+}
+
+MOE_DEVINL void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                          uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on `bar` when every MMA this thread issued so far has completed.
+MOE_DEVINL void umma_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_addr(bar))
+                 : "memory");
+}
+
+// 32 lanes x 32 consecutive float32 columns: thread i of the warp gets lane
+// (taddr.lane + i), columns taddr.col .. +31.
+MOE_DEVINL void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+        v[i] = __uint_as_float(r[i]);
+}
+
+// 2-D tiled TMA load (no multicast) of box {64 K values, rows} at (x, y).
+MOE_DEVINL void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
+MOE_DEVINL void cp_async16(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+MOE_DEVINL void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+MOE_DEVINL void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+MOE_DEVINL void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Work items: expert e contributes nrt x ceil(n_e / kGBN) items (weight-row
+// tile rt, token tile tt; tt fastest).
+struct GItem {
+    int e, rt, n, p0;
+};
+
+struct GTable {
+    int ibase[kGMaxE + 1];  // first item of each expert; ibase[E] = item count
+    int offs[kGMaxE + 1];   // expert offsets into the slot order
+    int scan[40];
+};
+
+// All threads of the CTA: fill the table from the expert offsets.
+__device__ void g_build_items(const int32_t *offsets, int E, int nrt, GTable &tb)
+{
+    for (int e = threadIdx.x; e <= E; e += blockDim.x)
+        tb.offs[e] = __ldcg(&offsets[e]);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const int n = tb.offs[e + 1] - tb.offs[e];
+        tb.ibase[e] = n > 0 ? nrt * ((n + kGBN - 1) / kGBN) : 0;
+    }
+    __syncthreads();
+    const int total = block_exclusive_scan(tb.ibase, E, tb.scan);
+    if (threadIdx.x == 0)
+        tb.ibase[E] = total;
+    __syncthreads();
+}
+
+MOE_DEVINL GItem g_item(const GTable &tb, int E, int i)
+{
+    int lo = 0, hi = E;  // ibase[lo] <= i < ibase[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (tb.ibase[mid] <= i)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    GItem it;
+    it.e = lo;
+    const int ne = tb.offs[lo + 1] - tb.offs[lo];
+    const int nt = (ne + kGBN - 1) / kGBN;
+    const int local = i - tb.ibase[lo];
+    it.rt = local / nt;
+    const int tt = local - it.rt * nt;
+    it.n = min(kGBN, ne - tt * kGBN);
+    it.p0 = tb.offs[lo] + tt * kGBN;
+    return it;
+}
+
+MOE_DEVINL int pad16(int n) { return (n + 15) & ~15; }
+
+// ---------------------------------------------------------------------------
+struct Gemm1Args {
+    const uint16_t *x;           // [T x d] bf16
+    const int32_t *offsets;      // [E + 1]
+    const int32_t *sorted_slot;  // [T*k1] slot ids (t*k1 + s) in expert order
+    uint16_t *h;                 // [T*k1 x I] bf16, row p = sorted position p
+    int T, d, E, I, k1;
+    WsHeader *hdr;
+};
+
+struct GSync {
+    uint64_t full[kG2Stages];
+    uint64_t empty[kG2Stages];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t drained;
+    uint32_t tmem_base;
+    int abort;
+};
+
+MOE_DEVINL uint8_t *g_align1024(uint8_t *p)
+{
+    const uint32_t a = smem_addr(p);
+    return p + (((a + 1023u) & ~1023u) - a);
+}
+
+inline size_t gemm1_smem_bytes() { return 1024 + (size_t)kG1Stages * kG1Stage + sizeof(GSync) + sizeof(GTable); }
+inline size_t gemm2_smem_bytes() { return 1024 + (size_t)kG2Stages * kG2Stage + sizeof(GSync) + sizeof(GTable); }
+
+// Gate/up GEMM with the SwiGLU epilogue.  Tensor memory: gate accumulator in
+// columns [0, 256), up accumulator in [256, 512).
+__global__ void __launch_bounds__(kG1Threads, 1)
+    k_gemm1(const __grid_constant__ CUtensorMap tm_gate, const __grid_constant__ CUtensorMap tm_up,
+            Gemm1Args a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *ring = g_align1024(smem_raw);
+    GSync &sy = *reinterpret_cast<GSync *>(ring + (size_t)kG1Stages * kG1Stage);
+    GTable &tb = *reinterpret_cast<GTable *>(&sy + 1);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    int *status = &a.hdr->status;
+
+    if (tid == 0) {
+        for (int s = 0; s < kG1Stages; ++s) {
+            mbar_init(&sy.full[s], 1 + kGGatherThreads);
+            mbar_init(&sy.empty[s], 1);
+        }
+        mbar_init(&sy.acc_full[0], 1);
+        mbar_init(&sy.acc_empty[0], kGEpiThreads / 32);
+        mbar_init(&sy.drained, 1);
+        sy.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == kGWarpMma) {
+        tmem_alloc(&sy.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sy.tmem_base;
+
+    pdl_wait();
+    pdl_trigger();
+    const int d = a.d, E = a.E, I = a.I;
+    const int nrt = I / kGBM;
+    const int nkb = d / kGBK;
+    g_build_items(a.offsets, E, nrt, tb);
+    const int n_items = tb.ibase[E];
+
+    if (warp == kGWarpTma) {
+        // -------------------------------------------------------- weight tiles
+        if (lane == 0) {
+            uint32_t g = 0;
+            for (int i = blockIdx.x; i < n_items && !*(volatile int *)&sy.abort; i += gridDim.x) {
+                const GItem it = g_item(tb, E, i);
+                const int row = it.e * I + it.rt * kGBM;
+                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                    const int s = g % kG1Stages;
+                    const uint32_t ph = (g / kG1Stages) & 1;
+                    if (!mbar_wait(&sy.empty[s], ph ^ 1, status)) {
+                        sy.abort = 1;
+                        break;
+                    }
+                    uint8_t *st = ring + (size_t)s * kG1Stage;
+                    mbar_arrive_expect_tx(&sy.full[s], 2 * kGTileA);
+                    tma_load_2d(st, &tm_gate, kb * kGBK, row, &sy.full[s]);
+                    tma_load_2d(st + kGTileA, &tm_up, kb * kGBK, row, &sy.full[s]);
+                }
+            }
+            // drain: every stage issued has landed before the CTA may leave
+            const uint32_t n_iss = g;
+            for (uint32_t q = n_iss > (uint32_t)kG1Stages ? n_iss - kG1Stages : 0; q < n_iss; ++q)
+                mbar_wait(&sy.full[q % kG1Stages], (q / kG1Stages) & 1, status);
+        }
+    } else if (warp == kGWarpMma) {
+        // -------------------------------------------------------- MMA issue
+        if (lane == 0) {
+            uint32_t g = 0, itc = 0;
+            for (int i = blockIdx.x; i < n_items && !*(volatile int *)&sy.abort; i += gridDim.x, ++itc) {
+                const GItem it = g_item(tb, E, i);
+                if (!mbar_wait(&sy.acc_empty[0], (itc & 1) ^ 1, status)) {
+                    sy.abort = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t idesc = umma_idesc_bf16(kGBM, pad16(it.n));
+                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                    const int s = g % kG1Stages;
+                    if (!mbar_wait(&sy.full[s], (g / kG1Stages) & 1, status)) {
+                        sy.abort = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t st = smem_addr(ring + (size_t)s * kG1Stage);
+#pragma unroll
+                    for (int kk = 0; kk < kGBK / 16; ++kk) {
+                        const uint64_t ag = umma_desc_sw128(st + kk * 32);
+                        const uint64_t au = umma_desc_sw128(st + kGTileA + kk * 32);
+                        const uint64_t bd = umma_desc_sw128(st + 2 * kGTileA + kk * 32);
+                        const uint32_t acc = (kb | kk) != 0;
+                        umma_bf16(tmem, ag, bd, idesc, acc);
+                        umma_bf16(tmem + 256, au, bd, idesc, acc);
+                    }
+                    umma_commit(&sy.empty[s]);
+                }
+                if (*(volatile int *)&sy.abort)
+                    break;
+                umma_commit(&sy.acc_full[0]);
+            }
+            // every MMA issued has completed before tensor memory is freed
+            umma_commit(&sy.drained);
+            mbar_wait(&sy.drained, 0, status);
+        }
+    } else if (warp >= 6) {
+        // -------------------------------------------------------- token gather
+        const int gt = tid - 6 * 32;  // 0..127
+        const int c = gt & 7;         // 16-byte chunk of the 128-byte row
+        const int rb = gt >> 3;       // rows rb + 16 j
+        const int k1 = a.k1;
+        uint32_t g = 0;
+        for (int i = blockIdx.x; i < n_items && !*(volatile int *)&sy.abort; i += gridDim.x) {
+            const GItem it = g_item(tb, E, i);
+            const int npad = pad16(it.n);
+            int tok[kGBN / 16];
+#pragma unroll
+            for (int j = 0; j < kGBN / 16; ++j) {
+                const int r = min(rb + 16 * j, it.n - 1);
+                tok[j] = __ldcg(&a.sorted_slot[it.p0 + r]) / k1;
+            }
+            for (int kb = 0; kb < nkb; ++kb, ++g) {
+                const int s = g % kG1Stages;
+                if (!mbar_wait(&sy.empty[s], ((g / kG1Stages) & 1) ^ 1, status)) {
+                    sy.abort = 1;
+                    break;
+                }
+                const uint32_t bst = smem_addr(ring + (size_t)s * kG1Stage + 2 * kGTileA);
+#pragma unroll
+                for (int j = 0; j < kGBN / 16; ++j) {
+                    const int r = rb + 16 * j;
+                    if (r < npad)
+                        cp_async16(bst + r * 128 + ((c ^ (r & 7)) << 4),
+                                   a.x + (size_t)tok[j] * d + kb * kGBK + c * 8);
+                }
+                cp_async_commit();
+                if (g >= kG1Stages - 1) {
+                    cp_async_wait<kG1Stages - 1>();
+                    fence_proxy_async_smem();
+                    mbar_arrive(&sy.full[(g - (kG1Stages - 1)) % kG1Stages]);
+                }
+            }
+        }
+        // the last stages' copies
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+        const uint32_t lo = g > (uint32_t)(kG1Stages - 1) ? g - (kG1Stages - 1) : 0;
+        for (uint32_t q = lo; q < g; ++q)
+            mbar_arrive(&sy.full[q % kG1Stages]);
+    } else {
+        // -------------------------------------------------------- epilogue (warps 0-3)
+        uint32_t itc = 0;
+        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+        for (int i = blockIdx.x; i < n_items && !*(volatile int *)&sy.abort; i += gridDim.x, ++itc) {
+            const GItem it = g_item(tb, E, i);
+            if (!mbar_wait(&sy.acc_full[0], itc & 1, status)) {
+                sy.abort = 1;
+                break;
+            }
+            tc_fence_after();
+            const int ch = it.rt * kGBM + warp * 32 + lane;  // this thread's channel
+            uint16_t *hcol = a.h + (size_t)it.p0 * I + ch;
+            for (int c0 = 0; c0 < it.n; c0 += 32) {
+                float gv[32], uv[32];
+                tmem_ld32(lane_addr + c0, gv);
+                tmem_ld32(lane_addr + 256 + c0, uv);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (c0 + j < it.n)
+                        hcol[(size_t)(c0 + j) * I] = f32_to_bf16_rn(silu_mul(gv[j], uv[j]));
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&sy.acc_empty[0]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kGWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------------------
+struct Gemm2Args {
+    const int32_t *offsets;      // [E + 1]
+    const int32_t *sorted_slot;  // [T*k1]
+    const float *topk_w;         // [T*k1] Eq. 2 weights by slot (combine mode)
+    float *y_acc;                // [T x d] float32, zero on entry (combine mode)
+    float *out;                  // [T*k1 x d] float32 per sorted position (out mode)
+    int T, d, E, I, k1;
+    int combine;                 // 1: weighted red.add into y_acc; 0: store rows of out
+    WsHeader *hdr;
+};
+
+// Down GEMM with the combine epilogue.  Two accumulator buffers of 256
+// columns each, so the epilogue of one item overlaps the MMAs of the next.
+__global__ void __launch_bounds__(kG2Threads, 1)
+    k_gemm2(const __grid_constant__ CUtensorMap tm_down, const __grid_constant__ CUtensorMap tm_h,
+            Gemm2Args a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *ring = g_align1024(smem_raw);
+    GSync &sy = *reinterpret_cast<GSync *>(ring + (size_t)kG2Stages * kG2Stage);
+    GTable &tb = *reinterpret_cast<GTable *>(&sy + 1);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    int *status = &a.hdr->status;
+
+    if (tid == 0) {
+        for (int s = 0; s < kG2Stages; ++s) {
+            mbar_init(&sy.full[s], 1);
+            mbar_init(&sy.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sy.acc_full[b], 1);
+            mbar_init(&sy.acc_empty[b], kGEpiThreads / 32);
+        }
+        mbar_init(&sy.drained, 1);
+        sy.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == kGWarpMma) {
+        tmem_alloc(&sy.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sy.tmem_base;
+
+    pdl_wait();
+    pdl_trigger();
+    const int d = a.d, E = a.E, I = a.I;
+    const int nrt = d / kGBM;
+    const int nkb = I / kGBK;
+    g_build_items(a.offsets, E, nrt, tb);
+    const int n_items = tb.ibase[E];
+
+    if (warp == kGWarpTma) {
+        if (lane == 0) {
+            uint32_t g = 0;
+            for (int i = blockIdx.x; i < n_items && !*(volatile int *)&sy.abort; i += gridDim.x) {
+                const GItem it = g_item(tb, E, i);
+                const int row = it.e * d + it.rt * kGBM;
+                const int nb = (it.n + 63) / 64;  // 64-row boxes of H
+                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                    const int s = g % kG2Stages;
+                    if (!mbar_wait(&sy.empty[s], ((g / kG2Stages) & 1) ^ 1, status)) {
+                        sy.abort = 1;
+                        break;
+                    }
+                    uint8_t *st = ring + (size_t)s * kG2Stage;
+                    mbar_arrive_expect_tx(&sy.full[s], kGTileA + nb * (kGTileB / 4));
+                    tma_load_2d(st, &tm_down, kb * kGBK, row, &sy.full[s]);
+                    for (int b = 0; b < nb; ++b)
+                        tma_load_2d(st + kGTileA + b * (kGTileB / 4), &tm_h, kb * kGBK,
+                                    it.p0 + 64 * b, &sy.full[s]);
+                }
+            }
+            const uint32_t n_iss = g;
+            for (uint32_t q = n_iss > (uint32_t)kG2Stages ? n_iss - kG2Stages : 0; q < n_iss; ++q)
+                mbar_wait(&sy.full[q % kG2Stages], (q / kG2Stages) & 1, status);
+        }
+    } else if (warp == kGWarpMma) {
+        if (lane == 0) {
+            uint32_t g = 0, itc = 0;
+            for (int i = blockIdx.x; i < n_items && !*(volatile int *)&sy.abort; i += gridDim.x, ++itc) {
+                const GItem it = g_item(tb, E, i);
+                const int buf = itc & 1;
+                if (!mbar_wait(&sy.acc_empty[buf], ((itc >> 1) & 1) ^ 1, status)) {
+                    sy.abort = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t idesc = umma_idesc_bf16(kGBM, pad16(it.n));
+                const uint32_t dt = tmem + buf * 256;
+                for (int kb = 0; kb < nkb; ++kb, ++g) {
+                    const int s = g % kG2Stages;
+                    if (!mbar_wait(&sy.full[s], (g / kG2Stages) & 1, status)) {
+                        sy.abort = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t st = smem_addr(ring + (size_t)s * kG2Stage);
+#pragma unroll
+                    for (int kk = 0; kk < kGBK / 16; ++kk)
+                        umma_bf16(dt, umma_desc_sw128(st + kk * 32),
+                                  umma_desc_sw128(st + kGTileA + kk * 32), idesc, (kb | kk) != 0);
+                    umma_commit(&sy.empty[s]);
+                }
+                if (*(volatile int *)&sy.abort)
+                    break;
+                umma_commit(&sy.acc_full[buf]);
+            }
+            umma_commit(&sy.drained);
+            mbar_wait(&sy.drained, 0, status);
+        }
+    } else {
+        // -------------------------------------------------------- epilogue (warps 0-3)
+        uint32_t itc = 0;
+        const int k1 = a.k1;
+        for (int i = blockIdx.x; i < n_items && !*(volatile int *)&sy.abort; i += gridDim.x, ++itc) {
+            const GItem it = g_item(tb, E, i);
+            const int buf = itc & 1;
+            // this lane's columns c*32 + lane: token and Eq. 2 weight (before the wait)
+            int tk[kGBN / 32];
+            float wt[kGBN / 32];
+#pragma unroll
+            for (int q = 0; q < kGBN / 32; ++q) {
+                const int col = q * 32 + lane;
+                tk[q] = 0;
+                wt[q] = 0.0f;
+                if (a.combine && col < it.n) {
+                    const int slot = __ldcg(&a.sorted_slot[it.p0 + col]);
+                    tk[q] = slot / k1;
+                    wt[q] = __ldcg(&a.topk_w[slot]);
+                }
+            }
+            if (!mbar_wait(&sy.acc_full[buf], (itc >> 1) & 1, status)) {
+                sy.abort = 1;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t taddr = tmem + buf * 256 + ((uint32_t)(warp * 32) << 16);
+            const int r = it.rt * kGBM + warp * 32 + lane;  // this thread's output row
+#pragma unroll
+            for (int q = 0; q < kGBN / 32; ++q) {
+                if (q * 32 < it.n) {
+                    float v[32];
+                    tmem_ld32(taddr + q * 32, v);
+                    if (a.combine) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int t = __shfl_sync(0xffffffffu, tk[q], j);
+                            const float w = __shfl_sync(0xffffffffu, wt[q], j);
+                            if (q * 32 + j < it.n)
+                                atomicAdd(&a.y_acc[(size_t)t * d + r], w * v[j]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (q * 32 + j < it.n)
+                                a.out[(size_t)(it.p0 + q * 32 + j) * d + r] = v[j];
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&sy.acc_empty[buf]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kGWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// The grouped path's shapes: whole 128-row weight tiles on both GEMMs.
+inline bool grouped_fits(int d, int E, int I) { return d % kGBM == 0 && I % kGBM == 0 && E <= kGMaxE; }
+
+}  // namespace moe

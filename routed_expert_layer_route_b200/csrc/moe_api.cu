@@ -13,6 +13,7 @@
 #include "../../include/moe_testing.h"
 #include "combine.cuh"
 #include "decode.cuh"
+#include "grouped.cuh"
 #include "route.cuh"
 #include "stream.cuh"
 
@@ -117,6 +118,11 @@ static int device_info(DevInfo *&out)
                                  decode_smem) != cudaSuccess ||
             cudaFuncSetAttribute(k_decode<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  decode_smem) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        if (cudaFuncSetAttribute(k_gemm1, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gemm1_smem_bytes()) != cudaSuccess ||
+            cudaFuncSetAttribute(k_gemm2, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gemm2_smem_bytes()) != cudaSuccess)
             return MOE_ERR_CUDA;
         const int small = 96 * 1024;
         if (cudaFuncSetAttribute(k_logits, cudaFuncAttributeMaxDynamicSharedMemorySize, small) !=
@@ -225,6 +231,102 @@ static int enqueue_decode(const void *x, const void *wg, const void *wu, const v
         return rc;
     return launch(k_finalize, dim3((d / 4 + 255) / 256), dim3(256), 0, s, true,
                   (const float *)at<float>(ws, L.y_acc), d, y, y_dtype);
+}
+
+
+// ------------------------------------------------------------------ grouped GEMM path
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime
+// (no link-time dependence on the driver library).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_tiled_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Row-major bf16 matrix [rows x inner] read in boxes of 64 inner values x
+// box_rows rows, 128-byte swizzle (the K-major operand layout of the MMAs).
+static int bf16_tile_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows,
+                         uint32_t box_rows)
+{
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (!enc)
+        return MOE_ERR_CUDA;
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {inner * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kGBK, box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+                           strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// The two grouped GEMMs over routed slots already grouped by expert
+// (offsets / sorted_slot).  combine: weighted red.add into y_acc (zeroed
+// before); otherwise per-slot rows of `out` in sorted order.
+static int enqueue_grouped(const void *x, const void *wg, const void *wu, const void *wd, int T,
+                           int d, int E, int I, int k1, const int32_t *offsets,
+                           const int32_t *sorted_slot, const float *topk_w, uint16_t *h,
+                           float *y_acc, float *out, WsHeader *hdr, int G, cudaStream_t s)
+{
+    CUtensorMap tg, tu, td, th;
+    int rc;
+    const uint64_t n = (uint64_t)T * k1;
+    if ((rc = bf16_tile_map(&tg, wg, d, (uint64_t)E * I, kGBM)) != MOE_OK ||
+        (rc = bf16_tile_map(&tu, wu, d, (uint64_t)E * I, kGBM)) != MOE_OK ||
+        (rc = bf16_tile_map(&td, wd, I, (uint64_t)E * d, kGBM)) != MOE_OK ||
+        (rc = bf16_tile_map(&th, h, I, n, 64)) != MOE_OK)
+        return rc;
+    Gemm1Args a1 = {};
+    a1.x = static_cast<const uint16_t *>(x);
+    a1.offsets = offsets;
+    a1.sorted_slot = sorted_slot;
+    a1.h = h;
+    a1.T = T;
+    a1.d = d;
+    a1.E = E;
+    a1.I = I;
+    a1.k1 = k1;
+    a1.hdr = hdr;
+    if ((rc = launch(k_gemm1, dim3(G), dim3(kG1Threads), gemm1_smem_bytes(), s, true, tg, tu,
+                     a1)) != MOE_OK)
+        return rc;
+    Gemm2Args a2 = {};
+    a2.offsets = offsets;
+    a2.sorted_slot = sorted_slot;
+    a2.topk_w = topk_w;
+    a2.y_acc = y_acc;
+    a2.out = out;
+    a2.T = T;
+    a2.d = d;
+    a2.E = E;
+    a2.I = I;
+    a2.k1 = k1;
+    a2.combine = y_acc != nullptr;
+    a2.hdr = hdr;
+    return launch(k_gemm2, dim3(G), dim3(kG2Threads), gemm2_smem_bytes(), s, true, td, th, a2);
+}
+
+// AUTO's choice of the tensor-core path: enough routed slots per expert to
+// fill MMA tiles, and whole 128-row weight tiles.
+static bool auto_grouped(int T, int d, int E, int I, int k1)
+{
+    return grouped_fits(d, E, I) && (long)T * k1 >= 16L * E;
 }
 
 }  // namespace moe
@@ -482,6 +584,14 @@ int moe_expert_ffn(const void *x_bf16, const int32_t *expert_offsets, const int3
     DevInfo *di;
     if ((rc = device_info(di)) != MOE_OK)
         return rc;
+    const bool grouped = flags == MOE_PATH_GROUPED || (flags == MOE_PATH_AUTO && auto_grouped(T, d, E, I, k1));
+    if (grouped) {
+        if (!grouped_fits(d, E, I))
+            return MOE_ERR_UNSUPPORTED_SHAPE;
+        return enqueue_grouped(x_bf16, w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I, k1,
+                               expert_offsets, sorted_slot, nullptr, at<uint16_t>(ws, L.h),
+                               nullptr, out, static_cast<WsHeader *>(ws), di->num_sms, s);
+    }
     if ((rc = launch(k_uniq_from_offsets, dim3(1), dim3(1024), 0, s, true, expert_offsets, E,
                      at<int32_t>(ws, L.uniq_count), at<int32_t>(ws, L.uniq_list))) != MOE_OK)
         return rc;
@@ -570,13 +680,30 @@ int moe_layer(const void *x_bf16, const void *w_router_bf16, const float *bias,
     const bool decode = down_cm && decode_fits(T, d, E, I, k1, G);
     if (down_cm && !decode)
         return MOE_ERR_UNSUPPORTED_SHAPE;  // channel-major down matrix: one-token calls only
-    float4 *y_acc = decode ? at<float4>(ws, L.y_acc) : nullptr;
+    const bool grouped = !down_cm && (path == MOE_PATH_GROUPED ||
+                                      (path == MOE_PATH_AUTO && auto_grouped(T, d, E, I, k1)));
+    if (grouped && !grouped_fits(d, E, I))
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    float4 *y_acc = decode || grouped ? at<float4>(ws, L.y_acc) : nullptr;
     if ((rc = enqueue_logits(x_bf16, w_router_bf16, bias, z, logits_out, T, d, E, s, y_acc,
                              T * d / 4)) != MOE_OK)
         return rc;
     if (decode)
         return enqueue_decode(x_bf16, w_gate_bf16, w_up_bf16, w_down_bf16, d, E, I, k1, k2, y,
                               y_dtype, topk_idx_out, topk_w_out, ws, G, s);
+    if (grouped) {
+        if ((rc = launch(k_topk, dim3(T), dim3(topk_threads(E)), permute_smem_bytes(E, T), s, true,
+                         (const float *)z, T, E, k1, k2, idx, w, topk_idx_out, topk_w_out, po,
+                         hdr)) != MOE_OK)
+            return rc;
+        if ((rc = enqueue_grouped(x_bf16, w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I, k1,
+                                  po.offsets, po.sorted_slot, w, at<uint16_t>(ws, L.h),
+                                  at<float>(ws, L.y_acc), nullptr, hdr, G, s)) != MOE_OK)
+            return rc;
+        const int n = T * d;
+        return launch(k_finalize, dim3((n / 4 + 255) / 256), dim3(256), 0, s, true,
+                      (const float *)at<float>(ws, L.y_acc), n, y, y_dtype);
+    }
     if (T > 1) {
         // one CTA per token ranks its probabilities; the last one to finish
         // builds the permutation tables

@@ -75,9 +75,10 @@ def check_layer_full(L, k1, k2, flags=moe.MOE_PATH_AUTO, tight=True, w_down=None
     return yy, ref
 
 
-def check_layer_sampled(L, k1, k2, tokens, flags=moe.MOE_PATH_AUTO, w_down=None):
+def check_layer_sampled(L, k1, k2, tokens, flags=moe.MOE_PATH_AUTO, w_down=None, tight=True):
     """Parity on sampled tokens; expert weights are fetched to the host only
-    for the experts those tokens use."""
+    for the experts those tokens use.  tight=False for the tensor-core path,
+    which rounds h to bf16 before the down projection."""
     y, idx, w, z = run_layer(L, k1, k2, flags=flags, w_down=w_down)
     tokens = np.asarray(tokens)
     zn = z.cpu().numpy()[tokens]
@@ -94,5 +95,6 @@ def check_layer_sampled(L, k1, k2, tokens, flags=moe.MOE_PATH_AUTO, w_down=None)
     assert np.array_equal(w.cpu().numpy()[tokens], ref["w"])
     yy = y.cpu().numpy()[tokens]
     err, rel = assert_close_layer(yy, ref["y"], "sampled layer")
-    assert rel <= 1e-4, rel
+    if tight:
+        assert rel <= 1e-4, rel
     return idx.cpu().numpy()

@@ -195,8 +195,69 @@ def test_large_full_size(T, k1, k2):
 
 @pytest.mark.parametrize("k1,k2", [(8, 16), (4, 16)])
 def test_prefill_full_size_sampled(k1, k2):
+    # AUTO runs the tensor-core grouped GEMMs at this batch size
     L = synth.make_layer(4096, 2048, 128, 768, seed=0, layer=0, device=DEV, bias="zipf")
-    idx = check_layer_sampled(L, k1, k2, [0, 1, 777, 2048, 4000, 4095])
+    tokens = [0, 1, 777, 2048, 4000, 4095]
+    idx = check_layer_sampled(L, k1, k2, tokens, tight=False)
     # Zipf bias: the most popular expert gets many more tokens than the least
     counts = np.bincount(idx.ravel(), minlength=128)
     assert counts.max() > 4 * max(1, np.median(counts))
+    # the streaming path on the same layer (float32 h: tight)
+    check_layer_sampled(L, k1, k2, tokens, flags=moe.MOE_PATH_STREAM)
+
+
+# ------------------------------------------------------------------ tensor-core grouped path
+GROUPED = moe.MOE_PATH_GROUPED
+GSMALL = [
+    # T, d, E, I, k1, k2, bias
+    (1, 128, 8, 128, 2, 4, None),
+    (16, 128, 16, 128, 4, 8, None),
+    (64, 256, 16, 256, 4, 16, "normal"),
+    (300, 256, 4, 128, 2, 4, None),      # > 256 slots per expert: several token tiles
+    (200, 512, 32, 384, 8, 8, "zipf"),   # ragged tiles, experts without tokens
+    (37, 384, 64, 128, 3, 1000, None),
+    (130, 128, 2, 256, 2, 2, None),      # k1 = E: every token in every expert
+]
+
+
+@pytest.mark.parametrize("T,d,E,I,k1,k2,bias", GSMALL)
+def test_layer_grouped_all_tokens(T, d, E, I, k1, k2, bias):
+    L = synth.make_layer(T, d, E, I, seed=T + d + E + 1, device=DEV, bias=bias)
+    check_layer_full(L, k1, k2, flags=GROUPED, tight=False)
+
+
+@pytest.mark.parametrize("T,d,E,I,k1", [(48, 256, 8, 128, 2), (520, 128, 4, 256, 2)])
+def test_expert_ffn_grouped_per_slot(T, d, E, I, k1):
+    L = synth.make_layer(T, d, E, I, seed=11, device=DEV, bias="normal")
+    ws = moe.workspace(T, d, E, I, k1, device=DEV)
+    idx = torch.empty(T, k1, dtype=torch.int32, device=DEV)
+    w = torch.empty(T, k1, dtype=torch.float32, device=DEV)
+    z = torch.empty(T, E, dtype=torch.float32, device=DEV)
+    moe.moe_route(L.x, L.w_router, L.bias, z, k1, k1, idx, w)
+    off = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    ss = torch.empty(T * k1, dtype=torch.int32, device=DEV)
+    sp = torch.empty(T * k1, dtype=torch.int32, device=DEV)
+    moe.moe_permute(idx, E, off, ss, sp)
+    out = torch.full((T * k1, d), float("nan"), dtype=torch.float32, device=DEV)
+    moe.moe_expert_ffn(L.x, off, ss, L.w_gate, L.w_up, L.w_down, k1, out, ws, flags=GROUPED)
+    torch.cuda.synchronize()
+    assert moe.moe_read_device_status(ws) == 0
+    ssn, idxn, on = ss.cpu().numpy(), idx.cpu().numpy(), out.cpu().numpy()
+    xf = (synth.to_numpy(L.x).astype(np.uint32) << 16).view(np.float32)
+    experts = {}
+    ref = np.empty_like(on)
+    for p in range(T * k1):
+        slot = int(ssn[p])
+        t, e = slot // k1, int(idxn.ravel()[slot])
+        if e not in experts:
+            experts[e] = (synth.to_numpy(L.w_gate[e]), synth.to_numpy(L.w_up[e]),
+                          synth.to_numpy(L.w_down[e]))
+        ref[p] = oracle.expert(xf[t], *experts[e])[1]
+    assert_close_layer(on, ref, "grouped expert outputs")
+
+
+def test_grouped_rejects_partial_tiles():
+    L = synth.make_layer(8, 192, 8, 128, seed=1, device=DEV)   # d not a multiple of 128
+    with pytest.raises(moe.MoeError) as ei:
+        run_layer(L, 2, 4, flags=GROUPED)
+    assert ei.value.status == moe.MOE_ERR_UNSUPPORTED_SHAPE
