@@ -44,7 +44,8 @@ WORKLOADS = {
                       sweep=[(4, 16), (8, 8), (8, 16), (8, 128), (4, 4), (4, 128)]),
     "decode_small_batch": dict(T=8, d=2048, E=128, I=768, layers=48, bias="normal",
                                sweep=[(4, 16), (8, 8)]),
-    "prefill": dict(T=4096, d=2048, E=128, I=768, layers=4, bias="zipf", sweep=[(8, 16), (4, 16)]),
+    "prefill": dict(T=4096, d=2048, E=128, I=768, layers=4, bias="zipf", sweep=[(8, 16), (4, 16)],
+                    grouped=True),
     "large": dict(T=1, d=4096, E=512, I=1024, layers=8, bias=None, sweep=[(5, 20), (10, 10)]),
 }
 
@@ -210,7 +211,11 @@ class Stack:
         self.wl = wl
         self.layers = []
         self.channel_major = wl["T"] == 1
-        self.flags = moe.MOE_WDOWN_CHANNEL_MAJOR if self.channel_major else moe.MOE_PATH_AUTO
+        # large batches: the tensor-core grouped GEMMs (what AUTO picks at >= 16
+        # routed slots per expert), named explicitly so the timed kernels are known
+        self.grouped = wl.get("grouped", False)
+        self.flags = (moe.MOE_WDOWN_CHANNEL_MAJOR if self.channel_major else
+                      moe.MOE_PATH_GROUPED if self.grouped else moe.MOE_PATH_STREAM)
         for l in range(wl["layers"]):
             L = synth.make_layer(wl["T"], wl["d"], wl["E"], wl["I"], seed=seed, layer=l,
                                  device=device, bias=wl["bias"])
@@ -279,6 +284,31 @@ def time_dominant_kernel(stack, k1, k2, ws_list, ys, stream, reps):
     return statistics.mean(ms[len(stack.layers):] or ms)  # first pass is warm-up
 
 
+def time_grouped_kernels(stack, k1, ws_list, stream, reps):
+    """Average durations (ms) of the token-row gather, the gate/up and the down
+    grouped GEMM, each launched alone (CUDA events on its stream) on the
+    routing tables the layer's last moe_layer call left in its workspace,
+    cycling the layers."""
+    from routed_expert_layer_route_b200 import moe
+    out = []
+    for which in (4, 1, 2):
+        pairs = []
+        with torch.cuda.stream(stream):
+            for r in range(reps):
+                for L, ws in zip(stack.layers, ws_list):
+                    s = torch.cuda.Event(enable_timing=True)
+                    e = torch.cuda.Event(enable_timing=True)
+                    s.record(stream)
+                    moe.moe_test_expert_grouped(L.x, L.w_gate, L.w_up, L.w_down, k1, which, ws,
+                                                stream=stream)
+                    e.record(stream)
+                    pairs.append((s, e))
+        stream.synchronize()
+        ms = [a.elapsed_time(b) for a, b in pairs]
+        out.append(statistics.mean(ms[len(stack.layers):] or ms))
+    return out
+
+
 def e2e_tokens_per_s(stack, k1, k2, ws_list, steps, warmup, stream):
     """Through the public API with host buffers: per step, pinned-host ->
     device copy of every layer's tokens, every layer's moe_layer call, and a
@@ -314,18 +344,19 @@ def e2e_tokens_per_s(stack, k1, k2, ws_list, steps, warmup, stream):
 
 
 # ---------------------------------------------------------------------- CPU oracle
-def cpu_oracle_rate(stack, k1, k2, budget_s=12.0):
+def cpu_oracle_rate(stack, k1, k2, budget_s=12.0, max_tokens=8):
     """The oracle as it stands, on the host cores: router logits, routing,
     the k1 experts and the combine, layer after layer until the time budget
-    is spent.  Returns (tokens/s for the whole stack, layers run, threads)."""
+    is spent, on the first min(T, max_tokens) tokens of each layer.  Returns
+    (tokens/s for the whole stack, layers run, threads, seconds)."""
     import oracle
     from routed_expert_layer_route_b200 import synth
     wl = stack.wl
-    T = wl["T"]
+    T = min(wl["T"], max_tokens)
     prepared = []
     # fetch only what the sample needs (router, bias, the routed experts)
     for L in stack.layers:
-        x = synth.to_numpy(L.x)
+        x = synth.to_numpy(L.x[:T])
         wr = synth.to_numpy(L.w_router)
         b = synth.to_numpy(L.bias)
         z = oracle.logits(x, wr, b)
@@ -333,7 +364,7 @@ def cpu_oracle_rate(stack, k1, k2, budget_s=12.0):
         experts = {int(e): (synth.to_numpy(L.w_gate[int(e)]), synth.to_numpy(L.w_up[int(e)]),
                             stack.down_hf(L, int(e))) for e in np.unique(idx)}
         prepared.append((x, wr, b, experts))
-        if len(prepared) >= 6:
+        if len(prepared) >= (6 if wl["T"] == 1 else 2):
             break
     t0 = time.perf_counter()
     n = 0
@@ -413,9 +444,11 @@ def run_native(args, world, rank):
         us = unique_experts(stack, k1, k2, ws_list, ys, stream)
         U = statistics.mean(us)
         bytes_layer = U * 3 * d * I * 2
+        flops_layer = T * (k1 * 6.0 * d * I + 2.0 * d * E)
         results.append({"k1": k1, "k2": k2, "ms_per_step": ms, "us_per_layer": ms * 1000 / Ln,
                         "tokens_per_s": world * T * 1000.0 / ms, "unique_experts_per_layer": U,
-                        "expert_GBps": bytes_layer / (ms / Ln * 1e-3) / 1e9})
+                        "expert_GBps": bytes_layer / (ms / Ln * 1e-3) / 1e9,
+                        "layer_TFLOPs": flops_layer / (ms / Ln * 1e-3) / 1e12})
 
     clocks.stop()
     clk, _ = clocks.summary(*head_win)
@@ -427,19 +460,46 @@ def run_native(args, world, rank):
     # dominant kernel alone, events on its own stream
     k1h, k2h = head
     _, ws_list, ys = graphs[head]
-    kern_ms = time_dominant_kernel(stack, k1h, k2h, ws_list, ys, stream, reps=3)
     U_head = results[0]["unique_experts_per_layer"]
     alg_bytes = U_head * 3 * d * I * 2
-    achieved = alg_bytes / (kern_ms * 1e-3) / 1e9
-    kname = "k_decode" if stack.channel_major else "k_stream"
-    traffic = recorded_traffic(args.workload, k1h, kname)
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-                "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
-                "kernel": "moe::" + kname,
-                "kernel_us": round(kern_ms * 1000, 2),
-                "algorithmic_bytes_per_launch": int(alg_bytes),
-                "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
-                if peak_kind == "measured" else "fallback 6650 GB/s"}
+    if stack.grouped:
+        gx_ms, g1_ms, g2_ms = time_grouped_kernels(stack, k1h, ws_list, stream, reps=3)
+        n_slots = T * k1h
+        f1 = 2.0 * n_slots * 2 * I * d   # gate and up
+        f2 = 2.0 * n_slots * I * d       # down
+        a1 = f1 / (g1_ms * 1e-3) / 1e12
+        a2 = f2 / (g2_ms * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "achieved": round(a1, 1), "peak": bf16_peak,
+                    "unit": "TFLOP/s", "frac": round(a1 / bf16_peak, 4),
+                    "traffic": recorded_traffic(args.workload, k1h, "k_gemm1"),
+                    "kernel": "moe::k_gemm1", "kernel_us": round(g1_ms * 1000, 2),
+                    "algorithmic_flops_per_launch": f1,
+                    "second_kernel": {"kernel": "moe::k_gemm2", "kernel_us": round(g2_ms * 1000, 2),
+                                      "algorithmic_flops_per_launch": f2,
+                                      "achieved": round(a2, 1),
+                                      "frac": round(a2 / bf16_peak, 4)},
+                    "gather_kernel": {"kernel": "moe::k_gather_rows",
+                                      "kernel_us": round(gx_ms * 1000, 2)},
+                    "both_gemms_frac": round((f1 + f2) / ((g1_ms + g2_ms) * 1e-3) / 1e12
+                                             / bf16_peak, 4),
+                    "hbm_bytes_per_layer": int(alg_bytes),
+                    "hbm_frac_both_gemms": round(alg_bytes / ((g1_ms + g2_ms) * 1e-3) / 1e9
+                                                 / hbm_peak, 4),
+                    "peak_source": "%s (MEASURED_PEAKS.json bf16_tflops, burst: kernels timed "
+                                   "alone)" % peak_kind if peak_kind == "measured"
+                    else "fallback 1590 TFLOP/s"}
+    else:
+        kern_ms = time_dominant_kernel(stack, k1h, k2h, ws_list, ys, stream, reps=3)
+        achieved = alg_bytes / (kern_ms * 1e-3) / 1e9
+        kname = "k_decode" if stack.channel_major else "k_stream"
+        traffic = recorded_traffic(args.workload, k1h, kname)
+        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
+                    "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
+                    "kernel": "moe::" + kname,
+                    "kernel_us": round(kern_ms * 1000, 2),
+                    "algorithmic_bytes_per_launch": int(alg_bytes),
+                    "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
+                    if peak_kind == "measured" else "fallback 6650 GB/s"}
 
     # end to end through the public API with host buffers
     e2e_val, h2d, d2h = e2e_tokens_per_s(stack, k1h, k2h, ws_list, max(3, args.steps // 4),
@@ -458,10 +518,13 @@ def run_native(args, world, rank):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, nl, thr, el = cpu_oracle_rate(stack, k1h, k2h)
         cpu = {"value": rate, "unit": "tokens/s", "cores": thr, "kind": "oracle",
-               "sample": "%d single-token layers of this workload (k1=%d, k2=%d) in %.1f s, "
-                         "per-layer time scaled to the %d-layer stack" % (nl, k1h, k2h, el, Ln)}
+               "sample": "%d layers of this workload, first %d token(s) of each (k1=%d, k2=%d), "
+                         "in %.1f s; per-layer time scaled to the %d-layer stack"
+                         % (nl, min(T, 8), k1h, k2h, el, Ln)}
 
-    per_step_launches = 3  # router, expert kernel, finalize (T == 1) / router, top-k, expert
+    # kernels per layer: router, decode kernel, finalize (one token); router, top-k,
+    # streaming kernel (small batch); router, top-k, two grouped GEMMs, finalize
+    per_step_launches = 5 if stack.grouped else 3
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
@@ -526,9 +589,10 @@ def run_reference(args, world, rank):
                                                     "k2=%d" % (args.workload, wl["layers"], wl["d"],
                                                                wl["E"], wl["I"], wl["T"], k1, k2)},
         "cpu_baseline": {"value": round(r_stack, 4), "unit": "tokens/s", "cores": thr,
-                         "kind": "oracle", "sample": "each step: single-token layers for 3 s, "
-                                                     "per-layer time scaled to the %d-layer stack"
-                                                     % wl["layers"]},
+                         "kind": "oracle", "sample": "each step: layers of this workload for 3 s, "
+                                                     "first %d token(s) of each; per-layer time "
+                                                     "scaled to the %d-layer stack"
+                                                     % (min(wl["T"], 8), wl["layers"])},
         "e2e": {"value": round(r_stack, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "wall_s": round(total, 2),

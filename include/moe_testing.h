@@ -36,6 +36,20 @@ int moe_test_expert_stream(const void *x_bf16, const void *w_gate_bf16, const vo
                            void *y, int y_dtype, int flags, void *ws, size_t ws_bytes,
                            void *stream);
 
+/* The kernels of the grouped tensor-core expert FFN launched alone, without
+ * programmatic dependent launch, on the routing tables a previous moe_layer
+ * call left in `ws` (same shapes, k1).  `which` is a bit set: 4 copies the
+ * routed tokens' x rows into expert order, 1 runs the gate/up GEMM with the
+ * SwiGLU epilogue (writes h), 2 the down GEMM with the weighted combine (adds
+ * into the workspace's float32 accumulator, whose contents are then
+ * meaningless); 8 alone runs the down GEMM storing per-slot rows (the
+ * moe_expert_ffn epilogue) over the gathered rows' space.  For timing the
+ * kernels separately.  Shapes must satisfy the
+ * grouped path (d and I multiples of 128).  Returns a moe_status. */
+int moe_test_expert_grouped(const void *x_bf16, const void *w_gate_bf16, const void *w_up_bf16,
+                            const void *w_down_bf16, int T, int d, int E, int I, int k1, int which,
+                            void *ws, size_t ws_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

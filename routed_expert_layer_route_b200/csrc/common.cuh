@@ -16,7 +16,8 @@ constexpr int kMaxGridCtas = 960;  // most CTAs a grid barrier can serve
 struct WsHeader {
     int status;             // device status word (moe_status), 0 = OK
     unsigned route_arrive;  // last-block hand-off counter of the top-k kernel
-    unsigned pad0[30];
+    unsigned decode_arrive; // last-block hand-off counter of the decode kernel
+    unsigned pad0[29];
     unsigned bar_go;        // grid barrier: generation released so far (own 128-byte line)
     unsigned pad1[31];
     unsigned bar_flag[kMaxGridCtas];  // grid barrier: generation each CTA has reached

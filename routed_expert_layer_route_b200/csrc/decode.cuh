@@ -12,8 +12,10 @@
 // (Eq. 2 weight w, "Paper of the Week #3", section "The Receipt").
 //
 // Design (one persistent CTA per SM, 12 consumer warps + 1 producer warp):
-//  * one token per call (T == 1): every CTA routes it itself from the
-//    router's logits (same fixed float32 sequence as the router kernels);
+//  * one token per call (T == 1): one warp of every CTA routes it from the
+//    router's logits in registers (warp_route: the same fixed float32
+//    sequence as the router kernels) while the others load x; each CTA's
+//    channel ranges are fixed before the kernel waits on the router;
 //  * the U activated experts are laid end to end as U*I channels and CTA b
 //    owns a contiguous range of floor(U*I/G) or one more channels;
 //  * the producer streams stages of n whole channels (gate rows, up rows,
@@ -24,8 +26,9 @@
 //    adds h * down_row into register partials for its fixed third of the
 //    output rows;
 //  * at the end the four groups' partials are summed in shared memory and
-//    added into the float32 accumulator y_acc with red.global.add;
-//    k_finalize converts y_acc to the output type after the kernel ends.
+//    added into the float32 accumulator y_acc with red.global.add; the last
+//    CTA to check in (a counter in the workspace header) converts y_acc to
+//    the output y.
 // Partial sums from different CTAs reach y_acc in a timing-dependent order,
 // so y can differ between runs in the last bits (stream.cuh holds the
 // deterministic two-phase kernel).
@@ -62,6 +65,8 @@ struct DecodeArgs {
     int32_t *uniq_count;
     int32_t *uniq_list;
     float *y_acc;  // [d] float32, zero on entry
+    void *y;       // [d] output (y_dtype); written by the last CTA to finish
+    int y_dtype;
     WsHeader *hdr;
 };
 
@@ -80,7 +85,7 @@ struct __align__(16) DecodeSmem {
     int nseg;
     int abort;
     int issued;
-    int pad;
+    int last;
 };
 
 struct DIter {
@@ -136,54 +141,8 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
         ds->abort = 0;
         ds->issued = 0;
         fence_mbar_init();
-    }
-    __syncthreads();
-
-    pdl_wait();
-    pdl_trigger();
-
-    // ------------------------------------------------------------ routing
-    // the token's x row goes out in the same round as the logits
-    for (int i = tid; i < (d >> 3); i += kSThreads)
-        reinterpret_cast<uint4 *>(area)[i] = reinterpret_cast<const uint4 *>(a.x)[i];
-    {
-        // the ring is idle until routing is known, so the routing scratch lives there
-        RouteSmem &rs = *reinterpret_cast<RouteSmem *>(ring);
-        float *zs = reinterpret_cast<float *>(ring + sizeof(RouteSmem));
-        for (int j = tid; j < E; j += kSThreads)
-            zs[j] = __ldcg(&a.logits[j]);
-        __syncthreads();
-        route_token_block(zs, E, k1, a.k2, rs, b == 0 ? a.topk_idx : nullptr,
-                          b == 0 ? a.topk_w : nullptr, b == 0 ? a.idx_copy : nullptr,
-                          b == 0 ? a.w_copy : nullptr);
-        if (tid < k1) {
-            const int e = rs.out_j[tid];
-            int p = 0;
-            for (int s = 0; s < k1; ++s)
-                p += rs.out_j[s] < e;
-            ds->ue[p] = e;
-            ds->uw[p] = rs.out_w[tid];
-            if (b == 0) {
-                a.uniq_list[p] = e;
-                a.sorted_slot[p] = tid;
-                a.slot_pos[tid] = p;
-            }
-        }
-        if (b == 0) {
-            if (tid == 0)
-                *a.uniq_count = k1;
-            for (int e = tid; e <= E; e += kSThreads) {
-                int c = 0;
-                for (int s = 0; s < k1; ++s)
-                    c += rs.out_j[s] < e;
-                a.offsets[e] = c;
-            }
-        }
-        __syncthreads();
-    }
-
-    // ------------------------------------------------------------ this CTA's segments
-    if (tid == 0) {
+        // this CTA's channel segments depend only on k1, I and the grid: the
+        // U = k1 activated experts laid end to end as U*I channels
         const unsigned tot = (unsigned)k1 * (unsigned)I;
         const unsigned c_lo = split_lo(tot, G, b), c_hi = split_lo(tot, G, b + 1);
         int ns = 0;
@@ -202,6 +161,57 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
             ns = 0;
         }
         ds->nseg = ns;
+    }
+    __syncthreads();
+
+    pdl_wait();
+    pdl_trigger();
+
+    // ------------------------------------------------------------ routing (one warp)
+    if (warp == 0) {
+        int j;
+        float wv;
+        if (E <= 128)
+            warp_route<4>(a.logits, E, k1, a.k2, lane, j, wv);
+        else if (E <= 256)
+            warp_route<8>(a.logits, E, k1, a.k2, lane, j, wv);
+        else if (E <= 512)
+            warp_route<16>(a.logits, E, k1, a.k2, lane, j, wv);
+        else
+            warp_route<32>(a.logits, E, k1, a.k2, lane, j, wv);
+        int p = 0;  // position of this lane's expert among the k1, ascending
+        for (int q = 0; q < k1; ++q)
+            p += __shfl_sync(0xffffffffu, j, q) < j;
+        if (lane < k1) {
+            ds->ue[p] = j;
+            ds->uw[p] = wv;
+            if (b == 0) {
+                a.topk_idx[lane] = j;
+                a.topk_w[lane] = wv;
+                if (a.idx_copy)
+                    a.idx_copy[lane] = j;
+                if (a.w_copy)
+                    a.w_copy[lane] = wv;
+                a.uniq_list[p] = j;
+                a.sorted_slot[p] = lane;
+                a.slot_pos[lane] = p;
+            }
+        }
+        __syncwarp();
+        if (b == 0) {
+            if (lane == 0)
+                *a.uniq_count = k1;
+            for (int e = lane; e <= E; e += 32) {
+                int cnt = 0;
+                for (int q = 0; q < k1; ++q)
+                    cnt += ds->ue[q] < e;
+                a.offsets[e] = cnt;
+            }
+        }
+    } else {
+        // the token's x row, meanwhile
+        for (int i = tid - 32; i < (d >> 3); i += kSThreads - 32)
+            reinterpret_cast<uint4 *>(area)[i] = reinterpret_cast<const uint4 *>(a.x)[i];
     }
     __syncthreads();
     const int nseg = ds->nseg;
@@ -350,6 +360,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
                 atomicAdd(&a.y_acc[r], sum);
             }
         }
+        __threadfence();  // the adds are visible before this CTA checks in below
     }
 
     __syncthreads();
@@ -360,6 +371,29 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
             const uint32_t parity = (uint32_t)((last / kDStages) & 1);
             mbar_wait(&full[s], parity, status);
         }
+    }
+
+    // ------------------------------------------------------------ y (last CTA to finish)
+    if (tid == 0) {
+        const unsigned prev = atomicAdd(&a.hdr->decode_arrive, 1u);
+        ds->last = prev == (unsigned)G - 1;
+    }
+    __syncthreads();
+    if (ds->last) {
+        __threadfence();
+        for (int i = tid * 4; i < d; i += kSThreads * 4) {
+            const float4 v = __ldcg(reinterpret_cast<const float4 *>(a.y_acc + i));
+            if (a.y_dtype == MOE_DTYPE_BF16) {
+                const uint32_t lo = f32_to_bf16_rn(v.x) | ((uint32_t)f32_to_bf16_rn(v.y) << 16);
+                const uint32_t hi = f32_to_bf16_rn(v.z) | ((uint32_t)f32_to_bf16_rn(v.w) << 16);
+                *reinterpret_cast<uint2 *>(reinterpret_cast<uint16_t *>(a.y) + i) =
+                    make_uint2(lo, hi);
+            } else {
+                *reinterpret_cast<float4 *>(reinterpret_cast<float *>(a.y) + i) = v;
+            }
+        }
+        if (tid == 0)
+            a.hdr->decode_arrive = 0u;
     }
 }
 

@@ -20,11 +20,13 @@
 // weight tiles and token rows through L2).  Warp roles:
 //   warps 0-3   epilogue: tensor memory -> registers (tcgen05.ld), SwiGLU or
 //               the weighted combine, global stores / float32 red.add;
-//   warp 4      TMA producer (weight tiles; for GEMM 2 also H tiles), no
-//               multicast;
-//   warp 5      allocates tensor memory and issues the MMAs (one thread);
-//   warps 6-9   (GEMM 1 only) gather the routed tokens' x rows with cp.async
-//               into the swizzled layout.
+//   warp 4      TMA producer, no multicast: weight tiles and token tiles
+//               (GEMM 1: the routed tokens' x rows, copied into expert order
+//               by k_gather_rows; GEMM 2: H), with an L2 prefetch stream a
+//               few k-blocks ahead of the loads;
+//   warp 5      allocates tensor memory and issues the MMAs (one thread).
+// The same down-GEMM kernel computes the router logits of large batches
+// (one group of T rows, W_r as the weight matrix, bias added).
 // Every wait is bounded: a wait that gives up records MOE_ERR_TIMEOUT and the
 // CTA drains what it issued and leaves.
 #pragma once
@@ -46,9 +48,8 @@ constexpr int kG2Stages = 4;              // A_down + B = 48 KB per stage
 constexpr int kG1Stage = 2 * kGTileA + kGTileB;
 constexpr int kG2Stage = kGTileA + kGTileB;
 constexpr int kGEpiThreads = 128;
-constexpr int kGGatherThreads = 128;
-constexpr int kG1Threads = kGEpiThreads + 64 + kGGatherThreads;  // 320
-constexpr int kG2Threads = kGEpiThreads + 64;                    // 192
+constexpr int kG1Threads = kGEpiThreads + 64;  // 192
+constexpr int kG2Threads = kGEpiThreads + 64;  // 192
 constexpr int kGMaxE = 1024;
 constexpr int kGWarpTma = 4, kGWarpMma = 5;
 
@@ -148,20 +149,33 @@ MOE_DEVINL void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uin
         : "memory");
 }
 
-MOE_DEVINL void cp_async16(uint32_t dst, const void *src)
+// Prefetch `bytes` (multiple of 16) of contiguous global memory into L2.
+MOE_DEVINL void bulk_prefetch_l2(const void *src, uint32_t bytes)
 {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
-MOE_DEVINL void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-MOE_DEVINL void cp_async_wait()
+
+// A weight tile's rows are one contiguous block (row-major weights): fetch it
+// into L2 front to back in 64 KB pieces, a DRAM-friendly order, before the
+// tiled loads walk it one 128-byte column strip at a time.
+MOE_DEVINL void prefetch_rows_l2(const uint16_t *base, size_t row0, int rows, int rowlen)
 {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+    const uint8_t *p = reinterpret_cast<const uint8_t *>(base + row0 * rowlen);
+    const size_t bytes = (size_t)rows * rowlen * 2;
+    for (size_t o = 0; o < bytes; o += 65536)
+        bulk_prefetch_l2(p + o, (uint32_t)min((size_t)65536, bytes - o));
 }
-MOE_DEVINL void fence_proxy_async_smem()
+
+// Prefetch one box of a 2-D map into L2 (no shared memory, no multicast).
+MOE_DEVINL void tma_prefetch_2d(const CUtensorMap *map, int x, int y)
 {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y)
+                 : "memory");
 }
+
+
 
 // ---------------------------------------------------------------------------
 // Work items: expert e contributes nrt x ceil(n_e / kGBN) items (weight-row
@@ -173,18 +187,23 @@ struct GItem {
 struct GTable {
     int ibase[kGMaxE + 1];  // first item of each expert; ibase[E] = item count
     int offs[kGMaxE + 1];   // expert offsets into the slot order
+    int bn;                 // tokens per tile (<= kGBN, multiple of 64)
     int scan[40];
 };
 
-// All threads of the CTA: fill the table from the expert offsets.
-__device__ void g_build_items(const int32_t *offsets, int E, int nrt, GTable &tb)
+// All threads of the CTA: fill the table from the expert offsets (or, with
+// offsets == nullptr, one group of single_n rows).
+__device__ void g_build_items(const int32_t *offsets, int E, int nrt, GTable &tb, int single_n = 0,
+                              int bn = kGBN)
 {
     for (int e = threadIdx.x; e <= E; e += blockDim.x)
-        tb.offs[e] = __ldcg(&offsets[e]);
+        tb.offs[e] = offsets ? __ldcg(&offsets[e]) : (e == 0 ? 0 : single_n);
+    if (threadIdx.x == 0)
+        tb.bn = bn;
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         const int n = tb.offs[e + 1] - tb.offs[e];
-        tb.ibase[e] = n > 0 ? nrt * ((n + kGBN - 1) / kGBN) : 0;
+        tb.ibase[e] = n > 0 ? nrt * ((n + bn - 1) / bn) : 0;
     }
     __syncthreads();
     const int total = block_exclusive_scan(tb.ibase, E, tb.scan);
@@ -206,23 +225,55 @@ MOE_DEVINL GItem g_item(const GTable &tb, int E, int i)
     GItem it;
     it.e = lo;
     const int ne = tb.offs[lo + 1] - tb.offs[lo];
-    const int nt = (ne + kGBN - 1) / kGBN;
+    const int bn = tb.bn;
+    const int nt = (ne + bn - 1) / bn;
     const int local = i - tb.ibase[lo];
     it.rt = local / nt;
     const int tt = local - it.rt * nt;
-    it.n = min(kGBN, ne - tt * kGBN);
-    it.p0 = tb.offs[lo] + tt * kGBN;
+    it.n = min(bn, ne - tt * bn);
+    it.p0 = tb.offs[lo] + tt * bn;
     return it;
 }
 
 MOE_DEVINL int pad16(int n) { return (n + 15) & ~15; }
 
+// L2 prefetch stream that runs kPF k-blocks ahead of the producer over this
+// CTA's (item, k-block) sequence: the weight tile (two maps for gate / up)
+// and the token tile of that k-block are fetched into L2 early, so the TMA
+// loads behind them find their data there.
+template <int kPF>
+struct GPrefetch {
+    int i, kb, nkb, step, E;
+    GItem it;
+    __device__ void init(const GTable &tb, int E_, int first, int step_, int nkb_, int n_items)
+    {
+        E = E_;
+        i = first;
+        step = step_;
+        nkb = nkb_;
+        kb = 0;
+        if (i < n_items)
+            it = g_item(tb, E, i);
+    }
+    __device__ void next(const GTable &tb, int n_items)
+    {
+        if (++kb == nkb) {
+            kb = 0;
+            i += step;
+            if (i < n_items)
+                it = g_item(tb, E, i);
+        }
+    }
+};
+
 // ---------------------------------------------------------------------------
 struct Gemm1Args {
-    const uint16_t *x;           // [T x d] bf16
+    const uint16_t *wg, *wu;     // [E x I x d] bf16 (the maps' memory, for the L2 prefetch)
     const int32_t *offsets;      // [E + 1]
     const int32_t *sorted_slot;  // [T*k1] slot ids (t*k1 + s) in expert order
     uint16_t *h;                 // [T*k1 x I] bf16, row p = sorted position p
+    float4 *zero;                // nullable: buffer to clear for the down GEMM's combine
+    int zero_n4;
     int T, d, E, I, k1;
     WsHeader *hdr;
 };
@@ -250,7 +301,7 @@ inline size_t gemm2_smem_bytes() { return 1024 + (size_t)kG2Stages * kG2Stage + 
 // columns [0, 256), up accumulator in [256, 512).
 __global__ void __launch_bounds__(kG1Threads, 1)
     k_gemm1(const __grid_constant__ CUtensorMap tm_gate, const __grid_constant__ CUtensorMap tm_up,
-            Gemm1Args a)
+            const __grid_constant__ CUtensorMap tm_xs, Gemm1Args a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *ring = g_align1024(smem_raw);
@@ -261,7 +312,7 @@ __global__ void __launch_bounds__(kG1Threads, 1)
 
     if (tid == 0) {
         for (int s = 0; s < kG1Stages; ++s) {
-            mbar_init(&sy.full[s], 1 + kGGatherThreads);
+            mbar_init(&sy.full[s], 1);
             mbar_init(&sy.empty[s], 1);
         }
         mbar_init(&sy.acc_full[0], 1);
@@ -288,23 +339,48 @@ __global__ void __launch_bounds__(kG1Threads, 1)
     const int n_items = tb.ibase[E];
 
     if (warp == kGWarpTma) {
-        // -------------------------------------------------------- weight tiles
+        // -------------------------------------------------------- weight and token tiles
         if (lane == 0) {
+            constexpr int kPF = 6;
+            GPrefetch<kPF> pf;  // token tiles, kPF k-blocks ahead
+            pf.init(tb, E, blockIdx.x, gridDim.x, nkb, n_items);
+            auto prefetch = [&]() {
+                if (pf.i < n_items)
+                    for (int b = 0; b * 64 < pf.it.n; ++b)
+                        tma_prefetch_2d(&tm_xs, pf.kb * kGBK, pf.it.p0 + 64 * b);
+                pf.next(tb, n_items);
+            };
+            for (int q = 0; q < kPF; ++q)
+                prefetch();
+            auto prefetch_weights = [&](int i) {  // a whole item's gate and up tiles
+                if (i < n_items) {
+                    const GItem w = g_item(tb, E, i);
+                    const size_t r0 = (size_t)w.e * I + w.rt * kGBM;
+                    prefetch_rows_l2(a.wg, r0, kGBM, d);
+                    prefetch_rows_l2(a.wu, r0, kGBM, d);
+                }
+            };
+            prefetch_weights(blockIdx.x);
             uint32_t g = 0;
             for (int i = blockIdx.x; i < n_items && !*(volatile int *)&sy.abort; i += gridDim.x) {
                 const GItem it = g_item(tb, E, i);
                 const int row = it.e * I + it.rt * kGBM;
+                prefetch_weights(i + gridDim.x);  // the next item's, one item ahead
+                const int nb = (it.n + 63) / 64;  // 64-row boxes of the sorted x rows
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
                     const int s = g % kG1Stages;
-                    const uint32_t ph = (g / kG1Stages) & 1;
-                    if (!mbar_wait(&sy.empty[s], ph ^ 1, status)) {
+                    if (!mbar_wait(&sy.empty[s], ((g / kG1Stages) & 1) ^ 1, status)) {
                         sy.abort = 1;
                         break;
                     }
                     uint8_t *st = ring + (size_t)s * kG1Stage;
-                    mbar_arrive_expect_tx(&sy.full[s], 2 * kGTileA);
+                    mbar_arrive_expect_tx(&sy.full[s], 2 * kGTileA + nb * (kGTileB / 4));
                     tma_load_2d(st, &tm_gate, kb * kGBK, row, &sy.full[s]);
                     tma_load_2d(st + kGTileA, &tm_up, kb * kGBK, row, &sy.full[s]);
+                    for (int b = 0; b < nb; ++b)
+                        tma_load_2d(st + 2 * kGTileA + b * (kGTileB / 4), &tm_xs, kb * kGBK,
+                                    it.p0 + 64 * b, &sy.full[s]);
+                    prefetch();
                 }
             }
             // drain: every stage issued has landed before the CTA may leave
@@ -351,52 +427,11 @@ __global__ void __launch_bounds__(kG1Threads, 1)
             umma_commit(&sy.drained);
             mbar_wait(&sy.drained, 0, status);
         }
-    } else if (warp >= 6) {
-        // -------------------------------------------------------- token gather
-        const int gt = tid - 6 * 32;  // 0..127
-        const int c = gt & 7;         // 16-byte chunk of the 128-byte row
-        const int rb = gt >> 3;       // rows rb + 16 j
-        const int k1 = a.k1;
-        uint32_t g = 0;
-        for (int i = blockIdx.x; i < n_items && !*(volatile int *)&sy.abort; i += gridDim.x) {
-            const GItem it = g_item(tb, E, i);
-            const int npad = pad16(it.n);
-            int tok[kGBN / 16];
-#pragma unroll
-            for (int j = 0; j < kGBN / 16; ++j) {
-                const int r = min(rb + 16 * j, it.n - 1);
-                tok[j] = __ldcg(&a.sorted_slot[it.p0 + r]) / k1;
-            }
-            for (int kb = 0; kb < nkb; ++kb, ++g) {
-                const int s = g % kG1Stages;
-                if (!mbar_wait(&sy.empty[s], ((g / kG1Stages) & 1) ^ 1, status)) {
-                    sy.abort = 1;
-                    break;
-                }
-                const uint32_t bst = smem_addr(ring + (size_t)s * kG1Stage + 2 * kGTileA);
-#pragma unroll
-                for (int j = 0; j < kGBN / 16; ++j) {
-                    const int r = rb + 16 * j;
-                    if (r < npad)
-                        cp_async16(bst + r * 128 + ((c ^ (r & 7)) << 4),
-                                   a.x + (size_t)tok[j] * d + kb * kGBK + c * 8);
-                }
-                cp_async_commit();
-                if (g >= kG1Stages - 1) {
-                    cp_async_wait<kG1Stages - 1>();
-                    fence_proxy_async_smem();
-                    mbar_arrive(&sy.full[(g - (kG1Stages - 1)) % kG1Stages]);
-                }
-            }
-        }
-        // the last stages' copies
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
-        const uint32_t lo = g > (uint32_t)(kG1Stages - 1) ? g - (kG1Stages - 1) : 0;
-        for (uint32_t q = lo; q < g; ++q)
-            mbar_arrive(&sy.full[q % kG1Stages]);
     } else {
         // -------------------------------------------------------- epilogue (warps 0-3)
+        if (a.zero)  // the down GEMM's accumulator (read only after this grid completes)
+            for (int q = blockIdx.x * kGEpiThreads + tid; q < a.zero_n4; q += gridDim.x * kGEpiThreads)
+                a.zero[q] = make_float4(0.f, 0.f, 0.f, 0.f);
         uint32_t itc = 0;
         const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
         for (int i = blockIdx.x; i < n_items && !*(volatile int *)&sy.abort; i += gridDim.x, ++itc) {
@@ -434,12 +469,17 @@ __global__ void __launch_bounds__(kG1Threads, 1)
 
 // ---------------------------------------------------------------------------
 struct Gemm2Args {
-    const int32_t *offsets;      // [E + 1]
+    const uint16_t *wd;          // [E x d x I] bf16 (the weight map's memory, for the L2 prefetch)
+    const int32_t *offsets;      // [E + 1]; nullptr: one group of single_n rows
     const int32_t *sorted_slot;  // [T*k1]
     const float *topk_w;         // [T*k1] Eq. 2 weights by slot (combine mode)
     float *y_acc;                // [T x d] float32, zero on entry (combine mode)
-    float *out;                  // [T*k1 x d] float32 per sorted position (out mode)
-    int T, d, E, I, k1;
+    float *out;                  // [rows x d] float32 per sorted position (store mode)
+    float *out_copy;             // nullable second destination of the store mode
+    const float *bias;           // nullable [d], added in the store mode
+    int single_n;
+    int bn;                      // tokens per tile: kGBN, or 64 to spread a small job
+    int T, d, E, I, k1;          // d: output rows of the weight matrix, I: K
     int combine;                 // 1: weighted red.add into y_acc; 0: store rows of out
     WsHeader *hdr;
 };
@@ -484,15 +524,34 @@ __global__ void __launch_bounds__(kG2Threads, 1)
     const int d = a.d, E = a.E, I = a.I;
     const int nrt = d / kGBM;
     const int nkb = I / kGBK;
-    g_build_items(a.offsets, E, nrt, tb);
+    g_build_items(a.offsets, E, nrt, tb, a.single_n, a.bn > 0 ? a.bn : kGBN);
     const int n_items = tb.ibase[E];
 
     if (warp == kGWarpTma) {
         if (lane == 0) {
+            constexpr int kPF = 8;
+            GPrefetch<kPF> pf;  // token tiles, kPF k-blocks ahead
+            pf.init(tb, E, blockIdx.x, gridDim.x, nkb, n_items);
+            auto prefetch = [&]() {
+                if (pf.i < n_items)
+                    for (int b = 0; b * 64 < pf.it.n; ++b)
+                        tma_prefetch_2d(&tm_h, pf.kb * kGBK, pf.it.p0 + 64 * b);
+                pf.next(tb, n_items);
+            };
+            for (int q = 0; q < kPF; ++q)
+                prefetch();
+            auto prefetch_weights = [&](int i) {  // a whole item's weight tile
+                if (i < n_items) {
+                    const GItem w = g_item(tb, E, i);
+                    prefetch_rows_l2(a.wd, (size_t)w.e * d + w.rt * kGBM, kGBM, I);
+                }
+            };
+            prefetch_weights(blockIdx.x);
             uint32_t g = 0;
             for (int i = blockIdx.x; i < n_items && !*(volatile int *)&sy.abort; i += gridDim.x) {
                 const GItem it = g_item(tb, E, i);
                 const int row = it.e * d + it.rt * kGBM;
+                prefetch_weights(i + gridDim.x);  // the next item's, one item ahead
                 const int nb = (it.n + 63) / 64;  // 64-row boxes of H
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
                     const int s = g % kG2Stages;
@@ -506,6 +565,7 @@ __global__ void __launch_bounds__(kG2Threads, 1)
                     for (int b = 0; b < nb; ++b)
                         tma_load_2d(st + kGTileA + b * (kGTileB / 4), &tm_h, kb * kGBK,
                                     it.p0 + 64 * b, &sy.full[s]);
+                    prefetch();
                 }
             }
             const uint32_t n_iss = g;
@@ -588,10 +648,16 @@ __global__ void __launch_bounds__(kG2Threads, 1)
                                 atomicAdd(&a.y_acc[(size_t)t * d + r], w * v[j]);
                         }
                     } else {
+                        const float b = a.bias ? __ldg(&a.bias[r]) : 0.0f;
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
-                            if (q * 32 + j < it.n)
-                                a.out[(size_t)(it.p0 + q * 32 + j) * d + r] = v[j];
+                            if (q * 32 + j < it.n) {
+                                const size_t o = (size_t)(it.p0 + q * 32 + j) * d + r;
+                                const float val = a.bias ? __fadd_rn(v[j], b) : v[j];
+                                a.out[o] = val;
+                                if (a.out_copy)
+                                    a.out_copy[o] = val;
+                            }
                     }
                 }
             }
@@ -607,6 +673,24 @@ __global__ void __launch_bounds__(kG2Threads, 1)
     if (warp == kGWarpMma) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
+    }
+}
+
+// xs[p] = x[sorted_slot[p] / k1]: the routed tokens' rows in expert order, the
+// token operand of the gate/up GEMM.  One warp per row, 16-byte vectors.
+__global__ void __launch_bounds__(256) k_gather_rows(const uint16_t *x, const int32_t *sorted_slot,
+                                                     int n, int d, int k1, uint16_t *xs)
+{
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int nv = d >> 3;
+    for (int p = blockIdx.x * 8 + (threadIdx.x >> 5); p < n; p += gridDim.x * 8) {
+        const int t = __ldcg(&sorted_slot[p]) / k1;
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * d);
+        uint4 *dst = reinterpret_cast<uint4 *>(xs + (size_t)p * d);
+        for (int v = lane; v < nv; v += 32)
+            dst[v] = __ldg(&src[v]);
     }
 }
 

@@ -30,8 +30,10 @@ static inline size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct WsLayout {
     size_t logits, idx, w, offsets, sorted_slot, slot_pos, uniq_count, uniq_list, h, out, y_acc,
-        total;
+        hist, total;
 };
+
+static inline int perm_chunks(int T) { return (T + kPermTok - 1) / kPermTok; }
 
 static WsLayout ws_layout(int T, int d, int E, int I, int k1)
 {
@@ -49,6 +51,7 @@ static WsLayout ws_layout(int T, int d, int E, int I, int k1)
     L.h = o;           o = align256(o + sizeof(float) * n * (size_t)I);
     L.out = o;         o = align256(o + sizeof(float) * n * (size_t)d);
     L.y_acc = o;       o = align256(o + sizeof(float) * (size_t)T * d);
+    L.hist = o;        o = align256(o + sizeof(int32_t) * (size_t)perm_chunks(T) * E);
     L.total = o;
     return L;
 }
@@ -189,9 +192,9 @@ static int enqueue_logits(const void *x, const void *wr, const float *bias, floa
 }
 
 // The single-pass decode path of moe_layer after the router (T == 1, down
-// matrix channel-major): the decode kernel (routing, gate/up, down partials
-// into y_acc) and the finalize kernel (y_acc -> y).  y_acc was cleared by the
-// router kernel.
+// matrix channel-major): one decode kernel (routing, gate/up, down partials
+// into y_acc, y written by its last CTA).  y_acc was cleared by the router
+// kernel.
 static int enqueue_decode(const void *x, const void *wg, const void *wu, const void *wdt, int d,
                           int E, int I, int k1, int k2, void *y, int y_dtype, int32_t *idx_copy,
                           float *w_copy, void *ws, int G, cudaStream_t s)
@@ -218,19 +221,15 @@ static int enqueue_decode(const void *x, const void *wg, const void *wu, const v
     a.uniq_count = at<int32_t>(ws, L.uniq_count);
     a.uniq_list = at<int32_t>(ws, L.uniq_list);
     a.y_acc = at<float>(ws, L.y_acc);
+    a.y = y;
+    a.y_dtype = y_dtype;
     a.hdr = static_cast<WsHeader *>(ws);
     const size_t smem = decode_smem_bytes(d);
-    int rc;
     if (d == 2048)
-        rc = launch(k_decode<8>, dim3(G), dim3(kSThreads), smem, s, true, a);
-    else if (d == 4096)
-        rc = launch(k_decode<16>, dim3(G), dim3(kSThreads), smem, s, true, a);
-    else
-        rc = launch(k_decode<0>, dim3(G), dim3(kSThreads), smem, s, true, a);
-    if (rc != MOE_OK)
-        return rc;
-    return launch(k_finalize, dim3((d / 4 + 255) / 256), dim3(256), 0, s, true,
-                  (const float *)at<float>(ws, L.y_acc), d, y, y_dtype);
+        return launch(k_decode<8>, dim3(G), dim3(kSThreads), smem, s, true, a);
+    if (d == 4096)
+        return launch(k_decode<16>, dim3(G), dim3(kSThreads), smem, s, true, a);
+    return launch(k_decode<0>, dim3(G), dim3(kSThreads), smem, s, true, a);
 }
 
 
@@ -279,34 +278,51 @@ static int bf16_tile_map(CUtensorMap *m, const void *base, uint64_t inner, uint6
 // The two grouped GEMMs over routed slots already grouped by expert
 // (offsets / sorted_slot).  combine: weighted red.add into y_acc (zeroed
 // before); otherwise per-slot rows of `out` in sorted order.
+// which: 4 gathers the token rows into expert order (xs), 1 runs the gate/up
+// GEMM, 2 the down GEMM (7: the whole expert FFN).
 static int enqueue_grouped(const void *x, const void *wg, const void *wu, const void *wd, int T,
                            int d, int E, int I, int k1, const int32_t *offsets,
-                           const int32_t *sorted_slot, const float *topk_w, uint16_t *h,
-                           float *y_acc, float *out, WsHeader *hdr, int G, cudaStream_t s)
+                           const int32_t *sorted_slot, const float *topk_w, uint16_t *xs,
+                           uint16_t *h, float *y_acc, float *out, WsHeader *hdr, int G,
+                           cudaStream_t s, int which = 7, bool pdl = true)
 {
-    CUtensorMap tg, tu, td, th;
+    CUtensorMap tg, tu, tx, td, th;
     int rc;
     const uint64_t n = (uint64_t)T * k1;
     if ((rc = bf16_tile_map(&tg, wg, d, (uint64_t)E * I, kGBM)) != MOE_OK ||
         (rc = bf16_tile_map(&tu, wu, d, (uint64_t)E * I, kGBM)) != MOE_OK ||
+        (rc = bf16_tile_map(&tx, xs, d, n, 64)) != MOE_OK ||
         (rc = bf16_tile_map(&td, wd, I, (uint64_t)E * d, kGBM)) != MOE_OK ||
         (rc = bf16_tile_map(&th, h, I, n, 64)) != MOE_OK)
         return rc;
+    if (which & 4) {
+        const int rows = (int)n;
+        const int grid = (rows + 7) / 8 < 8 * G ? (rows + 7) / 8 : 8 * G;
+        if ((rc = launch(k_gather_rows, dim3(grid), dim3(256), 0, s, pdl,
+                         static_cast<const uint16_t *>(x), sorted_slot, rows, d, k1, xs)) != MOE_OK)
+            return rc;
+    }
     Gemm1Args a1 = {};
-    a1.x = static_cast<const uint16_t *>(x);
+    a1.wg = static_cast<const uint16_t *>(wg);
+    a1.wu = static_cast<const uint16_t *>(wu);
     a1.offsets = offsets;
     a1.sorted_slot = sorted_slot;
     a1.h = h;
+    a1.zero = reinterpret_cast<float4 *>(y_acc);
+    a1.zero_n4 = y_acc ? T * d / 4 : 0;
     a1.T = T;
     a1.d = d;
     a1.E = E;
     a1.I = I;
     a1.k1 = k1;
     a1.hdr = hdr;
-    if ((rc = launch(k_gemm1, dim3(G), dim3(kG1Threads), gemm1_smem_bytes(), s, true, tg, tu,
-                     a1)) != MOE_OK)
+    if ((which & 1) && (rc = launch(k_gemm1, dim3(G), dim3(kG1Threads), gemm1_smem_bytes(), s,
+                                    pdl, tg, tu, tx, a1)) != MOE_OK)
         return rc;
+    if (!(which & 2))
+        return MOE_OK;
     Gemm2Args a2 = {};
+    a2.wd = static_cast<const uint16_t *>(wd);
     a2.offsets = offsets;
     a2.sorted_slot = sorted_slot;
     a2.topk_w = topk_w;
@@ -319,7 +335,69 @@ static int enqueue_grouped(const void *x, const void *wg, const void *wu, const 
     a2.k1 = k1;
     a2.combine = y_acc != nullptr;
     a2.hdr = hdr;
-    return launch(k_gemm2, dim3(G), dim3(kG2Threads), gemm2_smem_bytes(), s, true, td, th, a2);
+    return launch(k_gemm2, dim3(G), dim3(kG2Threads), gemm2_smem_bytes(), s, pdl, td, th, a2);
+}
+
+// Router logits of a large batch as a tensor-core GEMM (the down-GEMM kernel
+// with W_r as the weight matrix, the tokens in order as one group, bias added
+// in the epilogue): needs whole 128-row tiles of experts.
+static bool gemm_logits_ok(int T, int d, int E) { return E % kGBM == 0 && E <= kGMaxE && T >= 256; }
+
+static int enqueue_logits_gemm(const void *x, const void *wr, const float *bias, float *z,
+                               float *z_copy, int T, int d, int E, WsHeader *hdr, int G,
+                               cudaStream_t s)
+{
+    CUtensorMap tw, tx;
+    int rc;
+    if ((rc = bf16_tile_map(&tw, wr, d, E, kGBM)) != MOE_OK ||
+        (rc = bf16_tile_map(&tx, x, d, T, 64)) != MOE_OK)
+        return rc;
+    Gemm2Args a = {};
+    a.wd = static_cast<const uint16_t *>(wr);
+    a.out = z;
+    a.out_copy = z_copy;
+    a.bias = bias;
+    a.single_n = T;
+    a.bn = 64;  // 64-token tiles: enough work items to spread over the SMs
+    a.T = T;
+    a.d = E;  // output rows: the experts
+    a.I = d;  // K: the hidden size
+    a.E = 1;  // one group: every token
+    a.k1 = 1;
+    a.combine = 0;
+    a.hdr = hdr;
+    return launch(k_gemm2, dim3(G), dim3(kG2Threads), gemm2_smem_bytes(), s, true, tw, tx, a);
+}
+
+// Warp-per-token routing of T tokens from float32 logits.
+static int enqueue_route_warp(const float *z, int T, int E, int k1, int k2, int32_t *idx, float *w,
+                              int32_t *idx_copy, float *w_copy, cudaStream_t s)
+{
+    const dim3 grid((T + 7) / 8), block(256);
+#define MOE_ROUTE_WARP(R)                                                                        \
+    return launch(k_route_warp<R>, grid, block, 0, s, true, z, T, E, k1, k2, idx, w, idx_copy, \
+                  w_copy)
+    if (E <= 32) MOE_ROUTE_WARP(1);
+    if (E <= 64) MOE_ROUTE_WARP(2);
+    if (E <= 128) MOE_ROUTE_WARP(4);
+    if (E <= 256) MOE_ROUTE_WARP(8);
+    if (E <= 512) MOE_ROUTE_WARP(16);
+    MOE_ROUTE_WARP(32);
+#undef MOE_ROUTE_WARP
+}
+
+// Stable counting sort of T*k1 slots over chunks of kPermTok tokens (no
+// unique-expert list); hist: perm_chunks(T) x E ints of scratch.
+static int enqueue_perm_parallel(const int32_t *idx, int T, int k1, int E, int *hist, PermOut po,
+                                 int *status, cudaStream_t s)
+{
+    const int nch = perm_chunks(T);
+    int rc;
+    if ((rc = launch(k_perm_hist, dim3(nch), dim3(256), perm_hist_smem_bytes(E, k1), s, true, idx,
+                     T, k1, E, hist, status)) != MOE_OK)
+        return rc;
+    return launch(k_perm_scatter, dim3(nch), dim3(256), perm_scatter_smem_bytes(E, k1), s, true,
+                  idx, T, k1, E, (const int *)hist, po);
 }
 
 // AUTO's choice of the tensor-core path: enough routed slots per expert to
@@ -430,10 +508,7 @@ int moe_route(const void *x_bf16, const void *w_router_bf16, const float *bias, 
             return rc;
         z = zbuf;
     }
-    PermOut none = {};
-    return launch(k_topk, dim3(T), dim3(topk_threads(E)), 0, s, true, z, T, E, k1, k2, topk_idx,
-                  topk_w, (int32_t *)nullptr, (float *)nullptr, none,
-                  ws ? static_cast<WsHeader *>(ws) : (WsHeader *)nullptr);
+    return enqueue_route_warp(z, T, E, k1, k2, topk_idx, topk_w, nullptr, nullptr, s);
 }
 
 int moe_permute(const int32_t *topk_idx, int T, int k1, int E, int32_t *expert_offsets,
@@ -456,6 +531,11 @@ int moe_permute(const int32_t *topk_idx, int T, int k1, int E, int32_t *expert_o
         return rc;
     PermOut po = {expert_offsets, sorted_slot, slot_pos, nullptr, nullptr};
     int *status = ws ? &static_cast<WsHeader *>(ws)->status : nullptr;
+    // many slots and room for the chunk counts after the header: chunked kernels
+    const size_t hist_bytes = sizeof(int) * (size_t)perm_chunks(T) * E;
+    if ((long)T * k1 > 4096 && ws && ws_bytes >= sizeof(WsHeader) + hist_bytes)
+        return enqueue_perm_parallel(topk_idx, T, k1, E, at<int>(ws, sizeof(WsHeader)), po, status,
+                                     s);
     return launch(k_permute, dim3(1), dim3(1024), permute_smem_bytes(E, T), s, true, topk_idx, T,
                   k1, E, po, status);
 }
@@ -589,8 +669,9 @@ int moe_expert_ffn(const void *x_bf16, const int32_t *expert_offsets, const int3
         if (!grouped_fits(d, E, I))
             return MOE_ERR_UNSUPPORTED_SHAPE;
         return enqueue_grouped(x_bf16, w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I, k1,
-                               expert_offsets, sorted_slot, nullptr, at<uint16_t>(ws, L.h),
-                               nullptr, out, static_cast<WsHeader *>(ws), di->num_sms, s);
+                               expert_offsets, sorted_slot, nullptr, at<uint16_t>(ws, L.out),
+                               at<uint16_t>(ws, L.h), nullptr, out, static_cast<WsHeader *>(ws),
+                               di->num_sms, s);
     }
     if ((rc = launch(k_uniq_from_offsets, dim3(1), dim3(1024), 0, s, true, expert_offsets, E,
                      at<int32_t>(ws, L.uniq_count), at<int32_t>(ws, L.uniq_list))) != MOE_OK)
@@ -684,26 +765,38 @@ int moe_layer(const void *x_bf16, const void *w_router_bf16, const float *bias,
                                       (path == MOE_PATH_AUTO && auto_grouped(T, d, E, I, k1)));
     if (grouped && !grouped_fits(d, E, I))
         return MOE_ERR_UNSUPPORTED_SHAPE;
-    float4 *y_acc = decode || grouped ? at<float4>(ws, L.y_acc) : nullptr;
+    if (grouped) {
+        // router logits (tensor-core GEMM when the experts fill 128-row tiles),
+        // warp-per-token routing, the chunked stable permutation, the two
+        // grouped GEMMs (the first clears y_acc for the second's combine), y
+        if (gemm_logits_ok(T, d, E))
+            rc = enqueue_logits_gemm(x_bf16, w_router_bf16, bias, z, logits_out, T, d, E, hdr, G, s);
+        else
+            rc = enqueue_logits(x_bf16, w_router_bf16, bias, z, logits_out, T, d, E, s);
+        if (rc != MOE_OK)
+            return rc;
+        if ((rc = enqueue_route_warp(z, T, E, k1, k2, idx, w, topk_idx_out, topk_w_out, s)) !=
+            MOE_OK)
+            return rc;
+        if ((rc = enqueue_perm_parallel(idx, T, k1, E, at<int>(ws, L.hist), po, &hdr->status, s)) !=
+            MOE_OK)
+            return rc;
+        if ((rc = enqueue_grouped(x_bf16, w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I, k1,
+                                  po.offsets, po.sorted_slot, w, at<uint16_t>(ws, L.out),
+                                  at<uint16_t>(ws, L.h), at<float>(ws, L.y_acc), nullptr, hdr, G,
+                                  s)) != MOE_OK)
+            return rc;
+        const int n = T * d;
+        return launch(k_finalize, dim3((n / 4 + 255) / 256), dim3(256), 0, s, true,
+                      (const float *)at<float>(ws, L.y_acc), n, y, y_dtype);
+    }
+    float4 *y_acc = decode ? at<float4>(ws, L.y_acc) : nullptr;
     if ((rc = enqueue_logits(x_bf16, w_router_bf16, bias, z, logits_out, T, d, E, s, y_acc,
                              T * d / 4)) != MOE_OK)
         return rc;
     if (decode)
         return enqueue_decode(x_bf16, w_gate_bf16, w_up_bf16, w_down_bf16, d, E, I, k1, k2, y,
                               y_dtype, topk_idx_out, topk_w_out, ws, G, s);
-    if (grouped) {
-        if ((rc = launch(k_topk, dim3(T), dim3(topk_threads(E)), permute_smem_bytes(E, T), s, true,
-                         (const float *)z, T, E, k1, k2, idx, w, topk_idx_out, topk_w_out, po,
-                         hdr)) != MOE_OK)
-            return rc;
-        if ((rc = enqueue_grouped(x_bf16, w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I, k1,
-                                  po.offsets, po.sorted_slot, w, at<uint16_t>(ws, L.h),
-                                  at<float>(ws, L.y_acc), nullptr, hdr, G, s)) != MOE_OK)
-            return rc;
-        const int n = T * d;
-        return launch(k_finalize, dim3((n / 4 + 255) / 256), dim3(256), 0, s, true,
-                      (const float *)at<float>(ws, L.y_acc), n, y, y_dtype);
-    }
     if (T > 1) {
         // one CTA per token ranks its probabilities; the last one to finish
         // builds the permutation tables
@@ -789,6 +882,8 @@ int moe_test_expert_stream(const void *x_bf16, const void *w_gate_bf16, const vo
         a.uniq_count = at<int32_t>(ws, L.uniq_count);
         a.uniq_list = at<int32_t>(ws, L.uniq_list);
         a.y_acc = at<float>(ws, L.y_acc);
+        a.y = y;
+        a.y_dtype = y_dtype;
         a.hdr = static_cast<WsHeader *>(ws);
         const size_t smem = decode_smem_bytes(d);
         if (d == 2048)
@@ -808,6 +903,43 @@ int moe_test_num_sms(void)
     if (device_info(di) != MOE_OK)
         return 0;
     return di->num_sms;
+}
+
+int moe_test_expert_grouped(const void *x_bf16, const void *w_gate_bf16, const void *w_up_bf16,
+                            const void *w_down_bf16, int T, int d, int E, int I, int k1, int which,
+                            void *ws, size_t ws_bytes, void *stream)
+{
+    int rc = check_shape(T, d, E, I, k1);
+    if (rc != MOE_OK)
+        return rc;
+    if (which < 1 || which > 8)
+        return MOE_ERR_INVALID_ARG;
+    if (!grouped_fits(d, E, I))
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (T == 0)
+        return MOE_OK;
+    if (!x_bf16 || !w_gate_bf16 || !w_up_bf16 || !w_down_bf16 || !ws)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x_bf16) || !aligned16(w_gate_bf16) || !aligned16(w_up_bf16) ||
+        !aligned16(w_down_bf16) || (reinterpret_cast<uintptr_t>(ws) & 255))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(T, d, E, I, k1);
+    if (ws_bytes < L.total)
+        return MOE_ERR_WORKSPACE_TOO_SMALL;
+    DevInfo *di;
+    if ((rc = device_info(di)) != MOE_OK)
+        return rc;
+    if (which & 8)  // the down GEMM storing per-slot rows (the moe_expert_ffn epilogue)
+        return enqueue_grouped(x_bf16, w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I, k1,
+                               at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.sorted_slot),
+                               nullptr, at<uint16_t>(ws, L.out), at<uint16_t>(ws, L.h), nullptr,
+                               at<float>(ws, L.out), static_cast<WsHeader *>(ws), di->num_sms,
+                               static_cast<cudaStream_t>(stream), 2, false);
+    return enqueue_grouped(x_bf16, w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I, k1,
+                           at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.sorted_slot),
+                           at<float>(ws, L.w), at<uint16_t>(ws, L.out), at<uint16_t>(ws, L.h),
+                           at<float>(ws, L.y_acc), nullptr, static_cast<WsHeader *>(ws),
+                           di->num_sms, static_cast<cudaStream_t>(stream), which, false);
 }
 
 }  // extern "C"

@@ -397,6 +397,202 @@ __global__ void __launch_bounds__(1024) k_topk(const float *logits, int T, int E
 }
 
 // ---------------------------------------------------------------------------
+// warp_route: one warp routes one token from its E float32 logits z (global
+// memory), everything in registers.  Lane l holds logits j = l, l+32, ...
+// (R per lane, E <= 32 R), which is exactly the canonical partial-sum
+// assignment of the normaliser Z; the top-Kneed probabilities come out in
+// rank order by repeated warp arg-max on (p descending, j ascending) -- two
+// redux.sync per rank: the largest key, then the lowest index holding it --
+// so the top-k2 mass S is summed in rank order as it is found.  Same float
+// sequence, same bits as route_token_block.  Lane s < k1 returns the rank-s
+// expert in my_j and its Eq. 2 weight in my_w.  k_route_warp: one warp per
+// token of a batch.
+template <int R>
+__device__ __forceinline__ void warp_route(const float *z, int E, int k1, int k2, int lane,
+                                           int &my_j, float &my_w)
+{
+    const float kNegInf = -__int_as_float(0x7f800000);
+    float p[R];
+    float m = kNegInf;
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+        const int j = lane + 32 * i;
+        p[i] = j < E ? __ldcg(&z[j]) : kNegInf;
+        m = fmaxf(m, p[i]);
+    }
+    asm volatile("redux.sync.max.f32 %0, %0, 0xffffffff;" : "+f"(m));  // exact in any order
+    float Z = 0.0f;
+#pragma unroll
+    for (int i = 0; i < R; ++i)
+        if (lane + 32 * i < E) {
+            p[i] = expc(__fsub_rn(p[i], m));
+            Z = __fadd_rn(Z, p[i]);
+        }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1)
+        Z = __fadd_rn(Z, __shfl_xor_sync(0xffffffffu, Z, o));
+    // key = bits of p + 1 (p >= 0, so the bits order like the values); 0 = taken / absent
+    unsigned key[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i)
+        key[i] = lane + 32 * i < E ? __float_as_uint(__fdiv_rn(p[i], Z)) + 1u : 0u;
+
+    const int K = k2 < E ? k2 : E;
+    const bool renorm = k2 < E;
+    const int Kneed = renorm ? K : k1;
+    float S = 0.0f, my_p = 0.0f;
+    my_j = 0;
+    for (int r = 0; r < Kneed; ++r) {
+        unsigned kl = 0u;
+        int jl = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < R; ++i)
+            if (key[i] > kl) {  // strict: the lowest j among equal p in this lane
+                kl = key[i];
+                jl = lane + 32 * i;
+            }
+        const unsigned km = __reduce_max_sync(0xffffffffu, kl);
+        const int bj = (int)__reduce_min_sync(0xffffffffu, kl == km ? (unsigned)jl : 0xffffffffu);
+        const float bp = __uint_as_float(km - 1u);
+        if (lane == r) {
+            my_j = bj;
+            my_p = bp;
+        }
+        if (renorm)
+            S = __fadd_rn(S, bp);
+#pragma unroll
+        for (int i = 0; i < R; ++i)
+            if (lane + 32 * i == bj)
+                key[i] = 0u;
+    }
+    my_w = renorm ? __fdiv_rn(my_p, S) : my_p;
+}
+
+template <int R>
+__global__ void __launch_bounds__(256) k_route_warp(const float *logits, int T, int E, int k1,
+                                                    int k2, int32_t *idx, float *w,
+                                                    int32_t *idx_copy, float *w_copy)
+{
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= T)
+        return;
+    int my_j;
+    float my_w;
+    warp_route<R>(logits + (size_t)t * E, E, k1, k2, lane, my_j, my_w);
+    if (lane < k1) {
+        const size_t o = (size_t)t * k1 + lane;
+        idx[o] = my_j;
+        w[o] = my_w;
+        if (idx_copy)
+            idx_copy[o] = my_j;
+        if (w_copy)
+            w_copy[o] = my_w;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Large-batch permutation in two kernels over chunks of kPermTok tokens.
+// k_perm_hist: per-chunk expert counts into hist[chunk][E] (and the range /
+// repeat checks of the expert ids).  k_perm_scatter: every chunk turns the
+// counts into its starting position per expert (offsets of all experts plus
+// the counts of earlier chunks) and one warp walks the chunk's slots in
+// order, so the sort is stable by slot index.
+constexpr int kPermTok = 128;
+
+__global__ void __launch_bounds__(256) k_perm_hist(const int32_t *idx, int T, int k1, int E,
+                                                   int *hist, int *status)
+{
+    extern __shared__ int hsm[];  // cnt[E], ids[kPermTok * k1]
+    int *cnt = hsm, *ids = hsm + E;
+    pdl_wait();
+    pdl_trigger();
+    const int tid = threadIdx.x, nt = blockDim.x, b = blockIdx.x;
+    for (int e = tid; e < E; e += nt)
+        cnt[e] = 0;
+    const int t0 = b * kPermTok, t1 = min(T, t0 + kPermTok);
+    const int i0 = t0 * k1, m = (t1 - t0) * k1;
+    for (int i = tid; i < m; i += nt)
+        ids[i] = __ldcg(&idx[i0 + i]);
+    __syncthreads();
+    for (int i = tid; i < m; i += nt) {
+        const int e = ids[i];
+        if (e < 0 || e >= E) {
+            set_status(status, MOE_ERR_DEVICE_CHECK);
+            continue;
+        }
+        atomicAdd(&cnt[e], 1);
+        for (int q = i - i % k1; q < i; ++q)  // the same expert earlier in this token
+            if (ids[q] == e)
+                set_status(status, MOE_ERR_DEVICE_CHECK);
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += nt)
+        hist[(size_t)b * E + e] = cnt[e];
+}
+
+__global__ void __launch_bounds__(256) k_perm_scatter(const int32_t *idx, int T, int k1, int E,
+                                                      const int *hist, PermOut out)
+{
+    extern __shared__ int psm[];  // base[E], run[E], tot[E + 1], scan[40], ids[kPermTok * k1]
+    pdl_wait();
+    pdl_trigger();
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, b = blockIdx.x;
+    const int nch = gridDim.x;
+    int *base = psm, *run = base + E, *tot = run + E, *scan = tot + E + 1, *ids = scan + 40;
+    const int i0 = b * kPermTok * k1, i1 = min(T, (b + 1) * kPermTok) * k1;
+    for (int i = tid; i < i1 - i0; i += nt)
+        ids[i] = __ldcg(&idx[i0 + i]);
+    for (int e = tid; e < E; e += nt) {
+        int before = 0, all = 0;
+        for (int c = 0; c < nch; ++c) {
+            const int h = __ldcg(&hist[(size_t)c * E + e]);
+            all += h;
+            before += c < b ? h : 0;
+        }
+        base[e] = before;
+        tot[e] = all;
+        run[e] = 0;
+    }
+    if (tid == 0)
+        tot[E] = 0;
+    __syncthreads();
+    block_exclusive_scan(tot, E + 1, scan);  // tot[e] = offsets[e], tot[E] = T*k1 (valid ids)
+    if (b == 0)
+        for (int e = tid; e <= E; e += nt)
+            out.offsets[e] = tot[e];
+    for (int e = tid; e < E; e += nt)
+        base[e] += tot[e];
+    __syncthreads();
+    if (tid < 32) {
+        const unsigned lt = (1u << lane) - 1u;
+        for (int i = i0; i < i1; i += 32) {
+            const int slot = i + lane;
+            const int e = slot < i1 ? ids[slot - i0] : -1;
+            const bool valid = e >= 0 && e < E;
+            const unsigned grp = __match_any_sync(0xffffffffu, valid ? e : -1);
+            if (valid) {
+                const int pos = base[e] + run[e] + __popc(grp & lt);
+                out.sorted_slot[pos] = slot;
+                out.slot_pos[slot] = pos;
+            }
+            __syncwarp();
+            if (valid && lane == __ffs(grp) - 1)
+                run[e] += __popc(grp);
+            __syncwarp();
+        }
+    }
+}
+
+inline size_t perm_hist_smem_bytes(int E, int k1) { return sizeof(int) * ((size_t)E + kPermTok * k1); }
+inline size_t perm_scatter_smem_bytes(int E, int k1)
+{
+    return sizeof(int) * ((size_t)3 * E + 1 + 40 + kPermTok * k1);
+}
+
+// ---------------------------------------------------------------------------
 // k_logits: z[t, e] = sum_k x[t, k] W_r[e, k] (+ b[e]) with float32
 // accumulation.  One warp per (expert, chunk of up to 8 tokens).  The warp's
 // W_r row is loaded into registers before the programmatic-launch wait (the

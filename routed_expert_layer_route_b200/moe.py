@@ -56,6 +56,7 @@ SIGNATURES = {
     "moe_test_num_sms": (_i, []),
     "moe_test_expert_stream": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _i, _vp,
                                     _sz, _vp]),
+    "moe_test_expert_grouped": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
 }
 
 _lib = None
@@ -236,3 +237,15 @@ def moe_test_expert_stream(x, w_gate, w_up, w_down, k1, k2, y, ws, flags=MOE_PAT
     _check(lib().moe_test_expert_stream(_p(x), _p(w_gate), _p(w_up), _p(w_down), T, d, E, I, k1,
                                         k2, _p(y), y_dtype, flags, wsp, wsn, _stream(stream)),
            "moe_test_expert_stream")
+
+
+def moe_test_expert_grouped(x, w_gate, w_up, w_down, k1, which, ws, stream=None):
+    """Kernels of the grouped expert FFN alone (which, a bit set: 4 token-row
+    gather, 1 gate/up GEMM, 2 down GEMM) on the routing tables a previous
+    moe_layer call left in ws."""
+    T, d = x.shape
+    E, I, _ = w_gate.shape
+    wsp, wsn = _ws_args(ws)
+    _check(lib().moe_test_expert_grouped(_p(x), _p(w_gate), _p(w_up), _p(w_down), T, d, E, I, k1,
+                                         which, wsp, wsn, _stream(stream)),
+           "moe_test_expert_grouped")

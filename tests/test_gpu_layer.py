@@ -217,6 +217,8 @@ GSMALL = [
     (200, 512, 32, 384, 8, 8, "zipf"),   # ragged tiles, experts without tokens
     (37, 384, 64, 128, 3, 1000, None),
     (130, 128, 2, 256, 2, 2, None),      # k1 = E: every token in every expert
+    (256, 256, 128, 128, 4, 16, "normal"),  # router logits on the tensor cores too
+    (300, 128, 256, 128, 6, 6, None),    # two 128-expert logit tiles, ragged token tile
 ]
 
 

@@ -127,6 +127,34 @@ def test_permute_exact(T, k1, E):
     assert np.array_equal(g_off.cpu().numpy(), off)
     assert np.array_equal(g_ss.cpu().numpy(), ss)
     assert np.array_equal(g_sp.cpu().numpy(), sp)
+    if T * k1 > 4096:  # with a workspace: the chunked two-kernel sort
+        ws = moe.workspace(T, 64, E, 16, k1, device=DEV)
+        for t in (g_off, g_ss, g_sp):
+            t.fill_(-7)
+        moe.moe_permute(ti, E, g_off, g_ss, g_sp, ws=ws)
+        torch.cuda.synchronize()
+        assert moe.moe_read_device_status(ws) == 0
+        assert np.array_equal(g_off.cpu().numpy(), off)
+        assert np.array_equal(g_ss.cpu().numpy(), ss)
+        assert np.array_equal(g_sp.cpu().numpy(), sp)
+
+
+def test_permute_chunked_bad_expert_sets_device_status():
+    E, T, k1 = 64, 1024, 8
+    rng = np.random.default_rng(3)
+    idx = np.stack([rng.choice(E, k1, replace=False) for _ in range(T)]).astype(np.int32)
+    idx[5, 3] = 99
+    idx[700, 0] = -2
+    ws = moe.workspace(T, 64, E, 16, k1, device=DEV)
+    off = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    ss = torch.empty(T * k1, dtype=torch.int32, device=DEV)
+    sp = torch.empty(T * k1, dtype=torch.int32, device=DEV)
+    moe.moe_permute(torch.from_numpy(idx).to(DEV), E, off, ss, sp, ws=ws)
+    torch.cuda.synchronize()
+    assert moe.moe_read_device_status(ws) == moe.MOE_ERR_DEVICE_CHECK
+    assert int(off[-1]) == T * k1 - 2  # the two bad slots are dropped
+    good = np.sort(ss.cpu().numpy()[: T * k1 - 2])
+    assert np.array_equal(good, np.setdiff1d(np.arange(T * k1), [5 * k1 + 3, 700 * k1]))
 
 
 def test_permute_bad_expert_sets_device_status():
