@@ -17,7 +17,8 @@ struct WsHeader {
     int status;             // device status word (moe_status), 0 = OK
     unsigned route_arrive;  // last-block hand-off counter of the top-k kernel
     unsigned decode_arrive; // last-block hand-off counter of the decode kernel
-    unsigned pad0[29];
+    unsigned sched[8];      // work-item counters of the grouped GEMMs (next, done) x 3
+    unsigned pad0[21];
     unsigned bar_go;        // grid barrier: generation released so far (own 128-byte line)
     unsigned pad1[31];
     unsigned bar_flag[kMaxGridCtas];  // grid barrier: generation each CTA has reached

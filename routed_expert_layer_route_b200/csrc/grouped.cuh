@@ -15,15 +15,19 @@
 // costs little padding.  Both operands are K-major bf16 tiles of 64 K values
 // (one 128-byte row) in the 128-byte swizzled shared-memory layout.
 //
-// One persistent CTA per SM walks the work items (expert, weight-row tile,
-// token tile; token tile fastest, so CTAs that run at the same time share
-// weight tiles and token rows through L2).  Warp roles:
-//   warps 0-3   epilogue: tensor memory -> registers (tcgen05.ld), SwiGLU or
-//               the weighted combine, global stores / float32 red.add;
-//   warp 4      TMA producer, no multicast: weight tiles and token tiles
-//               (GEMM 1: the routed tokens' x rows, copied into expert order
-//               by k_gather_rows; GEMM 2: H), with an L2 prefetch stream a
-//               few k-blocks ahead of the loads;
+// One persistent CTA per SM takes work items (expert, weight-row tile, token
+// tile; token tile fastest) from a device-wide counter, so items are handed
+// out in order to whichever SM is free: neighbours in the order, which share
+// weight tiles and token rows, run at the same time and read them once from
+// DRAM, and the load balances itself.  Warp roles:
+//   warps 0-3, 6-9  epilogue: tensor memory -> registers (tcgen05.ld),
+//               SwiGLU or the weighted combine, global stores / float32
+//               red.add; warp w reads lane quarter w % 4, the two warps of a
+//               quarter split the token columns;
+//   warp 4      takes the items and publishes them to the other roles
+//               through a shared-memory queue; TMA producer, no multicast:
+//               weight tiles and token tiles (GEMM 1: the routed tokens' x
+//               rows, copied into expert order by k_gather_rows; GEMM 2: H);
 //   warp 5      allocates tensor memory and issues the MMAs (one thread).
 // The same down-GEMM kernel computes the router logits of large batches
 // (one group of T rows, W_r as the weight matrix, bias added).
@@ -47,9 +51,10 @@ constexpr int kG1Stages = 3;              // A_gate + A_up + B = 64 KB per stage
 constexpr int kG2Stages = 4;              // A_down + B = 48 KB per stage
 constexpr int kG1Stage = 2 * kGTileA + kGTileB;
 constexpr int kG2Stage = kGTileA + kGTileB;
-constexpr int kGEpiThreads = 128;
-constexpr int kG1Threads = kGEpiThreads + 64;  // 192
-constexpr int kG2Threads = kGEpiThreads + 64;  // 192
+constexpr int kGEpiWarps = 8;  // two per quarter of the tensor-memory lanes
+constexpr int kGEpiThreads = kGEpiWarps * 32;
+constexpr int kG1Threads = kGEpiThreads + 64;  // 320
+constexpr int kG2Threads = kGEpiThreads + 64;  // 320
 constexpr int kGMaxE = 1024;
 constexpr int kGWarpTma = 4, kGWarpMma = 5;
 
@@ -139,6 +144,23 @@ MOE_DEVINL void tmem_ld32(uint32_t taddr, float (&v)[32])
         v[i] = __uint_as_float(r[i]);
 }
 
+// 32 lanes x 16 consecutive float32 columns.
+MOE_DEVINL void tmem_ld16(uint32_t taddr, float (&v)[16])
+{
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        v[i] = __uint_as_float(r[i]);
+}
+
 // 2-D tiled TMA load (no multicast) of box {64 K values, rows} at (x, y).
 MOE_DEVINL void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar)
 {
@@ -148,34 +170,6 @@ MOE_DEVINL void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uin
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y)
         : "memory");
 }
-
-// Prefetch `bytes` (multiple of 16) of contiguous global memory into L2.
-MOE_DEVINL void bulk_prefetch_l2(const void *src, uint32_t bytes)
-{
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
-// A weight tile's rows are one contiguous block (row-major weights): fetch it
-// into L2 front to back in 64 KB pieces, a DRAM-friendly order, before the
-// tiled loads walk it one 128-byte column strip at a time.
-MOE_DEVINL void prefetch_rows_l2(const uint16_t *base, size_t row0, int rows, int rowlen)
-{
-    const uint8_t *p = reinterpret_cast<const uint8_t *>(base + row0 * rowlen);
-    const size_t bytes = (size_t)rows * rowlen * 2;
-    for (size_t o = 0; o < bytes; o += 65536)
-        bulk_prefetch_l2(p + o, (uint32_t)min((size_t)65536, bytes - o));
-}
-
-// Prefetch one box of a 2-D map into L2 (no shared memory, no multicast).
-MOE_DEVINL void tma_prefetch_2d(const CUtensorMap *map, int x, int y)
-{
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(x), "r"(y)
-                 : "memory");
-}
-
-
 
 // ---------------------------------------------------------------------------
 // Work items: expert e contributes nrt x ceil(n_e / kGBN) items (weight-row
@@ -237,55 +231,41 @@ MOE_DEVINL GItem g_item(const GTable &tb, int E, int i)
 
 MOE_DEVINL int pad16(int n) { return (n + 15) & ~15; }
 
-// L2 prefetch stream that runs kPF k-blocks ahead of the producer over this
-// CTA's (item, k-block) sequence: the weight tile (two maps for gate / up)
-// and the token tile of that k-block are fetched into L2 early, so the TMA
-// loads behind them find their data there.
-template <int kPF>
-struct GPrefetch {
-    int i, kb, nkb, step, E;
-    GItem it;
-    __device__ void init(const GTable &tb, int E_, int first, int step_, int nkb_, int n_items)
-    {
-        E = E_;
-        i = first;
-        step = step_;
-        nkb = nkb_;
-        kb = 0;
-        if (i < n_items)
-            it = g_item(tb, E, i);
-    }
-    __device__ void next(const GTable &tb, int n_items)
-    {
-        if (++kb == nkb) {
-            kb = 0;
-            i += step;
-            if (i < n_items)
-                it = g_item(tb, E, i);
-        }
-    }
-};
-
 // ---------------------------------------------------------------------------
-struct Gemm1Args {
-    const uint16_t *wg, *wu;     // [E x I x d] bf16 (the maps' memory, for the L2 prefetch)
-    const int32_t *offsets;      // [E + 1]
-    const int32_t *sorted_slot;  // [T*k1] slot ids (t*k1 + s) in expert order
-    uint16_t *h;                 // [T*k1 x I] bf16, row p = sorted position p
-    float4 *zero;                // nullable: buffer to clear for the down GEMM's combine
-    int zero_n4;
-    int T, d, E, I, k1;
-    WsHeader *hdr;
-};
+constexpr int kGQ = 4;  // depth of the work-item queue between the roles
 
 struct GSync {
     uint64_t full[kG2Stages];
     uint64_t empty[kG2Stages];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
+    uint64_t q_full[kGQ];   // the producer published item q_item[slot]
+    uint64_t q_empty[kGQ];  // the MMA thread and every epilogue warp are done with it
     uint64_t drained;
+    int q_item[kGQ];        // item index, -1: no more items
     uint32_t tmem_base;
     int abort;
+};
+
+// Position in the item queue: slot and phase parity.
+struct GQueue {
+    int slot;
+    uint32_t ph;
+    __device__ void advance()
+    {
+        if (++slot == kGQ) {
+            slot = 0;
+            ph ^= 1u;
+        }
+    }
+};
+
+// Device-wide item counters of one grouped launch: `next` hands out items,
+// `done` counts the CTAs that have left; the last CTA resets both, so each
+// launch finds them at zero (the workspace header starts zeroed).
+struct GSched {
+    unsigned *next;
+    unsigned *done;
 };
 
 MOE_DEVINL uint8_t *g_align1024(uint8_t *p)
@@ -293,6 +273,122 @@ MOE_DEVINL uint8_t *g_align1024(uint8_t *p)
     const uint32_t a = smem_addr(p);
     return p + (((a + 1023u) & ~1023u) - a);
 }
+
+MOE_DEVINL bool g_aborted(const GSync &sy) { return *(volatile const int *)&sy.abort != 0; }
+
+// Barrier set-up shared by the kernels (thread 0) and the tensor-memory
+// allocation (warp kGWarpMma, all 512 columns).
+MOE_DEVINL void g_setup(GSync &sy, int stages, int nacc, int tid, int warp)
+{
+    if (tid == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(&sy.full[s], 1);
+            mbar_init(&sy.empty[s], 1);
+        }
+        for (int b = 0; b < nacc; ++b) {
+            mbar_init(&sy.acc_full[b], 1);
+            mbar_init(&sy.acc_empty[b], kGEpiWarps);
+        }
+        for (int q = 0; q < kGQ; ++q) {
+            mbar_init(&sy.q_full[q], 1);
+            mbar_init(&sy.q_empty[q], 1 + kGEpiWarps);
+        }
+        mbar_init(&sy.drained, 1);
+        sy.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == kGWarpMma) {
+        tmem_alloc(&sy.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+}
+
+// Producer side of the queue: publish item `cur` (-1 ends the stream).
+MOE_DEVINL bool g_publish(GSync &sy, GQueue &q, int cur, int *status)
+{
+    if (!mbar_wait(&sy.q_empty[q.slot], q.ph ^ 1u, status))
+        return false;
+    sy.q_item[q.slot] = cur;
+    mbar_arrive(&sy.q_full[q.slot]);
+    q.advance();
+    return true;
+}
+
+// Consumer side, one thread (the MMA issuer): the next item index (-1: none
+// left, or a wait gave up).
+MOE_DEVINL int g_take(GSync &sy, GQueue &q, int *status)
+{
+    if (!mbar_wait(&sy.q_full[q.slot], q.ph, status)) {
+        sy.abort = 1;
+        return -1;
+    }
+    return *(volatile int *)&sy.q_item[q.slot];
+}
+
+MOE_DEVINL void g_release(GSync &sy, GQueue &q)
+{
+    mbar_arrive(&sy.q_empty[q.slot]);
+    q.advance();
+}
+
+// Consumer side, a whole warp (epilogue): lane 0 waits, every lane gets the
+// same answer, so the warp never splits before its warp-wide tcgen05.ld.
+MOE_DEVINL int g_take_warp(GSync &sy, GQueue &q, int *status, int lane)
+{
+    int cur = -1;
+    if (lane == 0)
+        cur = g_take(sy, q, status);
+    return __shfl_sync(0xffffffffu, cur, 0);
+}
+
+MOE_DEVINL void g_release_warp(GSync &sy, GQueue &q, int lane)
+{
+    __syncwarp();
+    if (lane == 0)
+        mbar_arrive(&sy.q_empty[q.slot]);
+    q.advance();
+}
+
+// Bounded wait by lane 0 for the whole warp.
+MOE_DEVINL bool g_wait_warp(uint64_t *bar, uint32_t parity, int *status, int lane)
+{
+    int ok = 1;
+    if (lane == 0)
+        ok = mbar_wait(bar, parity, status);
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// End of a grouped kernel: free tensor memory; the last CTA resets the counters.
+MOE_DEVINL void g_teardown(GSync &sy, uint32_t tmem, GSched sc, int tid, int warp)
+{
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kGWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+    if (tid == 0) {
+        __threadfence();
+        if (atomicAdd(sc.done, 1u) == gridDim.x - 1) {
+            *sc.next = 0u;
+            *sc.done = 0u;
+        }
+    }
+}
+
+struct Gemm1Args {
+    const int32_t *offsets;      // [E + 1]
+    const int32_t *sorted_slot;  // [T*k1] slot ids (t*k1 + s) in expert order
+    uint16_t *h;                 // [T*k1 x I] bf16, row p = sorted position p
+    float4 *zero;                // nullable: buffer to clear for the down GEMM's combine
+    int zero_n4;
+    int T, d, E, I, k1;
+    GSched sched;
+    WsHeader *hdr;
+};
 
 inline size_t gemm1_smem_bytes() { return 1024 + (size_t)kG1Stages * kG1Stage + sizeof(GSync) + sizeof(GTable); }
 inline size_t gemm2_smem_bytes() { return 1024 + (size_t)kG2Stages * kG2Stage + sizeof(GSync) + sizeof(GTable); }
@@ -310,24 +406,7 @@ __global__ void __launch_bounds__(kG1Threads, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     int *status = &a.hdr->status;
 
-    if (tid == 0) {
-        for (int s = 0; s < kG1Stages; ++s) {
-            mbar_init(&sy.full[s], 1);
-            mbar_init(&sy.empty[s], 1);
-        }
-        mbar_init(&sy.acc_full[0], 1);
-        mbar_init(&sy.acc_empty[0], kGEpiThreads / 32);
-        mbar_init(&sy.drained, 1);
-        sy.abort = 0;
-        fence_mbar_init();
-    }
-    if (warp == kGWarpMma) {
-        tmem_alloc(&sy.tmem_base, 512);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
+    g_setup(sy, kG1Stages, 1, tid, warp);
     const uint32_t tmem = sy.tmem_base;
 
     pdl_wait();
@@ -337,35 +416,24 @@ __global__ void __launch_bounds__(kG1Threads, 1)
     const int nkb = d / kGBK;
     g_build_items(a.offsets, E, nrt, tb);
     const int n_items = tb.ibase[E];
+    GQueue q = {0, 0u};
 
     if (warp == kGWarpTma) {
-        // -------------------------------------------------------- weight and token tiles
+        // -------------------------------------------------------- items, weight and token tiles
         if (lane == 0) {
-            constexpr int kPF = 6;
-            GPrefetch<kPF> pf;  // token tiles, kPF k-blocks ahead
-            pf.init(tb, E, blockIdx.x, gridDim.x, nkb, n_items);
-            auto prefetch = [&]() {
-                if (pf.i < n_items)
-                    for (int b = 0; b * 64 < pf.it.n; ++b)
-                        tma_prefetch_2d(&tm_xs, pf.kb * kGBK, pf.it.p0 + 64 * b);
-                pf.next(tb, n_items);
-            };
-            for (int q = 0; q < kPF; ++q)
-                prefetch();
-            auto prefetch_weights = [&](int i) {  // a whole item's gate and up tiles
-                if (i < n_items) {
-                    const GItem w = g_item(tb, E, i);
-                    const size_t r0 = (size_t)w.e * I + w.rt * kGBM;
-                    prefetch_rows_l2(a.wg, r0, kGBM, d);
-                    prefetch_rows_l2(a.wu, r0, kGBM, d);
-                }
-            };
-            prefetch_weights(blockIdx.x);
             uint32_t g = 0;
-            for (int i = blockIdx.x; i < n_items && !*(volatile int *)&sy.abort; i += gridDim.x) {
-                const GItem it = g_item(tb, E, i);
+            int i = (int)atomicAdd(a.sched.next, 1u);
+            while (true) {
+                const int cur = i < n_items && !g_aborted(sy) ? i : -1;
+                if (!g_publish(sy, q, cur, status)) {
+                    sy.abort = 1;
+                    break;
+                }
+                if (cur < 0)
+                    break;
+                i = (int)atomicAdd(a.sched.next, 1u);  // the next one, in flight meanwhile
+                const GItem it = g_item(tb, E, cur);
                 const int row = it.e * I + it.rt * kGBM;
-                prefetch_weights(i + gridDim.x);  // the next item's, one item ahead
                 const int nb = (it.n + 63) / 64;  // 64-row boxes of the sorted x rows
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
                     const int s = g % kG1Stages;
@@ -380,20 +448,22 @@ __global__ void __launch_bounds__(kG1Threads, 1)
                     for (int b = 0; b < nb; ++b)
                         tma_load_2d(st + 2 * kGTileA + b * (kGTileB / 4), &tm_xs, kb * kGBK,
                                     it.p0 + 64 * b, &sy.full[s]);
-                    prefetch();
                 }
             }
             // drain: every stage issued has landed before the CTA may leave
             const uint32_t n_iss = g;
-            for (uint32_t q = n_iss > (uint32_t)kG1Stages ? n_iss - kG1Stages : 0; q < n_iss; ++q)
-                mbar_wait(&sy.full[q % kG1Stages], (q / kG1Stages) & 1, status);
+            for (uint32_t r = n_iss > (uint32_t)kG1Stages ? n_iss - kG1Stages : 0; r < n_iss; ++r)
+                mbar_wait(&sy.full[r % kG1Stages], (r / kG1Stages) & 1, status);
         }
     } else if (warp == kGWarpMma) {
         // -------------------------------------------------------- MMA issue
         if (lane == 0) {
             uint32_t g = 0, itc = 0;
-            for (int i = blockIdx.x; i < n_items && !*(volatile int *)&sy.abort; i += gridDim.x, ++itc) {
-                const GItem it = g_item(tb, E, i);
+            while (true) {
+                const int cur = g_take(sy, q, status);
+                if (cur < 0)
+                    break;
+                const GItem it = g_item(tb, E, cur);
                 if (!mbar_wait(&sy.acc_empty[0], (itc & 1) ^ 1, status)) {
                     sy.abort = 1;
                     break;
@@ -419,36 +489,45 @@ __global__ void __launch_bounds__(kG1Threads, 1)
                     }
                     umma_commit(&sy.empty[s]);
                 }
-                if (*(volatile int *)&sy.abort)
+                if (g_aborted(sy))
                     break;
                 umma_commit(&sy.acc_full[0]);
+                g_release(sy, q);
+                ++itc;
             }
             // every MMA issued has completed before tensor memory is freed
             umma_commit(&sy.drained);
             mbar_wait(&sy.drained, 0, status);
         }
     } else {
-        // -------------------------------------------------------- epilogue (warps 0-3)
+        // -------------------------------------------------------- epilogue (warps 0-3, 6-9)
+        const int ew = warp < 4 ? warp : warp - 2;  // 0..7
+        const int lq = warp & 3;                    // tensor-memory lane quarter
+        const int eh = warp >= 6;                   // which half of the token columns
         if (a.zero)  // the down GEMM's accumulator (read only after this grid completes)
-            for (int q = blockIdx.x * kGEpiThreads + tid; q < a.zero_n4; q += gridDim.x * kGEpiThreads)
-                a.zero[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int r = blockIdx.x * kGEpiThreads + ew * 32 + lane; r < a.zero_n4;
+                 r += gridDim.x * kGEpiThreads)
+                a.zero[r] = make_float4(0.f, 0.f, 0.f, 0.f);
         uint32_t itc = 0;
-        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-        for (int i = blockIdx.x; i < n_items && !*(volatile int *)&sy.abort; i += gridDim.x, ++itc) {
-            const GItem it = g_item(tb, E, i);
-            if (!mbar_wait(&sy.acc_full[0], itc & 1, status)) {
+        const uint32_t lane_addr = tmem + ((uint32_t)(lq * 32) << 16);
+        while (true) {
+            const int cur = g_take_warp(sy, q, status, lane);
+            if (cur < 0)
+                break;
+            const GItem it = g_item(tb, E, cur);
+            if (!g_wait_warp(&sy.acc_full[0], itc & 1, status, lane)) {
                 sy.abort = 1;
                 break;
             }
             tc_fence_after();
-            const int ch = it.rt * kGBM + warp * 32 + lane;  // this thread's channel
+            const int ch = it.rt * kGBM + lq * 32 + lane;  // this thread's channel
             uint16_t *hcol = a.h + (size_t)it.p0 * I + ch;
-            for (int c0 = 0; c0 < it.n; c0 += 32) {
-                float gv[32], uv[32];
-                tmem_ld32(lane_addr + c0, gv);
-                tmem_ld32(lane_addr + 256 + c0, uv);
+            for (int c0 = 16 * eh; c0 < it.n; c0 += 32) {
+                float gv[16], uv[16];
+                tmem_ld16(lane_addr + c0, gv);
+                tmem_ld16(lane_addr + 256 + c0, uv);
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
+                for (int j = 0; j < 16; ++j)
                     if (c0 + j < it.n)
                         hcol[(size_t)(c0 + j) * I] = f32_to_bf16_rn(silu_mul(gv[j], uv[j]));
             }
@@ -456,20 +535,15 @@ __global__ void __launch_bounds__(kG1Threads, 1)
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&sy.acc_empty[0]);
+            g_release_warp(sy, q, lane);
+            ++itc;
         }
     }
-
-    tc_fence_before();
-    __syncthreads();
-    if (warp == kGWarpMma) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 512);
-    }
+    g_teardown(sy, tmem, a.sched, tid, warp);
 }
 
 // ---------------------------------------------------------------------------
 struct Gemm2Args {
-    const uint16_t *wd;          // [E x d x I] bf16 (the weight map's memory, for the L2 prefetch)
     const int32_t *offsets;      // [E + 1]; nullptr: one group of single_n rows
     const int32_t *sorted_slot;  // [T*k1]
     const float *topk_w;         // [T*k1] Eq. 2 weights by slot (combine mode)
@@ -481,6 +555,7 @@ struct Gemm2Args {
     int bn;                      // tokens per tile: kGBN, or 64 to spread a small job
     int T, d, E, I, k1;          // d: output rows of the weight matrix, I: K
     int combine;                 // 1: weighted red.add into y_acc; 0: store rows of out
+    GSched sched;
     WsHeader *hdr;
 };
 
@@ -497,26 +572,7 @@ __global__ void __launch_bounds__(kG2Threads, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     int *status = &a.hdr->status;
 
-    if (tid == 0) {
-        for (int s = 0; s < kG2Stages; ++s) {
-            mbar_init(&sy.full[s], 1);
-            mbar_init(&sy.empty[s], 1);
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&sy.acc_full[b], 1);
-            mbar_init(&sy.acc_empty[b], kGEpiThreads / 32);
-        }
-        mbar_init(&sy.drained, 1);
-        sy.abort = 0;
-        fence_mbar_init();
-    }
-    if (warp == kGWarpMma) {
-        tmem_alloc(&sy.tmem_base, 512);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
+    g_setup(sy, kG2Stages, 2, tid, warp);
     const uint32_t tmem = sy.tmem_base;
 
     pdl_wait();
@@ -526,32 +582,23 @@ __global__ void __launch_bounds__(kG2Threads, 1)
     const int nkb = I / kGBK;
     g_build_items(a.offsets, E, nrt, tb, a.single_n, a.bn > 0 ? a.bn : kGBN);
     const int n_items = tb.ibase[E];
+    GQueue q = {0, 0u};
 
     if (warp == kGWarpTma) {
         if (lane == 0) {
-            constexpr int kPF = 8;
-            GPrefetch<kPF> pf;  // token tiles, kPF k-blocks ahead
-            pf.init(tb, E, blockIdx.x, gridDim.x, nkb, n_items);
-            auto prefetch = [&]() {
-                if (pf.i < n_items)
-                    for (int b = 0; b * 64 < pf.it.n; ++b)
-                        tma_prefetch_2d(&tm_h, pf.kb * kGBK, pf.it.p0 + 64 * b);
-                pf.next(tb, n_items);
-            };
-            for (int q = 0; q < kPF; ++q)
-                prefetch();
-            auto prefetch_weights = [&](int i) {  // a whole item's weight tile
-                if (i < n_items) {
-                    const GItem w = g_item(tb, E, i);
-                    prefetch_rows_l2(a.wd, (size_t)w.e * d + w.rt * kGBM, kGBM, I);
-                }
-            };
-            prefetch_weights(blockIdx.x);
             uint32_t g = 0;
-            for (int i = blockIdx.x; i < n_items && !*(volatile int *)&sy.abort; i += gridDim.x) {
-                const GItem it = g_item(tb, E, i);
+            int i = (int)atomicAdd(a.sched.next, 1u);
+            while (true) {
+                const int cur = i < n_items && !g_aborted(sy) ? i : -1;
+                if (!g_publish(sy, q, cur, status)) {
+                    sy.abort = 1;
+                    break;
+                }
+                if (cur < 0)
+                    break;
+                i = (int)atomicAdd(a.sched.next, 1u);
+                const GItem it = g_item(tb, E, cur);
                 const int row = it.e * d + it.rt * kGBM;
-                prefetch_weights(i + gridDim.x);  // the next item's, one item ahead
                 const int nb = (it.n + 63) / 64;  // 64-row boxes of H
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
                     const int s = g % kG2Stages;
@@ -565,18 +612,20 @@ __global__ void __launch_bounds__(kG2Threads, 1)
                     for (int b = 0; b < nb; ++b)
                         tma_load_2d(st + kGTileA + b * (kGTileB / 4), &tm_h, kb * kGBK,
                                     it.p0 + 64 * b, &sy.full[s]);
-                    prefetch();
                 }
             }
             const uint32_t n_iss = g;
-            for (uint32_t q = n_iss > (uint32_t)kG2Stages ? n_iss - kG2Stages : 0; q < n_iss; ++q)
-                mbar_wait(&sy.full[q % kG2Stages], (q / kG2Stages) & 1, status);
+            for (uint32_t r = n_iss > (uint32_t)kG2Stages ? n_iss - kG2Stages : 0; r < n_iss; ++r)
+                mbar_wait(&sy.full[r % kG2Stages], (r / kG2Stages) & 1, status);
         }
     } else if (warp == kGWarpMma) {
         if (lane == 0) {
             uint32_t g = 0, itc = 0;
-            for (int i = blockIdx.x; i < n_items && !*(volatile int *)&sy.abort; i += gridDim.x, ++itc) {
-                const GItem it = g_item(tb, E, i);
+            while (true) {
+                const int cur = g_take(sy, q, status);
+                if (cur < 0)
+                    break;
+                const GItem it = g_item(tb, E, cur);
                 const int buf = itc & 1;
                 if (!mbar_wait(&sy.acc_empty[buf], ((itc >> 1) & 1) ^ 1, status)) {
                     sy.abort = 1;
@@ -599,60 +648,67 @@ __global__ void __launch_bounds__(kG2Threads, 1)
                                   umma_desc_sw128(st + kGTileA + kk * 32), idesc, (kb | kk) != 0);
                     umma_commit(&sy.empty[s]);
                 }
-                if (*(volatile int *)&sy.abort)
+                if (g_aborted(sy))
                     break;
                 umma_commit(&sy.acc_full[buf]);
+                g_release(sy, q);
+                ++itc;
             }
             umma_commit(&sy.drained);
             mbar_wait(&sy.drained, 0, status);
         }
     } else {
-        // -------------------------------------------------------- epilogue (warps 0-3)
+        // -------------------------------------------------------- epilogue (warps 0-3, 6-9)
+        const int lq = warp & 3;   // tensor-memory lane quarter
+        const int eh = warp >= 6;  // which half of the token column chunks
         uint32_t itc = 0;
         const int k1 = a.k1;
-        for (int i = blockIdx.x; i < n_items && !*(volatile int *)&sy.abort; i += gridDim.x, ++itc) {
-            const GItem it = g_item(tb, E, i);
+        while (true) {
+            const int cur = g_take_warp(sy, q, status, lane);
+            if (cur < 0)
+                break;
+            const GItem it = g_item(tb, E, cur);
             const int buf = itc & 1;
             // this lane's columns c*32 + lane: token and Eq. 2 weight (before the wait)
             int tk[kGBN / 32];
             float wt[kGBN / 32];
 #pragma unroll
-            for (int q = 0; q < kGBN / 32; ++q) {
-                const int col = q * 32 + lane;
-                tk[q] = 0;
-                wt[q] = 0.0f;
-                if (a.combine && col < it.n) {
+            for (int c = 0; c < kGBN / 32; ++c) {
+                const int col = c * 32 + lane;
+                tk[c] = 0;
+                wt[c] = 0.0f;
+                if (a.combine && (c & 1) == eh && col < it.n) {
                     const int slot = __ldcg(&a.sorted_slot[it.p0 + col]);
-                    tk[q] = slot / k1;
-                    wt[q] = __ldcg(&a.topk_w[slot]);
+                    tk[c] = slot / k1;
+                    wt[c] = __ldcg(&a.topk_w[slot]);
                 }
             }
-            if (!mbar_wait(&sy.acc_full[buf], (itc >> 1) & 1, status)) {
+            if (!g_wait_warp(&sy.acc_full[buf], (itc >> 1) & 1, status, lane)) {
                 sy.abort = 1;
                 break;
             }
             tc_fence_after();
-            const uint32_t taddr = tmem + buf * 256 + ((uint32_t)(warp * 32) << 16);
-            const int r = it.rt * kGBM + warp * 32 + lane;  // this thread's output row
+            const uint32_t taddr = tmem + buf * 256 + ((uint32_t)(lq * 32) << 16);
+            const int r = it.rt * kGBM + lq * 32 + lane;  // this thread's output row
 #pragma unroll
-            for (int q = 0; q < kGBN / 32; ++q) {
-                if (q * 32 < it.n) {
+            for (int c = 0; c < kGBN / 32; ++c) {
+                if ((c & 1) == eh && c * 32 < it.n) {
                     float v[32];
-                    tmem_ld32(taddr + q * 32, v);
+                    tmem_ld32(taddr + c * 32, v);
                     if (a.combine) {
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
-                            const int t = __shfl_sync(0xffffffffu, tk[q], j);
-                            const float w = __shfl_sync(0xffffffffu, wt[q], j);
-                            if (q * 32 + j < it.n)
+                            const int t = __shfl_sync(0xffffffffu, tk[c], j);
+                            const float w = __shfl_sync(0xffffffffu, wt[c], j);
+                            if (c * 32 + j < it.n)
                                 atomicAdd(&a.y_acc[(size_t)t * d + r], w * v[j]);
                         }
                     } else {
                         const float b = a.bias ? __ldg(&a.bias[r]) : 0.0f;
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
-                            if (q * 32 + j < it.n) {
-                                const size_t o = (size_t)(it.p0 + q * 32 + j) * d + r;
+                            if (c * 32 + j < it.n) {
+                                const size_t o = (size_t)(it.p0 + c * 32 + j) * d + r;
                                 const float val = a.bias ? __fadd_rn(v[j], b) : v[j];
                                 a.out[o] = val;
                                 if (a.out_copy)
@@ -665,15 +721,11 @@ __global__ void __launch_bounds__(kG2Threads, 1)
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&sy.acc_empty[buf]);
+            g_release_warp(sy, q, lane);
+            ++itc;
         }
     }
-
-    tc_fence_before();
-    __syncthreads();
-    if (warp == kGWarpMma) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 512);
-    }
+    g_teardown(sy, tmem, a.sched, tid, warp);
 }
 
 // xs[p] = x[sorted_slot[p] / k1]: the routed tokens' rows in expert order, the

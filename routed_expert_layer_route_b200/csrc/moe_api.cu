@@ -303,13 +303,12 @@ static int enqueue_grouped(const void *x, const void *wg, const void *wu, const 
             return rc;
     }
     Gemm1Args a1 = {};
-    a1.wg = static_cast<const uint16_t *>(wg);
-    a1.wu = static_cast<const uint16_t *>(wu);
     a1.offsets = offsets;
     a1.sorted_slot = sorted_slot;
     a1.h = h;
     a1.zero = reinterpret_cast<float4 *>(y_acc);
     a1.zero_n4 = y_acc ? T * d / 4 : 0;
+    a1.sched = {&hdr->sched[0], &hdr->sched[1]};
     a1.T = T;
     a1.d = d;
     a1.E = E;
@@ -322,7 +321,6 @@ static int enqueue_grouped(const void *x, const void *wg, const void *wu, const 
     if (!(which & 2))
         return MOE_OK;
     Gemm2Args a2 = {};
-    a2.wd = static_cast<const uint16_t *>(wd);
     a2.offsets = offsets;
     a2.sorted_slot = sorted_slot;
     a2.topk_w = topk_w;
@@ -334,6 +332,7 @@ static int enqueue_grouped(const void *x, const void *wg, const void *wu, const 
     a2.I = I;
     a2.k1 = k1;
     a2.combine = y_acc != nullptr;
+    a2.sched = {&hdr->sched[2], &hdr->sched[3]};
     a2.hdr = hdr;
     return launch(k_gemm2, dim3(G), dim3(kG2Threads), gemm2_smem_bytes(), s, pdl, td, th, a2);
 }
@@ -353,7 +352,6 @@ static int enqueue_logits_gemm(const void *x, const void *wr, const float *bias,
         (rc = bf16_tile_map(&tx, x, d, T, 64)) != MOE_OK)
         return rc;
     Gemm2Args a = {};
-    a.wd = static_cast<const uint16_t *>(wr);
     a.out = z;
     a.out_copy = z_copy;
     a.bias = bias;
@@ -365,6 +363,7 @@ static int enqueue_logits_gemm(const void *x, const void *wr, const float *bias,
     a.E = 1;  // one group: every token
     a.k1 = 1;
     a.combine = 0;
+    a.sched = {&hdr->sched[4], &hdr->sched[5]};
     a.hdr = hdr;
     return launch(k_gemm2, dim3(G), dim3(kG2Threads), gemm2_smem_bytes(), s, true, tw, tx, a);
 }
