@@ -262,50 +262,52 @@ def unique_experts(stack, k1, k2, ws_list, ys, stream):
     return us
 
 
-def time_dominant_kernel(stack, k1, k2, ws_list, ys, stream, reps):
-    """Average duration of the expert-streaming kernel launched alone (CUDA
-    events on its stream), cycling through the layers so weights come from
-    HBM, not L2."""
-    from routed_expert_layer_route_b200 import moe
-    starts, ends = [], []
+def graph_time_per_call(calls, stream, reps):
+    """Average device time of one call, the calls captured once into a CUDA
+    graph (so host-side work between launches is not on the device timeline)
+    and the graph replayed `reps` times between CUDA events on its stream."""
+    g = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
-        for r in range(reps):
-            for L, ws, y in zip(stack.layers, ws_list, ys):
-                s = torch.cuda.Event(enable_timing=True)
-                e = torch.cuda.Event(enable_timing=True)
-                s.record(stream)
-                moe.moe_test_expert_stream(L.x, L.w_gate, L.w_up, L.w_down, k1, k2, y, ws,
-                                           flags=stack.flags, stream=stream)
-                e.record(stream)
-                starts.append(s)
-                ends.append(e)
-    stream.synchronize()
-    ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
-    return statistics.mean(ms[len(stack.layers):] or ms)  # first pass is warm-up
+        for c in calls:  # one eager pass: first-use set-up stays outside capture
+            c()
+        stream.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            for c in calls:
+                c()
+        g.replay()  # warm
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e.record(stream)
+    e.synchronize()
+    ms = s.elapsed_time(e) / (reps * len(calls))
+    del g
+    return ms
+
+
+def time_dominant_kernel(stack, k1, k2, ws_list, ys, stream, reps):
+    """Average duration of the expert kernel launched alone (no programmatic
+    dependent launch), one launch per layer so weights come from HBM, not L2."""
+    from routed_expert_layer_route_b200 import moe
+    calls = [(lambda L=L, ws=ws, y=y: moe.moe_test_expert_stream(
+        L.x, L.w_gate, L.w_up, L.w_down, k1, k2, y, ws, flags=stack.flags, stream=stream))
+        for L, ws, y in zip(stack.layers, ws_list, ys)]
+    return graph_time_per_call(calls, stream, reps)
 
 
 def time_grouped_kernels(stack, k1, ws_list, stream, reps):
     """Average durations (ms) of the token-row gather, the gate/up and the down
-    grouped GEMM, each launched alone (CUDA events on its stream) on the
-    routing tables the layer's last moe_layer call left in its workspace,
-    cycling the layers."""
+    grouped GEMM, each launched alone on the routing tables the layer's last
+    moe_layer call left in its workspace, one launch per layer."""
     from routed_expert_layer_route_b200 import moe
     out = []
     for which in (4, 1, 2):
-        pairs = []
-        with torch.cuda.stream(stream):
-            for r in range(reps):
-                for L, ws in zip(stack.layers, ws_list):
-                    s = torch.cuda.Event(enable_timing=True)
-                    e = torch.cuda.Event(enable_timing=True)
-                    s.record(stream)
-                    moe.moe_test_expert_grouped(L.x, L.w_gate, L.w_up, L.w_down, k1, which, ws,
-                                                stream=stream)
-                    e.record(stream)
-                    pairs.append((s, e))
-        stream.synchronize()
-        ms = [a.elapsed_time(b) for a, b in pairs]
-        out.append(statistics.mean(ms[len(stack.layers):] or ms))
+        calls = [(lambda L=L, ws=ws, which=which: moe.moe_test_expert_grouped(
+            L.x, L.w_gate, L.w_up, L.w_down, k1, which, ws, stream=stream))
+            for L, ws in zip(stack.layers, ws_list)]
+        out.append(graph_time_per_call(calls, stream, reps))
     return out
 
 
@@ -489,7 +491,7 @@ def run_native(args, world, rank):
                                    "alone)" % peak_kind if peak_kind == "measured"
                     else "fallback 1590 TFLOP/s"}
     else:
-        kern_ms = time_dominant_kernel(stack, k1h, k2h, ws_list, ys, stream, reps=3)
+        kern_ms = time_dominant_kernel(stack, k1h, k2h, ws_list, ys, stream, reps=5)
         achieved = alg_bytes / (kern_ms * 1e-3) / 1e9
         kname = "k_decode" if stack.channel_major else "k_stream"
         traffic = recorded_traffic(args.workload, k1h, kname)

@@ -144,6 +144,59 @@ MOE_DEVINL void tmem_ld32(uint32_t taddr, float (&v)[32])
         v[i] = __uint_as_float(r[i]);
 }
 
+// Two 32-column loads (columns ta.. and tb..) with one wait: the wait is part
+// of the same asm statement, so no use of the outputs can move above it.
+MOE_DEVINL void tmem_ld32x2(uint32_t ta, uint32_t tb, float (&a)[32], float (&b)[32])
+{
+    uint32_t r[64];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]),
+          "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]),
+          "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]),
+          "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]),
+          "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]),
+          "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(ta), "r"(tb)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        a[i] = __uint_as_float(r[i]);
+        b[i] = __uint_as_float(r[32 + i]);
+    }
+}
+
+// silu(g) * u for the tensor-core path, whose h is rounded to bf16 next:
+// fast exp and divide (a few ulp of float32, far below the bf16 step).
+MOE_DEVINL float silu_mul_fast(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
+
+// Two floats to a bf16x2 word (round to nearest even), lo in the low half.
+MOE_DEVINL uint32_t pack_bf16x2(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// y[0..3] += v (16-byte aligned float32 vector), one vector reduction.
+MOE_DEVINL void red_add_v4(float *y, float v0, float v1, float v2, float v3)
+{
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(y), "f"(v0), "f"(v1),
+                 "f"(v2), "f"(v3)
+                 : "memory");
+}
+
 // 32 lanes x 16 consecutive float32 columns.
 MOE_DEVINL void tmem_ld16(uint32_t taddr, float (&v)[16])
 {
@@ -520,16 +573,23 @@ __global__ void __launch_bounds__(kG1Threads, 1)
                 break;
             }
             tc_fence_after();
-            const int ch = it.rt * kGBM + lq * 32 + lane;  // this thread's channel
-            uint16_t *hcol = a.h + (size_t)it.p0 * I + ch;
-            for (int c0 = 16 * eh; c0 < it.n; c0 += 32) {
-                float gv[16], uv[16];
-                tmem_ld16(lane_addr + c0, gv);
-                tmem_ld16(lane_addr + 256 + c0, uv);
+            // lane pairs (2m, 2m+1) store channels 2m, 2m+1 together: the even lane
+            // for token j, the odd lane for token j+1
+            const int odd = lane & 1;
+            uint16_t *hrow = a.h + (size_t)it.p0 * I + it.rt * kGBM + lq * 32 + (lane & ~1);
+            for (int c0 = 32 * eh; c0 < it.n; c0 += 64) {
+                float gv[32], uv[32];
+                tmem_ld32x2(lane_addr + c0, lane_addr + 256 + c0, gv, uv);
 #pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    if (c0 + j < it.n)
-                        hcol[(size_t)(c0 + j) * I] = f32_to_bf16_rn(silu_mul(gv[j], uv[j]));
+                for (int j = 0; j < 32; j += 2) {
+                    const float h0 = silu_mul_fast(gv[j], uv[j]);
+                    const float h1 = silu_mul_fast(gv[j + 1], uv[j + 1]);
+                    const float other = __shfl_xor_sync(0xffffffffu, odd ? h0 : h1, 1);
+                    const uint32_t pair = odd ? pack_bf16x2(other, h1) : pack_bf16x2(h0, other);
+                    const int tj = c0 + j + odd;
+                    if (tj < it.n)
+                        *reinterpret_cast<uint32_t *>(hrow + (size_t)tj * I) = pair;
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -690,18 +750,39 @@ __global__ void __launch_bounds__(kG2Threads, 1)
             tc_fence_after();
             const uint32_t taddr = tmem + buf * 256 + ((uint32_t)(lq * 32) << 16);
             const int r = it.rt * kGBM + lq * 32 + lane;  // this thread's output row
+            const int qd = lane & 3;                       // position in the lane quad
+            const int rq = it.rt * kGBM + lq * 32 + (lane & ~3);  // the quad's first row
 #pragma unroll
             for (int c = 0; c < kGBN / 32; ++c) {
                 if ((c & 1) == eh && c * 32 < it.n) {
                     float v[32];
                     tmem_ld32(taddr + c * 32, v);
                     if (a.combine) {
+                        // 4 x 4 transposes inside each lane quad: lane 4m+q gets rows
+                        // 4m..4m+3 of token column j0+q and adds them with one vector red
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const int t = __shfl_sync(0xffffffffu, tk[c], j);
-                            const float w = __shfl_sync(0xffffffffu, wt[c], j);
-                            if (c * 32 + j < it.n)
-                                atomicAdd(&a.y_acc[(size_t)t * d + r], w * v[j]);
+                        for (int j0 = 0; j0 < 32; j0 += 4) {
+                            float s0 = v[j0], s1 = v[j0 + 1], s2 = v[j0 + 2], s3 = v[j0 + 3];
+                            const bool hi = qd & 2, od = qd & 1;
+                            float t0 = __shfl_xor_sync(0xffffffffu, hi ? s0 : s2, 2);
+                            float t1 = __shfl_xor_sync(0xffffffffu, hi ? s1 : s3, 2);
+                            if (hi) {
+                                s0 = t0;
+                                s1 = t1;
+                            } else {
+                                s2 = t0;
+                                s3 = t1;
+                            }
+                            t0 = __shfl_xor_sync(0xffffffffu, od ? s0 : s1, 1);
+                            t1 = __shfl_xor_sync(0xffffffffu, od ? s2 : s3, 1);
+                            const float o0 = od ? t0 : s0, o1 = od ? s1 : t0;
+                            const float o2 = od ? t1 : s2, o3 = od ? s3 : t1;
+                            const int col = j0 + qd;
+                            const int t = __shfl_sync(0xffffffffu, tk[c], col);
+                            const float w = __shfl_sync(0xffffffffu, wt[c], col);
+                            if (c * 32 + col < it.n)
+                                red_add_v4(a.y_acc + (size_t)t * d + rq, w * o0, w * o1, w * o2,
+                                           w * o3);
                         }
                     } else {
                         const float b = a.bias ? __ldg(&a.bias[r]) : 0.0f;
