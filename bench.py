@@ -44,8 +44,7 @@ WORKLOADS = {
                       sweep=[(4, 16), (8, 8), (8, 16), (8, 128), (4, 4), (4, 128)]),
     "decode_small_batch": dict(T=8, d=2048, E=128, I=768, layers=48, bias="normal",
                                sweep=[(4, 16), (8, 8)]),
-    "prefill": dict(T=4096, d=2048, E=128, I=768, layers=4, bias="zipf", sweep=[(8, 16), (4, 16)],
-                    grouped=True),
+    "prefill": dict(T=4096, d=2048, E=128, I=768, layers=4, bias="zipf", sweep=[(8, 16), (4, 16)]),
     "large": dict(T=1, d=4096, E=512, I=1024, layers=8, bias=None, sweep=[(5, 20), (10, 10)]),
 }
 
@@ -211,9 +210,9 @@ class Stack:
         self.wl = wl
         self.layers = []
         self.channel_major = wl["T"] == 1
-        # large batches: the tensor-core grouped GEMMs (what AUTO picks at >= 16
-        # routed slots per expert), named explicitly so the timed kernels are known
-        self.grouped = wl.get("grouped", False)
+        # two or more tokens: the tensor-core grouped GEMMs (what AUTO picks when d
+        # and I fill 128-row tiles), named explicitly so the timed kernels are known
+        self.grouped = wl["T"] > 1 and wl["d"] % 128 == 0 and wl["I"] % 128 == 0
         self.flags = (moe.MOE_WDOWN_CHANNEL_MAJOR if self.channel_major else
                       moe.MOE_PATH_GROUPED if self.grouped else moe.MOE_PATH_STREAM)
         for l in range(wl["layers"]):
@@ -467,29 +466,44 @@ def run_native(args, world, rank):
     if stack.grouped:
         gx_ms, g1_ms, g2_ms = time_grouped_kernels(stack, k1h, ws_list, stream, reps=3)
         n_slots = T * k1h
-        f1 = 2.0 * n_slots * 2 * I * d   # gate and up
-        f2 = 2.0 * n_slots * I * d       # down
-        a1 = f1 / (g1_ms * 1e-3) / 1e12
-        a2 = f2 / (g2_ms * 1e-3) / 1e12
-        roofline = {"bound": "tensor", "achieved": round(a1, 1), "peak": bf16_peak,
-                    "unit": "TFLOP/s", "frac": round(a1 / bf16_peak, 4),
+        # algorithmic work of each GEMM: FLOPs, and bytes = the unique experts'
+        # weights + the token rows read + the rows written
+        f1 = 2.0 * n_slots * 2 * I * d                       # gate and up
+        b1 = U_head * 2 * d * I * 2 + n_slots * d * 2 + n_slots * I * 2
+        f2 = 2.0 * n_slots * I * d                           # down
+        b2 = U_head * d * I * 2 + n_slots * I * 2 + T * d * 4
+
+        def bound(f, b, ms):
+            t_tensor, t_hbm = f / (bf16_peak * 1e12), b / (hbm_peak * 1e9)
+            tf = f / (ms * 1e-3) / 1e12
+            gb = b / (ms * 1e-3) / 1e9
+            if t_tensor >= t_hbm:
+                return "tensor", tf, bf16_peak, "TFLOP/s", tf / bf16_peak, gb / hbm_peak
+            return "hbm", gb, hbm_peak, "GB/s", gb / hbm_peak, tf / bf16_peak
+
+        bd1, a1, p1, u1, fr1, other1 = bound(f1, b1, g1_ms)
+        bd2, a2, p2, u2, fr2, other2 = bound(f2, b2, g2_ms)
+        roofline = {"bound": bd1, "achieved": round(a1, 1), "peak": p1, "unit": u1,
+                    "frac": round(fr1, 4),
                     "traffic": recorded_traffic(args.workload, k1h, "k_gemm1"),
                     "kernel": "moe::k_gemm1", "kernel_us": round(g1_ms * 1000, 2),
-                    "algorithmic_flops_per_launch": f1,
+                    "algorithmic_flops_per_launch": f1, "algorithmic_bytes_per_launch": int(b1),
+                    "tensor_frac": round(f1 / (g1_ms * 1e-3) / 1e12 / bf16_peak, 4),
+                    "hbm_frac": round(b1 / (g1_ms * 1e-3) / 1e9 / hbm_peak, 4),
                     "second_kernel": {"kernel": "moe::k_gemm2", "kernel_us": round(g2_ms * 1000, 2),
+                                      "bound": bd2, "achieved": round(a2, 1), "unit": u2,
+                                      "frac": round(fr2, 4),
                                       "algorithmic_flops_per_launch": f2,
-                                      "achieved": round(a2, 1),
-                                      "frac": round(a2 / bf16_peak, 4)},
+                                      "algorithmic_bytes_per_launch": int(b2)},
                     "gather_kernel": {"kernel": "moe::k_gather_rows",
                                       "kernel_us": round(gx_ms * 1000, 2)},
-                    "both_gemms_frac": round((f1 + f2) / ((g1_ms + g2_ms) * 1e-3) / 1e12
-                                             / bf16_peak, 4),
-                    "hbm_bytes_per_layer": int(alg_bytes),
-                    "hbm_frac_both_gemms": round(alg_bytes / ((g1_ms + g2_ms) * 1e-3) / 1e9
+                    "both_gemms_tensor_frac": round((f1 + f2) / ((g1_ms + g2_ms) * 1e-3) / 1e12
+                                                    / bf16_peak, 4),
+                    "both_gemms_hbm_frac": round(alg_bytes / ((g1_ms + g2_ms) * 1e-3) / 1e9
                                                  / hbm_peak, 4),
-                    "peak_source": "%s (MEASURED_PEAKS.json bf16_tflops, burst: kernels timed "
-                                   "alone)" % peak_kind if peak_kind == "measured"
-                    else "fallback 1590 TFLOP/s"}
+                    "peak_source": "%s (MEASURED_PEAKS.json bf16_tflops burst and hbm_gbs: "
+                                   "kernels timed alone)" % peak_kind if peak_kind == "measured"
+                    else "fallback 1590 TFLOP/s, 6650 GB/s"}
     else:
         kern_ms = time_dominant_kernel(stack, k1h, k2h, ws_list, ys, stream, reps=5)
         achieved = alg_bytes / (kern_ms * 1e-3) / 1e9
@@ -510,11 +524,12 @@ def run_native(args, world, rank):
 
     # ratio of k1=4 to k1=8 layer time (same k2 where possible)
     by = {(r["k1"], r["k2"]): r for r in results}
-    ratio = None
-    if (4, 16) in by and (8, 16) in by:
-        ratio = by[(4, 16)]["us_per_layer"] / by[(8, 16)]["us_per_layer"]
-    elif (4, 4) in by and (8, 8) in by:
-        ratio = by[(4, 4)]["us_per_layer"] / by[(8, 8)]["us_per_layer"]
+    ratio, ratio_pair = None, None
+    for p4, p8 in (((4, 16), (8, 16)), ((4, 4), (8, 8)), ((4, 16), (8, 8)), ((5, 20), (10, 10))):
+        if p4 in by and p8 in by:
+            ratio = by[p4]["us_per_layer"] / by[p8]["us_per_layer"]
+            ratio_pair = "k1=%d,k2=%d over k1=%d,k2=%d" % (p4 + p8)
+            break
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -551,6 +566,7 @@ def run_native(args, world, rank):
         "clocks": clk,
         "sweep": results,
         "k1_4_over_k1_8_time_ratio": None if ratio is None else round(ratio, 4),
+        "k1_ratio_conditions": ratio_pair,
     }
     for g, _, _ in graphs.values():
         del g

@@ -76,10 +76,15 @@ typedef enum {
 #define MOE_DTYPE_BF16 1
 
 /* moe_layer / moe_expert_ffn flags: which expert-FFN path runs.
- * AUTO picks by batch size and shapes. */
+ * AUTO: one token with the channel-major down matrix -> DECODE; two or more
+ * tokens with d and I multiples of 128 -> GROUPED; otherwise STREAM. */
 #define MOE_PATH_AUTO 0
-#define MOE_PATH_STREAM 1  /* two-phase weight streaming, deterministic output        */
-#define MOE_PATH_GROUPED 2 /* tcgen05 grouped GEMM path (large batches)               */
+#define MOE_PATH_STREAM 1  /* two-phase weight streaming on CUDA cores, deterministic
+                              output                                                  */
+#define MOE_PATH_GROUPED 2 /* grouped GEMMs on the tcgen05 tensor cores (d, I multiples
+                              of 128); h rounded to bf16 before the down projection;
+                              the float32 combine runs in a timing-dependent order, so
+                              y may differ between runs in the last bits              */
 #define MOE_PATH_DECODE 3  /* one token: a single pass over the routed experts with the
                               down matrix channel-major (needs MOE_WDOWN_CHANNEL_MAJOR);
                               the float32 sum into y runs in a timing-dependent order,

@@ -18,6 +18,17 @@ MAX_ABS = 2e-2
 REL_L2 = 5e-3
 
 
+def takes_grouped_path(T, d, I, flags):
+    """The path moe_layer takes rounds h to bf16 (the tensor-core grouped
+    GEMMs): explicitly, or by AUTO for two or more tokens with d and I
+    multiples of 128 (the rule in include/moe.h)."""
+    path = flags & moe.MOE_PATH_MASK
+    if path == moe.MOE_PATH_GROUPED:
+        return True
+    return (path == moe.MOE_PATH_AUTO and not (flags & moe.MOE_WDOWN_CHANNEL_MAJOR)
+            and T >= 2 and d % 128 == 0 and I % 128 == 0)
+
+
 def rel_l2(a, b):
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
 
@@ -55,8 +66,13 @@ def run_layer(L, k1, k2, y_dtype=torch.float32, flags=moe.MOE_PATH_AUTO, ws=None
     return y, idx, w, z
 
 
-def check_layer_full(L, k1, k2, flags=moe.MOE_PATH_AUTO, tight=True, w_down=None):
-    """Whole-layer parity against oracle.layer (all tokens, all weights on host)."""
+def check_layer_full(L, k1, k2, flags=moe.MOE_PATH_AUTO, tight=None, w_down=None):
+    """Whole-layer parity against oracle.layer (all tokens, all weights on host).
+    tight (default: unless the path rounds h to bf16): float32 output within
+    1e-4 relative, i.e. only the summation order differs from the oracle."""
+    T, d = L.x.shape
+    if tight is None:
+        tight = not takes_grouped_path(T, d, L.w_gate.shape[1], flags)
     y, idx, w, z = run_layer(L, k1, k2, flags=flags, w_down=w_down)
     zn = z.cpu().numpy()
     # logits against the oracle's own
@@ -75,10 +91,12 @@ def check_layer_full(L, k1, k2, flags=moe.MOE_PATH_AUTO, tight=True, w_down=None
     return yy, ref
 
 
-def check_layer_sampled(L, k1, k2, tokens, flags=moe.MOE_PATH_AUTO, w_down=None, tight=True):
+def check_layer_sampled(L, k1, k2, tokens, flags=moe.MOE_PATH_AUTO, w_down=None, tight=None):
     """Parity on sampled tokens; expert weights are fetched to the host only
-    for the experts those tokens use.  tight=False for the tensor-core path,
-    which rounds h to bf16 before the down projection."""
+    for the experts those tokens use.  tight as for check_layer_full."""
+    T, d = L.x.shape
+    if tight is None:
+        tight = not takes_grouped_path(T, d, L.w_gate.shape[1], flags)
     y, idx, w, z = run_layer(L, k1, k2, flags=flags, w_down=w_down)
     tokens = np.asarray(tokens)
     zn = z.cpu().numpy()[tokens]

@@ -181,7 +181,9 @@ def test_decode_b1_full_size(k1, k2):
 @pytest.mark.parametrize("k1,k2", [(8, 8), (4, 16)])
 def test_decode_small_batch_full_size(T, k1, k2):
     L = synth.make_layer(T, 2048, 128, 768, seed=0, layer=1, device=DEV, bias="normal")
-    check_layer_sampled(L, k1, k2, list(range(T)) if T == 8 else [0, 5, 17, 31])
+    tokens = list(range(T)) if T == 8 else [0, 5, 17, 31]
+    check_layer_sampled(L, k1, k2, tokens)  # AUTO: the tensor-core path
+    check_layer_sampled(L, k1, k2, tokens, flags=moe.MOE_PATH_STREAM)
 
 
 @pytest.mark.parametrize("T", [1, 64])
@@ -198,7 +200,7 @@ def test_prefill_full_size_sampled(k1, k2):
     # AUTO runs the tensor-core grouped GEMMs at this batch size
     L = synth.make_layer(4096, 2048, 128, 768, seed=0, layer=0, device=DEV, bias="zipf")
     tokens = [0, 1, 777, 2048, 4000, 4095]
-    idx = check_layer_sampled(L, k1, k2, tokens, tight=False)
+    idx = check_layer_sampled(L, k1, k2, tokens)
     # Zipf bias: the most popular expert gets many more tokens than the least
     counts = np.bincount(idx.ravel(), minlength=128)
     assert counts.max() > 4 * max(1, np.median(counts))
