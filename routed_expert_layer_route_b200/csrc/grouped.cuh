@@ -436,8 +436,6 @@ struct Gemm1Args {
     const int32_t *offsets;      // [E + 1]
     const int32_t *sorted_slot;  // [T*k1] slot ids (t*k1 + s) in expert order
     uint16_t *h;                 // [T*k1 x I] bf16, row p = sorted position p
-    float4 *zero;                // nullable: buffer to clear for the down GEMM's combine
-    int zero_n4;
     int T, d, E, I, k1;
     GSched sched;
     WsHeader *hdr;
@@ -554,13 +552,8 @@ __global__ void __launch_bounds__(kG1Threads, 1)
         }
     } else {
         // -------------------------------------------------------- epilogue (warps 0-3, 6-9)
-        const int ew = warp < 4 ? warp : warp - 2;  // 0..7
         const int lq = warp & 3;                    // tensor-memory lane quarter
         const int eh = warp >= 6;                   // which half of the token columns
-        if (a.zero)  // the down GEMM's accumulator (read only after this grid completes)
-            for (int r = blockIdx.x * kGEpiThreads + ew * 32 + lane; r < a.zero_n4;
-                 r += gridDim.x * kGEpiThreads)
-                a.zero[r] = make_float4(0.f, 0.f, 0.f, 0.f);
         uint32_t itc = 0;
         const uint32_t lane_addr = tmem + ((uint32_t)(lq * 32) << 16);
         while (true) {
@@ -810,12 +803,17 @@ __global__ void __launch_bounds__(kG2Threads, 1)
 }
 
 // xs[p] = x[sorted_slot[p] / k1]: the routed tokens' rows in expert order, the
-// token operand of the gate/up GEMM.  One warp per row, 16-byte vectors.
+// token operand of the gate/up GEMM.  One warp per row, 16-byte vectors.  Also
+// clears the down GEMM's float32 accumulator (zero: nullable, zero_n4 float4s).
 __global__ void __launch_bounds__(256) k_gather_rows(const uint16_t *x, const int32_t *sorted_slot,
-                                                     int n, int d, int k1, uint16_t *xs)
+                                                     int n, int d, int k1, uint16_t *xs,
+                                                     float4 *zero, int zero_n4)
 {
     pdl_wait();
     pdl_trigger();
+    if (zero)
+        for (int q = blockIdx.x * 256 + threadIdx.x; q < zero_n4; q += gridDim.x * 256)
+            zero[q] = make_float4(0.f, 0.f, 0.f, 0.f);
     const int lane = threadIdx.x & 31;
     const int nv = d >> 3;
     for (int p = blockIdx.x * 8 + (threadIdx.x >> 5); p < n; p += gridDim.x * 8) {

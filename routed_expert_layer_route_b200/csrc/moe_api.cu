@@ -299,15 +299,14 @@ static int enqueue_grouped(const void *x, const void *wg, const void *wu, const 
         const int rows = (int)n;
         const int grid = (rows + 7) / 8 < 8 * G ? (rows + 7) / 8 : 8 * G;
         if ((rc = launch(k_gather_rows, dim3(grid), dim3(256), 0, s, pdl,
-                         static_cast<const uint16_t *>(x), sorted_slot, rows, d, k1, xs)) != MOE_OK)
+                         static_cast<const uint16_t *>(x), sorted_slot, rows, d, k1, xs,
+                         reinterpret_cast<float4 *>(y_acc), y_acc ? T * d / 4 : 0)) != MOE_OK)
             return rc;
     }
     Gemm1Args a1 = {};
     a1.offsets = offsets;
     a1.sorted_slot = sorted_slot;
     a1.h = h;
-    a1.zero = reinterpret_cast<float4 *>(y_acc);
-    a1.zero_n4 = y_acc ? T * d / 4 : 0;
     a1.sched = {&hdr->sched[0], &hdr->sched[1]};
     a1.T = T;
     a1.d = d;
