@@ -539,9 +539,10 @@ def run_native(args, world, rank):
                          "in %.1f s; per-layer time scaled to the %d-layer stack"
                          % (nl, min(T, 8), k1h, k2h, el, Ln)}
 
-    # kernels per layer: router, decode kernel, finalize (one token); router, top-k,
-    # streaming kernel (small batch); router, top-k, two grouped GEMMs, finalize
-    per_step_launches = 5 if stack.grouped else 3
+    # kernels per layer: router logits + decode kernel (one token); router logits,
+    # warp router, permutation (2), token-row gather, two grouped GEMMs, finalize
+    # (tensor-core path); router logits, top-k, streaming kernel (streaming path)
+    per_step_launches = 2 if stack.channel_major else (8 if stack.grouped else 3)
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
