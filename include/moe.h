@@ -75,6 +75,10 @@ typedef enum {
 #define MOE_DTYPE_F32 0
 #define MOE_DTYPE_BF16 1
 
+/* An unused slot of a variable-k (cascade) route: its topk_idx entry; its
+ * weight is 0.  The permutation skips such slots without a device check. */
+#define MOE_EMPTY_SLOT 0x7fffffff
+
 /* moe_layer / moe_expert_ffn flags: which expert-FFN path runs.
  * AUTO: one token with the channel-major down matrix -> DECODE; two or more
  * tokens with d and I multiples of 128 -> GROUPED; otherwise STREAM. */
@@ -141,7 +145,9 @@ int moe_route(const void *x_bf16, const void *w_router_bf16, const float *bias, 
  *  sorted_slot [T*k1]: slots ordered by (expert, slot index);
  *  slot_pos    [T*k1]: inverse, sorted_slot[slot_pos[i]] == i.
  *  An expert id outside [0, E) sets MOE_ERR_DEVICE_CHECK in the device status
- *  word when ws is given (the slot is then dropped).  ws may be NULL. */
+ *  word when ws is given (the slot is then dropped).  Slots holding
+ *  MOE_EMPTY_SLOT (variable-k routes) are skipped without a check; their
+ *  slot_pos entries are left as they were.  ws may be NULL. */
 int moe_permute(const int32_t *topk_idx, int T, int k1, int E, int32_t *expert_offsets,
                 int32_t *sorted_slot, int32_t *slot_pos, void *ws, size_t ws_bytes, void *stream);
 
@@ -176,6 +182,33 @@ int moe_layer(const void *x_bf16, const void *w_router_bf16, const float *bias,
               int E, int I, int k1, int k2, void *y, int y_dtype, int32_t *topk_idx_out,
               float *topk_w_out, float *logits_out, int flags, void *ws, size_t ws_bytes,
               void *stream);
+
+/* Variable number of experts per token (the "cascade ... cover" arm of
+ * "Reading the MoE measurement defects", kozo-lab, sections 4 and 6.2-6.3:
+ * each token runs experts in rank order until they cover a share tau of its
+ * probability mass).  Reading taken here: the mass after k experts is the
+ * float32 sum of the first k ranked probabilities in rank order (the same
+ * partial sums as the top-k2 mass of Eq. 2); token t takes k_t = the smallest
+ * k <= k1 whose mass is >= tau, else k1 (so 1 <= k_t <= k1).  Its weights are
+ * Eq. 2 with the fixed k2.  Routing outputs keep k1 slots per token; slots
+ * s >= k_t hold MOE_EMPTY_SLOT with weight 0.  topk_count [T] int32
+ * (nullable) receives k_t.  tau NaN: MOE_ERR_INVALID_ARG.  Other arguments
+ * as for moe_route. */
+int moe_route_cascade(const void *x_bf16, const void *w_router_bf16, const float *bias,
+                      float *logits, int T, int d, int E, int k1, int k2, float tau,
+                      int32_t *topk_idx, float *topk_w, int32_t *topk_count, void *ws,
+                      size_t ws_bytes, void *stream);
+
+/* moe_layer with the variable-k route of moe_route_cascade: y[t] sums only
+ * the token's k_t experts.  Runs on the one-token decode path (down matrix
+ * channel-major) and on the tensor-core grouped path (d, I multiples of 128);
+ * other shapes return MOE_ERR_UNSUPPORTED_SHAPE.  topk_count_out [T] int32
+ * (nullable) receives k_t.  Other arguments as for moe_layer. */
+int moe_layer_cascade(const void *x_bf16, const void *w_router_bf16, const float *bias,
+                      const void *w_gate_bf16, const void *w_up_bf16, const void *w_down_bf16,
+                      int T, int d, int E, int I, int k1, int k2, float tau, void *y, int y_dtype,
+                      int32_t *topk_idx_out, float *topk_w_out, int32_t *topk_count_out,
+                      float *logits_out, int flags, void *ws, size_t ws_bytes, void *stream);
 
 /* Channel-major copy of a down matrix, made once when the weights are
  * loaded: w_down_cm[e][c][r] = w_down[e][r][c] (w_down [E x d x I] bf16 ->

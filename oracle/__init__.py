@@ -45,6 +45,9 @@ def lib():
         L.oracle_softmax_f32.restype = None
         L.oracle_route_f32.argtypes = [f32p, ci, ci, ci, ci, i32p, f32p]
         L.oracle_route_f32.restype = ci
+        L.oracle_route_cascade_f32.argtypes = [f32p, ci, ci, ci, ci, ctypes.c_float, i32p, f32p,
+                                               i32p]
+        L.oracle_route_cascade_f32.restype = ci
         L.oracle_route_f64.argtypes = [f64p, ci, ci, ci, ci, i32p, f64p, f64p]
         L.oracle_route_f64.restype = ci
         L.oracle_logits.argtypes = [vp, ci, vp, ci, f32p, ci, ci, ci, f32p]
@@ -123,6 +126,48 @@ def route_f32(logits, k1, k2):
     return idx, w
 
 
+EMPTY_SLOT = 0x7fffffff  # an unused slot of a variable-k (cascade) route
+
+
+def route_cascade_f32(logits, kmax, k2, tau):
+    """Variable k per token: returns (idx [T x kmax], w [T x kmax], k [T]);
+    slots s >= k[t] hold EMPTY_SLOT and weight 0."""
+    z = _f32(logits)
+    T, E = z.shape
+    idx = np.empty((T, kmax), np.int32)
+    w = np.empty((T, kmax), np.float32)
+    k = np.empty(T, np.int32)
+    rc = lib().oracle_route_cascade_f32(_ptr(z, ctypes.c_float), T, E, kmax, k2, ctypes.c_float(tau),
+                                        _ptr(idx, ctypes.c_int32), _ptr(w, ctypes.c_float),
+                                        _ptr(k, ctypes.c_int32))
+    if rc != 0:
+        raise OracleError("oracle_route_cascade_f32: bad arguments (T=%d E=%d kmax=%d k2=%d)"
+                          % (T, E, kmax, k2))
+    return idx, w, k
+
+
+def layer_tokens_cascade(xrows, z_rows, fetch_expert, kmax, k2, tau):
+    """layer_tokens with the variable-k route: each token sums only its k[t]
+    experts.  Returns dict(y, idx, w, k)."""
+    idx, w, k = route_cascade_f32(z_rows, kmax, k2, tau)
+    n = idx.shape[0]
+    xa, xc = _wcode(xrows)
+    d = xa.shape[1]
+    xf_all = (xa.astype(np.uint32) << 16).view(np.float32) if xc == 1 else xa
+    y = np.empty((n, d), np.float32)
+    cache = {}
+    for t in range(n):
+        kt = int(k[t])
+        o = np.empty((kt, d), np.float32)
+        for s in range(kt):
+            e = int(idx[t, s])
+            if e not in cache:
+                cache[e] = fetch_expert(e)
+            _, o[s] = expert(xf_all[t], *cache[e], par=True)
+        y[t] = combine(o, w[t, :kt])
+    return {"y": y, "idx": idx, "w": w, "k": k}
+
+
 def route_f64(logits, k1, k2):
     z = np.ascontiguousarray(logits, dtype=np.float64)
     T, E = z.shape
@@ -188,7 +233,8 @@ def permute(idx, E):
                               _ptr(sorted_slot, ctypes.c_int32), _ptr(slot_pos, ctypes.c_int32))
     if rc != 0:
         raise OracleError("oracle_permute: expert index out of range")
-    return offsets, sorted_slot[:n], slot_pos[:n]
+    # slots holding EMPTY_SLOT are not placed (slot_pos -1)
+    return offsets, sorted_slot[:int(offsets[E])], slot_pos[:n]
 
 
 def layer(x, wr, bias, wg, wu, wd, k1, k2, logits_in=None):

@@ -46,6 +46,11 @@
  *  oracle_route_f32/_f64   pinned: Eq. 2 special cases and invariants,
  *                          brute-force subset enumeration, tie rule, the page's
  *                          router restated with library top-k
+ *  oracle_route_cascade_f32  pinned: tau below the top probability gives k = 1,
+ *                          tau above any reachable mass gives kmax, uniform
+ *                          logits give k = ceil(tau E) exactly, minimality by
+ *                          brute force (mass of the first k-1 < tau), equality
+ *                          with the fixed-k route on the taken prefix
  *  oracle_logits           pinned: library matmul (numpy) on exactly
  *                          representable inputs, bias shift
  *  oracle_expert           pinned: I=1 closed form, zero weights, library
@@ -67,6 +72,7 @@
 
 #define OR_OK 0
 #define OR_BAD_ARG (-1)
+#define ORACLE_EMPTY_SLOT 0x7fffffff /* an unused slot of a variable-k route */
 
 /* ------------------------------------------------------------------------ */
 /* element access: dtype 0 = float32, 1 = bfloat16 (upper half of a float32) */
@@ -294,6 +300,73 @@ int oracle_route_f32(const float *logits, int T, int E, int k1, int k2, int32_t 
 
 /* Double-precision twin: libm exp, plain index-order sums, the same ranking
  * and Eq. 2.  p_out (nullable) receives the [T x E] probabilities. */
+/* Variable k per token (the "cascade ... cover" arm of "Reading the MoE
+ * measurement defects", kozo-lab, sections 4 and 6.2-6.3): the experts are
+ * taken in rank order until their probability mass reaches tau.  Reading
+ * used here: the mass after k experts is the float32 sequential sum
+ * (((p_(0) + p_(1)) + ...) + p_(k-1)) from +0, the same partial sums as the
+ * top-k2 mass S; k_t = the smallest k <= kmax with mass >= tau, else kmax
+ * (so k_t >= 1).  Weights are Eq. 2 with the fixed k2 (kmax <= k2).  Output
+ * rows have kmax slots; slots s >= k_t hold ORACLE_EMPTY_SLOT and weight 0;
+ * count[t] = k_t (count nullable). */
+int oracle_route_cascade_f32(const float *logits, int T, int E, int kmax, int k2, float tau,
+                             int32_t *idx, float *w, int32_t *count)
+{
+    if (T < 0 || E < 1 || kmax < 1 || k2 < kmax || kmax > E)
+        return OR_BAD_ARG;
+    const int K = k2 < E ? k2 : E;
+    float *p = (float *)malloc(sizeof(float) * (size_t)E);
+    int *rank = (int *)malloc(sizeof(int) * (size_t)K);
+    char *taken = (char *)malloc((size_t)E);
+    if (!p || !rank || !taken) {
+        free(p);
+        free(rank);
+        free(taken);
+        return OR_BAD_ARG;
+    }
+    for (int t = 0; t < T; ++t) {
+        oracle_softmax_f32(logits + (size_t)t * E, E, p);
+        memset(taken, 0, (size_t)E);
+        for (int s = 0; s < K; ++s) {
+            int best = -1;
+            for (int j = 0; j < E; ++j)
+                if (!taken[j] && (best < 0 || before_f32(p, j, best)))
+                    best = j;
+            taken[best] = 1;
+            rank[s] = best;
+        }
+        int kt = kmax;
+        float M = 0.0f;
+        for (int s = 0; s < kmax; ++s) {
+            M = M + p[rank[s]];
+            if (M >= tau) {
+                kt = s + 1;
+                break;
+            }
+        }
+        float S = 0.0f;
+        if (k2 < E)
+            for (int s = 0; s < K; ++s)
+                S = S + p[rank[s]];
+        for (int s = 0; s < kmax; ++s) {
+            const size_t o = (size_t)t * kmax + s;
+            if (s < kt) {
+                idx[o] = rank[s];
+                w[o] = (k2 >= E) ? p[rank[s]] : p[rank[s]] / S;
+            } else {
+                idx[o] = ORACLE_EMPTY_SLOT;
+                w[o] = 0.0f;
+            }
+        }
+        if (count)
+            count[t] = kt;
+    }
+    free(p);
+    free(rank);
+    free(taken);
+    return OR_OK;
+}
+
 int oracle_route_f64(const double *logits, int T, int E, int k1, int k2, int32_t *idx, double *w,
                      double *p_out)
 {
@@ -432,6 +505,8 @@ int oracle_permute(const int32_t *idx, int T, int k1, int E, int32_t *offsets, i
     for (int e = 0; e <= E; ++e)
         offsets[e] = 0;
     for (int64_t i = 0; i < n; ++i) {
+        if (idx[i] == ORACLE_EMPTY_SLOT)
+            continue; /* an unused slot of a variable-k route: not placed */
         if (idx[i] < 0 || idx[i] >= E)
             return OR_BAD_ARG;
         offsets[idx[i] + 1] += 1;
@@ -444,6 +519,10 @@ int oracle_permute(const int32_t *idx, int T, int k1, int E, int32_t *offsets, i
     for (int e = 0; e < E; ++e)
         next[e] = offsets[e];
     for (int64_t i = 0; i < n; ++i) {
+        if (idx[i] == ORACLE_EMPTY_SLOT) {
+            slot_pos[i] = -1;
+            continue;
+        }
         int32_t pos = next[idx[i]]++;
         sorted_slot[pos] = (int32_t)i;
         slot_pos[i] = pos;

@@ -67,6 +67,9 @@ struct DecodeArgs {
     float *y_acc;  // [d] float32, zero on entry
     void *y;       // [d] output (y_dtype); written by the last CTA to finish
     int y_dtype;
+    int cascade;   // variable k: the first kt <= k1 ranked experts covering tau
+    float tau;
+    int32_t *count;  // nullable: kt
     WsHeader *hdr;
 };
 
@@ -116,6 +119,30 @@ __host__ __device__ inline int decode_channels_per_stage(int d)
     return n >= kWPS ? kWPS : (n < 1 ? 1 : n);
 }
 
+// This CTA's channel segments: the U activated experts laid end to end as
+// U*I channels, CTA b taking a balanced contiguous range.
+__device__ void decode_segments(DecodeSmem *ds, int U, int I, int G, int b, int *status)
+{
+    const unsigned tot = (unsigned)U * (unsigned)I;
+    const unsigned c_lo = split_lo(tot, G, b), c_hi = split_lo(tot, G, b + 1);
+    int ns = 0;
+    unsigned c = c_lo;
+    for (; c < c_hi && ns < kDMaxSeg;) {
+        const int u = (int)(c / (unsigned)I);
+        DSeg sg;
+        sg.u = u;
+        sg.a = (int)(c % (unsigned)I);
+        sg.b = (int)min((unsigned)I, c_hi - (unsigned)u * I);
+        ds->seg[ns++] = sg;
+        c = (unsigned)u * I + sg.b;
+    }
+    if (c < c_hi) {  // more segments than kDMaxSeg: the host rules this out
+        set_status(status, MOE_ERR_DEVICE_CHECK);
+        ns = 0;
+    }
+    ds->nseg = ns;
+}
+
 // VPL: d = 256*VPL for the single-token register path (x in registers when
 // VPL <= kXRegMax), 0 for the general token loop.
 template <int VPL>
@@ -141,26 +168,10 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
         ds->abort = 0;
         ds->issued = 0;
         fence_mbar_init();
-        // this CTA's channel segments depend only on k1, I and the grid: the
-        // U = k1 activated experts laid end to end as U*I channels
-        const unsigned tot = (unsigned)k1 * (unsigned)I;
-        const unsigned c_lo = split_lo(tot, G, b), c_hi = split_lo(tot, G, b + 1);
-        int ns = 0;
-        unsigned c = c_lo;
-        for (; c < c_hi && ns < kDMaxSeg;) {
-            const int u = (int)(c / (unsigned)I);
-            DSeg sg;
-            sg.u = u;
-            sg.a = (int)(c % (unsigned)I);
-            sg.b = (int)min((unsigned)I, c_hi - (unsigned)u * I);
-            ds->seg[ns++] = sg;
-            c = (unsigned)u * I + sg.b;
-        }
-        if (c < c_hi) {  // more segments than kDMaxSeg: the host rules this out
-            set_status(status, MOE_ERR_DEVICE_CHECK);
-            ns = 0;
-        }
-        ds->nseg = ns;
+        // this CTA's channel segments depend only on k1, I and the grid (with
+        // the cascade, on the routed count: computed after routing)
+        if (!a.cascade)
+            decode_segments(ds, k1, I, G, b, status);
     }
     __syncthreads();
 
@@ -169,22 +180,25 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
 
     // ------------------------------------------------------------ routing (one warp)
     if (warp == 0) {
-        int j;
+        int j, kt;
         float wv;
+        const bool cas = a.cascade != 0;
         if (E <= 128)
-            warp_route<4>(a.logits, E, k1, a.k2, lane, j, wv);
+            warp_route<4>(a.logits, E, k1, a.k2, lane, j, wv, cas, a.tau, &kt);
         else if (E <= 256)
-            warp_route<8>(a.logits, E, k1, a.k2, lane, j, wv);
+            warp_route<8>(a.logits, E, k1, a.k2, lane, j, wv, cas, a.tau, &kt);
         else if (E <= 512)
-            warp_route<16>(a.logits, E, k1, a.k2, lane, j, wv);
+            warp_route<16>(a.logits, E, k1, a.k2, lane, j, wv, cas, a.tau, &kt);
         else
-            warp_route<32>(a.logits, E, k1, a.k2, lane, j, wv);
-        int p = 0;  // position of this lane's expert among the k1, ascending
+            warp_route<32>(a.logits, E, k1, a.k2, lane, j, wv, cas, a.tau, &kt);
+        int p = 0;  // position of this lane's expert among the kt taken, ascending
         for (int q = 0; q < k1; ++q)
-            p += __shfl_sync(0xffffffffu, j, q) < j;
+            p += __shfl_sync(0xffffffffu, j, q) < j;  // empty slots never count
         if (lane < k1) {
-            ds->ue[p] = j;
-            ds->uw[p] = wv;
+            if (lane < kt) {
+                ds->ue[p] = j;
+                ds->uw[p] = wv;
+            }
             if (b == 0) {
                 a.topk_idx[lane] = j;
                 a.topk_w[lane] = wv;
@@ -192,18 +206,25 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
                     a.idx_copy[lane] = j;
                 if (a.w_copy)
                     a.w_copy[lane] = wv;
-                a.uniq_list[p] = j;
-                a.sorted_slot[p] = lane;
-                a.slot_pos[lane] = p;
+                if (lane < kt) {
+                    a.uniq_list[p] = j;
+                    a.sorted_slot[p] = lane;
+                }
+                a.slot_pos[lane] = lane < kt ? p : -1;
             }
         }
         __syncwarp();
+        if (cas && lane == 0)
+            decode_segments(ds, kt, I, G, b, status);
         if (b == 0) {
-            if (lane == 0)
-                *a.uniq_count = k1;
+            if (lane == 0) {
+                *a.uniq_count = kt;
+                if (a.count)
+                    *a.count = kt;
+            }
             for (int e = lane; e <= E; e += 32) {
                 int cnt = 0;
-                for (int q = 0; q < k1; ++q)
+                for (int q = 0; q < kt; ++q)
                     cnt += ds->ue[q] < e;
                 a.offsets[e] = cnt;
             }

@@ -803,11 +803,15 @@ __global__ void __launch_bounds__(kG2Threads, 1)
 }
 
 // xs[p] = x[sorted_slot[p] / k1]: the routed tokens' rows in expert order, the
-// token operand of the gate/up GEMM.  One warp per row, 16-byte vectors.  Also
-// clears the down GEMM's float32 accumulator (zero: nullable, zero_n4 float4s).
+// token operand of the gate/up GEMM.  One warp per row, 16-byte vectors; only
+// the offsets[E] placed slots (empty or dropped slots are not in the order),
+// and a slot id beyond the T*k1 slots records MOE_ERR_DEVICE_CHECK and is
+// skipped.  Also clears the down GEMM's float32 accumulator (zero: nullable,
+// zero_n4 float4s).
 __global__ void __launch_bounds__(256) k_gather_rows(const uint16_t *x, const int32_t *sorted_slot,
-                                                     int n, int d, int k1, uint16_t *xs,
-                                                     float4 *zero, int zero_n4)
+                                                     const int32_t *offsets, int E, int n, int d,
+                                                     int k1, uint16_t *xs, float4 *zero,
+                                                     int zero_n4, int *status)
 {
     pdl_wait();
     pdl_trigger();
@@ -816,8 +820,15 @@ __global__ void __launch_bounds__(256) k_gather_rows(const uint16_t *x, const in
             zero[q] = make_float4(0.f, 0.f, 0.f, 0.f);
     const int lane = threadIdx.x & 31;
     const int nv = d >> 3;
-    for (int p = blockIdx.x * 8 + (threadIdx.x >> 5); p < n; p += gridDim.x * 8) {
-        const int t = __ldcg(&sorted_slot[p]) / k1;
+    const int placed = min(n, __ldcg(&offsets[E]));
+    for (int p = blockIdx.x * 8 + (threadIdx.x >> 5); p < placed; p += gridDim.x * 8) {
+        const int slot = __ldcg(&sorted_slot[p]);
+        if (slot < 0 || slot >= n) {
+            if (lane == 0)
+                set_status(status, MOE_ERR_DEVICE_CHECK);
+            continue;
+        }
+        const int t = slot / k1;
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * d);
         uint4 *dst = reinterpret_cast<uint4 *>(xs + (size_t)p * d);
         for (int v = lane; v < nv; v += 32)

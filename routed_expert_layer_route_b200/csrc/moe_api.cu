@@ -197,7 +197,8 @@ static int enqueue_logits(const void *x, const void *wr, const float *bias, floa
 // kernel.
 static int enqueue_decode(const void *x, const void *wg, const void *wu, const void *wdt, int d,
                           int E, int I, int k1, int k2, void *y, int y_dtype, int32_t *idx_copy,
-                          float *w_copy, void *ws, int G, cudaStream_t s)
+                          float *w_copy, void *ws, int G, cudaStream_t s, bool cascade = false,
+                          float tau = 0.0f, int32_t *count = nullptr)
 {
     const WsLayout L = ws_layout(1, d, E, I, k1);
     DecodeArgs a = {};
@@ -223,6 +224,9 @@ static int enqueue_decode(const void *x, const void *wg, const void *wu, const v
     a.y_acc = at<float>(ws, L.y_acc);
     a.y = y;
     a.y_dtype = y_dtype;
+    a.cascade = cascade ? 1 : 0;
+    a.tau = tau;
+    a.count = count;
     a.hdr = static_cast<WsHeader *>(ws);
     const size_t smem = decode_smem_bytes(d);
     if (d == 2048)
@@ -299,8 +303,9 @@ static int enqueue_grouped(const void *x, const void *wg, const void *wu, const 
         const int rows = (int)n;
         const int grid = (rows + 7) / 8 < 8 * G ? (rows + 7) / 8 : 8 * G;
         if ((rc = launch(k_gather_rows, dim3(grid), dim3(256), 0, s, pdl,
-                         static_cast<const uint16_t *>(x), sorted_slot, rows, d, k1, xs,
-                         reinterpret_cast<float4 *>(y_acc), y_acc ? T * d / 4 : 0)) != MOE_OK)
+                         static_cast<const uint16_t *>(x), sorted_slot, offsets, E, rows, d, k1,
+                         xs, reinterpret_cast<float4 *>(y_acc), y_acc ? T * d / 4 : 0,
+                         &hdr->status)) != MOE_OK)
             return rc;
     }
     Gemm1Args a1 = {};
@@ -369,12 +374,13 @@ static int enqueue_logits_gemm(const void *x, const void *wr, const float *bias,
 
 // Warp-per-token routing of T tokens from float32 logits.
 static int enqueue_route_warp(const float *z, int T, int E, int k1, int k2, int32_t *idx, float *w,
-                              int32_t *idx_copy, float *w_copy, cudaStream_t s)
+                              int32_t *idx_copy, float *w_copy, cudaStream_t s,
+                              bool cascade = false, float tau = 0.0f, int32_t *count = nullptr)
 {
     const dim3 grid((T + 7) / 8), block(256);
 #define MOE_ROUTE_WARP(R)                                                                        \
     return launch(k_route_warp<R>, grid, block, 0, s, true, z, T, E, k1, k2, idx, w, idx_copy, \
-                  w_copy)
+                  w_copy, (int)cascade, tau, count)
     if (E <= 32) MOE_ROUTE_WARP(1);
     if (E <= 64) MOE_ROUTE_WARP(2);
     if (E <= 128) MOE_ROUTE_WARP(4);
@@ -467,9 +473,12 @@ int moe_read_device_status(void *ws, int *status_out, void *stream)
     return MOE_OK;
 }
 
-int moe_route(const void *x_bf16, const void *w_router_bf16, const float *bias, float *logits,
-              int T, int d, int E, int k1, int k2, int32_t *topk_idx, float *topk_w, void *ws,
-              size_t ws_bytes, void *stream)
+}  // extern "C" (route_impl below is internal)
+
+static int route_impl(const void *x_bf16, const void *w_router_bf16, const float *bias,
+                      float *logits, int T, int d, int E, int k1, int k2, int32_t *topk_idx,
+                      float *topk_w, void *ws, size_t ws_bytes, void *stream, bool cascade,
+                      float tau, int32_t *count)
 {
     int rc = check_route(E, k1, k2);
     if (rc != MOE_OK)
@@ -510,7 +519,29 @@ int moe_route(const void *x_bf16, const void *w_router_bf16, const float *bias, 
             return rc;
         z = zbuf;
     }
-    return enqueue_route_warp(z, T, E, k1, k2, topk_idx, topk_w, nullptr, nullptr, s);
+    return enqueue_route_warp(z, T, E, k1, k2, topk_idx, topk_w, nullptr, nullptr, s, cascade, tau,
+                              count);
+}
+
+extern "C" {
+
+int moe_route(const void *x_bf16, const void *w_router_bf16, const float *bias, float *logits,
+              int T, int d, int E, int k1, int k2, int32_t *topk_idx, float *topk_w, void *ws,
+              size_t ws_bytes, void *stream)
+{
+    return route_impl(x_bf16, w_router_bf16, bias, logits, T, d, E, k1, k2, topk_idx, topk_w, ws,
+                      ws_bytes, stream, false, 0.0f, nullptr);
+}
+
+int moe_route_cascade(const void *x_bf16, const void *w_router_bf16, const float *bias,
+                      float *logits, int T, int d, int E, int k1, int k2, float tau,
+                      int32_t *topk_idx, float *topk_w, int32_t *topk_count, void *ws,
+                      size_t ws_bytes, void *stream)
+{
+    if (tau != tau)
+        return MOE_ERR_INVALID_ARG;  // NaN
+    return route_impl(x_bf16, w_router_bf16, bias, logits, T, d, E, k1, k2, topk_idx, topk_w, ws,
+                      ws_bytes, stream, true, tau, topk_count);
 }
 
 int moe_permute(const int32_t *topk_idx, int T, int k1, int E, int32_t *expert_offsets,
@@ -716,11 +747,14 @@ int moe_combine(const float *expert_out, const int32_t *slot_pos, const float *t
                   true, expert_out, slot_pos, topk_w, T, d, k1, y, y_dtype, (int *)nullptr);
 }
 
-int moe_layer(const void *x_bf16, const void *w_router_bf16, const float *bias,
-              const void *w_gate_bf16, const void *w_up_bf16, const void *w_down_bf16, int T, int d,
-              int E, int I, int k1, int k2, void *y, int y_dtype, int32_t *topk_idx_out,
-              float *topk_w_out, float *logits_out, int flags, void *ws, size_t ws_bytes,
-              void *stream)
+}  // extern "C" (layer_impl below is internal)
+
+static int layer_impl(const void *x_bf16, const void *w_router_bf16, const float *bias,
+                      const void *w_gate_bf16, const void *w_up_bf16, const void *w_down_bf16,
+                      int T, int d, int E, int I, int k1, int k2, void *y, int y_dtype,
+                      int32_t *topk_idx_out, float *topk_w_out, float *logits_out, int flags,
+                      void *ws, size_t ws_bytes, void *stream, bool cascade, float tau,
+                      int32_t *count_out)
 {
     int rc = check_shape(T, d, E, I, k1);
     if (rc != MOE_OK)
@@ -767,6 +801,8 @@ int moe_layer(const void *x_bf16, const void *w_router_bf16, const float *bias,
                                       (path == MOE_PATH_AUTO && auto_grouped(T, d, E, I, k1)));
     if (grouped && !grouped_fits(d, E, I))
         return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (cascade && !decode && !grouped)
+        return MOE_ERR_UNSUPPORTED_SHAPE;  // the variable-k route runs on those two paths
     if (grouped) {
         // router logits (tensor-core GEMM when the experts fill 128-row tiles),
         // warp-per-token routing, the chunked stable permutation, the two
@@ -777,8 +813,8 @@ int moe_layer(const void *x_bf16, const void *w_router_bf16, const float *bias,
             rc = enqueue_logits(x_bf16, w_router_bf16, bias, z, logits_out, T, d, E, s);
         if (rc != MOE_OK)
             return rc;
-        if ((rc = enqueue_route_warp(z, T, E, k1, k2, idx, w, topk_idx_out, topk_w_out, s)) !=
-            MOE_OK)
+        if ((rc = enqueue_route_warp(z, T, E, k1, k2, idx, w, topk_idx_out, topk_w_out, s, cascade,
+                                     tau, count_out)) != MOE_OK)
             return rc;
         if ((rc = enqueue_perm_parallel(idx, T, k1, E, at<int>(ws, L.hist), po, &hdr->status, s)) !=
             MOE_OK)
@@ -798,7 +834,8 @@ int moe_layer(const void *x_bf16, const void *w_router_bf16, const float *bias,
         return rc;
     if (decode)
         return enqueue_decode(x_bf16, w_gate_bf16, w_up_bf16, w_down_bf16, d, E, I, k1, k2, y,
-                              y_dtype, topk_idx_out, topk_w_out, ws, G, s);
+                              y_dtype, topk_idx_out, topk_w_out, ws, G, s, cascade, tau,
+                              count_out);
     if (T > 1) {
         // one CTA per token ranks its probabilities; the last one to finish
         // builds the permutation tables
@@ -811,6 +848,32 @@ int moe_layer(const void *x_bf16, const void *w_router_bf16, const float *bias,
     return enqueue_stream(layer_stream_call(x_bf16, w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I,
                                             k1, k2, y, y_dtype, topk_idx_out, topk_w_out, ws),
                           s);
+}
+
+extern "C" {
+
+int moe_layer(const void *x_bf16, const void *w_router_bf16, const float *bias,
+              const void *w_gate_bf16, const void *w_up_bf16, const void *w_down_bf16, int T, int d,
+              int E, int I, int k1, int k2, void *y, int y_dtype, int32_t *topk_idx_out,
+              float *topk_w_out, float *logits_out, int flags, void *ws, size_t ws_bytes,
+              void *stream)
+{
+    return layer_impl(x_bf16, w_router_bf16, bias, w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I,
+                      k1, k2, y, y_dtype, topk_idx_out, topk_w_out, logits_out, flags, ws, ws_bytes,
+                      stream, false, 0.0f, nullptr);
+}
+
+int moe_layer_cascade(const void *x_bf16, const void *w_router_bf16, const float *bias,
+                      const void *w_gate_bf16, const void *w_up_bf16, const void *w_down_bf16,
+                      int T, int d, int E, int I, int k1, int k2, float tau, void *y, int y_dtype,
+                      int32_t *topk_idx_out, float *topk_w_out, int32_t *topk_count_out,
+                      float *logits_out, int flags, void *ws, size_t ws_bytes, void *stream)
+{
+    if (tau != tau)
+        return MOE_ERR_INVALID_ARG;  // NaN
+    return layer_impl(x_bf16, w_router_bf16, bias, w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I,
+                      k1, k2, y, y_dtype, topk_idx_out, topk_w_out, logits_out, flags, ws, ws_bytes,
+                      stream, true, tau, topk_count_out);
 }
 
 int moe_pack_w_down(const void *w_down_bf16, void *w_down_cm_bf16, int E, int d, int I,

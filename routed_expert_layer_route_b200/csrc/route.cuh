@@ -264,7 +264,7 @@ __device__ void permute_block(const int32_t *idx, int T, int k1, int E, PermOut 
         const int i = base + lane;
         int e = i < n ? __ldcg(&idx[i]) : -1;
         const bool valid = (e >= 0) & (e < E);
-        if (i < n && !valid)
+        if (i < n && !valid && e != MOE_EMPTY_SLOT)
             set_status(status, MOE_ERR_DEVICE_CHECK);
         const int key = valid ? e : -1;
         const unsigned grp = __match_any_sync(0xffffffffu, key);
@@ -397,29 +397,32 @@ __global__ void __launch_bounds__(1024) k_topk(const float *logits, int T, int E
 }
 
 // ---------------------------------------------------------------------------
-// warp_route: one warp routes one token from its E float32 logits z (global
-// memory), everything in registers.  Lane l holds logits j = l, l+32, ...
-// (R per lane, E <= 32 R), which is exactly the canonical partial-sum
-// assignment of the normaliser Z; the top-Kneed probabilities come out in
-// rank order by repeated warp arg-max on (p descending, j ascending) -- two
-// redux.sync per rank: the largest key, then the lowest index holding it --
-// so the top-k2 mass S is summed in rank order as it is found.  Same float
-// sequence, same bits as route_token_block.  Lane s < k1 returns the rank-s
-// expert in my_j and its Eq. 2 weight in my_w.  k_route_warp: one warp per
-// token of a batch.
+// warp_route_vals: one warp routes one token from its E float32 logits, held
+// as p[i] = z[lane + 32 i], everything in registers.  That assignment is
+// exactly the canonical partial-sum assignment of the normaliser Z; the
+// top-Kneed probabilities come out in rank order by repeated warp arg-max on
+// (p descending, j ascending) -- two redux.sync per rank: the largest key,
+// then the lowest index holding it -- so the top-k2 mass S is summed in rank
+// order as it is found.  Same float sequence, same bits as
+// route_token_block.  Lane s < k1 returns the rank-s expert in my_j and its
+// Eq. 2 weight in my_w.
+// Cascade (variable k per token, cascade = true; the "cascade ... cover" arm
+// of "Reading the MoE measurement defects", sections 4 and 6.2-6.3): the
+// experts are taken in rank order until their mass -- the same float32
+// rank-order partial sums as S -- reaches tau; kt = the smallest such
+// k <= k1, else k1, and lanes kt <= s < k1 return MOE_EMPTY_SLOT and weight
+// 0.  Without the cascade kt = k1.  k_route_warp: one warp per token.
 template <int R>
-__device__ __forceinline__ void warp_route(const float *z, int E, int k1, int k2, int lane,
-                                           int &my_j, float &my_w)
+__device__ __forceinline__ void warp_route_vals(float (&p)[R], int E, int k1, int k2, int lane,
+                                                int &my_j, float &my_w, bool cascade = false,
+                                                float tau = 0.0f, int *kt_out = nullptr)
 {
     const float kNegInf = -__int_as_float(0x7f800000);
-    float p[R];
     float m = kNegInf;
 #pragma unroll
-    for (int i = 0; i < R; ++i) {
-        const int j = lane + 32 * i;
-        p[i] = j < E ? __ldcg(&z[j]) : kNegInf;
-        m = fmaxf(m, p[i]);
-    }
+    for (int i = 0; i < R; ++i)
+        if (lane + 32 * i < E)
+            m = fmaxf(m, p[i]);
     asm volatile("redux.sync.max.f32 %0, %0, 0xffffffff;" : "+f"(m));  // exact in any order
     float Z = 0.0f;
 #pragma unroll
@@ -441,6 +444,8 @@ __device__ __forceinline__ void warp_route(const float *z, int E, int k1, int k2
     const bool renorm = k2 < E;
     const int Kneed = renorm ? K : k1;
     float S = 0.0f, my_p = 0.0f;
+    int kt = k1;
+    bool covered = false;
     my_j = 0;
     for (int r = 0; r < Kneed; ++r) {
         unsigned kl = 0u;
@@ -458,20 +463,45 @@ __device__ __forceinline__ void warp_route(const float *z, int E, int k1, int k2
             my_j = bj;
             my_p = bp;
         }
-        if (renorm)
-            S = __fadd_rn(S, bp);
+        S = __fadd_rn(S, bp);  // mass of the first r+1 ranks
+        if (cascade && !covered && r < k1 && S >= tau) {
+            covered = true;
+            kt = r + 1;
+        }
 #pragma unroll
         for (int i = 0; i < R; ++i)
             if (lane + 32 * i == bj)
                 key[i] = 0u;
     }
     my_w = renorm ? __fdiv_rn(my_p, S) : my_p;
+    if (lane >= kt && lane < k1) {
+        my_j = MOE_EMPTY_SLOT;
+        my_w = 0.0f;
+    }
+    if (kt_out)
+        *kt_out = kt;
+}
+
+// The same from E logits in global memory.
+template <int R>
+__device__ __forceinline__ void warp_route(const float *z, int E, int k1, int k2, int lane,
+                                           int &my_j, float &my_w, bool cascade = false,
+                                           float tau = 0.0f, int *kt_out = nullptr)
+{
+    float p[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+        const int j = lane + 32 * i;
+        p[i] = j < E ? __ldcg(&z[j]) : 0.0f;
+    }
+    warp_route_vals<R>(p, E, k1, k2, lane, my_j, my_w, cascade, tau, kt_out);
 }
 
 template <int R>
 __global__ void __launch_bounds__(256) k_route_warp(const float *logits, int T, int E, int k1,
                                                     int k2, int32_t *idx, float *w,
-                                                    int32_t *idx_copy, float *w_copy)
+                                                    int32_t *idx_copy, float *w_copy,
+                                                    int cascade, float tau, int32_t *count)
 {
     pdl_wait();
     pdl_trigger();
@@ -479,9 +509,11 @@ __global__ void __launch_bounds__(256) k_route_warp(const float *logits, int T, 
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= T)
         return;
-    int my_j;
+    int my_j, kt;
     float my_w;
-    warp_route<R>(logits + (size_t)t * E, E, k1, k2, lane, my_j, my_w);
+    warp_route<R>(logits + (size_t)t * E, E, k1, k2, lane, my_j, my_w, cascade != 0, tau, &kt);
+    if (count && lane == 0)
+        count[t] = kt;
     if (lane < k1) {
         const size_t o = (size_t)t * k1 + lane;
         idx[o] = my_j;
@@ -520,7 +552,8 @@ __global__ void __launch_bounds__(256) k_perm_hist(const int32_t *idx, int T, in
     for (int i = tid; i < m; i += nt) {
         const int e = ids[i];
         if (e < 0 || e >= E) {
-            set_status(status, MOE_ERR_DEVICE_CHECK);
+            if (e != MOE_EMPTY_SLOT)
+                set_status(status, MOE_ERR_DEVICE_CHECK);
             continue;
         }
         atomicAdd(&cnt[e], 1);

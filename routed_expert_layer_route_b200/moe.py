@@ -32,11 +32,13 @@ MOE_PATH_GROUPED = 2
 MOE_PATH_DECODE = 3
 MOE_PATH_MASK = 0xFF
 MOE_WDOWN_CHANNEL_MAJOR = 0x100
+MOE_EMPTY_SLOT = 0x7FFFFFFF
 
 # every symbol include/*.h declares, with (restype, argtypes)
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
 _sz = ctypes.c_size_t
+_f = ctypes.c_float
 SIGNATURES = {
     "moe_status_string": (ctypes.c_char_p, [_i]),
     "moe_version": (_i, []),
@@ -50,6 +52,10 @@ SIGNATURES = {
     "moe_combine": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _i, _vp]),
     "moe_layer": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp,
                        _vp, _i, _vp, _sz, _vp]),
+    "moe_route_cascade": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _sz,
+                               _vp]),
+    "moe_layer_cascade": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _i,
+                               _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp]),
     "moe_expert_ffn_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
     "moe_pack_w_down": (_i, [_vp, _vp, _i, _i, _i, _vp]),
     "moe_test_exp_c": (_i, [_vp, _vp, ctypes.c_int64, _vp]),
@@ -249,3 +255,33 @@ def moe_test_expert_grouped(x, w_gate, w_up, w_down, k1, which, ws, stream=None)
     _check(lib().moe_test_expert_grouped(_p(x), _p(w_gate), _p(w_up), _p(w_down), T, d, E, I, k1,
                                          which, wsp, wsn, _stream(stream)),
            "moe_test_expert_grouped")
+
+
+def moe_route_cascade(x, w_router, bias, logits, k1, k2, tau, topk_idx, topk_w, topk_count=None,
+                      ws=None, stream=None):
+    """Variable-k route (k_t <= k1 per token covering mass tau); unused slots
+    hold MOE_EMPTY_SLOT with weight 0."""
+    if x is None:
+        T, E = logits.shape
+        d = 0
+    else:
+        T, d = x.shape
+        E = w_router.shape[0]
+    wsp, wsn = _ws_args(ws)
+    _check(lib().moe_route_cascade(_p(x), _p(w_router), _p(bias), _p(logits), T, d, E, k1, k2,
+                                   float(tau), _p(topk_idx), _p(topk_w), _p(topk_count), wsp, wsn,
+                                   _stream(stream)), "moe_route_cascade")
+
+
+def moe_layer_cascade(x, w_router, bias, w_gate, w_up, w_down, k1, k2, tau, y, ws,
+                      topk_idx_out=None, topk_w_out=None, topk_count_out=None, logits_out=None,
+                      flags=MOE_PATH_AUTO, stream=None):
+    """moe_layer with the variable-k route."""
+    T, d = x.shape
+    E, I, _ = w_gate.shape
+    y_dtype = MOE_DTYPE_BF16 if y.dtype == torch.bfloat16 else MOE_DTYPE_F32
+    wsp, wsn = _ws_args(ws)
+    _check(lib().moe_layer_cascade(_p(x), _p(w_router), _p(bias), _p(w_gate), _p(w_up), _p(w_down),
+                                   T, d, E, I, k1, k2, float(tau), _p(y), y_dtype, _p(topk_idx_out),
+                                   _p(topk_w_out), _p(topk_count_out), _p(logits_out), flags, wsp,
+                                   wsn, _stream(stream)), "moe_layer_cascade")

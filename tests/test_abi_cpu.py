@@ -116,6 +116,26 @@ def test_other_calls_argument_checks(L):
                                     None) == moe.MOE_ERR_INVALID_ARG
 
 
+def test_cascade_argument_checks(L):
+    nan = float("nan")
+    r = L.moe_route_cascade(None, None, None, FAKE, 4, 0, 128, 8, 16, nan, FAKE, FAKE, None, None,
+                            0, None)
+    assert r == moe.MOE_ERR_INVALID_ARG                                # tau NaN
+    r = L.moe_route_cascade(None, None, None, FAKE, 4, 0, 128, 8, 4, 0.5, FAKE, FAKE, None, None, 0,
+                            None)
+    assert r == moe.MOE_ERR_INVALID_ARG                                # k2 < k1
+    r = L.moe_route_cascade(None, None, None, FAKE, 0, 0, 128, 8, 16, 0.9, FAKE, FAKE, None, None,
+                            0, None)
+    assert r == moe.MOE_OK                                             # T = 0
+
+    def lc(tau=0.7, k1=8, k2=8, T=1):
+        return L.moe_layer_cascade(FAKE, FAKE, None, FAKE, FAKE, FAKE, T, 2048, 128, 768, k1, k2,
+                                   tau, FAKE, 1, None, None, None, None, 0, FAKE, 1 << 40, None)
+    assert lc(tau=nan) == moe.MOE_ERR_INVALID_ARG
+    assert lc(k1=8, k2=4) == moe.MOE_ERR_INVALID_ARG
+    assert lc(T=0) == moe.MOE_OK
+
+
 def test_binding_raises_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(moe, "_lib", None)
     monkeypatch.setattr(moe, "LIB_PATH", str(tmp_path / "missing.so"))
