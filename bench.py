@@ -205,9 +205,10 @@ class Stack:
     at set-up (moe_pack_w_down; the original layout is then freed), and the
     layers run the single-pass decode path."""
 
-    def __init__(self, wl, seed, device):
+    def __init__(self, wl, seed, device, tau=None, router_std=None):
         from routed_expert_layer_route_b200 import moe, synth
         self.wl = wl
+        self.tau = tau  # not None: the variable-k (cascade) route
         self.layers = []
         self.channel_major = wl["T"] == 1
         # two or more tokens: the tensor-core grouped GEMMs (what AUTO picks when d
@@ -218,10 +219,26 @@ class Stack:
         for l in range(wl["layers"]):
             L = synth.make_layer(wl["T"], wl["d"], wl["E"], wl["I"], seed=seed, layer=l,
                                  device=device, bias=wl["bias"])
+            if router_std:  # router logits with this standard deviation (x is RMS-normalised)
+                scale = router_std / (0.02 * wl["d"] ** 0.5)
+                L.w_router = (L.w_router.float() * scale).to(torch.bfloat16)
             if self.channel_major:
                 L.w_down = moe.moe_pack_w_down(L.w_down)
             self.layers.append(L)
         torch.cuda.synchronize()
+
+    def call(self, L, k1, k2, y, ws, stream, idx=None, count=None, x=None, fixed=False):
+        """One layer through the public API: moe_layer, or moe_layer_cascade
+        when the stack routes with a cascade (unless fixed)."""
+        from routed_expert_layer_route_b200 import moe
+        x = L.x if x is None else x
+        if self.tau is None or fixed:
+            moe.moe_layer(x, L.w_router, L.bias, L.w_gate, L.w_up, L.w_down, k1, k2, y, ws,
+                          topk_idx_out=idx, flags=self.flags, stream=stream)
+        else:
+            moe.moe_layer_cascade(x, L.w_router, L.bias, L.w_gate, L.w_up, L.w_down, k1, k2,
+                                  self.tau, y, ws, topk_idx_out=idx, topk_count_out=count,
+                                  flags=self.flags, stream=stream)
 
     def down_hf(self, L, e):
         """Expert e's down matrix in the [d x I] layout (host copy for the oracle)."""
@@ -230,35 +247,34 @@ class Stack:
         return synth.to_numpy(wd.contiguous())
 
 
-def build_graph(stack, k1, k2, ws_list, ys, stream):
-    """Capture one step (every layer's moe_layer) into a CUDA graph."""
-    from routed_expert_layer_route_b200 import moe
+def build_graph(stack, k1, k2, ws_list, ys, stream, fixed=False):
+    """Capture one step (every layer's layer call) into a CUDA graph."""
     g = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
         # one eager pass first (module attribute set-up happens outside capture)
         for L, ws, y in zip(stack.layers, ws_list, ys):
-            moe.moe_layer(L.x, L.w_router, L.bias, L.w_gate, L.w_up, L.w_down, k1, k2, y, ws,
-                          flags=stack.flags, stream=stream)
+            stack.call(L, k1, k2, y, ws, stream, fixed=fixed)
         stream.synchronize()
         with torch.cuda.graph(g, stream=stream):
             for L, ws, y in zip(stack.layers, ws_list, ys):
-                moe.moe_layer(L.x, L.w_router, L.bias, L.w_gate, L.w_up, L.w_down, k1, k2, y, ws,
-                              flags=stack.flags, stream=stream)
+                stack.call(L, k1, k2, y, ws, stream, fixed=fixed)
     return g
 
 
 def unique_experts(stack, k1, k2, ws_list, ys, stream):
-    """Activated experts per layer, read back from the routing outputs."""
+    """Activated experts per layer and the mean experts per token, read back
+    from the routing outputs (empty slots of a cascade route excluded)."""
     from routed_expert_layer_route_b200 import moe
-    us = []
+    us, ks = [], []
     wl = stack.wl
     for L, ws, y in zip(stack.layers, ws_list, ys):
         idx = torch.empty(wl["T"], k1, dtype=torch.int32, device=L.x.device)
-        moe.moe_layer(L.x, L.w_router, L.bias, L.w_gate, L.w_up, L.w_down, k1, k2, y, ws,
-                      topk_idx_out=idx, flags=stack.flags, stream=stream)
+        stack.call(L, k1, k2, y, ws, stream, idx=idx)
         stream.synchronize()
-        us.append(int(torch.unique(idx).numel()))
-    return us
+        taken = idx[idx != moe.MOE_EMPTY_SLOT]
+        us.append(int(torch.unique(taken).numel()))
+        ks.append(taken.numel() / wl["T"])
+    return us, statistics.mean(ks)
 
 
 def graph_time_per_call(calls, stream, reps):
@@ -325,8 +341,7 @@ def e2e_tokens_per_s(stack, k1, k2, ws_list, steps, warmup, stream):
     def step():
         dev_x.copy_(host_x, non_blocking=True)
         for l, (L, ws) in enumerate(zip(stack.layers, ws_list)):
-            moe.moe_layer(dev_x[l], L.w_router, L.bias, L.w_gate, L.w_up, L.w_down, k1, k2,
-                          dev_y[l], ws, flags=stack.flags, stream=stream)
+            stack.call(L, k1, k2, dev_y[l], ws, stream, x=dev_x[l])
         host_y.copy_(dev_y, non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -394,12 +409,14 @@ def run_native(args, world, rank):
     sweep = list(wl["sweep"])
     if args.k1:
         sweep = [(args.k1, args.k2 or args.k1)]
+    elif args.cascade is not None:  # one cascade condition: cap k1 = 8, k2 = 8
+        sweep = [(8, args.k2 or 8)]
     head = sweep[0]
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.Stream()
     hbm_peak, bf16_peak, peak_kind = load_peaks()
 
-    stack = Stack(wl, seed=rank, device=dev)
+    stack = Stack(wl, seed=rank, device=dev, tau=args.cascade, router_std=args.router_std)
     T, d, E, I, Ln = wl["T"], wl["d"], wl["E"], wl["I"], wl["layers"]
     results = []
     graphs = {}
@@ -409,8 +426,10 @@ def run_native(args, world, rank):
         g = build_graph(stack, k1, k2, ws_list, ys, stream)
         graphs[(k1, k2)] = (g, ws_list, ys)
 
-    def timed(k1, k2, steps, warmup):
-        g = graphs[(k1, k2)][0]
+    def timed(*args_):
+        key, (steps, warmup) = (args_[0], args_[1:]) if isinstance(args_[0], tuple) else \
+            ((args_[0], args_[1]), args_[2:])
+        g = graphs[key][0]
         with torch.cuda.stream(stream):
             for _ in range(warmup):
                 g.replay()
@@ -442,14 +461,30 @@ def run_native(args, world, rank):
         ms = ms_step if (k1, k2) == head else timed(k1, k2, args.steps, args.warmup)[0]
         sweep_t1 = time.time()
         _, ws_list, ys = graphs[(k1, k2)]
-        us = unique_experts(stack, k1, k2, ws_list, ys, stream)
+        us, mean_k = unique_experts(stack, k1, k2, ws_list, ys, stream)
         U = statistics.mean(us)
         bytes_layer = U * 3 * d * I * 2
-        flops_layer = T * (k1 * 6.0 * d * I + 2.0 * d * E)
+        flops_layer = T * (mean_k * 6.0 * d * I + 2.0 * d * E)
         results.append({"k1": k1, "k2": k2, "ms_per_step": ms, "us_per_layer": ms * 1000 / Ln,
                         "tokens_per_s": world * T * 1000.0 / ms, "unique_experts_per_layer": U,
                         "expert_GBps": bytes_layer / (ms / Ln * 1e-3) / 1e9,
-                        "layer_TFLOPs": flops_layer / (ms / Ln * 1e-3) / 1e12})
+                        "layer_TFLOPs": flops_layer / (ms / Ln * 1e-3) / 1e12,
+                        "mean_experts_per_token": mean_k})
+
+    cascade = None
+    if stack.tau is not None:
+        # the same stack with the fixed k1 route: compute saved vs time saved
+        k1h_, k2h_ = head
+        _, ws_list, ys = graphs[head]
+        gf = build_graph(stack, k1h_, k2h_, ws_list, ys, stream, fixed=True)
+        graphs[("fixed",) + head] = (gf, ws_list, ys)
+        ms_fixed = timed(("fixed",) + head, args.steps, args.warmup)[0]
+        cascade = {"tau": stack.tau, "k1_cap": k1h_, "k2": k2h_,
+                   "mean_experts_per_token": results[0]["mean_experts_per_token"],
+                   "us_per_layer": results[0]["us_per_layer"],
+                   "fixed_k1_us_per_layer": ms_fixed * 1000 / Ln,
+                   "time_ratio_vs_fixed": results[0]["us_per_layer"] / (ms_fixed * 1000 / Ln),
+                   "compute_ratio_vs_fixed": results[0]["mean_experts_per_token"] / k1h_}
 
     clocks.stop()
     clk, _ = clocks.summary(*head_win)
@@ -463,7 +498,17 @@ def run_native(args, world, rank):
     _, ws_list, ys = graphs[head]
     U_head = results[0]["unique_experts_per_layer"]
     alg_bytes = U_head * 3 * d * I * 2
-    if stack.grouped:
+    if stack.tau is not None:
+        # the kernels alone are re-run only with the fixed route; for a cascade
+        # route the roofline is taken over the whole layer
+        lay_s = results[0]["us_per_layer"] * 1e-6
+        achieved = alg_bytes / lay_s / 1e9
+        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
+                    "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": None,
+                    "kernel": "whole layer (cascade route)", "kernel_us": round(lay_s * 1e6, 2),
+                    "algorithmic_bytes_per_launch": int(alg_bytes),
+                    "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind}
+    elif stack.grouped:
         gx_ms, g1_ms, g2_ms = time_grouped_kernels(stack, k1h, ws_list, stream, reps=3)
         n_slots = T * k1h
         # algorithmic work of each GEMM: FLOPs, and bytes = the unique experts'
@@ -532,7 +577,7 @@ def run_native(args, world, rank):
             break
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and stack.tau is None:
         rate, nl, thr, el = cpu_oracle_rate(stack, k1h, k2h)
         cpu = {"value": rate, "unit": "tokens/s", "cores": thr, "kind": "oracle",
                "sample": "%d layers of this workload, first %d token(s) of each (k1=%d, k2=%d), "
@@ -552,6 +597,7 @@ def run_native(args, world, rank):
                                % (args.workload, Ln, d, E, I, T, k1h, k2h),
                    "layers": Ln, "d": d, "E": E, "I": I, "T": T, "k1": k1h, "k2": k2h,
                    "bias": wl["bias"], "us_per_layer": round(ms_step * 1000 / Ln, 3),
+                   "cascade_tau": stack.tau, "router_logit_std": args.router_std,
                    "l2": "inputs larger than L2: every step reads the routed experts of all "
                          "%d layers (%.2f GB) from HBM" % (Ln, alg_bytes * Ln / 1e9),
                    "timing": "CUDA graph of the %d-layer step, CUDA events, max over ranks" % Ln,
@@ -566,6 +612,7 @@ def run_native(args, world, rank):
         "gpu_launches": per_step_launches * Ln * args.steps,
         "clocks": clk,
         "sweep": results,
+        "cascade": cascade,
         "k1_4_over_k1_8_time_ratio": None if ratio is None else round(ratio, 4),
         "k1_ratio_conditions": ratio_pair,
     }
@@ -630,6 +677,10 @@ def main():
     ap.add_argument("--T", type=int, default=0)
     ap.add_argument("--layers", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cascade", type=float, default=None, metavar="TAU",
+                    help="variable experts per token: the first k <= k1 covering mass TAU")
+    ap.add_argument("--router-std", type=float, default=None,
+                    help="scale the router so its logits have this standard deviation")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
