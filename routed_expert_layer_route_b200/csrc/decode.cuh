@@ -144,8 +144,9 @@ __device__ void decode_segments(DecodeSmem *ds, int U, int I, int G, int b, int 
 }
 
 // VPL: d = 256*VPL for the single-token register path (x in registers when
-// VPL <= kXRegMax), 0 for the general token loop.
-template <int VPL>
+// VPL <= kXRegMax), 0 for the general token loop.  CASCADE: the variable-k
+// route (a.cascade is then set).
+template <int VPL, bool CASCADE>
 __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -170,7 +171,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
         fence_mbar_init();
         // this CTA's channel segments depend only on k1, I and the grid (with
         // the cascade, on the routed count: computed after routing)
-        if (!a.cascade)
+        if constexpr (!CASCADE)
             decode_segments(ds, k1, I, G, b, status);
     }
     __syncthreads();
@@ -182,7 +183,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
     if (warp == 0) {
         int j, kt;
         float wv;
-        const bool cas = a.cascade != 0;
+        constexpr bool cas = CASCADE;
         if (E <= 128)
             warp_route<4>(a.logits, E, k1, a.k2, lane, j, wv, cas, a.tau, &kt);
         else if (E <= 256)
@@ -214,8 +215,10 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
             }
         }
         __syncwarp();
-        if (cas && lane == 0)
-            decode_segments(ds, kt, I, G, b, status);
+        if constexpr (CASCADE) {
+            if (lane == 0)
+                decode_segments(ds, kt, I, G, b, status);
+        }
         if (b == 0) {
             if (lane == 0) {
                 *a.uniq_count = kt;

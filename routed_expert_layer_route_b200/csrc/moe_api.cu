@@ -115,12 +115,13 @@ static int device_info(DevInfo *&out)
                                  stream_smem) != cudaSuccess)
             return MOE_ERR_CUDA;
         const int decode_smem = 227 * 1024;
-        if (cudaFuncSetAttribute(k_decode<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 decode_smem) != cudaSuccess ||
-            cudaFuncSetAttribute(k_decode<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 decode_smem) != cudaSuccess ||
-            cudaFuncSetAttribute(k_decode<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 decode_smem) != cudaSuccess)
+        const cudaFuncAttribute dsm = cudaFuncAttributeMaxDynamicSharedMemorySize;
+        if (cudaFuncSetAttribute(k_decode<0, false>, dsm, decode_smem) != cudaSuccess ||
+            cudaFuncSetAttribute(k_decode<8, false>, dsm, decode_smem) != cudaSuccess ||
+            cudaFuncSetAttribute(k_decode<16, false>, dsm, decode_smem) != cudaSuccess ||
+            cudaFuncSetAttribute(k_decode<0, true>, dsm, decode_smem) != cudaSuccess ||
+            cudaFuncSetAttribute(k_decode<8, true>, dsm, decode_smem) != cudaSuccess ||
+            cudaFuncSetAttribute(k_decode<16, true>, dsm, decode_smem) != cudaSuccess)
             return MOE_ERR_CUDA;
         if (cudaFuncSetAttribute(k_gemm1, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gemm1_smem_bytes()) != cudaSuccess ||
@@ -229,11 +230,19 @@ static int enqueue_decode(const void *x, const void *wg, const void *wu, const v
     a.count = count;
     a.hdr = static_cast<WsHeader *>(ws);
     const size_t smem = decode_smem_bytes(d);
+    const dim3 grid(G), block(kSThreads);
+    if (cascade) {
+        if (d == 2048)
+            return launch(k_decode<8, true>, grid, block, smem, s, true, a);
+        if (d == 4096)
+            return launch(k_decode<16, true>, grid, block, smem, s, true, a);
+        return launch(k_decode<0, true>, grid, block, smem, s, true, a);
+    }
     if (d == 2048)
-        return launch(k_decode<8>, dim3(G), dim3(kSThreads), smem, s, true, a);
+        return launch(k_decode<8, false>, grid, block, smem, s, true, a);
     if (d == 4096)
-        return launch(k_decode<16>, dim3(G), dim3(kSThreads), smem, s, true, a);
-    return launch(k_decode<0>, dim3(G), dim3(kSThreads), smem, s, true, a);
+        return launch(k_decode<16, false>, grid, block, smem, s, true, a);
+    return launch(k_decode<0, false>, grid, block, smem, s, true, a);
 }
 
 
@@ -952,10 +961,11 @@ int moe_test_expert_stream(const void *x_bf16, const void *w_gate_bf16, const vo
         a.hdr = static_cast<WsHeader *>(ws);
         const size_t smem = decode_smem_bytes(d);
         if (d == 2048)
-            return launch(k_decode<8>, dim3(di->num_sms), dim3(kSThreads), smem, s, false, a);
+            return launch(k_decode<8, false>, dim3(di->num_sms), dim3(kSThreads), smem, s, false, a);
         if (d == 4096)
-            return launch(k_decode<16>, dim3(di->num_sms), dim3(kSThreads), smem, s, false, a);
-        return launch(k_decode<0>, dim3(di->num_sms), dim3(kSThreads), smem, s, false, a);
+            return launch(k_decode<16, false>, dim3(di->num_sms), dim3(kSThreads), smem, s, false,
+                          a);
+        return launch(k_decode<0, false>, dim3(di->num_sms), dim3(kSThreads), smem, s, false, a);
     }
     return enqueue_stream(layer_stream_call(x_bf16, w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I,
                                             k1, k2, y, y_dtype, nullptr, nullptr, ws),
