@@ -294,3 +294,107 @@ def layer_tokens(xrows, z_rows, fetch_expert, k1, k2):
             _, o[s] = expert(xf_all[t], wg, wu, wd, par=True)
         y[t] = combine(o, w[t])
     return {"y": y, "idx": idx, "w": w}
+
+
+# ---------------------------------------------------------------------------
+# Channel top-k inside the activated experts ("Channel Selection for
+# Mixture-of-Experts Decoding Needs No Calibration Data", paperlayer.ai):
+# section 2 "Background" (channel c of a routed expert owns gate row c, up
+# row c and down column c), section 5.2 "Output-scaled scoring and exact
+# top-k computation" (score = router weight x down-column norm x activation
+# magnitude, in output units, so that channels of different experts compare
+# and the best ones are taken across a token's experts), section 5.3 (kept
+# channels are computed exactly).  The ternary sketch that screens channels
+# and the low-rank recovery of skipped ones are not part of this oracle: h is
+# computed exactly for every channel and skipped channels add nothing.
+
+
+def _widen(a):
+    a, code = _wcode(a)
+    return (a.astype(np.uint32) << 16).view(np.float32) if code == 1 else a
+
+
+def channel_norms(wd):
+    """Down-column norms of one expert: wd [d x I] (bf16 bits or float32) ->
+    float32 [I], n_c = sqrt(sum_r wd[r, c]^2) in float64, rounded once."""
+    w = _widen(wd).astype(np.float64)
+    return np.sqrt((w * w).sum(axis=0)).astype(np.float32)
+
+
+def channel_scores(h, w, norms):
+    """Output-scaled channel scores of one token: h [k x I] float32 channel
+    activations of its k slots, w [k] float32 Eq. 2 weights, norms [k x I]
+    float32 down-column norms of each slot's expert.  score = (w_s * n) * |h|,
+    two float32 products in that order, each rounded once."""
+    h = _f32(h)
+    wn = np.asarray(w, np.float32)[:, None] * _f32(norms)
+    return (wn * np.abs(h)).astype(np.float32)
+
+
+def channel_select(scores, keep):
+    """The `keep` best channels of one token over all its slots: flat indices
+    q = s*I + c (ascending) of the largest float32 scores, equal scores going
+    to the lower flat index (slot rank first, then channel).  Scores must be
+    finite and non-negative."""
+    s = np.asarray(scores, np.float32).ravel()
+    if not 1 <= keep <= s.size:
+        raise OracleError("channel_select: keep=%d outside [1, %d]" % (keep, s.size))
+    if not np.isfinite(s).all() or (s < 0).any():
+        raise OracleError("channel_select: scores must be finite and non-negative")
+    order = np.lexsort((np.arange(s.size), -s.astype(np.float64)))
+    return np.sort(order[:keep]).astype(np.int32)
+
+
+def channel_topk_tokens(xrows, z_rows, fetch_expert, fetch_norms, k1, k2, keep, scores_in=None,
+                        kept_in=None):
+    """Layer output with channel top-k for a few tokens.
+
+    xrows [n x d] float32 or bf16 bits, z_rows [n x E] float32 logits to route
+    on, fetch_expert(e) -> (wg [I x d], wu [I x d], wd [d x I]),
+    fetch_norms(e) -> float32 [I] down-column norms, keep channels per token.
+    Per token: route (Eq. 2), h [k1 x I] for every channel of its k1 experts
+    (oracle_expert), scores (channel_scores), the kept set (channel_select on
+    scores_in[t] when given, else on its own scores; kept_in[t] overrides
+    both), and y = sum over kept (s, c) of w_s * h[s, c] * wd_s[:, c],
+    accumulated in float64.  Returns dict(y [n x d] float32, idx, w, h,
+    norms, scores, kept [n x keep])."""
+    idx, w = route_f32(z_rows, k1, k2)
+    n = idx.shape[0]
+    xf_all = _widen(xrows)
+    d = xf_all.shape[1]
+    cache, ncache = {}, {}
+    hs, ns, ss, ks = [], [], [], []
+    y = np.empty((n, d), np.float32)
+    for t in range(n):
+        h = []
+        nrm = []
+        for s in range(k1):
+            e = int(idx[t, s])
+            if e not in cache:
+                cache[e] = fetch_expert(e)
+                ncache[e] = _f32(fetch_norms(e))
+            h.append(expert(xf_all[t], *cache[e], par=True)[0])
+            nrm.append(ncache[e])
+        h = np.stack(h)
+        nrm = np.stack(nrm)
+        I = h.shape[1]
+        sc = channel_scores(h, w[t], nrm)
+        if kept_in is not None:
+            kept = np.asarray(kept_in[t], np.int32)
+        else:
+            kept = channel_select(sc if scores_in is None else scores_in[t], keep)
+        acc = np.zeros(d, np.float64)
+        slot, ch = np.divmod(kept, I)
+        for s in range(k1):
+            cs = ch[slot == s]
+            if cs.size:
+                wd = _widen(cache[int(idx[t, s])][2]).astype(np.float64)
+                coef = float(w[t, s]) * h[s, cs].astype(np.float64)
+                acc += wd[:, cs] @ coef
+        y[t] = acc
+        hs.append(h)
+        ns.append(nrm)
+        ss.append(sc)
+        ks.append(kept)
+    return {"y": y, "idx": idx, "w": w, "h": np.stack(hs), "norms": np.stack(ns),
+            "scores": np.stack(ss), "kept": np.stack(ks)}
