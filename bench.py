@@ -205,10 +205,11 @@ class Stack:
     at set-up (moe_pack_w_down; the original layout is then freed), and the
     layers run the single-pass decode path."""
 
-    def __init__(self, wl, seed, device, tau=None, router_std=None):
+    def __init__(self, wl, seed, device, tau=None, router_std=None, keep_frac=None):
         from routed_expert_layer_route_b200 import moe, synth
         self.wl = wl
         self.tau = tau  # not None: the variable-k (cascade) route
+        self.keep_frac = keep_frac  # not None: channel top-k, this share of k1*I kept
         self.layers = []
         self.channel_major = wl["T"] == 1
         # two or more tokens: the tensor-core grouped GEMMs (what AUTO picks when d
@@ -224,15 +225,25 @@ class Stack:
                 L.w_router = (L.w_router.float() * scale).to(torch.bfloat16)
             if self.channel_major:
                 L.w_down = moe.moe_pack_w_down(L.w_down)
+                if keep_frac is not None:
+                    L.norms = moe.moe_channel_norms(L.w_down, channel_major=True)
             self.layers.append(L)
         torch.cuda.synchronize()
 
+    def keep(self, k1):
+        return max(1, int(round(self.keep_frac * k1 * self.wl["I"])))
+
     def call(self, L, k1, k2, y, ws, stream, idx=None, count=None, x=None, fixed=False):
         """One layer through the public API: moe_layer, or moe_layer_cascade
-        when the stack routes with a cascade (unless fixed)."""
+        when the stack routes with a cascade, or moe_layer_channel_topk with
+        channel top-k (unless fixed)."""
         from routed_expert_layer_route_b200 import moe
         x = L.x if x is None else x
-        if self.tau is None or fixed:
+        if self.keep_frac is not None and not fixed:
+            moe.moe_layer_channel_topk(x, L.w_router, L.bias, L.w_gate, L.w_up, L.w_down, L.norms,
+                                       k1, k2, self.keep(k1), y, ws, topk_idx_out=idx,
+                                       stream=stream)
+        elif self.tau is None or fixed:
             moe.moe_layer(x, L.w_router, L.bias, L.w_gate, L.w_up, L.w_down, k1, k2, y, ws,
                           topk_idx_out=idx, flags=self.flags, stream=stream)
         else:
@@ -390,7 +401,7 @@ def cpu_oracle_rate(stack, k1, k2, budget_s=12.0, max_tokens=8):
         oracle.layer_tokens(x, z, lambda e: experts[e], k1, k2)
         n += 1
         el = time.perf_counter() - t0
-        if el >= budget_s or n >= 4 * wl["layers"]:
+        if el >= budget_s or n >= 1000 * wl["layers"]:
             break
     per_layer = el / n
     return T / (per_layer * wl["layers"]), n, oracle.num_threads(), el
@@ -409,14 +420,18 @@ def run_native(args, world, rank):
     sweep = list(wl["sweep"])
     if args.k1:
         sweep = [(args.k1, args.k2 or args.k1)]
-    elif args.cascade is not None:  # one cascade condition: cap k1 = 8, k2 = 8
-        sweep = [(8, args.k2 or 8)]
+    elif args.cascade is not None or args.channel_keep is not None:
+        sweep = [(8, args.k2 or 8)]  # one condition: (cap) k1 = 8, k2 = 8
     head = sweep[0]
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.Stream()
     hbm_peak, bf16_peak, peak_kind = load_peaks()
 
-    stack = Stack(wl, seed=rank, device=dev, tau=args.cascade, router_std=args.router_std)
+    if args.channel_keep is not None and wl["T"] != 1:
+        raise SystemExit("--channel-keep: one-token workloads only (T = 1)")
+    stack = Stack(wl, seed=rank, device=dev, tau=args.cascade, router_std=args.router_std,
+                  keep_frac=args.channel_keep)
+    variant = stack.tau is not None or stack.keep_frac is not None
     T, d, E, I, Ln = wl["T"], wl["d"], wl["E"], wl["I"], wl["layers"]
     results = []
     graphs = {}
@@ -465,13 +480,33 @@ def run_native(args, world, rank):
         U = statistics.mean(us)
         bytes_layer = U * 3 * d * I * 2
         flops_layer = T * (mean_k * 6.0 * d * I + 2.0 * d * E)
+        if stack.keep_frac is not None:
+            # every gate/up row and norm of the routed experts, the kept down columns
+            bytes_layer = U * 2 * d * I * 2 + U * I * 4 + T * stack.keep(k1) * d * 2
+            flops_layer = T * (mean_k * 4.0 * d * I + 2.0 * stack.keep(k1) * d + 2.0 * d * E)
         results.append({"k1": k1, "k2": k2, "ms_per_step": ms, "us_per_layer": ms * 1000 / Ln,
+                        "bytes_per_layer": bytes_layer,
                         "tokens_per_s": world * T * 1000.0 / ms, "unique_experts_per_layer": U,
                         "expert_GBps": bytes_layer / (ms / Ln * 1e-3) / 1e9,
                         "layer_TFLOPs": flops_layer / (ms / Ln * 1e-3) / 1e12,
                         "mean_experts_per_token": mean_k})
 
     cascade = None
+    channel_topk = None
+    if stack.keep_frac is not None:
+        # the same stack through the full decode layer: bytes saved vs time saved
+        k1h_, k2h_ = head
+        _, ws_list, ys = graphs[head]
+        gf = build_graph(stack, k1h_, k2h_, ws_list, ys, stream, fixed=True)
+        graphs[("fixed",) + head] = (gf, ws_list, ys)
+        ms_fixed = timed(("fixed",) + head, args.steps, args.warmup)[0]
+        U0 = results[0]["unique_experts_per_layer"]
+        channel_topk = {"keep": stack.keep(k1h_), "keep_frac": stack.keep_frac, "k1": k1h_,
+                        "k2": k2h_, "channels_per_token": k1h_ * I,
+                        "us_per_layer": results[0]["us_per_layer"],
+                        "full_layer_us_per_layer": ms_fixed * 1000 / Ln,
+                        "time_ratio_vs_full": results[0]["us_per_layer"] / (ms_fixed * 1000 / Ln),
+                        "bytes_ratio_vs_full": results[0]["bytes_per_layer"] / (U0 * 3 * d * I * 2)}
     if stack.tau is not None:
         # the same stack with the fixed k1 route: compute saved vs time saved
         k1h_, k2h_ = head
@@ -497,15 +532,18 @@ def run_native(args, world, rank):
     k1h, k2h = head
     _, ws_list, ys = graphs[head]
     U_head = results[0]["unique_experts_per_layer"]
-    alg_bytes = U_head * 3 * d * I * 2
-    if stack.tau is not None:
+    alg_bytes = results[0]["bytes_per_layer"]
+    if variant:
         # the kernels alone are re-run only with the fixed route; for a cascade
-        # route the roofline is taken over the whole layer
+        # route or channel top-k the roofline is taken over the whole layer
         lay_s = results[0]["us_per_layer"] * 1e-6
         achieved = alg_bytes / lay_s / 1e9
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
                     "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": None,
-                    "kernel": "whole layer (cascade route)", "kernel_us": round(lay_s * 1e6, 2),
+                    "kernel": "whole layer (%s)" % ("cascade route" if stack.tau is not None else
+                                                    "channel top-k: k_logits, k_ctk_gateup, "
+                                                    "k_ctk_down"),
+                    "kernel_us": round(lay_s * 1e6, 2),
                     "algorithmic_bytes_per_launch": int(alg_bytes),
                     "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind}
     elif stack.grouped:
@@ -577,7 +615,7 @@ def run_native(args, world, rank):
             break
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and stack.tau is None:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not variant:
         rate, nl, thr, el = cpu_oracle_rate(stack, k1h, k2h)
         cpu = {"value": rate, "unit": "tokens/s", "cores": thr, "kind": "oracle",
                "sample": "%d layers of this workload, first %d token(s) of each (k1=%d, k2=%d), "
@@ -588,6 +626,8 @@ def run_native(args, world, rank):
     # warp router, permutation (2), token-row gather, two grouped GEMMs, finalize
     # (tensor-core path); router logits, top-k, streaming kernel (streaming path)
     per_step_launches = 2 if stack.channel_major else (8 if stack.grouped else 3)
+    if stack.keep_frac is not None:
+        per_step_launches = 1 + 2 * T  # router logits, then two kernels per token
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
@@ -598,6 +638,7 @@ def run_native(args, world, rank):
                    "layers": Ln, "d": d, "E": E, "I": I, "T": T, "k1": k1h, "k2": k2h,
                    "bias": wl["bias"], "us_per_layer": round(ms_step * 1000 / Ln, 3),
                    "cascade_tau": stack.tau, "router_logit_std": args.router_std,
+                   "channel_keep_frac": stack.keep_frac,
                    "l2": "inputs larger than L2: every step reads the routed experts of all "
                          "%d layers (%.2f GB) from HBM" % (Ln, alg_bytes * Ln / 1e9),
                    "timing": "CUDA graph of the %d-layer step, CUDA events, max over ranks" % Ln,
@@ -613,6 +654,7 @@ def run_native(args, world, rank):
         "clocks": clk,
         "sweep": results,
         "cascade": cascade,
+        "channel_topk": channel_topk,
         "k1_4_over_k1_8_time_ratio": None if ratio is None else round(ratio, 4),
         "k1_ratio_conditions": ratio_pair,
     }
@@ -679,6 +721,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cascade", type=float, default=None, metavar="TAU",
                     help="variable experts per token: the first k <= k1 covering mass TAU")
+    ap.add_argument("--channel-keep", type=float, default=None, metavar="FRAC",
+                    help="channel top-k: keep this share of each token's k1*I channels")
     ap.add_argument("--router-std", type=float, default=None,
                     help="scale the router so its logits have this standard deviation")
     args = ap.parse_args()

@@ -210,6 +210,45 @@ int moe_layer_cascade(const void *x_bf16, const void *w_router_bf16, const float
                       int32_t *topk_idx_out, float *topk_w_out, int32_t *topk_count_out,
                       float *logits_out, int flags, void *ws, size_t ws_bytes, void *stream);
 
+/* Channel top-k inside the activated experts ("Channel Selection for
+ * Mixture-of-Experts Decoding Needs No Calibration Data", paperlayer.ai,
+ * sections 2, 5.2 and 5.3).  Per token, every channel (s, c) of its k1 routed
+ * experts (slot s in rank order, channel c < I; flat index q = s*I + c) gets
+ * the output-scaled score
+ *     score[q] = (w_s * n[e_s][c]) * |h_c|     (two float32 products),
+ * the norm of that channel's contribution to y; the token keeps the `keep`
+ * channels with the largest scores over all its slots (equal scores go to
+ * the lower q) and
+ *     y[t, :] = sum over kept q of w_s * h_q * W_down[e_s][:, c]
+ * (kept channels exact; skipped channels add nothing: the pages' ternary
+ * sketch and low-rank recovery are not part of this call).  h is computed
+ * exactly for every channel, so every gate and up row of the routed experts
+ * is read; only the kept channels' down columns are.
+ *
+ * moe_channel_norms: n[e][c] = ||W_down[e][:, c]||_2 in float32 (float32
+ *   sum of squares, IEEE square root), norms [E x I] float32, from w_down in
+ *   the HF layout [E x d x I] (flags 0) or channel-major [E x I x d]
+ *   (flags MOE_WDOWN_CHANNEL_MAJOR, from moe_pack_w_down).  Computed once
+ *   when the weights are loaded.
+ * moe_layer_channel_topk: the layer with channel top-k.  w_down_cm is the
+ *   channel-major down matrix (moe_pack_w_down), norms from
+ *   moe_channel_norms.  1 <= keep <= k1*I <= 16384.  Tokens run one after
+ *   another (two kernels each).  Optional outputs (each nullable):
+ *   topk_idx_out / topk_w_out [T x k1], logits_out [T x E], h_out and
+ *   scores_out [T x k1 x I] float32, kept_out [T x keep] int32 (the kept
+ *   flat indices q, ascending).  Scores, h and the kept set are
+ *   deterministic; y sums the kept channels in a timing-dependent order (last
+ *   bits may differ between runs).  Non-finite activations leave the kept set
+ *   unspecified.  Other arguments and the workspace as for moe_layer. */
+int moe_channel_norms(const void *w_down_bf16, int E, int d, int I, int flags, float *norms,
+                      void *stream);
+int moe_layer_channel_topk(const void *x_bf16, const void *w_router_bf16, const float *bias,
+                           const void *w_gate_bf16, const void *w_up_bf16, const void *w_down_cm_bf16,
+                           const float *norms, int T, int d, int E, int I, int k1, int k2, int keep,
+                           void *y, int y_dtype, int32_t *topk_idx_out, float *topk_w_out,
+                           float *logits_out, float *h_out, float *scores_out, int32_t *kept_out,
+                           void *ws, size_t ws_bytes, void *stream);
+
 /* Channel-major copy of a down matrix, made once when the weights are
  * loaded: w_down_cm[e][c][r] = w_down[e][r][c] (w_down [E x d x I] bf16 ->
  * w_down_cm [E x I x d] bf16, separate buffers).  The channel decomposition

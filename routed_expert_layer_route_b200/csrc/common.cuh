@@ -214,6 +214,14 @@ MOE_DEVINL unsigned split_lo(unsigned n, unsigned G, unsigned b)
     return q * b + (b < r ? b : r);
 }
 
+// y[0..3] += v (16-byte aligned float32 vector), one vector reduction.
+MOE_DEVINL void red_add_v4(float *y, float v0, float v1, float v2, float v3)
+{
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(y), "f"(v0), "f"(v1),
+                 "f"(v2), "f"(v3)
+                 : "memory");
+}
+
 MOE_DEVINL uint4 ld_nc_v4(const void *p)
 {
     uint4 v;

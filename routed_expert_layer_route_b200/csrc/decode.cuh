@@ -26,9 +26,9 @@
 //    adds h * down_row into register partials for its fixed third of the
 //    output rows;
 //  * at the end the four groups' partials are summed in shared memory and
-//    added into the float32 accumulator y_acc with red.global.add; the last
-//    CTA to check in (a counter in the workspace header) converts y_acc to
-//    the output y.
+//    added into the float32 accumulator y_acc with 16-byte vector reductions
+//    (red.global.add.v4.f32); the last CTA to check in (a counter in the
+//    workspace header) converts y_acc to the output y.
 // Partial sums from different CTAs reach y_acc in a timing-dependent order,
 // so y can differ between runs in the last bits (stream.cuh holds the
 // deterministic two-phase kernel).
@@ -375,13 +375,18 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
             }
         }
         consumer_sync();
-        if (nseg > 0) {
-            for (int r = tid; r < d; r += kSC * 32) {
-                float sum = 0.0f;
+        if (nseg > 0) {  // one 16-byte vector reduction per four output rows
+            for (int r = tid * 4; r < d; r += kSC * 32 * 4) {
+                float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                for (int g = 0; g < kDStages; ++g)
-                    sum += red[(size_t)g * d + r];
-                atomicAdd(&a.y_acc[r], sum);
+                for (int g = 0; g < kDStages; ++g) {
+                    const float4 v = *reinterpret_cast<const float4 *>(red + (size_t)g * d + r);
+                    sum.x += v.x;
+                    sum.y += v.y;
+                    sum.z += v.z;
+                    sum.w += v.w;
+                }
+                red_add_v4(a.y_acc + r, sum.x, sum.y, sum.z, sum.w);
             }
         }
         __threadfence();  // the adds are visible before this CTA checks in below

@@ -189,14 +189,6 @@ MOE_DEVINL uint32_t pack_bf16x2(float lo, float hi)
     return r;
 }
 
-// y[0..3] += v (16-byte aligned float32 vector), one vector reduction.
-MOE_DEVINL void red_add_v4(float *y, float v0, float v1, float v2, float v3)
-{
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(y), "f"(v0), "f"(v1),
-                 "f"(v2), "f"(v3)
-                 : "memory");
-}
-
 // 32 lanes x 16 consecutive float32 columns.
 MOE_DEVINL void tmem_ld16(uint32_t taddr, float (&v)[16])
 {

@@ -12,6 +12,7 @@
 #include "../../include/moe.h"
 #include "../../include/moe_testing.h"
 #include "combine.cuh"
+#include "ctopk.cuh"
 #include "decode.cuh"
 #include "grouped.cuh"
 #include "route.cuh"
@@ -30,7 +31,7 @@ static inline size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct WsLayout {
     size_t logits, idx, w, offsets, sorted_slot, slot_pos, uniq_count, uniq_list, h, out, y_acc,
-        hist, total;
+        hist, ctk, total;
 };
 
 static inline int perm_chunks(int T) { return (T + kPermTok - 1) / kPermTok; }
@@ -52,6 +53,7 @@ static WsLayout ws_layout(int T, int d, int E, int I, int k1)
     L.out = o;         o = align256(o + sizeof(float) * n * (size_t)d);
     L.y_acc = o;       o = align256(o + sizeof(float) * (size_t)T * d);
     L.hist = o;        o = align256(o + sizeof(int32_t) * (size_t)perm_chunks(T) * E);
+    L.ctk = o;         o = align256(o + 2 * sizeof(float) * (size_t)k1 * I);  // one token's h, scores
     L.total = o;
     return L;
 }
@@ -127,6 +129,9 @@ static int device_info(DevInfo *&out)
                                  (int)gemm1_smem_bytes()) != cudaSuccess ||
             cudaFuncSetAttribute(k_gemm2, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gemm2_smem_bytes()) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        // scores of kCtkMaxN channels + at most 16 KiB of side-by-side row partials
+        if (cudaFuncSetAttribute(k_ctk_down, dsm, kCtkMaxN * 4 + 16 * 1024) != cudaSuccess)
             return MOE_ERR_CUDA;
         const int small = 96 * 1024;
         if (cudaFuncSetAttribute(k_logits, cudaFuncAttributeMaxDynamicSharedMemorySize, small) !=
@@ -883,6 +888,99 @@ int moe_layer_cascade(const void *x_bf16, const void *w_router_bf16, const float
     return layer_impl(x_bf16, w_router_bf16, bias, w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I,
                       k1, k2, y, y_dtype, topk_idx_out, topk_w_out, logits_out, flags, ws, ws_bytes,
                       stream, true, tau, topk_count_out);
+}
+
+int moe_channel_norms(const void *w_down_bf16, int E, int d, int I, int flags, float *norms,
+                      void *stream)
+{
+    if (E < 1 || E > kMaxE || d < kMinD || d > kMaxD || d % 64 || I < kMinI || I > kMaxI || I % 16)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if ((flags & ~MOE_WDOWN_CHANNEL_MAJOR) || !w_down_bf16 || !norms || !aligned16(w_down_bf16))
+        return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const uint16_t *wd = static_cast<const uint16_t *>(w_down_bf16);
+    if (flags & MOE_WDOWN_CHANNEL_MAJOR)
+        return launch(k_norms_cm, dim3((unsigned)(((long)E * I + 15) / 16)), dim3(512), 0, s, true,
+                      wd, E, I, d, norms);
+    return launch(k_norms_hf, dim3((I + 255) / 256, E), dim3(256), 0, s, true, wd, E, I, d, norms);
+}
+
+int moe_layer_channel_topk(const void *x_bf16, const void *w_router_bf16, const float *bias,
+                           const void *w_gate_bf16, const void *w_up_bf16, const void *w_down_cm_bf16,
+                           const float *norms, int T, int d, int E, int I, int k1, int k2, int keep,
+                           void *y, int y_dtype, int32_t *topk_idx_out, float *topk_w_out,
+                           float *logits_out, float *h_out, float *scores_out, int32_t *kept_out,
+                           void *ws, size_t ws_bytes, void *stream)
+{
+    int rc = check_shape(T, d, E, I, k1);
+    if (rc != MOE_OK)
+        return rc;
+    if ((rc = check_route(E, k1, k2)) != MOE_OK)
+        return rc;
+    const int N = k1 * I;
+    if (keep < 1 || keep > N || (y_dtype != MOE_DTYPE_F32 && y_dtype != MOE_DTYPE_BF16))
+        return MOE_ERR_INVALID_ARG;
+    if (N > kCtkMaxN)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (T == 0)
+        return MOE_OK;
+    if (!x_bf16 || !w_router_bf16 || !w_gate_bf16 || !w_up_bf16 || !w_down_cm_bf16 || !norms ||
+        !y || !ws)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x_bf16) || !aligned16(w_router_bf16) || !aligned16(w_gate_bf16) ||
+        !aligned16(w_up_bf16) || !aligned16(w_down_cm_bf16) || !aligned16(y) ||
+        (reinterpret_cast<uintptr_t>(ws) & 255))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(T, d, E, I, k1);
+    if (ws_bytes < L.total)
+        return MOE_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    DevInfo *di;
+    if ((rc = device_info(di)) != MOE_OK)
+        return rc;
+    const int G = di->num_sms;
+    if ((keep + G - 1) / G > kCtkMaxMine)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    float *z = at<float>(ws, L.logits);
+    float *y_acc = at<float>(ws, L.y_acc);
+    if ((rc = enqueue_logits(x_bf16, w_router_bf16, bias, z, logits_out, T, d, E, s,
+                             reinterpret_cast<float4 *>(y_acc), T * d / 4)) != MOE_OK)
+        return rc;
+    const size_t ysz = y_dtype == MOE_DTYPE_BF16 ? 2 : 4;
+    for (int t = 0; t < T; ++t) {  // one token after another (two kernels each)
+        CtkArgs a = {};
+        a.x = static_cast<const uint16_t *>(x_bf16) + (size_t)t * d;
+        a.wg = static_cast<const uint16_t *>(w_gate_bf16);
+        a.wu = static_cast<const uint16_t *>(w_up_bf16);
+        a.wdt = static_cast<const uint16_t *>(w_down_cm_bf16);
+        a.norms = norms;
+        a.logits = z + (size_t)t * E;
+        a.d = d;
+        a.E = E;
+        a.I = I;
+        a.k1 = k1;
+        a.k2 = k2;
+        a.keep = keep;
+        a.topk_idx = at<int32_t>(ws, L.idx) + (size_t)t * k1;
+        a.topk_w = at<float>(ws, L.w) + (size_t)t * k1;
+        a.idx_copy = topk_idx_out ? topk_idx_out + (size_t)t * k1 : nullptr;
+        a.w_copy = topk_w_out ? topk_w_out + (size_t)t * k1 : nullptr;
+        a.h = at<float>(ws, L.ctk);
+        a.score = a.h + N;
+        a.h_copy = h_out ? h_out + (size_t)t * N : nullptr;
+        a.score_copy = scores_out ? scores_out + (size_t)t * N : nullptr;
+        a.kept_out = kept_out ? kept_out + (size_t)t * keep : nullptr;
+        a.y_acc = y_acc + (size_t)t * d;
+        a.y = static_cast<char *>(y) + (size_t)t * d * ysz;
+        a.y_dtype = y_dtype;
+        a.hdr = static_cast<WsHeader *>(ws);
+        if ((rc = launch(k_ctk_gateup, dim3(G), dim3(kCtkThreads), (size_t)d * 2, s, true, a)) !=
+                MOE_OK ||
+            (rc = launch(k_ctk_down, dim3(G), dim3(kCtkThreads), ctk_down_smem_bytes(N, d), s, true,
+                         a)) != MOE_OK)
+            return rc;
+    }
+    return MOE_OK;
 }
 
 int moe_pack_w_down(const void *w_down_bf16, void *w_down_cm_bf16, int E, int d, int I,

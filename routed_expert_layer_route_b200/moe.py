@@ -58,6 +58,9 @@ SIGNATURES = {
                                _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp]),
     "moe_expert_ffn_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
     "moe_pack_w_down": (_i, [_vp, _vp, _i, _i, _i, _vp]),
+    "moe_channel_norms": (_i, [_vp, _i, _i, _i, _i, _vp, _vp]),
+    "moe_layer_channel_topk": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
+                                    _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_test_exp_c": (_i, [_vp, _vp, ctypes.c_int64, _vp]),
     "moe_test_num_sms": (_i, []),
     "moe_test_expert_stream": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _i, _vp,
@@ -203,6 +206,38 @@ def moe_pack_w_down(w_down, w_down_cm=None, stream=None):
     _check(lib().moe_pack_w_down(_p(w_down), _p(w_down_cm), E, d, I, _stream(stream)),
            "moe_pack_w_down")
     return w_down_cm
+
+
+def moe_channel_norms(w_down, channel_major=False, norms=None, stream=None):
+    """float32 [E x I] down-column norms of w_down: [E x d x I] (HF layout) or,
+    with channel_major, [E x I x d] (moe_pack_w_down's output)."""
+    if channel_major:
+        E, I, d = w_down.shape
+    else:
+        E, d, I = w_down.shape
+    if norms is None:
+        norms = torch.empty((E, I), dtype=torch.float32, device=w_down.device)
+    _check(lib().moe_channel_norms(_p(w_down), E, d, I,
+                                   MOE_WDOWN_CHANNEL_MAJOR if channel_major else 0, _p(norms),
+                                   _stream(stream)), "moe_channel_norms")
+    return norms
+
+
+def moe_layer_channel_topk(x, w_router, bias, w_gate, w_up, w_down_cm, norms, k1, k2, keep, y, ws,
+                           topk_idx_out=None, topk_w_out=None, logits_out=None, h_out=None,
+                           scores_out=None, kept_out=None, stream=None):
+    """The layer with channel top-k: each token keeps the `keep` channels of
+    its k1 experts with the largest w * ||down column|| * |h| (w_down_cm
+    channel-major, norms from moe_channel_norms)."""
+    T, d = x.shape
+    E, I, _ = w_gate.shape
+    y_dtype = MOE_DTYPE_BF16 if y.dtype == torch.bfloat16 else MOE_DTYPE_F32
+    wsp, wsn = _ws_args(ws)
+    _check(lib().moe_layer_channel_topk(_p(x), _p(w_router), _p(bias), _p(w_gate), _p(w_up),
+                                        _p(w_down_cm), _p(norms), T, d, E, I, k1, k2, int(keep),
+                                        _p(y), y_dtype, _p(topk_idx_out), _p(topk_w_out),
+                                        _p(logits_out), _p(h_out), _p(scores_out), _p(kept_out),
+                                        wsp, wsn, _stream(stream)), "moe_layer_channel_topk")
 
 
 def moe_combine(expert_out, slot_pos, topk_w, y, stream=None):
