@@ -234,6 +234,7 @@ __global__ void __launch_bounds__(kCtkThreads, 1) k_ctk_down(CtkArgs a)
     __syncthreads();  // hist0 is clear
     // first pass: 4096 buckets on bits 30..19 of the key (the exponent and the
     // top four mantissa bits: sixteen buckets per binade), no range needed
+#pragma unroll 4
     for (int i = tid; i < N; i += kCtkThreads) {
         const unsigned k = __float_as_uint(__ldcg(&a.score[i]));
         key[i] = k;
@@ -363,6 +364,7 @@ __global__ void __launch_bounds__(kCtkThreads, 1) k_ctk_down(CtkArgs a)
     const int s0 = min(N, warp * seg), s1 = min(N, s0 + seg);
     const unsigned lt = (1u << lane) - 1u;
     int ngt = 0, neq = 0;
+#pragma unroll 4
     for (int i0 = s0; i0 < s1; i0 += 32) {
         const int i = i0 + lane;
         const unsigned k = i < s1 ? key[i] : 0u;
@@ -384,6 +386,7 @@ __global__ void __launch_bounds__(kCtkThreads, 1) k_ctk_down(CtkArgs a)
     const int n_eq = K - tot_gt;  // keys equal to thr that are kept: the first n_eq
     const int p_lo = (int)split_lo((unsigned)K, G, b), p_hi = (int)split_lo((unsigned)K, G, b + 1);
     int pos = gt_before + min(eq_before, n_eq);
+#pragma unroll 4
     for (int i0 = s0; i0 < s1; i0 += 32) {
         const int i = i0 + lane;
         const unsigned k = i < s1 ? key[i] : 0u;
