@@ -398,3 +398,46 @@ def channel_topk_tokens(xrows, z_rows, fetch_expert, fetch_norms, k1, k2, keep, 
         ks.append(kept)
     return {"y": y, "idx": idx, "w": w, "h": np.stack(hs), "norms": np.stack(ns),
             "scores": np.stack(ss), "kept": np.stack(ks)}
+
+
+# ---------------------------------------------------------------------------
+# Expert skipping with the top-1 expert always kept (the shell of "ACE",
+# aimodeling.com, section "How ACE decides what to skip: GSP + RCR": a slot is
+# skipped only when two independent views both call it low-contribution, and
+# the top-1 expert is always retained).  Reading taken here: the first view is
+# a per-expert scalar looked up at inference (the page's offline statistic;
+# the caller supplies the table), the second is the slot's Eq. 2 weight (the
+# token's router-conditioned view); kept slots keep their Eq. 2 weights.
+
+
+def route_skip_f32(logits, k1, k2, table, th_e, th_w):
+    """route_f32, then slot s >= 1 of each token becomes EMPTY_SLOT (weight 0)
+    when table[e_s] < th_e and w_s < th_w (float32 comparisons).  Returns
+    (idx, w, count of kept slots per token)."""
+    idx, w = route_f32(logits, k1, k2)
+    tab = np.asarray(table, np.float32)
+    low = (tab[idx] < np.float32(th_e)) & (w < np.float32(th_w))
+    low[:, 0] = False  # the top-1 expert is always kept
+    idx = np.where(low, np.int32(EMPTY_SLOT), idx).astype(np.int32)
+    w = np.where(low, np.float32(0.0), w).astype(np.float32)
+    return idx, w, (~low).sum(axis=1).astype(np.int32)
+
+
+def layer_tokens_slots(xrows, idx, w, fetch_expert):
+    """Layer output for a few tokens from given routing outputs: y[t] sums
+    w[t, s] * FFN_{idx[t, s]}(x_t) over the slots that are not EMPTY_SLOT, in
+    slot order (oracle_expert, oracle_combine)."""
+    xf_all = _widen(xrows)
+    n, d = xf_all.shape
+    y = np.empty((n, d), np.float32)
+    cache = {}
+    for t in range(n):
+        slots = [s for s in range(idx.shape[1]) if idx[t, s] != EMPTY_SLOT]
+        o = np.empty((len(slots), d), np.float32)
+        for i, s in enumerate(slots):
+            e = int(idx[t, s])
+            if e not in cache:
+                cache[e] = fetch_expert(e)
+            _, o[i] = expert(xf_all[t], *cache[e], par=True)
+        y[t] = combine(o, w[t, slots]) if slots else 0.0
+    return y
