@@ -205,10 +205,11 @@ class Stack:
     at set-up (moe_pack_w_down; the original layout is then freed), and the
     layers run the single-pass decode path."""
 
-    def __init__(self, wl, seed, device, tau=None, router_std=None, keep_frac=None):
+    def __init__(self, wl, seed, device, tau=None, router_std=None, keep_frac=None, skip=None):
         from routed_expert_layer_route_b200 import moe, synth
         self.wl = wl
         self.tau = tau  # not None: the variable-k (cascade) route
+        self.skip = skip  # not None: (theta_expert, theta_weight) of expert skipping
         self.keep_frac = keep_frac  # not None: channel top-k, this share of k1*I kept
         self.layers = []
         self.channel_major = wl["T"] == 1
@@ -223,6 +224,9 @@ class Stack:
             if router_std:  # router logits with this standard deviation (x is RMS-normalised)
                 scale = router_std / (0.02 * wl["d"] ** 0.5)
                 L.w_router = (L.w_router.float() * scale).to(torch.bfloat16)
+            if skip is not None:  # the per-expert table: seeded uniform [0, 1) stand-in values
+                g = torch.Generator(device="cpu").manual_seed(1000003 * (seed + 1) + l)
+                L.skip_tab = torch.rand(wl["E"], generator=g).to(device)
             if self.channel_major:
                 L.w_down = moe.moe_pack_w_down(L.w_down)
                 if keep_frac is not None:
@@ -239,7 +243,11 @@ class Stack:
         channel top-k (unless fixed)."""
         from routed_expert_layer_route_b200 import moe
         x = L.x if x is None else x
-        if self.keep_frac is not None and not fixed:
+        if self.skip is not None and not fixed:
+            moe.moe_layer_skip(x, L.w_router, L.bias, L.w_gate, L.w_up, L.w_down, k1, k2,
+                               L.skip_tab, self.skip[0], self.skip[1], y, ws, topk_idx_out=idx,
+                               topk_count_out=count, flags=self.flags, stream=stream)
+        elif self.keep_frac is not None and not fixed:
             moe.moe_layer_channel_topk(x, L.w_router, L.bias, L.w_gate, L.w_up, L.w_down, L.norms,
                                        k1, k2, self.keep(k1), y, ws, topk_idx_out=idx,
                                        stream=stream)
@@ -420,7 +428,7 @@ def run_native(args, world, rank):
     sweep = list(wl["sweep"])
     if args.k1:
         sweep = [(args.k1, args.k2 or args.k1)]
-    elif args.cascade is not None or args.channel_keep is not None:
+    elif args.cascade is not None or args.channel_keep is not None or args.skip is not None:
         sweep = [(8, args.k2 or 8)]  # one condition: (cap) k1 = 8, k2 = 8
     head = sweep[0]
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -430,8 +438,8 @@ def run_native(args, world, rank):
     if args.channel_keep is not None and wl["T"] != 1:
         raise SystemExit("--channel-keep: one-token workloads only (T = 1)")
     stack = Stack(wl, seed=rank, device=dev, tau=args.cascade, router_std=args.router_std,
-                  keep_frac=args.channel_keep)
-    variant = stack.tau is not None or stack.keep_frac is not None
+                  keep_frac=args.channel_keep, skip=args.skip)
+    variant = stack.tau is not None or stack.keep_frac is not None or stack.skip is not None
     T, d, E, I, Ln = wl["T"], wl["d"], wl["E"], wl["I"], wl["layers"]
     results = []
     graphs = {}
@@ -507,14 +515,14 @@ def run_native(args, world, rank):
                         "full_layer_us_per_layer": ms_fixed * 1000 / Ln,
                         "time_ratio_vs_full": results[0]["us_per_layer"] / (ms_fixed * 1000 / Ln),
                         "bytes_ratio_vs_full": results[0]["bytes_per_layer"] / (U0 * 3 * d * I * 2)}
-    if stack.tau is not None:
+    if stack.tau is not None or stack.skip is not None:
         # the same stack with the fixed k1 route: compute saved vs time saved
         k1h_, k2h_ = head
         _, ws_list, ys = graphs[head]
         gf = build_graph(stack, k1h_, k2h_, ws_list, ys, stream, fixed=True)
         graphs[("fixed",) + head] = (gf, ws_list, ys)
         ms_fixed = timed(("fixed",) + head, args.steps, args.warmup)[0]
-        cascade = {"tau": stack.tau, "k1_cap": k1h_, "k2": k2h_,
+        cascade = {"tau": stack.tau, "skip_thresholds": stack.skip, "k1_cap": k1h_, "k2": k2h_,
                    "mean_experts_per_token": results[0]["mean_experts_per_token"],
                    "us_per_layer": results[0]["us_per_layer"],
                    "fixed_k1_us_per_layer": ms_fixed * 1000 / Ln,
@@ -541,7 +549,8 @@ def run_native(args, world, rank):
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
                     "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": None,
                     "kernel": "whole layer (%s)" % ("cascade route" if stack.tau is not None else
-                                                    "channel top-k: k_logits, k_ctk_gateup, "
+                                                    "expert skipping" if stack.skip is not None
+                                                    else "channel top-k: k_logits, k_ctk_gateup, "
                                                     "k_ctk_down"),
                     "kernel_us": round(lay_s * 1e6, 2),
                     "algorithmic_bytes_per_launch": int(alg_bytes),
@@ -638,7 +647,7 @@ def run_native(args, world, rank):
                    "layers": Ln, "d": d, "E": E, "I": I, "T": T, "k1": k1h, "k2": k2h,
                    "bias": wl["bias"], "us_per_layer": round(ms_step * 1000 / Ln, 3),
                    "cascade_tau": stack.tau, "router_logit_std": args.router_std,
-                   "channel_keep_frac": stack.keep_frac,
+                   "channel_keep_frac": stack.keep_frac, "skip_thresholds": stack.skip,
                    "l2": "inputs larger than L2: every step reads the routed experts of all "
                          "%d layers (%.2f GB) from HBM" % (Ln, alg_bytes * Ln / 1e9),
                    "timing": "CUDA graph of the %d-layer step, CUDA events, max over ranks" % Ln,
@@ -721,6 +730,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cascade", type=float, default=None, metavar="TAU",
                     help="variable experts per token: the first k <= k1 covering mass TAU")
+    ap.add_argument("--skip", type=float, nargs=2, default=None, metavar=("TH_E", "TH_W"),
+                    help="expert skipping (top-1 kept): skip a slot when its expert's table "
+                         "value < TH_E and its weight < TH_W (seeded uniform table)")
     ap.add_argument("--channel-keep", type=float, default=None, metavar="FRAC",
                     help="channel top-k: keep this share of each token's k1*I channels")
     ap.add_argument("--router-std", type=float, default=None,

@@ -210,6 +210,31 @@ int moe_layer_cascade(const void *x_bf16, const void *w_router_bf16, const float
                       int32_t *topk_idx_out, float *topk_w_out, int32_t *topk_count_out,
                       float *logits_out, int flags, void *ws, size_t ws_bytes, void *stream);
 
+/* Expert skipping with the top-1 expert always kept (the shell of "ACE",
+ * aimodeling.com, section "How ACE decides what to skip: GSP + RCR": a slot
+ * is skipped only when two views both call it low, and the top-1 expert is
+ * never skipped).  Reading taken here: the first view is a per-expert scalar
+ * table looked up at inference (expert_score [E] float32, device, 16-byte
+ * aligned; the page's offline statistic, supplied by the caller), the second
+ * is the slot's own Eq. 2 weight (the token's router-conditioned view).  Slot
+ * s >= 1 of token t is skipped when expert_score[e] < theta_expert AND
+ * topk_w[t, s] < theta_weight; skipped slots hold MOE_EMPTY_SLOT with weight
+ * 0, kept slots keep their Eq. 2 weights (no renormalisation over the kept
+ * set), and topk_count [T] (nullable) receives the kept count.  A NaN
+ * threshold or a null table: MOE_ERR_INVALID_ARG.  moe_layer_skip runs on the
+ * same paths as moe_layer_cascade.  Other arguments as for moe_route /
+ * moe_layer. */
+int moe_route_skip(const void *x_bf16, const void *w_router_bf16, const float *bias,
+                   float *logits, int T, int d, int E, int k1, int k2, const float *expert_score,
+                   float theta_expert, float theta_weight, int32_t *topk_idx, float *topk_w,
+                   int32_t *topk_count, void *ws, size_t ws_bytes, void *stream);
+int moe_layer_skip(const void *x_bf16, const void *w_router_bf16, const float *bias,
+                   const void *w_gate_bf16, const void *w_up_bf16, const void *w_down_bf16, int T,
+                   int d, int E, int I, int k1, int k2, const float *expert_score,
+                   float theta_expert, float theta_weight, void *y, int y_dtype,
+                   int32_t *topk_idx_out, float *topk_w_out, int32_t *topk_count_out,
+                   float *logits_out, int flags, void *ws, size_t ws_bytes, void *stream);
+
 /* Channel top-k inside the activated experts ("Channel Selection for
  * Mixture-of-Experts Decoding Needs No Calibration Data", paperlayer.ai,
  * sections 2, 5.2 and 5.3).  Per token, every channel (s, c) of its k1 routed

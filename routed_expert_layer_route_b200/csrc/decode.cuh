@@ -67,8 +67,7 @@ struct DecodeArgs {
     float *y_acc;  // [d] float32, zero on entry
     void *y;       // [d] output (y_dtype); written by the last CTA to finish
     int y_dtype;
-    int cascade;   // variable k: the first kt <= k1 ranked experts covering tau
-    float tau;
+    VarK vk;       // variable k: cascade or skip (kind 0 with the fixed-k kernel)
     int32_t *count;  // nullable: kt
     WsHeader *hdr;
 };
@@ -145,7 +144,7 @@ __device__ void decode_segments(DecodeSmem *ds, int U, int I, int G, int b, int 
 
 // VPL: d = 256*VPL for the single-token register path (x in registers when
 // VPL <= kXRegMax), 0 for the general token loop.  CASCADE: the variable-k
-// route (a.cascade is then set).
+// route (a.vk: cascade or skip).
 template <int VPL, bool CASCADE>
 __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
 {
@@ -183,20 +182,20 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
     if (warp == 0) {
         int j, kt;
         float wv;
-        constexpr bool cas = CASCADE;
+        const VarK vk = CASCADE ? a.vk : VarK();
         if (E <= 128)
-            warp_route<4>(a.logits, E, k1, a.k2, lane, j, wv, cas, a.tau, &kt);
+            warp_route<4>(a.logits, E, k1, a.k2, lane, j, wv, vk, &kt);
         else if (E <= 256)
-            warp_route<8>(a.logits, E, k1, a.k2, lane, j, wv, cas, a.tau, &kt);
+            warp_route<8>(a.logits, E, k1, a.k2, lane, j, wv, vk, &kt);
         else if (E <= 512)
-            warp_route<16>(a.logits, E, k1, a.k2, lane, j, wv, cas, a.tau, &kt);
+            warp_route<16>(a.logits, E, k1, a.k2, lane, j, wv, vk, &kt);
         else
-            warp_route<32>(a.logits, E, k1, a.k2, lane, j, wv, cas, a.tau, &kt);
+            warp_route<32>(a.logits, E, k1, a.k2, lane, j, wv, vk, &kt);
         int p = 0;  // position of this lane's expert among the kt taken, ascending
         for (int q = 0; q < k1; ++q)
             p += __shfl_sync(0xffffffffu, j, q) < j;  // empty slots never count
         if (lane < k1) {
-            if (lane < kt) {
+            if (j != MOE_EMPTY_SLOT) {  // taken (kt of the k1 slots)
                 ds->ue[p] = j;
                 ds->uw[p] = wv;
             }
@@ -207,11 +206,11 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
                     a.idx_copy[lane] = j;
                 if (a.w_copy)
                     a.w_copy[lane] = wv;
-                if (lane < kt) {
+                if (j != MOE_EMPTY_SLOT) {
                     a.uniq_list[p] = j;
                     a.sorted_slot[p] = lane;
                 }
-                a.slot_pos[lane] = lane < kt ? p : -1;
+                a.slot_pos[lane] = j != MOE_EMPTY_SLOT ? p : -1;
             }
         }
         __syncwarp();

@@ -203,8 +203,8 @@ static int enqueue_logits(const void *x, const void *wr, const float *bias, floa
 // kernel.
 static int enqueue_decode(const void *x, const void *wg, const void *wu, const void *wdt, int d,
                           int E, int I, int k1, int k2, void *y, int y_dtype, int32_t *idx_copy,
-                          float *w_copy, void *ws, int G, cudaStream_t s, bool cascade = false,
-                          float tau = 0.0f, int32_t *count = nullptr)
+                          float *w_copy, void *ws, int G, cudaStream_t s, VarK vk = VarK(),
+                          int32_t *count = nullptr)
 {
     const WsLayout L = ws_layout(1, d, E, I, k1);
     DecodeArgs a = {};
@@ -230,13 +230,12 @@ static int enqueue_decode(const void *x, const void *wg, const void *wu, const v
     a.y_acc = at<float>(ws, L.y_acc);
     a.y = y;
     a.y_dtype = y_dtype;
-    a.cascade = cascade ? 1 : 0;
-    a.tau = tau;
+    a.vk = vk;
     a.count = count;
     a.hdr = static_cast<WsHeader *>(ws);
     const size_t smem = decode_smem_bytes(d);
     const dim3 grid(G), block(kSThreads);
-    if (cascade) {
+    if (vk.kind != kVarFixed) {
         if (d == 2048)
             return launch(k_decode<8, true>, grid, block, smem, s, true, a);
         if (d == 4096)
@@ -389,12 +388,12 @@ static int enqueue_logits_gemm(const void *x, const void *wr, const float *bias,
 // Warp-per-token routing of T tokens from float32 logits.
 static int enqueue_route_warp(const float *z, int T, int E, int k1, int k2, int32_t *idx, float *w,
                               int32_t *idx_copy, float *w_copy, cudaStream_t s,
-                              bool cascade = false, float tau = 0.0f, int32_t *count = nullptr)
+                              VarK vk = VarK(), int32_t *count = nullptr)
 {
     const dim3 grid((T + 7) / 8), block(256);
 #define MOE_ROUTE_WARP(R)                                                                        \
     return launch(k_route_warp<R>, grid, block, 0, s, true, z, T, E, k1, k2, idx, w, idx_copy, \
-                  w_copy, (int)cascade, tau, count)
+                  w_copy, vk, count)
     if (E <= 32) MOE_ROUTE_WARP(1);
     if (E <= 64) MOE_ROUTE_WARP(2);
     if (E <= 128) MOE_ROUTE_WARP(4);
@@ -491,8 +490,8 @@ int moe_read_device_status(void *ws, int *status_out, void *stream)
 
 static int route_impl(const void *x_bf16, const void *w_router_bf16, const float *bias,
                       float *logits, int T, int d, int E, int k1, int k2, int32_t *topk_idx,
-                      float *topk_w, void *ws, size_t ws_bytes, void *stream, bool cascade,
-                      float tau, int32_t *count)
+                      float *topk_w, void *ws, size_t ws_bytes, void *stream, VarK vk,
+                      int32_t *count)
 {
     int rc = check_route(E, k1, k2);
     if (rc != MOE_OK)
@@ -533,8 +532,7 @@ static int route_impl(const void *x_bf16, const void *w_router_bf16, const float
             return rc;
         z = zbuf;
     }
-    return enqueue_route_warp(z, T, E, k1, k2, topk_idx, topk_w, nullptr, nullptr, s, cascade, tau,
-                              count);
+    return enqueue_route_warp(z, T, E, k1, k2, topk_idx, topk_w, nullptr, nullptr, s, vk, count);
 }
 
 extern "C" {
@@ -544,7 +542,7 @@ int moe_route(const void *x_bf16, const void *w_router_bf16, const float *bias, 
               size_t ws_bytes, void *stream)
 {
     return route_impl(x_bf16, w_router_bf16, bias, logits, T, d, E, k1, k2, topk_idx, topk_w, ws,
-                      ws_bytes, stream, false, 0.0f, nullptr);
+                      ws_bytes, stream, VarK(), nullptr);
 }
 
 int moe_route_cascade(const void *x_bf16, const void *w_router_bf16, const float *bias,
@@ -554,8 +552,37 @@ int moe_route_cascade(const void *x_bf16, const void *w_router_bf16, const float
 {
     if (tau != tau)
         return MOE_ERR_INVALID_ARG;  // NaN
+    VarK vk = {};
+    vk.kind = kVarCascade;
+    vk.tau = tau;
     return route_impl(x_bf16, w_router_bf16, bias, logits, T, d, E, k1, k2, topk_idx, topk_w, ws,
-                      ws_bytes, stream, true, tau, topk_count);
+                      ws_bytes, stream, vk, topk_count);
+}
+
+// The skip rule's arguments: a 16-byte aligned table and two thresholds, not NaN.
+static int skip_args(const float *tab, float th_e, float th_w, VarK &vk)
+{
+    if (!tab || !aligned16(tab) || th_e != th_e || th_w != th_w)
+        return MOE_ERR_INVALID_ARG;
+    vk = {};
+    vk.kind = kVarSkip;
+    vk.tab = tab;
+    vk.th_e = th_e;
+    vk.th_w = th_w;
+    return MOE_OK;
+}
+
+int moe_route_skip(const void *x_bf16, const void *w_router_bf16, const float *bias,
+                   float *logits, int T, int d, int E, int k1, int k2, const float *expert_score,
+                   float theta_expert, float theta_weight, int32_t *topk_idx, float *topk_w,
+                   int32_t *topk_count, void *ws, size_t ws_bytes, void *stream)
+{
+    VarK vk;
+    const int rc = skip_args(expert_score, theta_expert, theta_weight, vk);
+    if (rc != MOE_OK)
+        return rc;
+    return route_impl(x_bf16, w_router_bf16, bias, logits, T, d, E, k1, k2, topk_idx, topk_w, ws,
+                      ws_bytes, stream, vk, topk_count);
 }
 
 int moe_permute(const int32_t *topk_idx, int T, int k1, int E, int32_t *expert_offsets,
@@ -767,9 +794,9 @@ static int layer_impl(const void *x_bf16, const void *w_router_bf16, const float
                       const void *w_gate_bf16, const void *w_up_bf16, const void *w_down_bf16,
                       int T, int d, int E, int I, int k1, int k2, void *y, int y_dtype,
                       int32_t *topk_idx_out, float *topk_w_out, float *logits_out, int flags,
-                      void *ws, size_t ws_bytes, void *stream, bool cascade, float tau,
-                      int32_t *count_out)
+                      void *ws, size_t ws_bytes, void *stream, VarK vk, int32_t *count_out)
 {
+    const bool cascade = vk.kind != kVarFixed;  // a variable-k route (cascade or skip)
     int rc = check_shape(T, d, E, I, k1);
     if (rc != MOE_OK)
         return rc;
@@ -827,8 +854,8 @@ static int layer_impl(const void *x_bf16, const void *w_router_bf16, const float
             rc = enqueue_logits(x_bf16, w_router_bf16, bias, z, logits_out, T, d, E, s);
         if (rc != MOE_OK)
             return rc;
-        if ((rc = enqueue_route_warp(z, T, E, k1, k2, idx, w, topk_idx_out, topk_w_out, s, cascade,
-                                     tau, count_out)) != MOE_OK)
+        if ((rc = enqueue_route_warp(z, T, E, k1, k2, idx, w, topk_idx_out, topk_w_out, s, vk,
+                                     count_out)) != MOE_OK)
             return rc;
         if ((rc = enqueue_perm_parallel(idx, T, k1, E, at<int>(ws, L.hist), po, &hdr->status, s)) !=
             MOE_OK)
@@ -848,8 +875,7 @@ static int layer_impl(const void *x_bf16, const void *w_router_bf16, const float
         return rc;
     if (decode)
         return enqueue_decode(x_bf16, w_gate_bf16, w_up_bf16, w_down_bf16, d, E, I, k1, k2, y,
-                              y_dtype, topk_idx_out, topk_w_out, ws, G, s, cascade, tau,
-                              count_out);
+                              y_dtype, topk_idx_out, topk_w_out, ws, G, s, vk, count_out);
     if (T > 1) {
         // one CTA per token ranks its probabilities; the last one to finish
         // builds the permutation tables
@@ -874,7 +900,7 @@ int moe_layer(const void *x_bf16, const void *w_router_bf16, const float *bias,
 {
     return layer_impl(x_bf16, w_router_bf16, bias, w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I,
                       k1, k2, y, y_dtype, topk_idx_out, topk_w_out, logits_out, flags, ws, ws_bytes,
-                      stream, false, 0.0f, nullptr);
+                      stream, VarK(), nullptr);
 }
 
 int moe_layer_cascade(const void *x_bf16, const void *w_router_bf16, const float *bias,
@@ -885,9 +911,28 @@ int moe_layer_cascade(const void *x_bf16, const void *w_router_bf16, const float
 {
     if (tau != tau)
         return MOE_ERR_INVALID_ARG;  // NaN
+    VarK vk = {};
+    vk.kind = kVarCascade;
+    vk.tau = tau;
     return layer_impl(x_bf16, w_router_bf16, bias, w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I,
                       k1, k2, y, y_dtype, topk_idx_out, topk_w_out, logits_out, flags, ws, ws_bytes,
-                      stream, true, tau, topk_count_out);
+                      stream, vk, topk_count_out);
+}
+
+int moe_layer_skip(const void *x_bf16, const void *w_router_bf16, const float *bias,
+                   const void *w_gate_bf16, const void *w_up_bf16, const void *w_down_bf16, int T,
+                   int d, int E, int I, int k1, int k2, const float *expert_score,
+                   float theta_expert, float theta_weight, void *y, int y_dtype,
+                   int32_t *topk_idx_out, float *topk_w_out, int32_t *topk_count_out,
+                   float *logits_out, int flags, void *ws, size_t ws_bytes, void *stream)
+{
+    VarK vk;
+    const int rc = skip_args(expert_score, theta_expert, theta_weight, vk);
+    if (rc != MOE_OK)
+        return rc;
+    return layer_impl(x_bf16, w_router_bf16, bias, w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I,
+                      k1, k2, y, y_dtype, topk_idx_out, topk_w_out, logits_out, flags, ws, ws_bytes,
+                      stream, vk, topk_count_out);
 }
 
 int moe_channel_norms(const void *w_down_bf16, int E, int d, int I, int flags, float *norms,

@@ -397,6 +397,26 @@ __global__ void __launch_bounds__(1024) k_topk(const float *logits, int T, int E
 }
 
 // ---------------------------------------------------------------------------
+// Variable experts per token.  kind 0: the fixed k1.  kind 1, cascade (the
+// "cascade ... cover" arm of "Reading the MoE measurement defects", sections
+// 4 and 6.2-6.3): the first kt <= k1 ranked experts whose mass reaches tau.
+// kind 2, skip (the expert-skipping shell of "ACE", aimodeling.com, section
+// "How ACE decides what to skip: GSP + RCR": two views must both call a slot
+// low before it is skipped, and the top-1 expert is always kept): slot
+// s >= 1 is skipped when tab[e_s] < th_e (the per-expert offline scalar,
+// looked up) and its Eq. 2 weight w_s < th_w (the token's router-conditioned
+// view); kept slots keep their Eq. 2 weights.  Unused slots hold
+// MOE_EMPTY_SLOT with weight 0 -- a suffix for the cascade, anywhere after
+// slot 0 for skip.
+struct VarK {
+    int kind;
+    float tau;
+    const float *tab;  // [E] (skip)
+    float th_e, th_w;
+};
+constexpr int kVarFixed = 0, kVarCascade = 1, kVarSkip = 2;
+
+// ---------------------------------------------------------------------------
 // warp_route_vals: one warp routes one token from its E float32 logits, held
 // as p[i] = z[lane + 32 i], everything in registers.  That assignment is
 // exactly the canonical partial-sum assignment of the normaliser Z; the
@@ -406,17 +426,19 @@ __global__ void __launch_bounds__(1024) k_topk(const float *logits, int T, int E
 // order as it is found.  Same float sequence, same bits as
 // route_token_block.  Lane s < k1 returns the rank-s expert in my_j and its
 // Eq. 2 weight in my_w.
-// Cascade (variable k per token, cascade = true; the "cascade ... cover" arm
-// of "Reading the MoE measurement defects", sections 4 and 6.2-6.3): the
-// experts are taken in rank order until their mass -- the same float32
-// rank-order partial sums as S -- reaches tau; kt = the smallest such
-// k <= k1, else k1, and lanes kt <= s < k1 return MOE_EMPTY_SLOT and weight
-// 0.  Without the cascade kt = k1.  k_route_warp: one warp per token.
+// With a VarK (above): for the cascade the experts are taken in rank order
+// until their mass -- the same float32 rank-order partial sums as S --
+// reaches tau; kt = the smallest such k <= k1, else k1, and lanes
+// kt <= s < k1 return MOE_EMPTY_SLOT and weight 0; for skip the skipped lanes
+// return MOE_EMPTY_SLOT and weight 0.  kt = the slots taken (k1 when fixed).
+// k_route_warp: one warp per token.
 template <int R>
 __device__ __forceinline__ void warp_route_vals(float (&p)[R], int E, int k1, int k2, int lane,
-                                                int &my_j, float &my_w, bool cascade = false,
-                                                float tau = 0.0f, int *kt_out = nullptr)
+                                                int &my_j, float &my_w, VarK vk = VarK(),
+                                                int *kt_out = nullptr)
 {
+    const bool cascade = vk.kind == kVarCascade;
+    const float tau = vk.tau;
     const float kNegInf = -__int_as_float(0x7f800000);
     float m = kNegInf;
 #pragma unroll
@@ -478,6 +500,13 @@ __device__ __forceinline__ void warp_route_vals(float (&p)[R], int E, int k1, in
         my_j = MOE_EMPTY_SLOT;
         my_w = 0.0f;
     }
+    if (vk.kind == kVarSkip) {
+        if (lane >= 1 && lane < k1 && __ldg(&vk.tab[my_j]) < vk.th_e && my_w < vk.th_w) {
+            my_j = MOE_EMPTY_SLOT;
+            my_w = 0.0f;
+        }
+        kt = __popc(__ballot_sync(0xffffffffu, lane < k1 && my_j != MOE_EMPTY_SLOT));
+    }
     if (kt_out)
         *kt_out = kt;
 }
@@ -485,8 +514,8 @@ __device__ __forceinline__ void warp_route_vals(float (&p)[R], int E, int k1, in
 // The same from E logits in global memory.
 template <int R>
 __device__ __forceinline__ void warp_route(const float *z, int E, int k1, int k2, int lane,
-                                           int &my_j, float &my_w, bool cascade = false,
-                                           float tau = 0.0f, int *kt_out = nullptr)
+                                           int &my_j, float &my_w, VarK vk = VarK(),
+                                           int *kt_out = nullptr)
 {
     float p[R];
 #pragma unroll
@@ -494,14 +523,14 @@ __device__ __forceinline__ void warp_route(const float *z, int E, int k1, int k2
         const int j = lane + 32 * i;
         p[i] = j < E ? __ldcg(&z[j]) : 0.0f;
     }
-    warp_route_vals<R>(p, E, k1, k2, lane, my_j, my_w, cascade, tau, kt_out);
+    warp_route_vals<R>(p, E, k1, k2, lane, my_j, my_w, vk, kt_out);
 }
 
 template <int R>
 __global__ void __launch_bounds__(256) k_route_warp(const float *logits, int T, int E, int k1,
                                                     int k2, int32_t *idx, float *w,
                                                     int32_t *idx_copy, float *w_copy,
-                                                    int cascade, float tau, int32_t *count)
+                                                    VarK vk, int32_t *count)
 {
     pdl_wait();
     pdl_trigger();
@@ -511,7 +540,7 @@ __global__ void __launch_bounds__(256) k_route_warp(const float *logits, int T, 
         return;
     int my_j, kt;
     float my_w;
-    warp_route<R>(logits + (size_t)t * E, E, k1, k2, lane, my_j, my_w, cascade != 0, tau, &kt);
+    warp_route<R>(logits + (size_t)t * E, E, k1, k2, lane, my_j, my_w, vk, &kt);
     if (count && lane == 0)
         count[t] = kt;
     if (lane < k1) {

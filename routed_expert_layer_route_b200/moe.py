@@ -56,6 +56,10 @@ SIGNATURES = {
                                _vp]),
     "moe_layer_cascade": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _i,
                                _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp]),
+    "moe_route_skip": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _f, _f, _vp, _vp, _vp,
+                            _vp, _sz, _vp]),
+    "moe_layer_skip": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _f, _f, _vp,
+                            _i, _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp]),
     "moe_expert_ffn_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
     "moe_pack_w_down": (_i, [_vp, _vp, _i, _i, _i, _vp]),
     "moe_channel_norms": (_i, [_vp, _i, _i, _i, _i, _vp, _vp]),
@@ -206,6 +210,37 @@ def moe_pack_w_down(w_down, w_down_cm=None, stream=None):
     _check(lib().moe_pack_w_down(_p(w_down), _p(w_down_cm), E, d, I, _stream(stream)),
            "moe_pack_w_down")
     return w_down_cm
+
+
+def moe_route_skip(x, w_router, bias, logits, k1, k2, expert_score, theta_expert, theta_weight,
+                   topk_idx, topk_w, topk_count=None, ws=None, stream=None):
+    """Routing with expert skipping (top-1 kept); x None routes the given logits."""
+    if x is not None:
+        T, d = x.shape
+        E = w_router.shape[0]
+    else:
+        T, E = logits.shape
+        d = 0
+    wsp, wsn = _ws_args(ws)
+    _check(lib().moe_route_skip(_p(x), _p(w_router), _p(bias), _p(logits), T, d, E, k1, k2,
+                                _p(expert_score), float(theta_expert), float(theta_weight),
+                                _p(topk_idx), _p(topk_w), _p(topk_count), wsp, wsn,
+                                _stream(stream)), "moe_route_skip")
+
+
+def moe_layer_skip(x, w_router, bias, w_gate, w_up, w_down, k1, k2, expert_score, theta_expert,
+                   theta_weight, y, ws, topk_idx_out=None, topk_w_out=None, topk_count_out=None,
+                   logits_out=None, flags=MOE_PATH_AUTO, stream=None):
+    """moe_layer with expert skipping (top-1 kept)."""
+    T, d = x.shape
+    E, I, _ = w_gate.shape
+    y_dtype = MOE_DTYPE_BF16 if y.dtype == torch.bfloat16 else MOE_DTYPE_F32
+    wsp, wsn = _ws_args(ws)
+    _check(lib().moe_layer_skip(_p(x), _p(w_router), _p(bias), _p(w_gate), _p(w_up), _p(w_down),
+                                T, d, E, I, k1, k2, _p(expert_score), float(theta_expert),
+                                float(theta_weight), _p(y), y_dtype, _p(topk_idx_out),
+                                _p(topk_w_out), _p(topk_count_out), _p(logits_out), flags, wsp,
+                                wsn, _stream(stream)), "moe_layer_skip")
 
 
 def moe_channel_norms(w_down, channel_major=False, norms=None, stream=None):
