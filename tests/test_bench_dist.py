@@ -67,3 +67,26 @@ def test_single_rank_rate_needs_no_process_group():
     import bench
     rate, ms = bench.job_rate(4, 2.0, 1)
     assert ms == 2.0 and rate == pytest.approx(2000.0)
+
+
+def test_cpu_oracle_rate_scales_to_the_whole_stack():
+    # the sampled layers' time per layer is charged for every layer of the stack
+    sys.path.insert(0, ROOT)
+    import bench
+    from routed_expert_layer_route_b200 import synth
+
+    class SmallStack:
+        wl = {"T": 1, "layers": 3}
+
+        def __init__(self):
+            self.layers = [synth.make_layer(1, 64, 8, 32, seed=0, layer=l, device="cpu")
+                           for l in range(3)]
+
+        def down_hf(self, L, e):
+            return synth.to_numpy(L.w_down[e])
+
+    st = SmallStack()
+    r_own, n_own, _, _ = bench.cpu_oracle_rate(st, 2, 4, budget_s=0.3)
+    r_48, n_48, _, _ = bench.cpu_oracle_rate(st, 2, 4, budget_s=0.3, stack_layers=48)
+    assert n_own > 10 and n_48 > 10
+    assert r_48 < r_own / 4  # 16x fewer tokens/s for a 16x deeper stack, within timing noise
