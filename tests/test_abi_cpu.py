@@ -141,3 +141,41 @@ def test_binding_raises_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(moe, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError):
         moe.lib()
+
+
+def test_skip_argument_checks(L):
+    nan, inf = float("nan"), float("inf")
+
+    def rs(tab=FAKE, th_e=0.5, th_w=0.1, k1=8, k2=16, T=4):
+        return L.moe_route_skip(None, None, None, FAKE, T, 0, 128, k1, k2, tab, th_e, th_w, FAKE,
+                                FAKE, None, None, 0, None)
+    assert rs(tab=None) == moe.MOE_ERR_INVALID_ARG                      # no table
+    assert rs(th_e=nan) == moe.MOE_ERR_INVALID_ARG
+    assert rs(th_w=nan) == moe.MOE_ERR_INVALID_ARG
+    assert rs(k1=8, k2=4) == moe.MOE_ERR_INVALID_ARG                    # k2 < k1
+    assert rs(th_w=inf, T=0) == moe.MOE_OK                              # T = 0, infinite threshold
+
+    def ls(tab=FAKE, th_e=0.5, th_w=0.1, T=1):
+        return L.moe_layer_skip(FAKE, FAKE, None, FAKE, FAKE, FAKE, T, 2048, 128, 768, 8, 8, tab,
+                                th_e, th_w, FAKE, 1, None, None, None, None, 0, FAKE, 1 << 40, None)
+    assert ls(tab=None) == moe.MOE_ERR_INVALID_ARG
+    assert ls(th_e=nan) == moe.MOE_ERR_INVALID_ARG
+    assert ls(T=0) == moe.MOE_OK
+
+
+def test_channel_topk_argument_checks(L):
+    def lc(keep=100, k1=8, k2=8, I=768, T=1, y_dtype=1, norms=FAKE):
+        return L.moe_layer_channel_topk(FAKE, FAKE, None, FAKE, FAKE, FAKE, norms, T, 2048, 128, I,
+                                        k1, k2, keep, FAKE, y_dtype, None, None, None, None, None,
+                                        None, FAKE, 1 << 40, None)
+    assert lc(keep=0) == moe.MOE_ERR_INVALID_ARG
+    assert lc(keep=8 * 768 + 1) == moe.MOE_ERR_INVALID_ARG               # more than k1*I
+    assert lc(y_dtype=7) == moe.MOE_ERR_INVALID_ARG
+    assert lc(k1=8, k2=4) == moe.MOE_ERR_INVALID_ARG
+    assert lc(I=4096, keep=100) == moe.MOE_ERR_UNSUPPORTED_SHAPE         # 8*4096 channels > 16384
+    assert lc(T=0) == moe.MOE_OK
+    assert lc(norms=None) == moe.MOE_ERR_INVALID_ARG
+    r = L.moe_channel_norms(FAKE, 128, 2048, 770, 0, FAKE, None)         # I % 16 != 0
+    assert r == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    r = L.moe_channel_norms(FAKE, 128, 2048, 768, 0x7, FAKE, None)       # unknown flag
+    assert r == moe.MOE_ERR_INVALID_ARG
