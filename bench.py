@@ -605,6 +605,7 @@ def run_native(args, world, rank):
         traffic = recorded_traffic(args.workload, k1h, kname)
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
                     "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
+                    "frac_of_nominal_8000_GBps": round(achieved / 8000.0, 4),
                     "kernel": "moe::" + kname,
                     "kernel_us": round(kern_ms * 1000, 2),
                     "algorithmic_bytes_per_launch": int(alg_bytes),
