@@ -166,3 +166,13 @@ def test_channel_topk_argument_checks():
     with pytest.raises(moe.MoeError) as ei:
         _run(big, 8, 8, 100)
     assert ei.value.status == moe.MOE_ERR_UNSUPPORTED_SHAPE
+
+
+@pytest.mark.parametrize("T,d,E,I,k1,k2,keep", [
+    (1, 64, 1024, 16, 32, 64, 1),        # the widest route (1024 experts), smallest experts
+    (1, 64, 1024, 16, 32, 2000, 512),    # k2 > E: no renormalisation, every channel kept
+    (2, 128, 64, 512, 32, 32, 16384),    # the most channels a token may have (32 x 512)
+])
+def test_layer_channel_topk_edge_shapes(T, d, E, I, k1, k2, keep):
+    L = synth.make_layer(T, d, E, I, seed=E + I, device=DEV, bias="normal")
+    _check(L, k1, k2, keep, _run(L, k1, k2, keep))

@@ -136,3 +136,14 @@ def test_skip_argument_checks():
     with pytest.raises(moe.MoeError) as ei:
         _run(L2, 4, 8, tab, 0.5, 0.5, moe.MOE_PATH_AUTO)
     assert ei.value.status == moe.MOE_ERR_UNSUPPORTED_SHAPE
+
+
+def test_layer_skip_edge_shapes():
+    # 32 slots of 1024 experts on the decode path; every slot but the first skipped
+    d, E, I, k1, k2 = 64, 1024, 16, 32, 32
+    L = _peaky(1, d, E, I, seed=77)
+    tab = torch.zeros(E, dtype=torch.float32, device=DEV)
+    out = _run(L, k1, k2, tab, 1.0, math.inf, moe.MOE_WDOWN_CHANNEL_MAJOR,
+               w_down=moe.moe_pack_w_down(L.w_down))
+    k = _check(L, k1, k2, tab, 1.0, math.inf, out, [0])
+    assert k[0] == 1
