@@ -179,3 +179,18 @@ def test_channel_topk_argument_checks(L):
     assert r == moe.MOE_ERR_UNSUPPORTED_SHAPE
     r = L.moe_channel_norms(FAKE, 128, 2048, 768, 0x7, FAKE, None)       # unknown flag
     assert r == moe.MOE_ERR_INVALID_ARG
+
+
+def test_headers_are_plain_c(tmp_path):
+    # the boundary is a C ABI: both headers compile as strict C99, no C++ or CUDA types
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_headers.c"
+    src.write_text('#include "moe.h"\n#include "moe_testing.h"\nint main(void) { return 0; }\n')
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    r = subprocess.run([gcc, "-std=c99", "-pedantic", "-Wall", "-Wextra", "-Werror",
+                        "-fsyntax-only", "-I", inc, str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
