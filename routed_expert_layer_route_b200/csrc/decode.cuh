@@ -28,7 +28,10 @@
 //  * at the end the four groups' partials are summed in shared memory and
 //    added into the float32 accumulator y_acc with 16-byte vector reductions
 //    (red.global.add.v4.f32); the last CTA to check in (a counter in the
-//    workspace header) converts y_acc to the output y.
+//    workspace header) converts y_acc to the output y, and the first one
+//    writes the routing outputs and permutation tables (every CTA holds the
+//    route; writing them out before the stream delayed that CTA, and the
+//    layer, by a microsecond or more).
 // Partial sums from different CTAs reach y_acc in a timing-dependent order,
 // so y can differ between runs in the last bits (stream.cuh holds the
 // deterministic two-phase kernel).
@@ -83,11 +86,16 @@ struct __align__(16) DecodeSmem {
     float hs[kDStages][kWPS];  // w*h of the stage's channels, per group
     int ue[kDMaxK1];           // the activated experts, ascending
     float uw[kDMaxK1];         // their Eq. 2 weights
+    int sj[kDMaxK1];           // the route by slot: expert (or MOE_EMPTY_SLOT),
+    float sw[kDMaxK1];         //   weight,
+    int sp[kDMaxK1];           //   position among the taken experts (-1: empty)
     DSeg seg[kDMaxSeg];
     int nseg;
+    int kt;                    // slots taken
     int abort;
     int issued;
-    int last;
+    int first;                 // this CTA checked in first: it writes the route out
+    int last;                  // this CTA checked in last: it writes y
 };
 
 struct DIter {
@@ -199,37 +207,18 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
                 ds->ue[p] = j;
                 ds->uw[p] = wv;
             }
-            if (b == 0) {
-                a.topk_idx[lane] = j;
-                a.topk_w[lane] = wv;
-                if (a.idx_copy)
-                    a.idx_copy[lane] = j;
-                if (a.w_copy)
-                    a.w_copy[lane] = wv;
-                if (j != MOE_EMPTY_SLOT) {
-                    a.uniq_list[p] = j;
-                    a.sorted_slot[p] = lane;
-                }
-                a.slot_pos[lane] = j != MOE_EMPTY_SLOT ? p : -1;
-            }
+            // kept for the routing outputs, written after the stream by the
+            // first CTA to finish (off the path the layer's time waits on)
+            ds->sj[lane] = j;
+            ds->sw[lane] = wv;
+            ds->sp[lane] = j != MOE_EMPTY_SLOT ? p : -1;
         }
+        if (lane == 0)
+            ds->kt = kt;
         __syncwarp();
         if constexpr (CASCADE) {
             if (lane == 0)
                 decode_segments(ds, kt, I, G, b, status);
-        }
-        if (b == 0) {
-            if (lane == 0) {
-                *a.uniq_count = kt;
-                if (a.count)
-                    *a.count = kt;
-            }
-            for (int e = lane; e <= E; e += 32) {
-                int cnt = 0;
-                for (int q = 0; q < kt; ++q)
-                    cnt += ds->ue[q] < e;
-                a.offsets[e] = cnt;
-            }
         }
     } else {
         // the token's x row, meanwhile
@@ -404,9 +393,40 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
     // ------------------------------------------------------------ y (last CTA to finish)
     if (tid == 0) {
         const unsigned prev = atomicAdd(&a.hdr->decode_arrive, 1u);
+        ds->first = prev == 0u;
         ds->last = prev == (unsigned)G - 1;
     }
     __syncthreads();
+    if (ds->first && warp == 0) {
+        // the routing outputs and the permutation tables of the one token
+        const int kt = ds->kt;
+        if (lane < k1) {
+            const int j = ds->sj[lane], p = ds->sp[lane];
+            const float wv = ds->sw[lane];
+            a.topk_idx[lane] = j;
+            a.topk_w[lane] = wv;
+            if (a.idx_copy)
+                a.idx_copy[lane] = j;
+            if (a.w_copy)
+                a.w_copy[lane] = wv;
+            if (p >= 0) {
+                a.uniq_list[p] = j;
+                a.sorted_slot[p] = lane;
+            }
+            a.slot_pos[lane] = p;
+        }
+        if (lane == 0) {
+            *a.uniq_count = kt;
+            if (a.count)
+                *a.count = kt;
+        }
+        for (int e = lane; e <= E; e += 32) {
+            int cnt = 0;
+            for (int q = 0; q < kt; ++q)
+                cnt += ds->ue[q] < e;
+            a.offsets[e] = cnt;
+        }
+    }
     if (ds->last) {
         __threadfence();
         for (int i = tid * 4; i < d; i += kSThreads * 4) {
