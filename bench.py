@@ -266,6 +266,23 @@ class Stack:
         return synth.to_numpy(wd.contiguous())
 
 
+class OracleLayers:
+    """The workload's layers for the oracle arm: the same seeded synthetic
+    inputs as Stack (synth.make_layer), in the layouts the oracle reads, with
+    nothing from the product library (libmoe.so is never loaded on that arm)."""
+
+    def __init__(self, wl, seed, device):
+        from routed_expert_layer_route_b200 import synth
+        self.wl = wl
+        self.layers = [synth.make_layer(wl["T"], wl["d"], wl["E"], wl["I"], seed=seed, layer=l,
+                                        device=device, bias=wl["bias"])
+                       for l in range(wl["layers"])]
+
+    def down_hf(self, L, e):
+        from routed_expert_layer_route_b200 import synth
+        return synth.to_numpy(L.w_down[e].contiguous())
+
+
 def build_graph(stack, k1, k2, ws_list, ys, stream, fixed=False):
     """Capture one step (every layer's layer call) into a CUDA graph."""
     g = torch.cuda.CUDAGraph()
@@ -322,8 +339,9 @@ def graph_time_per_call(calls, stream, reps):
 
 
 def time_dominant_kernel(stack, k1, k2, ws_list, ys, stream, reps):
-    """Average duration of the expert kernel launched alone (no programmatic
-    dependent launch), one launch per layer so weights come from HBM, not L2."""
+    """Average duration of the streaming expert kernel launched alone (no
+    programmatic dependent launch), one launch per layer so weights come from
+    HBM, not L2 (batches on the CUDA-core streaming path)."""
     from routed_expert_layer_route_b200 import moe
     calls = [(lambda L=L, ws=ws, y=y: moe.moe_test_expert_stream(
         L.x, L.w_gate, L.w_up, L.w_down, k1, k2, y, ws, flags=stack.flags, stream=stream))
@@ -349,7 +367,6 @@ def e2e_tokens_per_s(stack, k1, k2, ws_list, steps, warmup, stream):
     """Through the public API with host buffers: per step, pinned-host ->
     device copy of every layer's tokens, every layer's moe_layer call, and a
     device -> pinned-host copy of every layer's output."""
-    from routed_expert_layer_route_b200 import moe
     wl = stack.wl
     T, d, L_ = wl["T"], wl["d"], wl["layers"]
     host_x = torch.stack([L.x for L in stack.layers]).cpu().pin_memory()
@@ -417,11 +434,9 @@ def cpu_oracle_rate(stack, k1, k2, budget_s=12.0, max_tokens=8, stack_layers=Non
     return T / (per_layer * (stack_layers or wl["layers"])), n, oracle.num_threads(), el
 
 
-# ---------------------------------------------------------------------- main
-def run_native(args, world, rank):
-    from routed_expert_layer_route_b200 import build as pkg_build
-    from routed_expert_layer_route_b200 import moe
-    pkg_build.build()
+# ---------------------------------------------------------------------- measurement
+def workload_of(args):
+    """The workload dict and its (k1, k2) sweep from the command line."""
     wl = dict(WORKLOADS[args.workload])
     if args.T:
         wl["T"] = args.T
@@ -432,10 +447,257 @@ def run_native(args, world, rank):
         sweep = [(args.k1, args.k2 or args.k1)]
     elif args.cascade is not None or args.channel_keep is not None or args.skip is not None:
         sweep = [(8, args.k2 or 8)]  # one condition: (cap) k1 = 8, k2 = 8
+    return wl, sweep
+
+
+def workload_config(name, wl, head, world):
+    """The line's config: what was run (both arms print this same dict)."""
+    T, d, E, I, Ln = wl["T"], wl["d"], wl["E"], wl["I"], wl["layers"]
+    k1, k2 = head
+    one = T == 1
+    return {"workload": "%s: %d layers, d=%d, E=%d, I=%d, T=%d per rank, k1=%d, k2=%d"
+                        % (name, Ln, d, E, I, T, k1, k2),
+            "layers": Ln, "d": d, "E": E, "I": I, "T": T, "k1": k1, "k2": k2,
+            "bias": wl["bias"],
+            "l2": "inputs larger than L2: every step reads the routed experts of all %d layers "
+                  "(%.1f GB of expert weights) from HBM" % (Ln, Ln * E * 3 * d * I * 2 / 1e9),
+            "timing": "CUDA graph of the %d-layer step, CUDA events, max over ranks" % Ln,
+            "w_down_layout": "channel-major [E x I x d], packed once at set-up" if one
+            else "[E x d x I]",
+            "parallelism": "replicas" if world > 1 else "single GPU"}
+
+
+def line_config(args, wl, head, world):
+    """workload_config plus the variant switches of the command line."""
+    c = workload_config(args.workload, wl, head, world)
+    c.update({"cascade_tau": args.cascade, "router_logit_std": args.router_std,
+              "channel_keep_frac": args.channel_keep,
+              "skip_thresholds": list(args.skip) if args.skip is not None else None})
+    return c
+
+
+def timed_graph(graph, steps, warmup, world, stream):
+    """Device time of `steps` replays of a CUDA graph, `warmup` replays first,
+    barrier + synchronize on both sides; the max over ranks."""
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            graph.replay()
+    stream.synchronize()
+    barrier(world)
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    h0 = time.time()
+    s.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(steps):
+            graph.replay()
+    e.record(stream)
+    e.synchronize()
+    h1 = time.time()
+    barrier(world)
+    return allreduce_max(s.elapsed_time(e), world) / steps, (h0, h1)
+
+
+def layer_work(stack, k1, U, mean_k):
+    """Algorithmic bytes and FLOPs of one layer: the unique routed experts'
+    weights, U*3*d*I*2 bytes, and T*(k*6*d*I + 2*d*E) FLOPs (channel top-k:
+    every gate/up row, the norms and the kept down columns)."""
+    wl = stack.wl
+    T, d, E, I = wl["T"], wl["d"], wl["E"], wl["I"]
+    if stack.keep_frac is not None:
+        b = U * 2 * d * I * 2 + U * I * 4 + T * stack.keep(k1) * d * 2
+        f = T * (mean_k * 4.0 * d * I + 2.0 * stack.keep(k1) * d + 2.0 * d * E)
+        return b, f
+    return U * 3 * d * I * 2, T * (mean_k * 6.0 * d * I + 2.0 * d * E)
+
+
+def measure_sweep(stack, sweep, args, world, stream, peaks):
+    """Every (k1, k2) condition: one CUDA graph of the whole step each, timed
+    by the contract's protocol; unique experts read back from the routing.
+    Returns (results, graphs, headline ms, headline window)."""
+    from routed_expert_layer_route_b200 import moe
+    hbm_peak, bf16_peak, _ = peaks
+    wl = stack.wl
+    T, d, E, I, Ln = wl["T"], wl["d"], wl["E"], wl["I"], wl["layers"]
+    dev = stack.layers[0].x.device
+    graphs = {}
+    for (k1, k2) in sweep:
+        ws_list = [moe.workspace(T, d, E, I, k1, device=dev) for _ in range(Ln)]
+        ys = [torch.empty(T, d, dtype=torch.bfloat16, device=dev) for _ in range(Ln)]
+        graphs[(k1, k2)] = (build_graph(stack, k1, k2, ws_list, ys, stream), ws_list, ys)
+    results, head_ms, head_win = [], None, None
+    for (k1, k2) in sweep:
+        g, ws_list, ys = graphs[(k1, k2)]
+        ms, win = timed_graph(g, args.steps, args.warmup, world, stream)
+        if head_ms is None:
+            head_ms, head_win = ms, win
+        us, mean_k = unique_experts(stack, k1, k2, ws_list, ys, stream)
+        U = statistics.mean(us)
+        b, f = layer_work(stack, k1, U, mean_k)
+        lay_s = ms / Ln * 1e-3
+        results.append({"k1": k1, "k2": k2, "ms_per_step": ms, "us_per_layer": ms * 1000 / Ln,
+                        "tokens_per_s": world * T * 1000.0 / ms, "unique_experts_per_layer": U,
+                        "mean_experts_per_token": mean_k, "bytes_per_layer": b,
+                        "flops_per_layer": f, "expert_GBps": b / lay_s / 1e9,
+                        "hbm_frac": b / lay_s / 1e9 / hbm_peak,
+                        "layer_TFLOPs": f / lay_s / 1e12,
+                        "tensor_frac": f / lay_s / 1e12 / bf16_peak})
+    return results, graphs, head_ms, head_win
+
+
+def k1_ratio(results):
+    """Layer time of k1 = 4 over k1 = 8 (same k2 where possible)."""
+    by = {(r["k1"], r["k2"]): r for r in results}
+    for p4, p8 in (((4, 16), (8, 16)), ((4, 4), (8, 8)), ((4, 16), (8, 8)), ((5, 20), (10, 10))):
+        if p4 in by and p8 in by:
+            return (round(by[p4]["us_per_layer"] / by[p8]["us_per_layer"], 4),
+                    "k1=%d,k2=%d over k1=%d,k2=%d" % (p4 + p8))
+    return None, None
+
+
+def peak_note(kind, what):
+    return ("measured (MEASURED_PEAKS.json %s)" % what) if kind == "measured" else \
+        "fallback 6650 GB/s, 1590 TFLOP/s"
+
+
+def roofline_record(stack, workload, head, res, graphs, stream, peaks, variant):
+    """Roofline of the dominant kernel of the headline condition.
+    One token: the layer is one kernel (router, routing, expert FFN, combine),
+    so its average duration in the timed graph is the layer time; bound by
+    HBM on the unique routed experts' bytes.  Tensor-core batches: the gate/up
+    grouped GEMM alone (and the down GEMM), with the bound that binds for its
+    FLOPs and its weight bytes.  CUDA-core streaming batches: that kernel alone."""
+    hbm_peak, bf16_peak, kind = peaks
+    wl = stack.wl
+    T, d, E, I, Ln = wl["T"], wl["d"], wl["E"], wl["I"], wl["layers"]
+    k1, k2 = head
+    _, ws_list, ys = graphs[head]
+    U = res["unique_experts_per_layer"]
+    alg_bytes = res["bytes_per_layer"]
+    if variant or stack.channel_major:
+        lay_s = res["us_per_layer"] * 1e-6
+        achieved = alg_bytes / lay_s / 1e9
+        kname = ("whole layer (cascade route)" if stack.tau is not None else
+                 "whole layer (expert skipping)" if stack.skip is not None else
+                 "whole layer (channel top-k: k_logits, k_ctk_gateup, k_ctk_down)"
+                 if stack.keep_frac is not None else "moe::k_decode")
+        return {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(achieved / hbm_peak, 4),
+                "traffic": None if variant else recorded_traffic(workload, k1, "k_decode"),
+                "frac_of_nominal_8000_GBps": round(achieved / 8000.0, 4),
+                "kernel": kname, "kernel_us": round(lay_s * 1e6, 3),
+                "launches_per_layer": 1 if not variant or stack.keep_frac is None else 3,
+                "algorithmic_bytes_per_launch": int(alg_bytes),
+                "duration_from": "the headline's timed CUDA graph (one kernel per layer)",
+                "peak_source": peak_note(kind, "hbm_gbs")}
+    if stack.grouped:
+        gx_ms, g1_ms, g2_ms = time_grouped_kernels(stack, k1, ws_list, stream, reps=3)
+        n_slots = T * k1
+        # algorithmic work of each GEMM: FLOPs, and the unique experts' weight
+        # bytes (the gathered token rows and h are traffic of this design)
+        f1 = 2.0 * n_slots * 2 * I * d
+        b1 = U * 2 * d * I * 2
+        f2 = 2.0 * n_slots * I * d
+        b2 = U * d * I * 2
+
+        def bound(f, b, ms):
+            t_tensor, t_hbm = f / (bf16_peak * 1e12), b / (hbm_peak * 1e9)
+            tf = f / (ms * 1e-3) / 1e12
+            gb = b / (ms * 1e-3) / 1e9
+            if t_tensor >= t_hbm:
+                return "tensor", tf, bf16_peak, "TFLOP/s", tf / bf16_peak
+            return "hbm", gb, hbm_peak, "GB/s", gb / hbm_peak
+
+        bd1, a1, p1, u1, fr1 = bound(f1, b1, g1_ms)
+        bd2, a2, p2, u2, fr2 = bound(f2, b2, g2_ms)
+        return {"bound": bd1, "achieved": round(a1, 1), "peak": p1, "unit": u1,
+                "frac": round(fr1, 4), "traffic": recorded_traffic(workload, k1, "k_gemm1"),
+                "kernel": "moe::k_gemm1", "kernel_us": round(g1_ms * 1000, 2),
+                "algorithmic_flops_per_launch": f1, "algorithmic_bytes_per_launch": int(b1),
+                "tensor_frac": round(f1 / (g1_ms * 1e-3) / 1e12 / bf16_peak, 4),
+                "hbm_frac": round(b1 / (g1_ms * 1e-3) / 1e9 / hbm_peak, 4),
+                "second_kernel": {"kernel": "moe::k_gemm2", "kernel_us": round(g2_ms * 1000, 2),
+                                  "bound": bd2, "achieved": round(a2, 1), "unit": u2,
+                                  "frac": round(fr2, 4), "algorithmic_flops_per_launch": f2,
+                                  "algorithmic_bytes_per_launch": int(b2)},
+                "gather_kernel": {"kernel": "moe::k_gather_rows",
+                                  "kernel_us": round(gx_ms * 1000, 2)},
+                "duration_from": "CUDA graph of one launch per layer, kernel alone",
+                "peak_source": peak_note(kind, "bf16_tflops burst and hbm_gbs: kernels timed "
+                                               "alone")}
+    kern_ms = time_dominant_kernel(stack, k1, k2, ws_list, ys, stream, reps=5)
+    achieved = alg_bytes / (kern_ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+            "frac": round(achieved / hbm_peak, 4),
+            "traffic": recorded_traffic(workload, k1, "k_stream"),
+            "kernel": "moe::k_stream", "kernel_us": round(kern_ms * 1000, 2),
+            "algorithmic_bytes_per_launch": int(alg_bytes),
+            "duration_from": "CUDA graph of one launch per layer, kernel alone",
+            "peak_source": peak_note(kind, "hbm_gbs")}
+
+
+def layer_roofline(res, peaks):
+    """The whole layer against its roofline time max(FLOPs / bf16 peak,
+    unique expert bytes / HBM bandwidth)."""
+    hbm_peak, bf16_peak, _ = peaks
+    t_f = res["flops_per_layer"] / (bf16_peak * 1e12)
+    t_b = res["bytes_per_layer"] / (hbm_peak * 1e9)
+    t = res["us_per_layer"] * 1e-6
+    return {"bound": "tensor" if t_f >= t_b else "hbm",
+            "roofline_us": round(max(t_f, t_b) * 1e6, 2),
+            "frac_of_roofline_time": round(max(t_f, t_b) / t, 4),
+            "layer_TFLOPs": round(res["layer_TFLOPs"], 1),
+            "tensor_frac": round(res["tensor_frac"], 4), "hbm_frac": round(res["hbm_frac"], 4)}
+
+
+# workloads timed after the headline in the default run, each a sub-record
+EXTRA_WORKLOADS = [
+    ("decode_small_batch", {"T": 8}), ("decode_small_batch", {"T": 32}),
+    ("decode_small_batch", {"T": 64}), ("prefill", {}),
+    ("large", {"T": 1}), ("large", {"T": 64}),
+]
+
+
+def extra_record(name, over, args, world, rank, stream, peaks):
+    """One more workload, timed like the headline: its sweep, unique experts,
+    the k1 ratio and the roofline of its dominant kernel."""
+    wl = dict(WORKLOADS[name])
+    wl.update(over)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stack = Stack(wl, seed=rank, device=dev)
+    res, graphs, _, _ = measure_sweep(stack, wl["sweep"], args, world, stream, peaks)
+    roof = roofline_record(stack, name, wl["sweep"][0], res[0], graphs, stream, peaks, False)
+    ratio, pair = k1_ratio(res)
+    rec = {"workload": workload_config(name, wl, wl["sweep"][0], world)["workload"],
+           "T": wl["T"], "layers": wl["layers"],
+           "conditions": [{k: (round(v, 4) if isinstance(v, float) else v) for k, v in r.items()}
+                          for r in res],
+           "k1_ratio": ratio, "k1_ratio_conditions": pair, "roofline": roof,
+           "layer_roofline": [dict(layer_roofline(r, peaks), k1=r["k1"], k2=r["k2"]) for r in res]}
+    for g, _, _ in graphs.values():
+        del g
+    graphs.clear()
+    del stack
+    release_memory()
+    return rec
+
+
+def release_memory():
+    import gc
+    gc.collect()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def run_native(args, world, rank):
+    from routed_expert_layer_route_b200 import build as pkg_build
+    pkg_build.build()
+    wl, sweep = workload_of(args)
     head = sweep[0]
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.Stream()
-    hbm_peak, bf16_peak, peak_kind = load_peaks()
+    peaks = load_peaks()
+    hbm_peak, bf16_peak, peak_kind = peaks
 
     if args.channel_keep is not None and wl["T"] != 1:
         raise SystemExit("--channel-keep: one-token workloads only (T = 1)")
@@ -443,188 +705,59 @@ def run_native(args, world, rank):
                   keep_frac=args.channel_keep, skip=args.skip)
     variant = stack.tau is not None or stack.keep_frac is not None or stack.skip is not None
     T, d, E, I, Ln = wl["T"], wl["d"], wl["E"], wl["I"], wl["layers"]
-    results = []
-    graphs = {}
-    for (k1, k2) in sweep:
-        ws_list = [moe.workspace(T, d, E, I, k1, device=dev) for _ in range(Ln)]
-        ys = [torch.empty(T, d, dtype=torch.bfloat16, device=dev) for _ in range(Ln)]
-        g = build_graph(stack, k1, k2, ws_list, ys, stream)
-        graphs[(k1, k2)] = (g, ws_list, ys)
 
-    def timed(*args_):
-        key, (steps, warmup) = (args_[0], args_[1:]) if isinstance(args_[0], tuple) else \
-            ((args_[0], args_[1]), args_[2:])
-        g = graphs[key][0]
-        with torch.cuda.stream(stream):
-            for _ in range(warmup):
-                g.replay()
-        stream.synchronize()
-        barrier(world)
-        s = torch.cuda.Event(enable_timing=True)
-        e = torch.cuda.Event(enable_timing=True)
-        h0 = time.time()
-        s.record(stream)
-        with torch.cuda.stream(stream):
-            for _ in range(steps):
-                g.replay()
-        e.record(stream)
-        e.synchronize()
-        h1 = time.time()
-        barrier(world)
-        ms = s.elapsed_time(e)
-        return job_rate(T * steps, ms, world)[1] / steps, (h0, h1)
-
-    # headline: the timed region of the contract (clocks sampled around it)
+    # headline: the timed region of the contract (clocks sampled around it),
+    # then every other (k1, k2) condition of the sweep by the same protocol
     clocks = ClockSampler(smi_index(torch.cuda.current_device()))
     clocks.start()
-    ms_step, head_win = timed(*head, args.steps, args.warmup)
+    results, graphs, ms_step, head_win = measure_sweep(stack, sweep, args, world, stream, peaks)
+    sweep_t1 = time.time()
     value = world * T * 1000.0 / ms_step
-    sweep_t0 = head_win[0]
-
-    # every (k1, k2) condition of the sweep, same protocol, outside the headline region
-    for (k1, k2) in sweep:
-        ms = ms_step if (k1, k2) == head else timed(k1, k2, args.steps, args.warmup)[0]
-        sweep_t1 = time.time()
-        _, ws_list, ys = graphs[(k1, k2)]
-        us, mean_k = unique_experts(stack, k1, k2, ws_list, ys, stream)
-        U = statistics.mean(us)
-        bytes_layer = U * 3 * d * I * 2
-        flops_layer = T * (mean_k * 6.0 * d * I + 2.0 * d * E)
-        if stack.keep_frac is not None:
-            # every gate/up row and norm of the routed experts, the kept down columns
-            bytes_layer = U * 2 * d * I * 2 + U * I * 4 + T * stack.keep(k1) * d * 2
-            flops_layer = T * (mean_k * 4.0 * d * I + 2.0 * stack.keep(k1) * d + 2.0 * d * E)
-        results.append({"k1": k1, "k2": k2, "ms_per_step": ms, "us_per_layer": ms * 1000 / Ln,
-                        "bytes_per_layer": bytes_layer,
-                        "tokens_per_s": world * T * 1000.0 / ms, "unique_experts_per_layer": U,
-                        "expert_GBps": bytes_layer / (ms / Ln * 1e-3) / 1e9,
-                        "layer_TFLOPs": flops_layer / (ms / Ln * 1e-3) / 1e12,
-                        "mean_experts_per_token": mean_k})
 
     cascade = None
     channel_topk = None
-    if stack.keep_frac is not None:
-        # the same stack through the full decode layer: bytes saved vs time saved
+    if variant:
+        # the same stack with the fixed-k1 full layer: compute / bytes saved vs time saved
         k1h_, k2h_ = head
         _, ws_list, ys = graphs[head]
         gf = build_graph(stack, k1h_, k2h_, ws_list, ys, stream, fixed=True)
         graphs[("fixed",) + head] = (gf, ws_list, ys)
-        ms_fixed = timed(("fixed",) + head, args.steps, args.warmup)[0]
-        U0 = results[0]["unique_experts_per_layer"]
-        channel_topk = {"keep": stack.keep(k1h_), "keep_frac": stack.keep_frac, "k1": k1h_,
-                        "k2": k2h_, "channels_per_token": k1h_ * I,
-                        "us_per_layer": results[0]["us_per_layer"],
-                        "full_layer_us_per_layer": ms_fixed * 1000 / Ln,
-                        "time_ratio_vs_full": results[0]["us_per_layer"] / (ms_fixed * 1000 / Ln),
-                        "bytes_ratio_vs_full": results[0]["bytes_per_layer"] / (U0 * 3 * d * I * 2)}
-    if stack.tau is not None or stack.skip is not None:
-        # the same stack with the fixed k1 route: compute saved vs time saved
-        k1h_, k2h_ = head
-        _, ws_list, ys = graphs[head]
-        gf = build_graph(stack, k1h_, k2h_, ws_list, ys, stream, fixed=True)
-        graphs[("fixed",) + head] = (gf, ws_list, ys)
-        ms_fixed = timed(("fixed",) + head, args.steps, args.warmup)[0]
-        cascade = {"tau": stack.tau, "skip_thresholds": stack.skip, "k1_cap": k1h_, "k2": k2h_,
-                   "mean_experts_per_token": results[0]["mean_experts_per_token"],
-                   "us_per_layer": results[0]["us_per_layer"],
-                   "fixed_k1_us_per_layer": ms_fixed * 1000 / Ln,
-                   "time_ratio_vs_fixed": results[0]["us_per_layer"] / (ms_fixed * 1000 / Ln),
-                   "compute_ratio_vs_fixed": results[0]["mean_experts_per_token"] / k1h_}
+        ms_fixed = timed_graph(gf, args.steps, args.warmup, world, stream)[0]
+        fixed_us = ms_fixed * 1000 / Ln
+        if stack.keep_frac is not None:
+            U0 = results[0]["unique_experts_per_layer"]
+            channel_topk = {"keep": stack.keep(k1h_), "keep_frac": stack.keep_frac, "k1": k1h_,
+                            "k2": k2h_, "channels_per_token": k1h_ * I,
+                            "us_per_layer": results[0]["us_per_layer"],
+                            "full_layer_us_per_layer": fixed_us,
+                            "time_ratio_vs_full": results[0]["us_per_layer"] / fixed_us,
+                            "bytes_ratio_vs_full": results[0]["bytes_per_layer"]
+                            / (U0 * 3 * d * I * 2)}
+        else:
+            cascade = {"tau": stack.tau, "skip_thresholds": stack.skip, "k1_cap": k1h_,
+                       "k2": k2h_, "mean_experts_per_token": results[0]["mean_experts_per_token"],
+                       "us_per_layer": results[0]["us_per_layer"],
+                       "fixed_k1_us_per_layer": fixed_us,
+                       "time_ratio_vs_fixed": results[0]["us_per_layer"] / fixed_us,
+                       "compute_ratio_vs_fixed": results[0]["mean_experts_per_token"] / k1h_}
 
     clocks.stop()
     clk, _ = clocks.summary(*head_win)
     if clk is None:  # timed region shorter than the sampling period: use the sweep's
-        clk, _ = clocks.summary(sweep_t0, sweep_t1)
+        clk, _ = clocks.summary(head_win[0], sweep_t1)
         if clk is not None:
             clk["window"] = "headline and sweep timed regions"
 
-    # dominant kernel alone, events on its own stream
+    roofline = roofline_record(stack, args.workload, head, results[0], graphs, stream, peaks,
+                               variant)
     k1h, k2h = head
     _, ws_list, ys = graphs[head]
-    U_head = results[0]["unique_experts_per_layer"]
-    alg_bytes = results[0]["bytes_per_layer"]
-    if variant:
-        # the kernels alone are re-run only with the fixed route; for a cascade
-        # route or channel top-k the roofline is taken over the whole layer
-        lay_s = results[0]["us_per_layer"] * 1e-6
-        achieved = alg_bytes / lay_s / 1e9
-        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
-                    "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": None,
-                    "kernel": "whole layer (%s)" % ("cascade route" if stack.tau is not None else
-                                                    "expert skipping" if stack.skip is not None
-                                                    else "channel top-k: k_logits, k_ctk_gateup, "
-                                                    "k_ctk_down"),
-                    "kernel_us": round(lay_s * 1e6, 2),
-                    "algorithmic_bytes_per_launch": int(alg_bytes),
-                    "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind}
-    elif stack.grouped:
-        gx_ms, g1_ms, g2_ms = time_grouped_kernels(stack, k1h, ws_list, stream, reps=3)
-        n_slots = T * k1h
-        # algorithmic work of each GEMM: FLOPs, and bytes = the unique experts'
-        # weights + the token rows read + the rows written
-        f1 = 2.0 * n_slots * 2 * I * d                       # gate and up
-        b1 = U_head * 2 * d * I * 2 + n_slots * d * 2 + n_slots * I * 2
-        f2 = 2.0 * n_slots * I * d                           # down
-        b2 = U_head * d * I * 2 + n_slots * I * 2 + T * d * 4
-
-        def bound(f, b, ms):
-            t_tensor, t_hbm = f / (bf16_peak * 1e12), b / (hbm_peak * 1e9)
-            tf = f / (ms * 1e-3) / 1e12
-            gb = b / (ms * 1e-3) / 1e9
-            if t_tensor >= t_hbm:
-                return "tensor", tf, bf16_peak, "TFLOP/s", tf / bf16_peak, gb / hbm_peak
-            return "hbm", gb, hbm_peak, "GB/s", gb / hbm_peak, tf / bf16_peak
-
-        bd1, a1, p1, u1, fr1, other1 = bound(f1, b1, g1_ms)
-        bd2, a2, p2, u2, fr2, other2 = bound(f2, b2, g2_ms)
-        roofline = {"bound": bd1, "achieved": round(a1, 1), "peak": p1, "unit": u1,
-                    "frac": round(fr1, 4),
-                    "traffic": recorded_traffic(args.workload, k1h, "k_gemm1"),
-                    "kernel": "moe::k_gemm1", "kernel_us": round(g1_ms * 1000, 2),
-                    "algorithmic_flops_per_launch": f1, "algorithmic_bytes_per_launch": int(b1),
-                    "tensor_frac": round(f1 / (g1_ms * 1e-3) / 1e12 / bf16_peak, 4),
-                    "hbm_frac": round(b1 / (g1_ms * 1e-3) / 1e9 / hbm_peak, 4),
-                    "second_kernel": {"kernel": "moe::k_gemm2", "kernel_us": round(g2_ms * 1000, 2),
-                                      "bound": bd2, "achieved": round(a2, 1), "unit": u2,
-                                      "frac": round(fr2, 4),
-                                      "algorithmic_flops_per_launch": f2,
-                                      "algorithmic_bytes_per_launch": int(b2)},
-                    "gather_kernel": {"kernel": "moe::k_gather_rows",
-                                      "kernel_us": round(gx_ms * 1000, 2)},
-                    "both_gemms_tensor_frac": round((f1 + f2) / ((g1_ms + g2_ms) * 1e-3) / 1e12
-                                                    / bf16_peak, 4),
-                    "both_gemms_hbm_frac": round(alg_bytes / ((g1_ms + g2_ms) * 1e-3) / 1e9
-                                                 / hbm_peak, 4),
-                    "peak_source": "%s (MEASURED_PEAKS.json bf16_tflops burst and hbm_gbs: "
-                                   "kernels timed alone)" % peak_kind if peak_kind == "measured"
-                    else "fallback 1590 TFLOP/s, 6650 GB/s"}
-    else:
-        kern_ms = time_dominant_kernel(stack, k1h, k2h, ws_list, ys, stream, reps=5)
-        achieved = alg_bytes / (kern_ms * 1e-3) / 1e9
-        kname = "k_decode" if stack.channel_major else "k_stream"
-        traffic = recorded_traffic(args.workload, k1h, kname)
-        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
-                    "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
-                    "frac_of_nominal_8000_GBps": round(achieved / 8000.0, 4),
-                    "kernel": "moe::" + kname,
-                    "kernel_us": round(kern_ms * 1000, 2),
-                    "algorithmic_bytes_per_launch": int(alg_bytes),
-                    "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
-                    if peak_kind == "measured" else "fallback 6650 GB/s"}
 
     # end to end through the public API with host buffers
     e2e_val, h2d, d2h = e2e_tokens_per_s(stack, k1h, k2h, ws_list, max(3, args.steps // 4),
                                          args.warmup, stream)
     e2e_val = world * T * 1000.0 / allreduce_max(T * 1000.0 / e2e_val, world)
-
-    # ratio of k1=4 to k1=8 layer time (same k2 where possible)
-    by = {(r["k1"], r["k2"]): r for r in results}
-    ratio, ratio_pair = None, None
-    for p4, p8 in (((4, 16), (8, 16)), ((4, 4), (8, 8)), ((4, 16), (8, 8)), ((5, 20), (10, 10))):
-        if p4 in by and p8 in by:
-            ratio = by[p4]["us_per_layer"] / by[p8]["us_per_layer"]
-            ratio_pair = "k1=%d,k2=%d over k1=%d,k2=%d" % (p4 + p8)
-            break
+    ratio, ratio_pair = k1_ratio(results)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not variant:
@@ -634,29 +767,20 @@ def run_native(args, world, rank):
                          "in %.1f s; per-layer time scaled to the %d-layer stack"
                          % (nl, min(T, 8), k1h, k2h, el, Ln)}
 
-    # kernels per layer: router logits + decode kernel (one token); router logits,
-    # warp router, permutation (2), token-row gather, two grouped GEMMs, finalize
-    # (tensor-core path); router logits, top-k, streaming kernel (streaming path)
-    per_step_launches = 2 if stack.channel_major else (8 if stack.grouped else 3)
+    # kernels per layer: the one-token layer kernel; router logits, warp router,
+    # permutation (2), token-row gather, two grouped GEMMs, finalize (tensor-core
+    # path); router logits, top-k, streaming kernel (streaming path)
+    per_step_launches = 1 if stack.channel_major else (8 if stack.grouped else 3)
     if stack.keep_frac is not None:
         per_step_launches = 1 + 2 * T  # router logits, then two kernels per token
+    config = line_config(args, wl, head, world)
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "us_per_layer": round(ms_step * 1000 / Ln, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,0.02) weights, RMS-normalised N(0,1) tokens)",
-        "config": {"workload": "%s: %d layers, d=%d, E=%d, I=%d, T=%d per rank, k1=%d, k2=%d"
-                               % (args.workload, Ln, d, E, I, T, k1h, k2h),
-                   "layers": Ln, "d": d, "E": E, "I": I, "T": T, "k1": k1h, "k2": k2h,
-                   "bias": wl["bias"], "us_per_layer": round(ms_step * 1000 / Ln, 3),
-                   "cascade_tau": stack.tau, "router_logit_std": args.router_std,
-                   "channel_keep_frac": stack.keep_frac, "skip_thresholds": stack.skip,
-                   "l2": "inputs larger than L2: every step reads the routed experts of all "
-                         "%d layers (%.2f GB) from HBM" % (Ln, alg_bytes * Ln / 1e9),
-                   "timing": "CUDA graph of the %d-layer step, CUDA events, max over ranks" % Ln,
-                   "w_down_layout": "channel-major [E x I x d], packed once at set-up"
-                   if stack.channel_major else "[E x d x I]",
-                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "config": config,
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_val, 3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
@@ -667,12 +791,31 @@ def run_native(args, world, rank):
         "sweep": results,
         "cascade": cascade,
         "channel_topk": channel_topk,
-        "k1_4_over_k1_8_time_ratio": None if ratio is None else round(ratio, 4),
+        "k1_4_over_k1_8_time_ratio": ratio,
         "k1_ratio_conditions": ratio_pair,
     }
     for g, _, _ in graphs.values():
         del g
     graphs.clear()
+    del stack
+    release_memory()
+
+    # the other workloads (small batches, prefill, the large model), each a
+    # sub-record with its own sweep, unique experts, k1 ratio and roofline
+    default = (args.workload == "decode_b1" and not args.k1 and not args.T and not args.layers
+               and not variant and not args.no_extra)
+    if default:
+        extra = {}
+        for name, over in EXTRA_WORKLOADS:
+            key = name + "".join("_%s%d" % kv for kv in sorted(over.items()))
+            extra[key] = extra_record(name, over, args, world, rank, stream, peaks)
+        line["workloads"] = extra
+        line["k1_ratio_by_batch"] = {
+            "T=1": {"ratio": ratio, "conditions": ratio_pair},
+            **{"T=%d" % extra[k]["T"]: {"ratio": extra[k]["k1_ratio"],
+                                        "conditions": extra[k]["k1_ratio_conditions"]}
+               for k in ("decode_small_batch_T8", "decode_small_batch_T32",
+                         "decode_small_batch_T64")}}
     return line
 
 
@@ -680,16 +823,12 @@ def run_reference(args, world, rank):
     """The oracle as it stands on the host cores, on the same workload."""
     if rank != 0:
         return None
-    wl = dict(WORKLOADS[args.workload])
-    if args.T:
-        wl["T"] = args.T
-    if args.layers:
-        wl["layers"] = args.layers
-    k1, k2 = (args.k1, args.k2 or args.k1) if args.k1 else wl["sweep"][0]
+    wl, sweep = workload_of(args)
+    k1, k2 = sweep[0]
     dev = torch.device("cuda", torch.cuda.current_device())
     small = dict(wl)
     small["layers"] = min(6, wl["layers"])
-    stack = Stack(small, seed=0, device=dev)
+    stack = OracleLayers(small, seed=0, device=dev)
     rates = []
     # each step a bounded sample: the whole run stays near two minutes at any K
     step_s = max(0.05, min(3.0, 120.0 / max(1, args.steps + args.warmup)))
@@ -707,9 +846,7 @@ def run_reference(args, world, rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1000.0 * wl["T"] / r_stack, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32 (bf16 inputs widened)",
-        "data": "synthetic", "config": {"workload": "%s: %d layers, d=%d, E=%d, I=%d, T=%d, k1=%d, "
-                                                    "k2=%d" % (args.workload, wl["layers"], wl["d"],
-                                                               wl["E"], wl["I"], wl["T"], k1, k2)},
+        "data": "synthetic", "config": line_config(args, wl, (k1, k2), world),
         "cpu_baseline": {"value": round(r_stack, 4), "unit": "tokens/s", "cores": thr,
                          "kind": "oracle", "sample": "each step: layers of this workload for "
                                                      "%.2f s, first %d token(s) of each; per-layer "
@@ -733,6 +870,9 @@ def main():
     ap.add_argument("--T", type=int, default=0)
     ap.add_argument("--layers", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="time only the chosen workload (the default run also times the small "
+                         "batches, prefill and the large model as sub-records)")
     ap.add_argument("--cascade", type=float, default=None, metavar="TAU",
                     help="variable experts per token: the first k <= k1 covering mass TAU")
     ap.add_argument("--skip", type=float, nargs=2, default=None, metavar=("TH_E", "TH_W"),

@@ -109,9 +109,10 @@ int moe_version(void);
  * Returns 0 when the shapes are invalid. */
 size_t moe_workspace_size(int T, int d, int E, int I, int k1);
 
-/* Zero the workspace's header (status word and the counters and flags the
- * kernels use for cross-block hand-off).  Enqueued on `stream`.  Call it once
- * before the first use, and again after a call recorded MOE_ERR_TIMEOUT. */
+/* Zero the whole workspace: the header (status word, the counters and flags
+ * the kernels use for cross-block hand-off) and the accumulators the kernels
+ * keep zero between calls.  Enqueued on `stream`.  Call it once before the
+ * first use, and again after a call recorded MOE_ERR_TIMEOUT. */
 int moe_workspace_init(void *ws, size_t ws_bytes, void *stream);
 
 /* Copy the workspace's device status word into *status_out (MOE_OK or a
@@ -299,18 +300,28 @@ int moe_pack_w_down(const void *w_down_bf16, void *w_down_cm_bf16, int E, int d,
  *    routed slots must fit the array), and the usual shape limits; larger
  *    shapes return MOE_ERR_SCRATCH_LIMIT and enqueue nothing.
  *  - The first call on a device looks up the array's device address (once
- *    per device, with that device current); make that first call outside any
- *    stream capture.
+ *    per device, with that device current) and keeps it for the life of the
+ *    process; make that first call outside any stream capture.  The address
+ *    is not looked up again, so calls after cudaDeviceReset on that device
+ *    are not supported.
  *  - Every call on a device shares the one array, and each call clears the
  *    part that must start at zero.  Calls whose work overlaps on the GPU
  *    (e.g. on two streams at once) race on the array; order them on one
  *    stream.
- *  - Device-side problems (bounded waits, index checks) cannot be read back
- *    through a workspace; they leave out unspecified. */
+ *  - Device-side problems (a bounded wait that gave up, an index check)
+ *    leave out unspecified and are recorded in the array's status word,
+ *    which calls do not clear: read it with moe_noalloc_read_status. */
 int moe_expert_ffn_noalloc(const void *x_bf16, const int32_t *expert_offsets,
                            const int32_t *sorted_slot, const void *w_gate_bf16,
                            const void *w_up_bf16, const void *w_down_bf16, int T, int d, int E,
                            int I, int k1, float *out, void *stream);
+
+/* The device status word of moe_expert_ffn_noalloc on the current device:
+ * copied into *status_out (host memory; MOE_OK or the first device-side
+ * moe_status any call recorded since the last read) and cleared.  Enqueued on
+ * `stream` after the calls to check, then synchronises `stream`.  Allocates
+ * nothing.  The paper has no counterpart. */
+int moe_noalloc_read_status(int *status_out, void *stream);
 
 #ifdef __cplusplus
 }

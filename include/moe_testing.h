@@ -22,6 +22,22 @@ int moe_test_exp_c(const float *x, float *y, int64_t n, void *stream);
  * device (0 if no device). */
 int moe_test_num_sms(void);
 
+/* Set how long the library's bounded device waits (mbarrier phases,
+ * cross-CTA flags, the grid barrier, the one-token layer's router exchange)
+ * spin before they give up and record MOE_ERR_TIMEOUT, for the current
+ * device, in nanoseconds (default 2e9).  Synchronous.  For tests that make a
+ * wait run out; set it back afterwards.  Returns a moe_status. */
+int moe_test_set_wait_limit_ns(uint64_t ns);
+
+/* Launch one CTA that waits, with the library's bounded waits, on something
+ * nothing ever completes: which 0, a flag in the workspace header; 1, an
+ * mbarrier phase no thread arrives on; 2, the one-token layer's router
+ * exchange for a tag no CTA publishes.  The wait gives up at the wait limit,
+ * records MOE_ERR_TIMEOUT in the workspace's status word and the kernel
+ * returns; the context stays usable.  Enqueued on `stream`.  Returns a
+ * moe_status. */
+int moe_test_wait_never_set(void *ws, size_t ws_bytes, int which, void *stream);
+
 /* Re-run only the expert kernel of the last moe_layer call made with this
  * workspace, these shapes and these flags, reusing the logits (T == 1, where
  * the kernel routes the token itself) or the routing tables (T > 1) that call

@@ -1,5 +1,6 @@
-// decode.cuh -- the small-batch layer kernel: one pass over the routed
-// experts' weights, each byte read once from HBM, no grid-wide barrier.
+// decode.cuh -- the one-token layer kernel: router logits, routing, the
+// routed experts' SwiGLU FFN and the weighted combine in one launch, each
+// weight byte read once from HBM.
 //
 // Structure of an expert ("Channel Selection for Mixture-of-Experts Decoding
 // Needs No Calibration Data", section 2 "Background"): a gated MLP whose
@@ -8,33 +9,36 @@
 // k_pack_w_down), a channel is three contiguous rows, and a CTA that owns
 // channels [c0, c1) of an expert finishes that expert's share of the output
 // alone:
-//     y[t, :] += w[t, e] * sum_{c in [c0, c1)} h_c(x_t) * down_row_c
-// (Eq. 2 weight w, "Paper of the Week #3", section "The Receipt").
+//     y[:] += w_e * sum_{c in [c0, c1)} h_c(x) * down_row_c
+// (Eq. 2 weight w_e, "Paper of the Week #3", section "The Receipt").
 //
-// Design (one persistent CTA per SM, 12 consumer warps + 1 producer warp):
-//  * one token per call (T == 1): one warp of every CTA routes it from the
-//    router's logits in registers (warp_route: the same fixed float32
-//    sequence as the router kernels) while the others load x; each CTA's
-//    channel ranges are fixed before the kernel waits on the router;
+// Design (one CTA per SM, cooperative launch; 12 consumer warps + 1 producer
+// warp):
+//  * router: CTA b dots x with router rows b, b+G, ... (fetched into shared
+//    memory before the programmatic-launch wait -- weights no earlier kernel
+//    writes -- with an L2 evict-last policy), writes the logits and counts
+//    them on a release counter in the workspace header (spread over lines);
+//    warp 0 of every CTA waits for all E, reads them back, forms the float32
+//    softmax, selects the top min(k2, E) in rank order from a candidate set
+//    and applies Eq. 2 -- the fixed float32 sequence the oracle follows;
 //  * the U activated experts are laid end to end as U*I channels and CTA b
 //    owns a contiguous range of floor(U*I/G) or one more channels;
 //  * the producer streams stages of n whole channels (gate rows, up rows,
-//    down rows: three contiguous bulk copies) through a ring of kStages
+//    down rows: three contiguous bulk copies) through a ring of kDStages
 //    shared-memory slots; each slot is served by kWPS consumer warps;
 //  * per stage, warp i of the slot's group forms h for channel i (times the
 //    token's Eq. 2 weight), the group meets at a named barrier, and each warp
 //    adds h * down_row into register partials for its fixed third of the
 //    output rows;
-//  * at the end the four groups' partials are summed in shared memory and
-//    added into the float32 accumulator y_acc with 16-byte vector reductions
-//    (red.global.add.v4.f32); the last CTA to check in (a counter in the
-//    workspace header) converts y_acc to the output y, and the first one
-//    writes the routing outputs and permutation tables (every CTA holds the
-//    route; writing them out before the stream delayed that CTA, and the
-//    layer, by a microsecond or more).
-// Partial sums from different CTAs reach y_acc in a timing-dependent order,
-// so y can differ between runs in the last bits (stream.cuh holds the
-// deterministic two-phase kernel).
+//  * combine: the four groups' partials are summed in shared memory and added
+//    into a float32 accumulator with 16-byte vector reductions (CTAs that
+//    finish early add theirs while others still stream); one fence and one
+//    ticket per CTA; the last CTA converts the accumulator to y and clears it
+//    for the next call.  Partial sums reach the accumulator in a
+//    timing-dependent order, so y can differ between runs in the last bits.
+// Call numbers (decode_seq in the header) pick one of four counters per call;
+// each call clears the counter two calls ahead, so no counter is reset on the
+// critical path.
 #pragma once
 #include "common.cuh"
 #include "route.cuh"
@@ -57,6 +61,12 @@ struct DecodeArgs {
     const uint16_t *wu;   // [E x I x d]
     const uint16_t *wdt;  // [E x I x d]: down matrix, channel-major
     int d, E, I, k1, k2;
+    // router: wr [E x d] (+ bias [E], nullable) -- the kernel forms the
+    // logits itself, writes them to `logits` (and logits_out, nullable); with
+    // wr null it routes from the float32 logits already in `logits`
+    const uint16_t *wr;
+    const float *bias;
+    float *logits_out;
     const float *logits;  // [E] float32
     int32_t *topk_idx;
     float *topk_w;
@@ -67,8 +77,8 @@ struct DecodeArgs {
     int32_t *slot_pos;
     int32_t *uniq_count;
     int32_t *uniq_list;
-    float *y_acc;  // [d] float32, zero on entry
-    void *y;       // [d] output (y_dtype); written by the last CTA to finish
+    float *yacc;   // [d] float32 accumulator, zero on entry; the last CTA clears it again
+    void *y;       // [d] output (y_dtype)
     int y_dtype;
     VarK vk;       // variable k: cascade or skip (kind 0 with the fixed-k kernel)
     int32_t *count;  // nullable: kt
@@ -82,6 +92,9 @@ struct DSeg {
     int b;  // one past the last channel
 };
 
+constexpr int kDMaxRouterRows = 8;          // router rows one CTA dots with x
+constexpr int kDRouteOff = 128 * 1024;      // ring offset of the routing scratch
+
 struct __align__(16) DecodeSmem {
     float hs[kDStages][kWPS];  // w*h of the stage's channels, per group
     int ue[kDMaxK1];           // the activated experts, ascending
@@ -94,8 +107,8 @@ struct __align__(16) DecodeSmem {
     int kt;                    // slots taken
     int abort;
     int issued;
-    int first;                 // this CTA checked in first: it writes the route out
     int last;                  // this CTA checked in last: it writes y
+    unsigned call;             // this call's number (decode_seq + 1)
 };
 
 struct DIter {
@@ -150,6 +163,71 @@ __device__ void decode_segments(DecodeSmem *ds, int U, int I, int G, int b, int 
     ds->nseg = ns;
 }
 
+// Arrival i of a spread count (release: this thread's earlier accesses, and
+// those it observed through a CTA barrier, come first).
+MOE_DEVINL void spread_arrive(SpreadCount *sc, unsigned i)
+{
+    fence_release_gpu();
+    atomicAdd(&sc->c[i % kSpread][0], 1u);
+}
+
+// One warp waits (bounded) until a spread count has seen n arrivals numbered
+// 0..n-1: lane l reads counter l % kSpread, whose share is the arrivals i
+// with i % kSpread == l % kSpread; then every lane acquires.  Gives up at the
+// wait limit: records MOE_ERR_TIMEOUT and returns false (on every lane).
+MOE_DEVINL bool warp_wait_spread(const SpreadCount *sc, unsigned n, int lane, int *status)
+{
+    const unsigned q = (unsigned)lane % kSpread;
+    const unsigned want = n > q ? (n - q + kSpread - 1) / kSpread : 0u;
+    const unsigned *p = &sc->c[q][0];
+    bool ok = true;
+    if (!__all_sync(0xffffffffu, ld_relaxed_u32(p) >= want)) {
+        const uint64_t t0 = global_ns();
+        const uint64_t lim = wait_limit_ns();
+        while (!__all_sync(0xffffffffu, ld_relaxed_u32(p) >= want)) {
+            if (global_ns() - t0 > lim) {
+                if (lane == 0)
+                    set_status(status, MOE_ERR_TIMEOUT);
+                ok = false;
+                break;
+            }
+            __nanosleep(32);
+        }
+    }
+    fence_acquire_gpu();
+    return ok;
+}
+
+// Warp 0 routes the token: its E logits into registers -- once the router
+// exchange counts all E published (bounded wait; every lane acquires, so each
+// lane's reads follow the logits), or directly when the logits were given --
+// the float32 softmax as keys, the Kneed best in rank order into sel_p /
+// sel_j, and Eq. 2 (lane s < k1: slot s).
+template <int R>
+__device__ __forceinline__ void decode_route(const DecodeArgs &a, bool fused, unsigned slot,
+                                             int lane, DecodeSmem *ds, int *status, VarK vk,
+                                             float *sel_p, int *sel_j, unsigned *cand_k,
+                                             int *cand_j, int &my_j, float &my_w, int &kt)
+{
+    const int E = a.E;
+    float p[R];
+    bool ok = true;
+    if (fused)  // every lane acquires, so each lane's reads below follow the logits
+        ok = warp_wait_spread(&a.hdr->xcnt[slot], (unsigned)E, lane, status);
+    if (!ok && lane == 0)
+        ds->abort = 1;
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+        const int j = lane + 32 * i;
+        p[i] = j < E && ok ? __ldcg(&a.logits[j]) : 0.0f;
+    }
+    unsigned key[R];
+    warp_softmax_keys<R>(p, E, lane, key);
+    const int Kneed = a.k2 < E ? a.k2 : a.k1;
+    warp_select_ranked<R>(key, Kneed, lane, sel_p, sel_j, cand_k, cand_j);
+    route_finish(sel_p, sel_j, E, a.k1, a.k2, lane, my_j, my_w, vk, &kt);
+}
+
 // VPL: d = 256*VPL for the single-token register path (x in registers when
 // VPL <= kXRegMax), 0 for the general token loop.  CASCADE: the variable-k
 // route (a.vk: cascade or skip).
@@ -160,19 +238,30 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
     uint8_t *ring = smem;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + kDStages * kDStageBytes);
     uint64_t *empty = full + kDStages;
-    DecodeSmem *ds = reinterpret_cast<DecodeSmem *>(empty + kDStages);
+    uint64_t *rbar = empty + kDStages;  // the router rows' bulk copies (2 slots: alignment)
+    DecodeSmem *ds = reinterpret_cast<DecodeSmem *>(rbar + 2);
     uint8_t *area = reinterpret_cast<uint8_t *>(ds + 1);  // the token's x row, d bf16
+    // routing scratch in the ring, which is idle until the route is known
+    // (the router rows occupy its first kDMaxRouterRows * d * 2 <= kDRouteOff bytes)
+    float *sel_p = reinterpret_cast<float *>(ring + kDRouteOff);  // [Kneed] in rank order
+    int *sel_j = reinterpret_cast<int *>(sel_p + kMaxExperts);
+    unsigned *cand_k = reinterpret_cast<unsigned *>(sel_j + kMaxExperts);  // [64] candidates
+    int *cand_j = reinterpret_cast<int *>(cand_k + 64);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = gridDim.x, b = blockIdx.x;
     int *status = &a.hdr->status;
     const int d = a.d, E = a.E, I = a.I, k1 = a.k1;
+    const bool fused = a.wr != nullptr;
+    const int nr = fused && b < E ? (E - 1 - b) / G + 1 : 0;  // router rows e = b + G*i
+    const int nvec = d >> 3;                                   // 16-byte vectors per row
 
     if (tid == 0) {
         for (int s = 0; s < kDStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kWPS);
         }
+        mbar_init(rbar, 1);
         ds->abort = 0;
         ds->issued = 0;
         fence_mbar_init();
@@ -182,48 +271,129 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
             decode_segments(ds, k1, I, G, b, status);
     }
     __syncthreads();
+    // this CTA's router rows: weights no earlier kernel writes, so they are
+    // fetched before the dependency wait and overlap the previous kernel
+    if (warp == kSC && lane == 0 && nr > 0) {
+        const uint64_t keep = l2_evict_last_policy();  // the router, read by every call
+        mbar_arrive_expect_tx(rbar, (uint32_t)(nr * d * 2));
+        for (int i = 0; i < nr; ++i)
+            bulk_g2s(ring + (size_t)i * d * 2, a.wr + (size_t)(b + G * i) * d, (uint32_t)(d * 2),
+                     rbar, keep);
+    }
 
     pdl_wait();
     pdl_trigger();
 
-    // ------------------------------------------------------------ routing (one warp)
-    if (warp == 0) {
-        int j, kt;
-        float wv;
-        const VarK vk = CASCADE ? a.vk : VarK();
-        if (E <= 128)
-            warp_route<4>(a.logits, E, k1, a.k2, lane, j, wv, vk, &kt);
-        else if (E <= 256)
-            warp_route<8>(a.logits, E, k1, a.k2, lane, j, wv, vk, &kt);
-        else if (E <= 512)
-            warp_route<16>(a.logits, E, k1, a.k2, lane, j, wv, vk, &kt);
-        else
-            warp_route<32>(a.logits, E, k1, a.k2, lane, j, wv, vk, &kt);
-        int p = 0;  // position of this lane's expert among the kt taken, ascending
-        for (int q = 0; q < k1; ++q)
-            p += __shfl_sync(0xffffffffu, j, q) < j;  // empty slots never count
-        if (lane < k1) {
-            if (j != MOE_EMPTY_SLOT) {  // taken (kt of the k1 slots)
-                ds->ue[p] = j;
-                ds->uw[p] = wv;
+    if (warp < kSC) {
+        const unsigned call = ld_relaxed_u32(&a.hdr->decode_seq) + 1u;
+        const unsigned slot = call & 3u;
+        if (b == 0 && tid < kSpread)  // the count of the call two ahead starts at zero
+            a.hdr->xcnt[(call + 2u) & 3u].c[tid][0] = 0u;
+        // ------------------------------------------------------------ router logits
+        // warp i < nr: router row b + G*i in router_step's order (the order of
+        // k_logits), its x vectors all in flight at once; warp 0 also keeps
+        // the token's x row in shared memory for the FFN
+        const uint4 *xg = reinterpret_cast<const uint4 *>(a.x);
+        const bool xreg = nvec <= 32 * kLogitsMaxVec;
+        uint4 xq[kLogitsMaxVec];
+        if ((warp == 0 || warp < nr) && xreg) {
+#pragma unroll
+            for (int i = 0; i < kLogitsMaxVec; ++i) {
+                const int v = lane + 32 * i;
+                xq[i] = v < nvec ? xg[v] : make_uint4(0, 0, 0, 0);
             }
-            // kept for the routing outputs, written after the stream by the
-            // first CTA to finish (off the path the layer's time waits on)
-            ds->sj[lane] = j;
-            ds->sw[lane] = wv;
-            ds->sp[lane] = j != MOE_EMPTY_SLOT ? p : -1;
         }
-        if (lane == 0)
-            ds->kt = kt;
-        __syncwarp();
-        if constexpr (CASCADE) {
-            if (lane == 0)
-                decode_segments(ds, kt, I, G, b, status);
+        if (warp == 0) {
+            if (xreg) {
+#pragma unroll
+                for (int i = 0; i < kLogitsMaxVec; ++i)
+                    if (lane + 32 * i < nvec)
+                        reinterpret_cast<uint4 *>(area)[lane + 32 * i] = xq[i];
+            } else {
+                for (int v = lane; v < nvec; v += 32)
+                    reinterpret_cast<uint4 *>(area)[v] = xg[v];
+            }
         }
-    } else {
-        // the token's x row, meanwhile
-        for (int i = tid - 32; i < (d >> 3); i += kSThreads - 32)
-            reinterpret_cast<uint4 *>(area)[i] = reinterpret_cast<const uint4 *>(a.x)[i];
+        if (warp < nr) {
+            if (!mbar_wait(rbar, 0, status))
+                ds->abort = 1;
+            const uint4 *row = reinterpret_cast<const uint4 *>(ring + (size_t)warp * d * 2);
+            float a0 = 0.0f, a1 = 0.0f;
+            if (xreg) {
+#pragma unroll
+                for (int i = 0; i < kLogitsMaxVec; ++i)
+                    if (lane + 32 * i < nvec)
+                        router_step(a0, a1, i, row[lane + 32 * i], xq[i]);
+            } else {
+                int i = 0;
+                for (int v = lane; v < nvec; v += 32, ++i)
+                    router_step(a0, a1, i, row[v], xg[v]);
+            }
+            float z = warp_sum(a0 + a1);
+            const int e = b + G * warp;
+            if (a.bias)
+                z = z + a.bias[e];
+            if (lane == 0) {
+                const_cast<float *>(a.logits)[e] = z;
+                if (a.logits_out)
+                    a.logits_out[e] = z;
+                spread_arrive(&a.hdr->xcnt[slot], (unsigned)e);  // the logit before the count
+            }
+        }
+
+        // ------------------------------------------------------------ routing (warp 0)
+        if (warp == 0) {
+            int j, kt;
+            float wv;
+            const VarK vk = CASCADE ? a.vk : VarK();
+            if (E <= 128)
+                decode_route<4>(a, fused, slot, lane, ds, status, vk, sel_p, sel_j, cand_k,
+                                cand_j, j, wv, kt);
+            else if (E <= 256)
+                decode_route<8>(a, fused, slot, lane, ds, status, vk, sel_p, sel_j, cand_k,
+                                cand_j, j, wv, kt);
+            else if (E <= 512)
+                decode_route<16>(a, fused, slot, lane, ds, status, vk, sel_p, sel_j, cand_k,
+                                 cand_j, j, wv, kt);
+            else
+                decode_route<32>(a, fused, slot, lane, ds, status, vk, sel_p, sel_j, cand_k,
+                                 cand_j, j, wv, kt);
+            if (MOE_CHECKS) {  // the route: experts in range, kt slots taken
+                const bool bad = (lane < k1 && j != MOE_EMPTY_SLOT && (j < 0 || j >= E)) ||
+                                 kt < 0 || kt > k1;
+                if (__any_sync(0xffffffffu, bad)) {
+                    if (lane == 0) {
+                        set_status(status, MOE_ERR_DEVICE_CHECK);
+                        ds->abort = 1;
+                    }
+                    j = lane < k1 ? MOE_EMPTY_SLOT : 0;
+                    kt = 0;
+                }
+            }
+            int p = 0;  // position of this lane's expert among the kt taken, ascending
+            for (int q = 0; q < k1; ++q)
+                p += __shfl_sync(0xffffffffu, j, q) < j;  // empty slots never count
+            if (lane < k1) {
+                if (j != MOE_EMPTY_SLOT) {  // taken (kt of the k1 slots)
+                    ds->ue[p] = j;
+                    ds->uw[p] = wv;
+                }
+                // kept for the routing outputs, which CTA 0 writes at the end
+                // (off the path the layer's time waits on)
+                ds->sj[lane] = j;
+                ds->sw[lane] = wv;
+                ds->sp[lane] = j != MOE_EMPTY_SLOT ? p : -1;
+            }
+            if (lane == 0) {
+                ds->kt = kt;
+                ds->call = call;
+            }
+            __syncwarp();
+            if constexpr (CASCADE) {
+                if (lane == 0)
+                    decode_segments(ds, kt, I, G, b, status);
+            }
+        }
     }
     __syncthreads();
     const int nseg = ds->nseg;
@@ -235,13 +405,13 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
             const uint64_t pol = l2_evict_first_policy();
             DIter it;
             it.init(ds->seg, nseg, nch);
-            int slot = 0;
+            int slot_r = 0;
             uint32_t ph = 0;
             int issued = 0;
             while (it.valid()) {
                 if (*(volatile int *)&ds->abort)
                     break;
-                if (!mbar_wait(&empty[slot], ph ^ 1u, status)) {
+                if (!mbar_wait(&empty[slot_r], ph ^ 1u, status)) {
                     ds->abort = 1;
                     break;
                 }
@@ -249,15 +419,15 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
                 const int e = ds->ue[ds->seg[it.s].u];
                 const size_t row0 = (size_t)e * I + it.c;
                 const uint32_t bytes = (uint32_t)n * d * 2;
-                uint8_t *dst = ring + (size_t)slot * kDStageBytes;
-                mbar_arrive_expect_tx(&full[slot], 3 * bytes);
-                bulk_g2s(dst, a.wg + row0 * d, bytes, &full[slot], pol);
-                bulk_g2s(dst + bytes, a.wu + row0 * d, bytes, &full[slot], pol);
-                bulk_g2s(dst + 2 * bytes, a.wdt + row0 * d, bytes, &full[slot], pol);
+                uint8_t *dst = ring + (size_t)slot_r * kDStageBytes;
+                mbar_arrive_expect_tx(&full[slot_r], 3 * bytes);
+                bulk_g2s(dst, a.wg + row0 * d, bytes, &full[slot_r], pol);
+                bulk_g2s(dst + bytes, a.wu + row0 * d, bytes, &full[slot_r], pol);
+                bulk_g2s(dst + 2 * bytes, a.wdt + row0 * d, bytes, &full[slot_r], pol);
                 ++issued;
                 it.next();
-                if (++slot == kDStages) {
-                    slot = 0;
+                if (++slot_r == kDStages) {
+                    slot_r = 0;
                     ph ^= 1u;
                 }
             }
@@ -268,7 +438,6 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
         // ------------------------------------------------------------ consumers
         const int group = warp / kWPS;
         const int gl = warp % kWPS;
-        const int nvec = d >> 3;  // 16-byte vectors per row
         // this warp's output rows: vectors v = gl*32 + lane + kWPS*32*j, j < RV
         constexpr int RV = VPL > 0 ? (VPL * 32 + kWPS * 32 - 1) / (kWPS * 32) : kDMaxRowVec;
         static_assert(RV <= kDMaxRowVec, "row partials");
@@ -350,7 +519,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
             it.next();
         }
 
-        // ------------------------------------------------------------ reduce and add
+        // ------------------------------------------------------------ this CTA's partial row
         consumer_sync();  // every warp is past its last stage: the ring is free
         float *red = reinterpret_cast<float *>(ring);  // [kDStages][d]
 #pragma unroll
@@ -363,21 +532,23 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
             }
         }
         consumer_sync();
-        if (nseg > 0) {  // one 16-byte vector reduction per four output rows
+        // the four groups' partials summed and added into the accumulator with
+        // 16-byte vector reductions; CTAs that finish early add theirs while
+        // the others still stream
+        if (nseg > 0) {
             for (int r = tid * 4; r < d; r += kSC * 32 * 4) {
-                float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+                float4 sum = *reinterpret_cast<const float4 *>(red + r);
 #pragma unroll
-                for (int g = 0; g < kDStages; ++g) {
+                for (int g = 1; g < kDStages; ++g) {
                     const float4 v = *reinterpret_cast<const float4 *>(red + (size_t)g * d + r);
                     sum.x += v.x;
                     sum.y += v.y;
                     sum.z += v.z;
                     sum.w += v.w;
                 }
-                red_add_v4(a.y_acc + r, sum.x, sum.y, sum.z, sum.w);
+                red_add_v4(a.yacc + r, sum.x, sum.y, sum.z, sum.w);
             }
         }
-        __threadfence();  // the adds are visible before this CTA checks in below
     }
 
     __syncthreads();
@@ -389,15 +560,37 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
             mbar_wait(&full[s], parity, status);
         }
     }
+    if (warp == kSC)
+        return;
 
-    // ------------------------------------------------------------ y (last CTA to finish)
+    // ------------------------------------------------------------ y (last CTA to check in)
     if (tid == 0) {
+        fence_acq_rel_gpu();  // this CTA's reductions before its ticket; others' after
         const unsigned prev = atomicAdd(&a.hdr->decode_arrive, 1u);
-        ds->first = prev == 0u;
         ds->last = prev == (unsigned)G - 1;
     }
-    __syncthreads();
-    if (ds->first && warp == 0) {
+    consumer_sync();
+    if (ds->last) {
+        for (int i = tid * 4; i < d; i += kSC * 32 * 4) {
+            const float4 v = __ldcg(reinterpret_cast<const float4 *>(a.yacc + i));
+            if (a.y_dtype == MOE_DTYPE_BF16) {
+                const uint32_t lo = f32_to_bf16_rn(v.x) | ((uint32_t)f32_to_bf16_rn(v.y) << 16);
+                const uint32_t hi = f32_to_bf16_rn(v.z) | ((uint32_t)f32_to_bf16_rn(v.w) << 16);
+                *reinterpret_cast<uint2 *>(reinterpret_cast<uint16_t *>(a.y) + i) =
+                    make_uint2(lo, hi);
+            } else {
+                *reinterpret_cast<float4 *>(reinterpret_cast<float *>(a.y) + i) = v;
+            }
+            __stcg(reinterpret_cast<float4 *>(a.yacc + i), make_float4(0.f, 0.f, 0.f, 0.f));
+        }
+        if (tid == 0) {
+            a.hdr->decode_arrive = 0u;
+            // every CTA read the call number before it took its ticket
+            a.hdr->decode_seq = ds->call;
+        }
+    }
+
+    if (b == 0 && warp == 0) {
         // the routing outputs and the permutation tables of the one token
         const int kt = ds->kt;
         if (lane < k1) {
@@ -421,43 +614,31 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
                 *a.count = kt;
         }
         for (int e = lane; e <= E; e += 32) {
-            int cnt = 0;
+            int c = 0;
             for (int q = 0; q < kt; ++q)
-                cnt += ds->ue[q] < e;
-            a.offsets[e] = cnt;
+                c += ds->ue[q] < e;
+            a.offsets[e] = c;
         }
-    }
-    if (ds->last) {
-        __threadfence();
-        for (int i = tid * 4; i < d; i += kSThreads * 4) {
-            const float4 v = __ldcg(reinterpret_cast<const float4 *>(a.y_acc + i));
-            if (a.y_dtype == MOE_DTYPE_BF16) {
-                const uint32_t lo = f32_to_bf16_rn(v.x) | ((uint32_t)f32_to_bf16_rn(v.y) << 16);
-                const uint32_t hi = f32_to_bf16_rn(v.z) | ((uint32_t)f32_to_bf16_rn(v.w) << 16);
-                *reinterpret_cast<uint2 *>(reinterpret_cast<uint16_t *>(a.y) + i) =
-                    make_uint2(lo, hi);
-            } else {
-                *reinterpret_cast<float4 *>(reinterpret_cast<float *>(a.y) + i) = v;
-            }
-        }
-        if (tid == 0)
-            a.hdr->decode_arrive = 0u;
     }
 }
 
 inline size_t decode_smem_bytes(int d)
 {
-    return (size_t)kDStages * kDStageBytes + 2 * kDStages * sizeof(uint64_t) + sizeof(DecodeSmem) +
-           (size_t)d * 2;
+    return (size_t)kDStages * kDStageBytes + (2 * kDStages + 2) * sizeof(uint64_t) +
+           sizeof(DecodeSmem) + (size_t)d * 2;
 }
 
 // The single-pass path serves one token per call (T == 1) whose output rows
-// fit the register partials, with the down matrix channel-major.
+// fit the register partials, with the down matrix channel-major; each CTA's
+// router rows fit the ring below the routing scratch.
 inline bool decode_fits(int T, int d, int E, int I, int k1, int G)
 {
-    if (T != 1 || k1 > kDMaxK1 || (d >> 3) > kWPS * 32 * kDMaxRowVec)
+    if (T != 1 || k1 > kDMaxK1 || (d >> 3) > kWPS * 32 * kDMaxRowVec || E > kMaxExperts)
         return false;
     if (decode_smem_bytes(d) > 227 * 1024 || (size_t)kDStages * d * 4 > (size_t)kDStages * kDStageBytes)
+        return false;
+    const int rows = (E + G - 1) / G;
+    if (rows > kDMaxRouterRows || (size_t)rows * d * 2 > (size_t)kDRouteOff)
         return false;
     const long chmax = ((long)k1 * I + G - 1) / G;
     const long nseg = (chmax + I - 1) / I + 1;

@@ -227,19 +227,40 @@ struct GTable {
     int ibase[kGMaxE + 1];  // first item of each expert; ibase[E] = item count
     int offs[kGMaxE + 1];   // expert offsets into the slot order
     int bn;                 // tokens per tile (<= kGBN, multiple of 64)
+    int bad;                // checked build: the offsets failed their check
     int scan[40];
 };
 
 // All threads of the CTA: fill the table from the expert offsets (or, with
-// offsets == nullptr, one group of single_n rows).
-__device__ void g_build_items(const int32_t *offsets, int E, int nrt, GTable &tb, int single_n = 0,
-                              int bn = kGBN)
+// offsets == nullptr, one group of single_n rows).  nmax: the rows the
+// offsets may address; the checked build verifies 0 <= offs[0] <= ... <=
+// offs[E] <= nmax and, if not, records MOE_ERR_DEVICE_CHECK and leaves no
+// items.
+__device__ void g_build_items(const int32_t *offsets, int E, int nrt, GTable &tb, int nmax,
+                              int *status, int single_n = 0, int bn = kGBN)
 {
     for (int e = threadIdx.x; e <= E; e += blockDim.x)
         tb.offs[e] = offsets ? __ldcg(&offsets[e]) : (e == 0 ? 0 : single_n);
-    if (threadIdx.x == 0)
+    if (threadIdx.x == 0) {
         tb.bn = bn;
+        tb.bad = 0;
+    }
     __syncthreads();
+    if (MOE_CHECKS) {
+        for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+            const int o = tb.offs[e];
+            if (o < 0 || o > nmax || (e < E && o > tb.offs[e + 1]))
+                tb.bad = 1;
+        }
+        __syncthreads();
+        if (tb.bad) {
+            if (threadIdx.x == 0)
+                set_status(status, MOE_ERR_DEVICE_CHECK);
+            for (int e = threadIdx.x; e <= E; e += blockDim.x)
+                tb.offs[e] = 0;
+        }
+        __syncthreads();
+    }
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         const int n = tb.offs[e + 1] - tb.offs[e];
         tb.ibase[e] = n > 0 ? nrt * ((n + bn - 1) / bn) : 0;
@@ -457,7 +478,7 @@ __global__ void __launch_bounds__(kG1Threads, 1)
     const int d = a.d, E = a.E, I = a.I;
     const int nrt = I / kGBM;
     const int nkb = d / kGBK;
-    g_build_items(a.offsets, E, nrt, tb);
+    g_build_items(a.offsets, E, nrt, tb, a.T * a.k1, status);
     const int n_items = tb.ibase[E];
     GQueue q = {0, 0u};
 
@@ -625,7 +646,8 @@ __global__ void __launch_bounds__(kG2Threads, 1)
     const int d = a.d, E = a.E, I = a.I;
     const int nrt = d / kGBM;
     const int nkb = I / kGBK;
-    g_build_items(a.offsets, E, nrt, tb, a.single_n, a.bn > 0 ? a.bn : kGBN);
+    g_build_items(a.offsets, E, nrt, tb, a.offsets ? a.T * a.k1 : a.single_n, status, a.single_n,
+                  a.bn > 0 ? a.bn : kGBN);
     const int n_items = tb.ibase[E];
     GQueue q = {0, 0u};
 
@@ -724,6 +746,10 @@ __global__ void __launch_bounds__(kG2Threads, 1)
                 wt[c] = 0.0f;
                 if (a.combine && (c & 1) == eh && col < it.n) {
                     const int slot = __ldcg(&a.sorted_slot[it.p0 + col]);
+                    if (MOE_CHECKS && (slot < 0 || slot >= a.T * k1)) {
+                        set_status(status, MOE_ERR_DEVICE_CHECK);
+                        continue;  // weight 0 into token 0: adds nothing
+                    }
                     tk[c] = slot / k1;
                     wt[c] = __ldcg(&a.topk_w[slot]);
                 }

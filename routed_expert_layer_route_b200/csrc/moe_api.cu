@@ -31,7 +31,7 @@ static inline size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct WsLayout {
     size_t logits, idx, w, offsets, sorted_slot, slot_pos, uniq_count, uniq_list, h, out, y_acc,
-        hist, ctk, total;
+        hist, ctk, dyacc, total;
 };
 
 static inline int perm_chunks(int T) { return (T + kPermTok - 1) / kPermTok; }
@@ -54,6 +54,8 @@ static WsLayout ws_layout(int T, int d, int E, int I, int k1)
     L.y_acc = o;       o = align256(o + sizeof(float) * (size_t)T * d);
     L.hist = o;        o = align256(o + sizeof(int32_t) * (size_t)perm_chunks(T) * E);
     L.ctk = o;         o = align256(o + 2 * sizeof(float) * (size_t)k1 * I);  // one token's h, scores
+    // one token: the decode kernel's accumulator (kept zero between calls)
+    L.dyacc = o;       o = align256(o + (T == 1 ? sizeof(float) * (size_t)d : 0));
     L.total = o;
     return L;
 }
@@ -148,20 +150,36 @@ static int device_info(DevInfo *&out)
 }
 
 // ------------------------------------------------------------------ launch
+// Launch options: kPdl chains the kernel to the previous one on the stream by
+// programmatic dependent launch (the kernel calls griddepcontrol.wait before
+// it reads anything an earlier kernel wrote); kCoop makes it a cooperative
+// launch, which the runtime places only when every CTA of the grid can be
+// resident at once (kernels whose CTAs wait on one another need that).
+constexpr int kPdl = 1, kCoop = 2;
+
 template <typename... KArgs, typename... Args>
 static int launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                  bool pdl, Args &&...args)
+                  int opts, Args &&...args)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = pdl ? attr : nullptr;
-    cfg.numAttrs = pdl ? 1 : 0;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    if (opts & kPdl) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    if (opts & kCoop) {
+        attr[n].id = cudaLaunchAttributeCooperative;
+        attr[n].val.cooperative = 1;
+        ++n;
+    }
+    cfg.attrs = n ? attr : nullptr;
+    cfg.numAttrs = n;
     const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
     return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -197,11 +215,11 @@ static int enqueue_logits(const void *x, const void *wr, const float *bias, floa
     return launch(k_logits, dim3(grid), dim3(kLogitsWarps * 32), 0, s, true, a);
 }
 
-// The single-pass decode path of moe_layer after the router (T == 1, down
-// matrix channel-major): one decode kernel (routing, gate/up, down partials
-// into y_acc, y written by its last CTA).  y_acc was cleared by the router
-// kernel.
-static int enqueue_decode(const void *x, const void *wg, const void *wu, const void *wdt, int d,
+// The single-pass decode path of moe_layer (T == 1, down matrix
+// channel-major): one kernel -- router logits, routing, gate/up, down
+// partials into y_acc, y written by its last CTA.
+static int enqueue_decode(const void *x, const void *wr, const float *bias, float *logits_out,
+                          const void *wg, const void *wu, const void *wdt, int d,
                           int E, int I, int k1, int k2, void *y, int y_dtype, int32_t *idx_copy,
                           float *w_copy, void *ws, int G, cudaStream_t s, VarK vk = VarK(),
                           int32_t *count = nullptr)
@@ -217,6 +235,9 @@ static int enqueue_decode(const void *x, const void *wg, const void *wu, const v
     a.I = I;
     a.k1 = k1;
     a.k2 = k2;
+    a.wr = static_cast<const uint16_t *>(wr);
+    a.bias = bias;
+    a.logits_out = logits_out;
     a.logits = at<float>(ws, L.logits);
     a.topk_idx = at<int32_t>(ws, L.idx);
     a.topk_w = at<float>(ws, L.w);
@@ -227,7 +248,7 @@ static int enqueue_decode(const void *x, const void *wg, const void *wu, const v
     a.slot_pos = at<int32_t>(ws, L.slot_pos);
     a.uniq_count = at<int32_t>(ws, L.uniq_count);
     a.uniq_list = at<int32_t>(ws, L.uniq_list);
-    a.y_acc = at<float>(ws, L.y_acc);
+    a.yacc = at<float>(ws, L.dyacc);
     a.y = y;
     a.y_dtype = y_dtype;
     a.vk = vk;
@@ -237,16 +258,16 @@ static int enqueue_decode(const void *x, const void *wg, const void *wu, const v
     const dim3 grid(G), block(kSThreads);
     if (vk.kind != kVarFixed) {
         if (d == 2048)
-            return launch(k_decode<8, true>, grid, block, smem, s, true, a);
+            return launch(k_decode<8, true>, grid, block, smem, s, kPdl | kCoop, a);
         if (d == 4096)
-            return launch(k_decode<16, true>, grid, block, smem, s, true, a);
-        return launch(k_decode<0, true>, grid, block, smem, s, true, a);
+            return launch(k_decode<16, true>, grid, block, smem, s, kPdl | kCoop, a);
+        return launch(k_decode<0, true>, grid, block, smem, s, kPdl | kCoop, a);
     }
     if (d == 2048)
-        return launch(k_decode<8, false>, grid, block, smem, s, true, a);
+        return launch(k_decode<8, false>, grid, block, smem, s, kPdl | kCoop, a);
     if (d == 4096)
-        return launch(k_decode<16, false>, grid, block, smem, s, true, a);
-    return launch(k_decode<0, false>, grid, block, smem, s, true, a);
+        return launch(k_decode<16, false>, grid, block, smem, s, kPdl | kCoop, a);
+    return launch(k_decode<0, false>, grid, block, smem, s, kPdl | kCoop, a);
 }
 
 
@@ -464,8 +485,9 @@ int moe_workspace_init(void *ws, size_t ws_bytes, void *stream)
 {
     if (!ws || ws_bytes < sizeof(WsHeader) || (reinterpret_cast<uintptr_t>(ws) & 255))
         return MOE_ERR_INVALID_ARG;
-    return cudaMemsetAsync(ws, 0, sizeof(WsHeader), static_cast<cudaStream_t>(stream)) ==
-                   cudaSuccess
+    // all of it: the header's counters and the accumulators that kernels keep
+    // zero between calls
+    return cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)) == cudaSuccess
                ? MOE_OK
                : MOE_ERR_CUDA;
 }
@@ -663,17 +685,22 @@ static int enqueue_stream(const StreamCall &c, cudaStream_t s, bool pdl = true)
     a.y = c.y;
     a.y_dtype = c.y_dtype;
     a.hdr = c.hdr;
+    // One CTA per SM, and the CTAs meet at a grid-wide barrier between the
+    // two phases: the launch is cooperative, so the runtime places the grid
+    // only when all of it can be resident at once (else the launch fails
+    // instead of the barrier timing out).
     const unsigned grid = (unsigned)(di->num_sms < kMaxGridCtas ? di->num_sms : kMaxGridCtas);
+    const int opts = (pdl ? kPdl : 0) | kCoop;
     switch (stream_variant(c.T, c.d, c.I, c.k1)) {
     case 1:
         return launch(k_stream<8, 3>, dim3(grid), dim3(kSThreads), stream_smem_bytes(), s,
-                      pdl, a);
+                      opts, a);
     case 2:
         return launch(k_stream<16, 4>, dim3(grid), dim3(kSThreads), stream_smem_bytes(), s,
-                      pdl, a);
+                      opts, a);
     default:
         return launch(k_stream<0, 0>, dim3(grid), dim3(kSThreads), stream_smem_bytes(), s,
-                      pdl, a);
+                      opts, a);
     }
 }
 
@@ -869,13 +896,12 @@ static int layer_impl(const void *x_bf16, const void *w_router_bf16, const float
         return launch(k_finalize, dim3((n / 4 + 255) / 256), dim3(256), 0, s, true,
                       (const float *)at<float>(ws, L.y_acc), n, y, y_dtype);
     }
-    float4 *y_acc = decode ? at<float4>(ws, L.y_acc) : nullptr;
-    if ((rc = enqueue_logits(x_bf16, w_router_bf16, bias, z, logits_out, T, d, E, s, y_acc,
-                             T * d / 4)) != MOE_OK)
-        return rc;
     if (decode)
-        return enqueue_decode(x_bf16, w_gate_bf16, w_up_bf16, w_down_bf16, d, E, I, k1, k2, y,
-                              y_dtype, topk_idx_out, topk_w_out, ws, G, s, vk, count_out);
+        return enqueue_decode(x_bf16, w_router_bf16, bias, logits_out, w_gate_bf16, w_up_bf16,
+                              w_down_bf16, d, E, I, k1, k2, y, y_dtype, topk_idx_out, topk_w_out,
+                              ws, G, s, vk, count_out);
+    if ((rc = enqueue_logits(x_bf16, w_router_bf16, bias, z, logits_out, T, d, E, s)) != MOE_OK)
+        return rc;
     if (T > 1) {
         // one CTA per token ranks its probabilities; the last one to finish
         // builds the permutation tables
@@ -1098,21 +1124,86 @@ int moe_test_expert_stream(const void *x_bf16, const void *w_gate_bf16, const vo
         a.slot_pos = at<int32_t>(ws, L.slot_pos);
         a.uniq_count = at<int32_t>(ws, L.uniq_count);
         a.uniq_list = at<int32_t>(ws, L.uniq_list);
-        a.y_acc = at<float>(ws, L.y_acc);
+            a.yacc = at<float>(ws, L.dyacc);
         a.y = y;
         a.y_dtype = y_dtype;
         a.hdr = static_cast<WsHeader *>(ws);
         const size_t smem = decode_smem_bytes(d);
         if (d == 2048)
-            return launch(k_decode<8, false>, dim3(di->num_sms), dim3(kSThreads), smem, s, false, a);
-        if (d == 4096)
-            return launch(k_decode<16, false>, dim3(di->num_sms), dim3(kSThreads), smem, s, false,
+            return launch(k_decode<8, false>, dim3(di->num_sms), dim3(kSThreads), smem, s, kCoop,
                           a);
-        return launch(k_decode<0, false>, dim3(di->num_sms), dim3(kSThreads), smem, s, false, a);
+        if (d == 4096)
+            return launch(k_decode<16, false>, dim3(di->num_sms), dim3(kSThreads), smem, s, kCoop,
+                          a);
+        return launch(k_decode<0, false>, dim3(di->num_sms), dim3(kSThreads), smem, s, kCoop, a);
     }
     return enqueue_stream(layer_stream_call(x_bf16, w_gate_bf16, w_up_bf16, w_down_bf16, T, d, E, I,
                                             k1, k2, y, y_dtype, nullptr, nullptr, ws),
                           s, false);
+}
+
+int moe_test_set_wait_limit_ns(uint64_t ns)
+{
+    if (ns == 0)
+        return MOE_ERR_INVALID_ARG;
+    const unsigned long long v = ns;
+    return cudaMemcpyToSymbol(g_moe_wait_limit_ns, &v, sizeof(v)) == cudaSuccess ? MOE_OK
+                                                                                 : MOE_ERR_CUDA;
+}
+
+}  // extern "C" (the wait kernel below is internal)
+
+namespace moe {
+// One CTA waits on something nothing will ever complete, with the library's
+// own bounded waits: which 0, a header flag (the grid barrier's release flag,
+// one generation ahead); 1, an mbarrier phase nobody arrives on; 2, the
+// one-token layer's router exchange, for a tag no CTA publishes.  Each wait
+// gives up at the wait limit and records MOE_ERR_TIMEOUT.
+__global__ void k_test_wait_never_set(WsHeader *hdr, int which)
+{
+    __shared__ uint64_t bar;
+    __shared__ float sel_p[kMaxExperts];
+    __shared__ int sel_j[kMaxExperts];
+    __shared__ unsigned cand_k[64];
+    __shared__ int cand_j[64];
+    __shared__ DecodeSmem ds;
+    int *status = &hdr->status;
+    if (which == 0) {
+        if (threadIdx.x == 0)
+            wait_flag_eq(&hdr->bar_go, ld_relaxed_u32(&hdr->bar_go) + 1u, status);
+    } else if (which == 1) {
+        if (threadIdx.x == 0) {
+            mbar_init(&bar, 1);
+            fence_mbar_init();
+            mbar_wait(&bar, 0, status);
+        }
+    } else if (threadIdx.x < 32) {
+        DecodeArgs a = {};
+        a.hdr = hdr;
+        a.E = 16;
+        a.k1 = 2;
+        a.k2 = 4;
+        // not read (the wait gives up first), but a valid global address
+        a.logits = reinterpret_cast<const float *>(hdr->bar_flag);
+        // the counter pair of the call two ahead: zero until that call runs
+        const unsigned slot = (ld_relaxed_u32(&hdr->decode_seq) + 3u) & 3u;
+        int j, kt;
+        float wv;
+        decode_route<4>(a, true, slot, threadIdx.x, &ds, status, VarK(), sel_p, sel_j, cand_k,
+                        cand_j, j, wv, kt);
+    }
+}
+}  // namespace moe
+
+extern "C" {
+
+int moe_test_wait_never_set(void *ws, size_t ws_bytes, int which, void *stream)
+{
+    if (!ws || ws_bytes < sizeof(WsHeader) || (reinterpret_cast<uintptr_t>(ws) & 255) ||
+        which < 0 || which > 2)
+        return MOE_ERR_INVALID_ARG;
+    return launch(k_test_wait_never_set, dim3(1), dim3(64), 0, static_cast<cudaStream_t>(stream),
+                  0, static_cast<WsHeader *>(ws), which);
 }
 
 int moe_test_num_sms(void)
@@ -1223,8 +1314,11 @@ extern "C" int moe_expert_ffn_noalloc(const void *x_bf16, const int32_t *expert_
     void *scratch = nullptr;
     if ((rc = noalloc_scratch(scratch)) != MOE_OK)
         return rc;
-    // the grid-barrier counters and the status word must start at zero
-    if (cudaMemsetAsync(scratch, 0, sizeof(WsHeader), s) != cudaSuccess)
+    // the grid-barrier counters and flags must start at zero; the status word
+    // (the header's first int) is kept, so problems of earlier calls stay
+    // visible until moe_noalloc_read_status reads and clears it
+    if (cudaMemsetAsync(static_cast<char *>(scratch) + sizeof(int), 0,
+                        sizeof(WsHeader) - sizeof(int), s) != cudaSuccess)
         return MOE_ERR_CUDA;
     int32_t *uniq_count = at<int32_t>(scratch, kNoAllocUOffset);
     int32_t *uniq_list = at<int32_t>(scratch, kNoAllocUOffset + 256);
@@ -1251,4 +1345,24 @@ extern "C" int moe_expert_ffn_noalloc(const void *x_bf16, const int32_t *expert_
     c.out = out;
     c.hdr = static_cast<WsHeader *>(scratch);
     return enqueue_stream(c, s);
+}
+
+extern "C" int moe_noalloc_read_status(int *status_out, void *stream)
+{
+    if (!status_out)
+        return MOE_ERR_INVALID_ARG;
+    void *scratch = nullptr;
+    int rc = noalloc_scratch(scratch);
+    if (rc != MOE_OK)
+        return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int v = 0;
+    if (cudaMemcpyAsync(&v, scratch, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (cudaMemsetAsync(scratch, 0, sizeof(int), s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    *status_out = v;
+    return MOE_OK;
 }

@@ -4,7 +4,9 @@ include/moe.h; arguments are torch tensors on the current CUDA device (or
 None where the C call takes NULL).  A non-OK status raises MoeError.
 
 There is no fallback: if libmoe.so is missing or fails to load, every call
-raises.
+raises.  With MOE_LIB_VARIANT=checks in the environment the checked build
+libmoe_checks.so is loaded instead (the same calls; kernels also verify the
+index tables they otherwise trust).
 """
 import ctypes
 import os
@@ -12,7 +14,10 @@ import os
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libmoe.so")
+LIB_VARIANT = os.environ.get("MOE_LIB_VARIANT", "")
+if LIB_VARIANT not in ("", "checks"):
+    raise RuntimeError("MOE_LIB_VARIANT must be unset or 'checks', not %r" % LIB_VARIANT)
+LIB_PATH = os.path.join(HERE, "libmoe_checks.so" if LIB_VARIANT == "checks" else "libmoe.so")
 
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = -1
@@ -61,12 +66,15 @@ SIGNATURES = {
     "moe_layer_skip": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _f, _f, _vp,
                             _i, _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp]),
     "moe_expert_ffn_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
+    "moe_noalloc_read_status": (_i, [ctypes.POINTER(_i), _vp]),
     "moe_pack_w_down": (_i, [_vp, _vp, _i, _i, _i, _vp]),
     "moe_channel_norms": (_i, [_vp, _i, _i, _i, _i, _vp, _vp]),
     "moe_layer_channel_topk": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
                                     _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_test_exp_c": (_i, [_vp, _vp, ctypes.c_int64, _vp]),
     "moe_test_num_sms": (_i, []),
+    "moe_test_set_wait_limit_ns": (_i, [ctypes.c_uint64]),
+    "moe_test_wait_never_set": (_i, [_vp, _sz, _i, _vp]),
     "moe_test_expert_stream": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _i, _vp,
                                     _sz, _vp]),
     "moe_test_expert_grouped": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
@@ -86,8 +94,8 @@ def lib():
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise RuntimeError("libmoe.so not built (%s); run python -m "
-                               "routed_expert_layer_route_b200.build" % LIB_PATH)
+            raise RuntimeError("%s not built; run python -m routed_expert_layer_route_b200.build%s"
+                               % (LIB_PATH, " --checks" if LIB_VARIANT else ""))
         L = ctypes.CDLL(LIB_PATH)
         for name, (res, args) in SIGNATURES.items():
             f = getattr(L, name)
@@ -202,6 +210,15 @@ def moe_expert_ffn_noalloc(x, expert_offsets, sorted_slot, w_gate, w_up, w_down,
                                         _stream(stream)), "moe_expert_ffn_noalloc")
 
 
+def moe_noalloc_read_status(stream=None):
+    """The device status of moe_expert_ffn_noalloc calls on the current device
+    since the last read (0 = OK); reading clears it.  Synchronises the stream."""
+    v = ctypes.c_int(0)
+    _check(lib().moe_noalloc_read_status(ctypes.byref(v), _stream(stream)),
+           "moe_noalloc_read_status")
+    return v.value
+
+
 def moe_pack_w_down(w_down, w_down_cm=None, stream=None):
     """Channel-major copy [E x I x d] of a down matrix [E x d x I] (bf16)."""
     E, d, I = w_down.shape
@@ -302,6 +319,16 @@ def moe_test_exp_c(x, y, stream=None):
 
 def moe_test_num_sms():
     return lib().moe_test_num_sms()
+
+
+def moe_test_set_wait_limit_ns(ns):
+    _check(lib().moe_test_set_wait_limit_ns(int(ns)), "moe_test_set_wait_limit_ns")
+
+
+def moe_test_wait_never_set(ws, which, stream=None):
+    wsp, wsn = _ws_args(ws)
+    _check(lib().moe_test_wait_never_set(wsp, wsn, int(which), _stream(stream)),
+           "moe_test_wait_never_set")
 
 
 def moe_test_expert_stream(x, w_gate, w_up, w_down, k1, k2, y, ws, flags=MOE_PATH_AUTO,

@@ -91,13 +91,19 @@ def check_layer_full(L, k1, k2, flags=moe.MOE_PATH_AUTO, tight=None, w_down=None
     return yy, ref
 
 
-def check_layer_sampled(L, k1, k2, tokens, flags=moe.MOE_PATH_AUTO, w_down=None, tight=None):
+def check_layer_sampled(L, k1, k2, tokens, flags=moe.MOE_PATH_AUTO, w_down=None, tight=None,
+                        by_expert=False):
     """Parity on sampled tokens; expert weights are fetched to the host only
-    for the experts those tokens use.  tight as for check_layer_full."""
+    for the experts those tokens use.  tokens: a list, or a function of the
+    GPU's routing [T x k1] returning the list.  by_expert: fetch each expert
+    once and drop it after use (oracle_layer_by_expert), for many tokens of a
+    large layer.  tight as for check_layer_full."""
     T, d = L.x.shape
     if tight is None:
         tight = not takes_grouped_path(T, d, L.w_gate.shape[1], flags)
     y, idx, w, z = run_layer(L, k1, k2, flags=flags, w_down=w_down)
+    if callable(tokens):
+        tokens = tokens(idx.cpu().numpy())
     tokens = np.asarray(tokens)
     zn = z.cpu().numpy()[tokens]
     xs = synth.to_numpy(L.x[torch.as_tensor(tokens, device=L.x.device)])
@@ -108,7 +114,10 @@ def check_layer_sampled(L, k1, k2, tokens, flags=moe.MOE_PATH_AUTO, w_down=None,
     def fetch(e):
         return (synth.to_numpy(L.w_gate[e]), synth.to_numpy(L.w_up[e]), synth.to_numpy(L.w_down[e]))
 
-    ref = oracle.layer_tokens(xs, zn, fetch, k1, k2)
+    if by_expert:
+        ref = oracle_layer_by_expert(L, tokens, zn, k1, k2)
+    else:
+        ref = oracle.layer_tokens(xs, zn, fetch, k1, k2)
     assert np.array_equal(idx.cpu().numpy()[tokens], ref["idx"])
     assert np.array_equal(w.cpu().numpy()[tokens], ref["w"])
     yy = y.cpu().numpy()[tokens]
@@ -116,3 +125,55 @@ def check_layer_sampled(L, k1, k2, tokens, flags=moe.MOE_PATH_AUTO, w_down=None,
     if tight:
         assert rel <= 1e-4, rel
     return idx.cpu().numpy()
+
+
+def oracle_layer_by_expert(L, tokens, z_rows, k1, k2):
+    """oracle.layer_tokens for many sampled tokens of a large layer, with
+    each routed expert's weights brought to the host once and dropped after
+    use (the same oracle steps: route the given float32 logits, every routed
+    slot through oracle.expert, oracle.combine in slot order)."""
+    idx, w = oracle.route_f32(z_rows, k1, k2)
+    xs = synth.to_numpy(L.x[torch.as_tensor(np.asarray(tokens), device=L.x.device)])
+    xf = (xs.astype(np.uint32) << 16).view(np.float32)
+    n, d = xf.shape
+    o = np.empty((n, k1, d), np.float32)
+    for e in np.unique(idx):
+        e = int(e)
+        wg, wu, wd = (synth.to_numpy(L.w_gate[e]), synth.to_numpy(L.w_up[e]),
+                      synth.to_numpy(L.w_down[e]))
+        for t, s in zip(*np.nonzero(idx == e)):
+            o[t, s] = oracle.expert(xf[t], wg, wu, wd)[1]
+    y = np.stack([oracle.combine(o[t], w[t]) for t in range(n)]) if n else np.empty((0, d))
+    return {"y": y, "idx": idx, "w": w}
+
+
+def tile_boundary_tokens(idx, E, n, seed, tile=256, half=128):
+    """Up to n tokens of a routed batch that exercise the grouped GEMMs' token
+    tiles: the routed tokens (in the stable expert order the permutation
+    builds) at positions 0, half-1, half, tile-1, tile, ... of every expert
+    and every token of the busiest expert's last, partial tile; the rest
+    drawn at random (seeded).  idx: [T x k1] routing of the batch."""
+    T, k1 = idx.shape
+    flat = idx.ravel()
+    order = np.argsort(flat, kind="stable")   # slots in expert order, stable by slot
+    counts = np.bincount(flat, minlength=E)
+    offs = np.concatenate([[0], np.cumsum(counts)])
+    pick = []
+    busiest = int(np.argmax(counts))
+    c = int(counts[busiest])
+    last0 = (c - 1) // tile * tile if c else 0
+    pick += [int(order[offs[busiest] + j]) // k1 for j in range(last0, c)]
+    for e in np.argsort(-counts, kind="stable"):
+        for j in range(0, int(counts[e]), half):
+            for q in (j - 1, j):
+                if 0 <= q < counts[e]:
+                    pick.append(int(order[offs[e] + q]) // k1)
+    seen, out = set(), []
+    for t in pick:
+        if t not in seen and len(out) < n:
+            seen.add(t)
+            out.append(t)
+    rng = np.random.default_rng(seed)
+    rest = np.setdiff1d(np.arange(T), np.asarray(out, np.int64))
+    extra = rng.choice(rest, size=min(len(rest), n - len(out)), replace=False)
+    return sorted(out + [int(t) for t in extra])

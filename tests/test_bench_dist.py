@@ -90,3 +90,30 @@ def test_cpu_oracle_rate_scales_to_the_whole_stack():
     r_48, n_48, _, _ = bench.cpu_oracle_rate(st, 2, 4, budget_s=0.3, stack_layers=48)
     assert n_own > 10 and n_48 > 10
     assert r_48 < r_own / 4  # 16x fewer tokens/s for a 16x deeper stack, within timing noise
+
+
+def test_reference_arm_inputs_leave_the_product_library_unloaded():
+    # the oracle arm builds its layers from the seeded generators alone
+    import subprocess
+    code = ("import sys; sys.path.insert(0, %r); import bench\n"
+            "wl = dict(bench.WORKLOADS['decode_b1']); wl.update(d=64, E=8, I=32, layers=2)\n"
+            "st = bench.OracleLayers(wl, 0, 'cpu')\n"
+            "assert st.down_hf(st.layers[0], 3).shape == (64, 32)\n"
+            "assert 'routed_expert_layer_route_b200.moe' not in sys.modules\n"
+            "print('ok')" % ROOT)
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", out.stderr
+
+
+def test_both_arms_report_the_same_config():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    class A:
+        workload, T, layers, k1, k2 = "decode_b1", 0, 0, 0, 0
+        cascade = channel_keep = skip = router_std = None
+    wl, sweep = bench.workload_of(A())
+    c = bench.line_config(A(), wl, sweep[0], 1)
+    assert c["workload"].startswith("decode_b1: 48 layers, d=2048, E=128, I=768, T=1")
+    assert (c["k1"], c["k2"]) == (4, 16)
+    assert "us_per_layer" not in c  # measured values stay out of the shared config

@@ -15,7 +15,13 @@ What is compared, and how:
     take the selection from);
   * the kept set bit for bit against the oracle's selection on the GPU's
     scores;
-  * y within the layer tolerance against the oracle's y over that kept set.
+  * y within the layer tolerance against the oracle's y over that kept set;
+  * and end to end with nothing taken from the GPU but its logits: the oracle
+    computes its own down-column norms, h, scores and kept set; that kept set
+    must equal the GPU's except for swaps between channels whose oracle
+    scores lie within SWAP_REL of the keep-th best oracle score (float32
+    rounding of h can only reorder such near-ties); with no swap, y within
+    the layer tolerance of the oracle's own y.
 """
 import numpy as np
 import pytest
@@ -28,6 +34,10 @@ from parity import assert_close_layer, logits_bound
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0")
+# relative width of the score band around the keep-th best oracle score in
+# which the two kept sets may differ: h agrees to ~1e-6 relative (float32
+# sums in another order), so scores that far apart are never reordered
+SWAP_REL = 1e-4
 
 
 @pytest.mark.parametrize("E,d,I", [(8, 256, 96), (4, 64, 16), (3, 6144, 32), (16, 2048, 768)])
@@ -90,7 +100,35 @@ def _check(L, k1, k2, keep, g, tokens=None):
         assert np.array_equal(g["scores"][t], want), "score formula"
         assert np.array_equal(g["kept"][t], oracle.channel_select(g["scores"][t], keep)), "kept set"
     assert_close_layer(g["y"][tokens], ref["y"], "channel top-k layer")
+    _check_own_selection(L, k1, k2, keep, g, tokens, xs, fetch)
     return ref
+
+
+def _check_own_selection(L, k1, k2, keep, g, tokens, xs, fetch):
+    """The oracle's own kept set (own norms, h and scores) against the GPU's."""
+    wd = {}
+
+    def own_norms(e):
+        if e not in wd:
+            wd[e] = oracle.channel_norms(synth.to_numpy(L.w_down[e]))
+        return wd[e]
+
+    own = oracle.channel_topk_tokens(xs, g["z"][tokens], fetch, own_norms, k1, k2, keep)
+    swaps = 0
+    for i, t in enumerate(tokens):
+        sc = own["scores"][i].ravel().astype(np.float64)
+        kth = np.sort(sc)[::-1][keep - 1]
+        a, b = set(own["kept"][i].tolist()), set(g["kept"][t].tolist())
+        diff = sorted(a ^ b)
+        assert len(a - b) == len(b - a)
+        for q in diff:
+            assert abs(sc[q] - kth) <= SWAP_REL * kth, \
+                "token %d channel %d: score %.9g vs keep-th %.9g" % (t, q, sc[q], kth)
+        swaps += len(a - b)
+        if not diff:
+            assert_close_layer(g["y"][t], own["y"][i], "channel top-k, oracle's own kept set")
+    print("channel top-k own selection: %d near-tie swaps over %d tokens" % (swaps, len(tokens)))
+    return swaps
 
 
 @pytest.mark.parametrize("T,d,E,I,k1,k2,keeps", [

@@ -13,7 +13,8 @@ import torch
 import oracle
 from routed_expert_layer_route_b200 import moe, synth
 
-from parity import (assert_close_layer, check_layer_full, check_layer_sampled, run_layer)
+from parity import (assert_close_layer, check_layer_full, check_layer_sampled, run_layer,
+                    tile_boundary_tokens)
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0")
@@ -189,23 +190,31 @@ def test_decode_small_batch_full_size(T, k1, k2):
 @pytest.mark.parametrize("T", [1, 64])
 @pytest.mark.parametrize("k1,k2", [(10, 10), (5, 20)])
 def test_large_full_size(T, k1, k2):
+    # every token of the batch, each routed expert's weights fetched once
     L = synth.make_layer(T, 4096, 512, 1024, seed=0, layer=0, device=DEV)
-    check_layer_sampled(L, k1, k2, [0] if T == 1 else [0, 9, 40, 63])
+    check_layer_sampled(L, k1, k2, list(range(T)), by_expert=True)
     if T == 1:
         check_layer_sampled(L, k1, k2, [0], flags=CM, w_down=moe.moe_pack_w_down(L.w_down))
 
 
 @pytest.mark.parametrize("k1,k2", [(8, 16), (4, 16)])
 def test_prefill_full_size_sampled(k1, k2):
-    # AUTO runs the tensor-core grouped GEMMs at this batch size
+    # AUTO runs the tensor-core grouped GEMMs at this batch size; 256 tokens:
+    # every token of the busiest expert's last, partial token tile, the tokens
+    # at the 128- and 256-row token-tile boundaries of the experts, the first
+    # and last token, the rest drawn at random
     L = synth.make_layer(4096, 2048, 128, 768, seed=0, layer=0, device=DEV, bias="zipf")
-    tokens = [0, 1, 777, 2048, 4000, 4095]
-    idx = check_layer_sampled(L, k1, k2, tokens)
+
+    def pick(idx):
+        return sorted(set(tile_boundary_tokens(idx, 128, 254, seed=k1)) | {0, 4095})
+
+    idx = check_layer_sampled(L, k1, k2, pick, by_expert=True)
     # Zipf bias: the most popular expert gets many more tokens than the least
     counts = np.bincount(idx.ravel(), minlength=128)
     assert counts.max() > 4 * max(1, np.median(counts))
-    # the streaming path on the same layer (float32 h: tight)
-    check_layer_sampled(L, k1, k2, tokens, flags=moe.MOE_PATH_STREAM)
+    # the streaming path on the same layer (float32 h: tight), 64 of its tokens
+    check_layer_sampled(L, k1, k2, lambda i: tile_boundary_tokens(i, 128, 64, seed=k1 + 1),
+                        flags=moe.MOE_PATH_STREAM, by_expert=True)
 
 
 # ------------------------------------------------------------------ tensor-core grouped path
