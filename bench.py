@@ -522,8 +522,11 @@ def measure_sweep(stack, sweep, args, world, stream, peaks):
     dev = stack.layers[0].x.device
     graphs = {}
     for (k1, k2) in sweep:
-        ws_list = [moe.workspace(T, d, E, I, k1, device=dev) for _ in range(Ln)]
+        # zeroed on the stream the layers run on (a side stream, which does not
+        # wait for the default one by itself)
+        ws_list = [moe.workspace(T, d, E, I, k1, device=dev, stream=stream) for _ in range(Ln)]
         ys = [torch.empty(T, d, dtype=torch.bfloat16, device=dev) for _ in range(Ln)]
+        stream.wait_stream(torch.cuda.current_stream())
         graphs[(k1, k2)] = (build_graph(stack, k1, k2, ws_list, ys, stream), ws_list, ys)
     results, head_ms, head_win = [], None, None
     for (k1, k2) in sweep:
@@ -808,6 +811,8 @@ def run_native(args, world, rank):
         extra = {}
         for name, over in EXTRA_WORKLOADS:
             key = name + "".join("_%s%d" % kv for kv in sorted(over.items()))
+            if rank == 0:
+                print("bench: workload %s" % key, file=sys.stderr, flush=True)
             extra[key] = extra_record(name, over, args, world, rank, stream, peaks)
         line["workloads"] = extra
         line["k1_ratio_by_batch"] = {

@@ -103,6 +103,26 @@ MOE_DEVINL float dot8_bf16(const uint4 w, const float *x, float acc)
     return acc;
 }
 
+// Paired float32 arithmetic (sm_100): two float32 lanes in one 64-bit
+// register, low half first.  ffma2: both halves a*b + c, each rounded once.
+MOE_DEVINL uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+// The two bf16 of a 32-bit word (element 0 in the low half) as a float32 pair.
+MOE_DEVINL uint64_t bf16x2_pair(uint32_t v)
+{
+    return ((uint64_t)(v & 0xffff0000u) << 32) | (uint64_t)(v << 16);
+}
+MOE_DEVINL uint64_t f32_pair(float lo, float hi)
+{
+    return ((uint64_t)__float_as_uint(hi) << 32) | (uint64_t)__float_as_uint(lo);
+}
+MOE_DEVINL float pair_lo(uint64_t p) { return __uint_as_float((uint32_t)p); }
+MOE_DEVINL float pair_hi(uint64_t p) { return __uint_as_float((uint32_t)(p >> 32)); }
+
 MOE_DEVINL float warp_sum(float v)
 {
 #pragma unroll
@@ -167,6 +187,25 @@ MOE_DEVINL bool mbar_wait(uint64_t *bar, uint32_t parity, int *status)
     const uint64_t t0 = global_ns();
     const uint64_t lim = wait_limit_ns();
     while (!mbar_try_wait(bar, parity)) {
+        if (global_ns() - t0 > lim) {
+            set_status(status, MOE_ERR_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+// mbar_wait that also ends (false) once the CTA's abort flag is set, so a
+// warp that waits on a slot other warps gave up on leaves promptly.
+MOE_DEVINL bool mbar_wait_live(uint64_t *bar, uint32_t parity, const int *abort, int *status)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = global_ns();
+    const uint64_t lim = wait_limit_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*(const volatile int *)abort)
+            return false;
         if (global_ns() - t0 > lim) {
             set_status(status, MOE_ERR_TIMEOUT);
             return false;

@@ -19,7 +19,7 @@
 //    writes -- with an L2 evict-last policy), writes the logits and counts
 //    them on a release counter in the workspace header (spread over lines);
 //    warp 0 of every CTA waits for all E, reads them back, forms the float32
-//    softmax, selects the top min(k2, E) in rank order from a candidate set
+//    softmax, takes the top min(k2, E) in rank order by repeated warp arg-max
 //    and applies Eq. 2 -- the fixed float32 sequence the oracle follows;
 //  * the U activated experts are laid end to end as U*I channels and CTA b
 //    owns a contiguous range of floor(U*I/G) or one more channels;
@@ -46,14 +46,15 @@
 
 namespace moe {
 
-constexpr int kDStageBytes = 48 * 1024;   // one ring stage of the decode kernel
-constexpr int kDStages = 4;
+constexpr int kDStageBytes = 36 * 1024;   // one ring slot of the decode kernel
+constexpr int kDSlots = 6;                // ring slots (stages in flight)
+constexpr int kDStages = 4;               // consumer groups (kWPS warps each)
 constexpr int kDMaxRowVec = 6;            // 16-byte row vectors per lane (d <= 4608)
 constexpr int kDMaxK1 = 32;
 constexpr int kDMaxSeg = 8;               // expert segments of one CTA's channels
 constexpr int kGroupBar0 = 2;             // named barriers 2..5: one per slot group
 
-static_assert(kSC == kDStages * kWPS, "decode kernel: one group of consumer warps per slot");
+static_assert(kSC == kDStages * kWPS, "decode kernel: the consumer warps split into groups");
 
 struct DecodeArgs {
     const uint16_t *x;    // [1 x d]
@@ -93,10 +94,10 @@ struct DSeg {
 };
 
 constexpr int kDMaxRouterRows = 8;          // router rows one CTA dots with x
-constexpr int kDRouteOff = 128 * 1024;      // ring offset of the routing scratch
+constexpr int kDRouterBytes = 128 * 1024;   // ring bytes the router rows may use
 
 struct __align__(16) DecodeSmem {
-    float hs[kDStages][kWPS];  // w*h of the stage's channels, per group
+    float hs[kDStages][2][kWPS];  // w*h of the stage's channels, per group and stage parity
     int ue[kDMaxK1];           // the activated experts, ascending
     float uw[kDMaxK1];         // their Eq. 2 weights
     int sj[kDMaxK1];           // the route by slot: expert (or MOE_EMPTY_SLOT),
@@ -167,8 +168,8 @@ __device__ void decode_segments(DecodeSmem *ds, int U, int I, int G, int b, int 
 // those it observed through a CTA barrier, come first).
 MOE_DEVINL void spread_arrive(SpreadCount *sc, unsigned i)
 {
-    fence_release_gpu();
-    atomicAdd(&sc->c[i % kSpread][0], 1u);
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&sc->c[i % kSpread][0])
+                 : "memory");
 }
 
 // One warp waits (bounded) until a spread count has seen n arrivals numbered
@@ -185,7 +186,8 @@ MOE_DEVINL bool warp_wait_spread(const SpreadCount *sc, unsigned n, int lane, in
         const uint64_t t0 = global_ns();
         const uint64_t lim = wait_limit_ns();
         while (!__all_sync(0xffffffffu, ld_relaxed_u32(p) >= want)) {
-            if (global_ns() - t0 > lim) {
+            // the whole warp gives up together (lanes read the clock apart)
+            if (__any_sync(0xffffffffu, global_ns() - t0 > lim)) {
                 if (lane == 0)
                     set_status(status, MOE_ERR_TIMEOUT);
                 ok = false;
@@ -201,18 +203,17 @@ MOE_DEVINL bool warp_wait_spread(const SpreadCount *sc, unsigned n, int lane, in
 // Warp 0 routes the token: its E logits into registers -- once the router
 // exchange counts all E published (bounded wait; every lane acquires, so each
 // lane's reads follow the logits), or directly when the logits were given --
-// the float32 softmax as keys, the Kneed best in rank order into sel_p /
-// sel_j, and Eq. 2 (lane s < k1: slot s).
+// then warp_route_vals: the float32 softmax, the top min(k2, E) by repeated
+// warp arg-max in rank order, Eq. 2 (lane s < k1: slot s).
 template <int R>
 __device__ __forceinline__ void decode_route(const DecodeArgs &a, bool fused, unsigned slot,
                                              int lane, DecodeSmem *ds, int *status, VarK vk,
-                                             float *sel_p, int *sel_j, unsigned *cand_k,
-                                             int *cand_j, int &my_j, float &my_w, int &kt)
+                                             int &my_j, float &my_w, int &kt)
 {
     const int E = a.E;
     float p[R];
     bool ok = true;
-    if (fused)  // every lane acquires, so each lane's reads below follow the logits
+    if (fused)
         ok = warp_wait_spread(&a.hdr->xcnt[slot], (unsigned)E, lane, status);
     if (!ok && lane == 0)
         ds->abort = 1;
@@ -221,11 +222,40 @@ __device__ __forceinline__ void decode_route(const DecodeArgs &a, bool fused, un
         const int j = lane + 32 * i;
         p[i] = j < E && ok ? __ldcg(&a.logits[j]) : 0.0f;
     }
-    unsigned key[R];
-    warp_softmax_keys<R>(p, E, lane, key);
-    const int Kneed = a.k2 < E ? a.k2 : a.k1;
-    warp_select_ranked<R>(key, Kneed, lane, sel_p, sel_j, cand_k, cand_j);
-    route_finish(sel_p, sel_j, E, a.k1, a.k2, lane, my_j, my_w, vk, &kt);
+    warp_route_vals<R>(p, E, a.k1, a.k2, lane, my_j, my_w, vk, &kt);
+}
+
+// One channel of the single-token register path with paired float32 FMAs:
+// g = gate_row . x, u = up_row . x with x held as float32 pairs, four partial
+// chains per dot product (pairs of 16-byte vectors alternate), then SiLU(g)*u.
+template <int VPL>
+__device__ __forceinline__ float pair_channel(const uint4 *grow, const uint4 *urow,
+                                              const uint64_t (&xp)[VPL][4], int lane)
+{
+    uint64_t g0 = 0, g1 = 0, u0 = 0, u1 = 0;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+        const uint4 wg = grow[lane + 32 * i];
+        const uint4 wu = urow[lane + 32 * i];
+        uint64_t &g = (i & 1) ? g1 : g0;
+        uint64_t &u = (i & 1) ? u1 : u0;
+        g = ffma2(bf16x2_pair(wg.x), xp[i][0], g);
+        u = ffma2(bf16x2_pair(wu.x), xp[i][0], u);
+        g = ffma2(bf16x2_pair(wg.y), xp[i][1], g);
+        u = ffma2(bf16x2_pair(wu.y), xp[i][1], u);
+        g = ffma2(bf16x2_pair(wg.z), xp[i][2], g);
+        u = ffma2(bf16x2_pair(wu.z), xp[i][2], u);
+        g = ffma2(bf16x2_pair(wg.w), xp[i][3], g);
+        u = ffma2(bf16x2_pair(wu.w), xp[i][3], u);
+    }
+    float g = (pair_lo(g0) + pair_hi(g0)) + (pair_lo(g1) + pair_hi(g1));
+    float u = (pair_lo(u0) + pair_hi(u0)) + (pair_lo(u1) + pair_hi(u1));
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        g += __shfl_xor_sync(0xffffffffu, g, o);
+        u += __shfl_xor_sync(0xffffffffu, u, o);
+    }
+    return silu_mul(g, u);
 }
 
 // VPL: d = 256*VPL for the single-token register path (x in registers when
@@ -236,17 +266,11 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t *ring = smem;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kDStages * kDStageBytes);
-    uint64_t *empty = full + kDStages;
-    uint64_t *rbar = empty + kDStages;  // the router rows' bulk copies (2 slots: alignment)
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kDSlots * kDStageBytes);
+    uint64_t *empty = full + kDSlots;
+    uint64_t *rbar = empty + kDSlots;  // the router rows' bulk copies (2 slots: alignment)
     DecodeSmem *ds = reinterpret_cast<DecodeSmem *>(rbar + 2);
     uint8_t *area = reinterpret_cast<uint8_t *>(ds + 1);  // the token's x row, d bf16
-    // routing scratch in the ring, which is idle until the route is known
-    // (the router rows occupy its first kDMaxRouterRows * d * 2 <= kDRouteOff bytes)
-    float *sel_p = reinterpret_cast<float *>(ring + kDRouteOff);  // [Kneed] in rank order
-    int *sel_j = reinterpret_cast<int *>(sel_p + kMaxExperts);
-    unsigned *cand_k = reinterpret_cast<unsigned *>(sel_j + kMaxExperts);  // [64] candidates
-    int *cand_j = reinterpret_cast<int *>(cand_k + 64);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = gridDim.x, b = blockIdx.x;
@@ -257,7 +281,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
     const int nvec = d >> 3;                                   // 16-byte vectors per row
 
     if (tid == 0) {
-        for (int s = 0; s < kDStages; ++s) {
+        for (int s = 0; s < kDSlots; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kWPS);
         }
@@ -347,17 +371,13 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
             float wv;
             const VarK vk = CASCADE ? a.vk : VarK();
             if (E <= 128)
-                decode_route<4>(a, fused, slot, lane, ds, status, vk, sel_p, sel_j, cand_k,
-                                cand_j, j, wv, kt);
+                decode_route<4>(a, fused, slot, lane, ds, status, vk, j, wv, kt);
             else if (E <= 256)
-                decode_route<8>(a, fused, slot, lane, ds, status, vk, sel_p, sel_j, cand_k,
-                                cand_j, j, wv, kt);
+                decode_route<8>(a, fused, slot, lane, ds, status, vk, j, wv, kt);
             else if (E <= 512)
-                decode_route<16>(a, fused, slot, lane, ds, status, vk, sel_p, sel_j, cand_k,
-                                 cand_j, j, wv, kt);
+                decode_route<16>(a, fused, slot, lane, ds, status, vk, j, wv, kt);
             else
-                decode_route<32>(a, fused, slot, lane, ds, status, vk, sel_p, sel_j, cand_k,
-                                 cand_j, j, wv, kt);
+                decode_route<32>(a, fused, slot, lane, ds, status, vk, j, wv, kt);
             if (MOE_CHECKS) {  // the route: experts in range, kt slots taken
                 const bool bad = (lane < k1 && j != MOE_EMPTY_SLOT && (j < 0 || j >= E)) ||
                                  kt < 0 || kt > k1;
@@ -411,7 +431,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
             while (it.valid()) {
                 if (*(volatile int *)&ds->abort)
                     break;
-                if (!mbar_wait(&empty[slot_r], ph ^ 1u, status)) {
+                if (!mbar_wait_live(&empty[slot_r], ph ^ 1u, &ds->abort, status)) {
                     ds->abort = 1;
                     break;
                 }
@@ -426,7 +446,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
                 bulk_g2s(dst + 2 * bytes, a.wdt + row0 * d, bytes, &full[slot_r], pol);
                 ++issued;
                 it.next();
-                if (++slot_r == kDStages) {
+                if (++slot_r == kDSlots) {
                     slot_r = 0;
                     ph ^= 1u;
                 }
@@ -448,13 +468,27 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
             for (int k = 0; k < 8; ++k)
                 yp[j][k] = 0.0f;
 
-        uint4 xv[VPL > 0 && VPL <= kXRegMax ? VPL : 1];
+        // x: float32 pairs in registers (register path), else read from shared memory
+        constexpr bool kPairs = VPL > 0 && VPL <= kXRegMax;
+        uint64_t xp[kPairs ? VPL : 1][4];
+        uint64_t yq[kPairs ? RV : 1][4];  // the row partials as pairs (register path)
         const uint4 *xs = reinterpret_cast<const uint4 *>(area);
-        if constexpr (VPL > 0 && VPL <= kXRegMax) {
+        if constexpr (kPairs) {
 #pragma unroll
-            for (int i = 0; i < VPL; ++i)
-                xv[i] = xs[lane + 32 * i];
+            for (int i = 0; i < VPL; ++i) {
+                const uint4 v = xs[lane + 32 * i];
+                xp[i][0] = bf16x2_pair(v.x);
+                xp[i][1] = bf16x2_pair(v.y);
+                xp[i][2] = bf16x2_pair(v.z);
+                xp[i][3] = bf16x2_pair(v.w);
+            }
+#pragma unroll
+            for (int j = 0; j < RV; ++j)
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    yq[j][q] = 0;
         }
+        uint4 xv[1];  // unused by the pair path
 
         DIter it;
         it.init(ds->seg, nseg, nch);
@@ -462,12 +496,28 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
         while (it.valid()) {
             const int n = it.count();
             if (sidx % kDStages == group) {
-                const uint32_t parity = (uint32_t)((sidx / kDStages) & 1);
-                const bool ok =
-                    !*(volatile int *)&ds->abort && mbar_wait(&full[group], parity, status);
-                if (!ok)
+                // stage sidx: group sidx % kDStages, slot sidx % kDSlots, the
+                // slot's use number rnd.  A slot's stages alternate between two
+                // groups, so a group comes back to a slot two phases of its
+                // full barrier later, which parity alone cannot tell from the
+                // phase before: it first waits until the other group has
+                // consumed the slot's previous stage (that stage's full phase
+                // done), then on this stage's full phase.  A warp hands a slot
+                // back only after a successful wait, so the producer refills a
+                // slot only once its previous copies have landed.
+                const int slot = sidx % kDSlots;
+                const int rnd = sidx / kDSlots;
+                const int hb = (sidx / kDStages) & 1;  // the group's h buffer
+                bool ok = !*(volatile int *)&ds->abort;
+                if (ok && rnd > 0)
+                    ok = mbar_wait_live(&empty[slot], (uint32_t)((rnd - 1) & 1), &ds->abort,
+                                        status);
+                if (ok)
+                    ok = mbar_wait_live(&full[slot], (uint32_t)(rnd & 1), &ds->abort, status);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok && lane == 0)
                     ds->abort = 1;
-                const uint8_t *stg = ring + (size_t)group * kDStageBytes;
+                const uint8_t *stg = ring + (size_t)slot * kDStageBytes;
                 const size_t rb = (size_t)n * d * 2;  // bytes of one of the three row blocks
                 const float wgt = ds->uw[ds->seg[it.s].u];
                 // (1) w * h for channel gl of the stage
@@ -475,7 +525,9 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
                     const uint4 *grow = reinterpret_cast<const uint4 *>(stg + (size_t)gl * d * 2);
                     const uint4 *urow = reinterpret_cast<const uint4 *>(stg + rb + (size_t)gl * d * 2);
                     float hval;
-                    if constexpr (VPL > 0) {
+                    if constexpr (kPairs) {
+                        hval = pair_channel<VPL>(grow, urow, xp, lane);
+                    } else if constexpr (VPL > 0) {
                         hval = fast_channel<VPL>(grow, urow, xv, xs, lane);
                     } else {
                         float r0[kTokChunk], r1[kTokChunk];
@@ -487,14 +539,32 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
                         hval = silu_mul(r0[0], r1[0]);
                     }
                     if (lane == 0)
-                        ds->hs[group][gl] = hval * wgt;
+                        ds->hs[group][hb][gl] = hval * wgt;
                 }
                 named_bar_sync(kGroupBar0 + group, kWPS * 32);  // the group's h are in shared memory
                 // (2) y partial += w*h * down row, for this warp's rows
-                if (ok) {
+                if (ok && kPairs) {
                     const uint8_t *drows = stg + 2 * rb;
                     for (int i = 0; i < n; ++i) {
-                        const float hv = ds->hs[group][i];
+                        const float hv = ds->hs[group][hb][i];
+                        const uint64_t h2 = f32_pair(hv, hv);
+                        const uint4 *drow = reinterpret_cast<const uint4 *>(drows + (size_t)i * d * 2);
+#pragma unroll
+                        for (int j = 0; j < (kPairs ? RV : 1); ++j) {
+                            const int v = gl * 32 + lane + kWPS * 32 * j;
+                            if (v < nvec) {
+                                const uint4 w = drow[v];
+                                yq[j][0] = ffma2(bf16x2_pair(w.x), h2, yq[j][0]);
+                                yq[j][1] = ffma2(bf16x2_pair(w.y), h2, yq[j][1]);
+                                yq[j][2] = ffma2(bf16x2_pair(w.z), h2, yq[j][2]);
+                                yq[j][3] = ffma2(bf16x2_pair(w.w), h2, yq[j][3]);
+                            }
+                        }
+                    }
+                } else if (ok) {
+                    const uint8_t *drows = stg + 2 * rb;
+                    for (int i = 0; i < n; ++i) {
+                        const float hv = ds->hs[group][hb][i];
                         const uint4 *drow = reinterpret_cast<const uint4 *>(drows + (size_t)i * d * 2);
 #pragma unroll
                         for (int j = 0; j < RV; ++j) {
@@ -509,16 +579,27 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
                         }
                     }
                 }
-                // hand the slot back (hs[group] is next written after this
-                // group's next stage wait, which needs these arrivals)
+                // hand the slot back; hs[group] alternates by stage parity, and a
+                // warp reaches the group's stage after next only past the next
+                // stage's group barrier, which every warp of the group passes
+                // after it has read this stage's values
                 __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&empty[group]);
+                if (ok && lane == 0)
+                    mbar_arrive(&empty[slot]);
             }
             ++sidx;
             it.next();
         }
 
+        if constexpr (kPairs) {
+#pragma unroll
+            for (int j = 0; j < RV; ++j)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    yp[j][2 * q] = pair_lo(yq[j][q]);
+                    yp[j][2 * q + 1] = pair_hi(yq[j][q]);
+                }
+        }
         // ------------------------------------------------------------ this CTA's partial row
         consumer_sync();  // every warp is past its last stage: the ring is free
         float *red = reinterpret_cast<float *>(ring);  // [kDStages][d]
@@ -554,9 +635,9 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
     __syncthreads();
     if (tid == 0 && ds->abort) {
         const int issued = ds->issued;
-        for (int s = 0; s < kDStages && s < issued; ++s) {
-            const int last = issued - 1 - ((issued - 1 - s) % kDStages);
-            const uint32_t parity = (uint32_t)((last / kDStages) & 1);
+        for (int s = 0; s < kDSlots && s < issued; ++s) {
+            const int last = issued - 1 - ((issued - 1 - s) % kDSlots);
+            const uint32_t parity = (uint32_t)((last / kDSlots) & 1);
             mbar_wait(&full[s], parity, status);
         }
     }
@@ -565,8 +646,13 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
 
     // ------------------------------------------------------------ y (last CTA to check in)
     if (tid == 0) {
-        fence_acq_rel_gpu();  // this CTA's reductions before its ticket; others' after
-        const unsigned prev = atomicAdd(&a.hdr->decode_arrive, 1u);
+        // release: this CTA's reductions before its ticket; acquire: the
+        // reductions of every CTA that took a ticket before, for the last one
+        unsigned prev;
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                     : "=r"(prev)
+                     : "l"(&a.hdr->decode_arrive)
+                     : "memory");
         ds->last = prev == (unsigned)G - 1;
     }
     consumer_sync();
@@ -624,21 +710,21 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
 
 inline size_t decode_smem_bytes(int d)
 {
-    return (size_t)kDStages * kDStageBytes + (2 * kDStages + 2) * sizeof(uint64_t) +
+    return (size_t)kDSlots * kDStageBytes + (2 * kDSlots + 2) * sizeof(uint64_t) +
            sizeof(DecodeSmem) + (size_t)d * 2;
 }
 
 // The single-pass path serves one token per call (T == 1) whose output rows
 // fit the register partials, with the down matrix channel-major; each CTA's
-// router rows fit the ring below the routing scratch.
+// router rows fit the ring.
 inline bool decode_fits(int T, int d, int E, int I, int k1, int G)
 {
     if (T != 1 || k1 > kDMaxK1 || (d >> 3) > kWPS * 32 * kDMaxRowVec || E > kMaxExperts)
         return false;
-    if (decode_smem_bytes(d) > 227 * 1024 || (size_t)kDStages * d * 4 > (size_t)kDStages * kDStageBytes)
+    if (decode_smem_bytes(d) > 227 * 1024 || (size_t)kDStages * d * 4 > (size_t)kDSlots * kDStageBytes)
         return false;
     const int rows = (E + G - 1) / G;
-    if (rows > kDMaxRouterRows || (size_t)rows * d * 2 > (size_t)kDRouteOff)
+    if (rows > kDMaxRouterRows || (size_t)rows * d * 2 > (size_t)kDRouterBytes)
         return false;
     const long chmax = ((long)k1 * I + G - 1) / G;
     const long nseg = (chmax + I - 1) / I + 1;

@@ -1162,10 +1162,6 @@ namespace moe {
 __global__ void k_test_wait_never_set(WsHeader *hdr, int which)
 {
     __shared__ uint64_t bar;
-    __shared__ float sel_p[kMaxExperts];
-    __shared__ int sel_j[kMaxExperts];
-    __shared__ unsigned cand_k[64];
-    __shared__ int cand_j[64];
     __shared__ DecodeSmem ds;
     int *status = &hdr->status;
     if (which == 0) {
@@ -1189,8 +1185,7 @@ __global__ void k_test_wait_never_set(WsHeader *hdr, int which)
         const unsigned slot = (ld_relaxed_u32(&hdr->decode_seq) + 3u) & 3u;
         int j, kt;
         float wv;
-        decode_route<4>(a, true, slot, threadIdx.x, &ds, status, VarK(), sel_p, sel_j, cand_k,
-                        cand_j, j, wv, kt);
+        decode_route<4>(a, true, slot, threadIdx.x, &ds, status, VarK(), j, wv, kt);
     }
 }
 }  // namespace moe

@@ -526,164 +526,6 @@ __device__ __forceinline__ void warp_route(const float *z, int E, int k1, int k2
     warp_route_vals<R>(p, E, k1, k2, lane, my_j, my_w, vk, kt_out);
 }
 
-// ---------------------------------------------------------------------------
-// The same routing for one token in one warp, with the ranking done on a
-// candidate set (the layer kernel's router):
-//  * warp_softmax_keys: m, e_j = expc(z_j - m), the canonical 32-partial
-//    normaliser Z, p_j = e_j / Z -- the float sequence of warp_route_vals --
-//    left as keys (bits of p_j + 1, 0 = no expert) in the lane's registers;
-//  * warp_select_ranked: the Kneed (<= 32) largest keys in rank order
-//    (p descending, expert index ascending) into sel_p / sel_j (shared
-//    memory).  The Kneed-th largest of the 32 lane maxima is a lower bound
-//    for the Kneed-th largest key, so only keys at or above it can be
-//    selected; those candidates (typically a few more than Kneed) are ranked
-//    among themselves.  With more than 64 candidates (many equal keys) the
-//    repeated warp arg-max of warp_route_vals ranks instead.  Either way the
-//    selection is the one the oracle's ordering defines;
-//  * route_finish: Eq. 2 on sel_p / sel_j (below).
-template <int R>
-__device__ __forceinline__ void warp_softmax_keys(float (&p)[R], int E, int lane, unsigned (&key)[R])
-{
-    const float kNegInf = -__int_as_float(0x7f800000);
-    float m = kNegInf;
-#pragma unroll
-    for (int i = 0; i < R; ++i)
-        if (lane + 32 * i < E)
-            m = fmaxf(m, p[i]);
-    asm volatile("redux.sync.max.f32 %0, %0, 0xffffffff;" : "+f"(m));
-    float Z = 0.0f;
-#pragma unroll
-    for (int i = 0; i < R; ++i)
-        if (lane + 32 * i < E) {
-            p[i] = expc(__fsub_rn(p[i], m));
-            Z = __fadd_rn(Z, p[i]);
-        }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1)
-        Z = __fadd_rn(Z, __shfl_xor_sync(0xffffffffu, Z, o));
-#pragma unroll
-    for (int i = 0; i < R; ++i)
-        key[i] = lane + 32 * i < E ? __float_as_uint(__fdiv_rn(p[i], Z)) + 1u : 0u;
-}
-
-// cand: shared scratch of 64 (key, index) pairs.  Kneed <= E; the candidate
-// path serves Kneed <= 32, the arg-max any Kneed.
-template <int R>
-__device__ __forceinline__ void warp_select_ranked(unsigned (&key)[R], int Kneed, int lane,
-                                                   float *sel_p, int *sel_j, unsigned *cand_k,
-                                                   int *cand_j)
-{
-    constexpr unsigned kFull = 0xffffffffu;
-    int nc = 65;  // candidates; more than 64 (or Kneed > 32): the arg-max below
-    if (Kneed <= 32) {
-        unsigned km = 0u;
-#pragma unroll
-        for (int i = 0; i < R; ++i)
-            km = max(km, key[i]);
-        // rank of this lane's maximum among the 32 (ties: lower lane first)
-        int rl = 0;
-#pragma unroll
-        for (int q = 0; q < 32; ++q) {
-            const unsigned v = __shfl_sync(kFull, km, q);
-            rl += (v > km) | ((v == km) & (q < lane));
-        }
-        const unsigned lead = __ballot_sync(kFull, rl == Kneed - 1);  // exactly one lane
-        const unsigned theta = __shfl_sync(kFull, km, __ffs(lead) - 1);
-        // candidates: keys >= theta, compacted in (i, lane) order
-        const unsigned below = (1u << lane) - 1u;
-        nc = 0;
-#pragma unroll
-        for (int i = 0; i < R; ++i) {
-            const bool c = key[i] != 0u && key[i] >= theta;
-            const unsigned bal = __ballot_sync(kFull, c);
-            const int pos = nc + __popc(bal & below);
-            if (c && pos < 64) {
-                cand_k[pos] = key[i];
-                cand_j[pos] = lane + 32 * i;
-            }
-            nc += __popc(bal);
-        }
-        __syncwarp();
-    }
-    if (nc <= 64) {
-        for (int c = lane; c < nc; c += 32) {
-            const unsigned k = cand_k[c];
-            const int j = cand_j[c];
-            int r = 0;
-            for (int q = 0; q < nc; ++q) {
-                const unsigned kq = cand_k[q];
-                r += (kq > k) | ((kq == k) & (cand_j[q] < j));
-            }
-            if (r < Kneed) {
-                sel_p[r] = __uint_as_float(k - 1u);
-                sel_j[r] = j;
-            }
-        }
-    } else {
-        // many equal keys: repeated arg-max, largest key then lowest index
-        for (int r = 0; r < Kneed; ++r) {
-            unsigned kl = 0u;
-            int jl = 0x7fffffff;
-#pragma unroll
-            for (int i = 0; i < R; ++i)
-                if (key[i] > kl) {
-                    kl = key[i];
-                    jl = lane + 32 * i;
-                }
-            const unsigned kmax = __reduce_max_sync(kFull, kl);
-            const int bj = (int)__reduce_min_sync(kFull, kl == kmax ? (unsigned)jl : 0xffffffffu);
-            if (lane == 0) {
-                sel_p[r] = __uint_as_float(kmax - 1u);
-                sel_j[r] = bj;
-            }
-#pragma unroll
-            for (int i = 0; i < R; ++i)
-                if (lane + 32 * i == bj)
-                    key[i] = 0u;
-        }
-    }
-    __syncwarp();
-}
-
-// Lane s < k1 gets the rank-s expert and its weight (MOE_EMPTY_SLOT / 0 for
-// a slot the variable-k route leaves out); kt = the slots taken.
-__device__ __forceinline__ void route_finish(const float *sel_p, const int *sel_j, int E, int k1,
-                                             int k2, int lane, int &my_j, float &my_w, VarK vk,
-                                             int *kt_out)
-{
-    const bool cascade = vk.kind == kVarCascade;
-    const int K = k2 < E ? k2 : E;
-    const bool renorm = k2 < E;
-    const int Kneed = renorm ? K : k1;
-    float S = 0.0f;
-    int kt = k1;
-    bool covered = false;
-#pragma unroll 8
-    for (int r = 0; r < Kneed; ++r) {
-        S = __fadd_rn(S, sel_p[r]);  // mass of the first r+1 ranks
-        if (cascade && !covered && r < k1 && S >= vk.tau) {
-            covered = true;
-            kt = r + 1;
-        }
-    }
-    const float my_p = lane < Kneed ? sel_p[lane] : 0.0f;
-    my_j = lane < Kneed ? sel_j[lane] : 0;
-    my_w = renorm ? __fdiv_rn(my_p, S) : my_p;
-    if (lane >= kt && lane < k1) {
-        my_j = MOE_EMPTY_SLOT;
-        my_w = 0.0f;
-    }
-    if (vk.kind == kVarSkip) {
-        if (lane >= 1 && lane < k1 && __ldg(&vk.tab[my_j]) < vk.th_e && my_w < vk.th_w) {
-            my_j = MOE_EMPTY_SLOT;
-            my_w = 0.0f;
-        }
-        kt = __popc(__ballot_sync(0xffffffffu, lane < k1 && my_j != MOE_EMPTY_SLOT));
-    }
-    if (kt_out)
-        *kt_out = kt;
-}
-
 template <int R>
 __global__ void __launch_bounds__(256) k_route_warp(const float *logits, int T, int E, int k1,
                                                     int k2, int32_t *idx, float *w,

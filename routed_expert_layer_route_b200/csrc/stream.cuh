@@ -494,7 +494,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_stream(StreamArgs a)
             while (it.valid()) {
                 if (*(volatile int *)&ss->abort)
                     break;
-                if (!mbar_wait(&empty[slot], ph ^ 1u, status)) {
+                if (!mbar_wait_live(&empty[slot], ph ^ 1u, &ss->abort, status)) {
                     ss->abort = 1;
                     break;
                 }
@@ -532,15 +532,20 @@ __global__ void __launch_bounds__(kSThreads, 1) k_stream(StreamArgs a)
 
         // Wait for stage sidx if this warp serves its slot; returns the stage
         // buffer, or nullptr when this warp skips the stage (not its slot) or
-        // the launch aborted.  Every served stage is handed back with release().
+        // the launch aborted.  Every stage acquired is handed back with
+        // release(); one not acquired is not, so the producer refills a slot
+        // only once its copies have landed.
         auto acquire = [&](bool &mine) -> const uint8_t * {
             mine = (sidx % kStages) == group;
             if (!mine)
                 return nullptr;
             const uint32_t parity = (uint32_t)((sidx / kStages) & 1);
-            const bool ok = !*(volatile int *)&ss->abort && mbar_wait(&full[group], parity, status);
+            bool ok = !*(volatile int *)&ss->abort &&
+                      mbar_wait_live(&full[group], parity, &ss->abort, status);
+            ok = __all_sync(0xffffffffu, ok);
             if (!ok) {
-                ss->abort = 1;
+                if (lane == 0)
+                    ss->abort = 1;
                 return nullptr;
             }
             return ring + (size_t)group * kStageBytes;
@@ -616,7 +621,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_stream(StreamArgs a)
                         }
                     }
                 }
-                if (mine)
+                if (stg)
                     release();
                 ++sidx;
                 it.next();
@@ -726,7 +731,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_stream(StreamArgs a)
                         }
                     }
                 }
-                if (mine)
+                if (stg)
                     release();
                 ++sidx;
                 it.next();

@@ -150,13 +150,15 @@ def moe_read_device_status(ws, stream=None):
     return v.value
 
 
-def workspace(T, d, E, I, k1, device=None):
-    """Allocate (torch) and initialise a workspace for these shapes."""
+def workspace(T, d, E, I, k1, device=None, stream=None):
+    """Allocate (torch) and initialise a workspace for these shapes.  The
+    zeroing is enqueued on `stream` (default: the current stream): give the
+    stream the layer calls will run on, or order the two streams yourself."""
     n = moe_workspace_size(T, d, E, I, k1)
     if n == 0:
         raise MoeError(MOE_ERR_UNSUPPORTED_SHAPE, "moe_workspace_size")
     ws = torch.empty(n, dtype=torch.uint8, device=device or torch.device("cuda"))
-    moe_workspace_init(ws)
+    moe_workspace_init(ws, stream)
     return ws
 
 
