@@ -72,6 +72,25 @@ def test_decode_path_single_token(d, E, I, k1, k2):
     check_layer_full(L, k1, k2, flags=CM, w_down=wdc)
 
 
+@pytest.mark.parametrize("E,k1,k2,group", [(128, 8, 16, 2), (128, 4, 128, 4), (128, 32, 127, 128),
+                                           (64, 6, 20, 3), (16, 4, 8, 16), (100, 5, 9, 7),
+                                           (512, 10, 20, 4)])
+def test_decode_route_ties(E, k1, k2, group):
+    """Equal logits on the one-token path: router rows repeated in runs of
+    `group` give bit-equal logits, so the rank order must fall back to the
+    lower expert index (the tie rule of the page's router, restated in the
+    oracle).  group = E: every logit equal, p = 1/E."""
+    d, I = 256, 32
+    L = synth.make_layer(1, d, E, I, seed=E + k1 + group, device=DEV)
+    L.w_router = L.w_router[torch.arange(E, device=DEV) // group * group].contiguous()
+    wdc = moe.moe_pack_w_down(L.w_down)
+    _, idx, _, z = run_layer(L, k1, k2, flags=CM, w_down=wdc)
+    zn = z.cpu().numpy()[0]
+    for g0 in range(0, E, group):  # the repeated rows give bit-equal logits
+        assert np.all(zn[g0:g0 + group] == zn[g0])
+    check_layer_full(L, k1, k2, flags=CM, w_down=wdc)
+
+
 def test_channel_major_down_needs_one_token():
     L = synth.make_layer(2, 256, 16, 32, seed=7, device=DEV)
     wdc = moe.moe_pack_w_down(L.w_down)
