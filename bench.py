@@ -612,10 +612,13 @@ def roofline_record(stack, workload, head, res, graphs, stream, peaks, variant):
             return "hbm", gb, hbm_peak, "GB/s", gb / hbm_peak
 
         bd1, a1, p1, u1, fr1 = bound(f1, b1, g1_ms)
+        # the gate/up GEMM runs on CTA pairs when I is a multiple of 256
+        from routed_expert_layer_route_b200 import moe
+        g1_name = "k_gemm1_pair" if I % 256 == 0 and moe.moe_test_gemm1_pairs() > 0 else "k_gemm1"
         bd2, a2, p2, u2, fr2 = bound(f2, b2, g2_ms)
         return {"bound": bd1, "achieved": round(a1, 1), "peak": p1, "unit": u1,
-                "frac": round(fr1, 4), "traffic": recorded_traffic(workload, k1, "k_gemm1"),
-                "kernel": "moe::k_gemm1", "kernel_us": round(g1_ms * 1000, 2),
+                "frac": round(fr1, 4), "traffic": recorded_traffic(workload, k1, g1_name),
+                "kernel": "moe::" + g1_name, "kernel_us": round(g1_ms * 1000, 2),
                 "algorithmic_flops_per_launch": f1, "algorithmic_bytes_per_launch": int(b1),
                 "tensor_frac": round(f1 / (g1_ms * 1e-3) / 1e12 / bf16_peak, 4),
                 "hbm_frac": round(b1 / (g1_ms * 1e-3) / 1e9 / hbm_peak, 4),

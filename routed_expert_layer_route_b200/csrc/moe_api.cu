@@ -14,6 +14,7 @@
 #include "combine.cuh"
 #include "ctopk.cuh"
 #include "decode.cuh"
+#include "gemm_pair.cuh"
 #include "grouped.cuh"
 #include "route.cuh"
 #include "stream.cuh"
@@ -96,7 +97,12 @@ static int check_route(int E, int k1, int k2)
 struct DevInfo {
     bool ready = false;
     int num_sms = 0;
+    int gemm1_pairs = 0;  // CTA pairs of k_gemm1_pair resident at once (0: not launchable)
 };
+
+// Which gate/up GEMM kernel the grouped path uses (test hook): 0 the pair
+// kernel where the shapes allow it, 1 always the single-CTA kernel.
+static int g_gemm1_single = 0;
 static DevInfo g_dev[64];
 static std::mutex g_dev_mu;
 
@@ -130,8 +136,30 @@ static int device_info(DevInfo *&out)
         if (cudaFuncSetAttribute(k_gemm1, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gemm1_smem_bytes()) != cudaSuccess ||
             cudaFuncSetAttribute(k_gemm2, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)gemm2_smem_bytes()) != cudaSuccess)
+                                 (int)gemm2_smem_bytes()) != cudaSuccess ||
+            cudaFuncSetAttribute(k_gemm1_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gemm1_pair_smem_bytes()) != cudaSuccess)
             return MOE_ERR_CUDA;
+        {
+            // how many CTA pairs of the pair kernel the device holds at once
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(2 * (di.num_sms / 2));
+            cfg.blockDim = dim3(kGPThreads);
+            cfg.dynamicSmemBytes = gemm1_pair_smem_bytes();
+            cudaLaunchAttribute at;
+            at.id = cudaLaunchAttributeClusterDimension;
+            at.val.clusterDim.x = 2;
+            at.val.clusterDim.y = 1;
+            at.val.clusterDim.z = 1;
+            cfg.attrs = &at;
+            cfg.numAttrs = 1;
+            int nc = 0;
+            if (cudaOccupancyMaxActiveClusters(&nc, k_gemm1_pair, &cfg) != cudaSuccess) {
+                cudaGetLastError();
+                nc = 0;
+            }
+            di.gemm1_pairs = nc < di.num_sms / 2 ? nc : di.num_sms / 2;
+        }
         // scores of kCtkMaxN channels + at most 16 KiB of side-by-side row partials
         if (cudaFuncSetAttribute(k_ctk_down, dsm, kCtkMaxN * 4 + 16 * 1024) != cudaSuccess)
             return MOE_ERR_CUDA;
@@ -154,8 +182,9 @@ static int device_info(DevInfo *&out)
 // programmatic dependent launch (the kernel calls griddepcontrol.wait before
 // it reads anything an earlier kernel wrote); kCoop makes it a cooperative
 // launch, which the runtime places only when every CTA of the grid can be
-// resident at once (kernels whose CTAs wait on one another need that).
-constexpr int kPdl = 1, kCoop = 2;
+// resident at once (kernels whose CTAs wait on one another need that);
+// kPair launches clusters of two CTAs (the pair kernels).
+constexpr int kPdl = 1, kCoop = 2, kPair = 4;
 
 template <typename... KArgs, typename... Args>
 static int launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
@@ -166,7 +195,7 @@ static int launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cu
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[2];
+    cudaLaunchAttribute attr[3];
     int n = 0;
     if (opts & kPdl) {
         attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -176,6 +205,13 @@ static int launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cu
     if (opts & kCoop) {
         attr[n].id = cudaLaunchAttributeCooperative;
         attr[n].val.cooperative = 1;
+        ++n;
+    }
+    if (opts & kPair) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = 2;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
         ++n;
     }
     cfg.attrs = n ? attr : nullptr;
@@ -353,9 +389,20 @@ static int enqueue_grouped(const void *x, const void *wg, const void *wu, const 
     a1.I = I;
     a1.k1 = k1;
     a1.hdr = hdr;
-    if ((which & 1) && (rc = launch(k_gemm1, dim3(G), dim3(kG1Threads), gemm1_smem_bytes(), s,
-                                    pdl, tg, tu, tx, a1)) != MOE_OK)
-        return rc;
+    if (which & 1) {
+        // the pair kernel when the weight rows come in whole 256-row tiles
+        DevInfo *di;
+        if ((rc = device_info(di)) != MOE_OK)
+            return rc;
+        if (I % kGPRows == 0 && di->gemm1_pairs > 0 && !g_gemm1_single)
+            rc = launch(k_gemm1_pair, dim3(2 * di->gemm1_pairs), dim3(kGPThreads),
+                        gemm1_pair_smem_bytes(), s, (pdl ? kPdl : 0) | kPair, tg, tu, tx, a1);
+        else
+            rc = launch(k_gemm1, dim3(G), dim3(kG1Threads), gemm1_smem_bytes(), s, pdl, tg, tu,
+                        tx, a1);
+        if (rc != MOE_OK)
+            return rc;
+    }
     if (!(which & 2))
         return MOE_OK;
     Gemm2Args a2 = {};
@@ -1199,6 +1246,22 @@ int moe_test_wait_never_set(void *ws, size_t ws_bytes, int which, void *stream)
         return MOE_ERR_INVALID_ARG;
     return launch(k_test_wait_never_set, dim3(1), dim3(64), 0, static_cast<cudaStream_t>(stream),
                   0, static_cast<WsHeader *>(ws), which);
+}
+
+int moe_test_set_gemm1_single(int single)
+{
+    if (single != 0 && single != 1)
+        return MOE_ERR_INVALID_ARG;
+    g_gemm1_single = single;
+    return MOE_OK;
+}
+
+int moe_test_gemm1_pairs(void)
+{
+    DevInfo *di;
+    if (device_info(di) != MOE_OK)
+        return -1;
+    return di->gemm1_pairs;
 }
 
 int moe_test_num_sms(void)

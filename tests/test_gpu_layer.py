@@ -249,17 +249,37 @@ GSMALL = [
     (130, 128, 2, 256, 2, 2, None),      # k1 = E: every token in every expert
     (256, 256, 128, 128, 4, 16, "normal"),  # router logits on the tensor cores too
     (300, 128, 256, 128, 6, 6, None),    # two 128-expert logit tiles, ragged token tile
+    # I a multiple of 256: the gate/up GEMM runs on CTA pairs (256-row tiles)
+    (600, 256, 4, 512, 2, 4, None),      # 300 slots per expert: a full and a ragged token tile
+    (77, 256, 16, 768, 5, 9, "zipf"),    # three 256-row tiles, tiles of a few tokens
+    (9, 128, 8, 256, 1, 2, None),        # token tiles of one to a few tokens (N = 16)
+    (520, 384, 2, 256, 1, 2, "normal"),  # k1 = 1: token tiles of 256 exactly and a remainder
 ]
 
 
+@pytest.fixture(params=["pair", "single"])
+def gemm1_kernel(request):
+    """Run a grouped-path test with the CTA-pair gate/up GEMM (where I allows
+    it) and again with the single-CTA one."""
+    moe.moe_test_set_gemm1_single(1 if request.param == "single" else 0)
+    yield request.param
+    moe.moe_test_set_gemm1_single(0)
+
+
+def test_gemm1_pair_kernel_launchable():
+    # a B200 holds many clusters of two of these CTAs; the pair kernel is the default
+    assert moe.moe_test_gemm1_pairs() >= 1
+
+
 @pytest.mark.parametrize("T,d,E,I,k1,k2,bias", GSMALL)
-def test_layer_grouped_all_tokens(T, d, E, I, k1, k2, bias):
+def test_layer_grouped_all_tokens(T, d, E, I, k1, k2, bias, gemm1_kernel):
     L = synth.make_layer(T, d, E, I, seed=T + d + E + 1, device=DEV, bias=bias)
     check_layer_full(L, k1, k2, flags=GROUPED, tight=False)
 
 
-@pytest.mark.parametrize("T,d,E,I,k1", [(48, 256, 8, 128, 2), (520, 128, 4, 256, 2)])
-def test_expert_ffn_grouped_per_slot(T, d, E, I, k1):
+@pytest.mark.parametrize("T,d,E,I,k1", [(48, 256, 8, 128, 2), (520, 128, 4, 256, 2),
+                                       (300, 256, 6, 512, 3)])
+def test_expert_ffn_grouped_per_slot(T, d, E, I, k1, gemm1_kernel):
     L = synth.make_layer(T, d, E, I, seed=11, device=DEV, bias="normal")
     ws = moe.workspace(T, d, E, I, k1, device=DEV)
     idx = torch.empty(T, k1, dtype=torch.int32, device=DEV)
