@@ -614,7 +614,7 @@ def roofline_record(stack, workload, head, res, graphs, stream, peaks, variant):
         bd1, a1, p1, u1, fr1 = bound(f1, b1, g1_ms)
         # the gate/up GEMM runs on CTA pairs when I is a multiple of 256
         from routed_expert_layer_route_b200 import moe
-        g1_name = "k_gemm1_pair" if I % 256 == 0 and moe.moe_test_gemm1_pairs() > 0 else "k_gemm1"
+        g1_name = "k_gemm1_pair" if I % 256 == 0 and moe.moe_test_grouped_pairs(1) > 0 else "k_gemm1"
         bd2, a2, p2, u2, fr2 = bound(f2, b2, g2_ms)
         return {"bound": bd1, "achieved": round(a1, 1), "peak": p1, "unit": u1,
                 "frac": round(fr1, 4), "traffic": recorded_traffic(workload, k1, g1_name),

@@ -22,17 +22,17 @@ int moe_test_exp_c(const float *x, float *y, int64_t n, void *stream);
  * device (0 if no device). */
 int moe_test_num_sms(void);
 
-/* Gate/up GEMM of the grouped path: single = 1 makes every later call use
- * the single-CTA kernel (k_gemm1); 0 (the default) uses the CTA-pair kernel
- * (k_gemm1_pair) whenever I is a multiple of 256 and the device holds at
- * least one pair.  Process-wide, not thread-safe; for tests and timing.
- * Returns a moe_status. */
-int moe_test_set_gemm1_single(int single);
+/* Grouped GEMMs of the tensor-core path: single = 1 makes every later call
+ * use the single-CTA kernels (k_gemm1, k_gemm2); 0 (the default) runs the
+ * gate/up GEMM on the CTA-pair kernel (k_gemm1_pair) when I is a multiple
+ * of 256 and the device holds at least one pair.  Process-wide, not
+ * thread-safe; for tests and timing.  Returns a moe_status. */
+int moe_test_set_grouped_single(int single);
 
-/* CTA pairs of the pair GEMM the current device holds at once (the pair
- * kernel's grid is twice this); 0 if it cannot be launched, -1 without a
- * device. */
-int moe_test_gemm1_pairs(void);
+/* CTA pairs of a pair GEMM the current device holds at once (the kernel's
+ * grid is twice this): which 1, the gate/up GEMM (the one pair kernel); 0 if
+ * it cannot be launched; -1 without a device or for another `which`. */
+int moe_test_grouped_pairs(int which);
 
 /* Set how long the library's bounded device waits (mbarrier phases,
  * cross-CTA flags, the grid barrier, the one-token layer's router exchange)

@@ -31,18 +31,17 @@
 
 namespace moe {
 
-constexpr int kGPStages = 4;
 constexpr int kGPTileB = (kGBN / 2) * kGBK * 2;  // 16 KB: half of a token tile
-constexpr int kGPStage = 2 * kGTileA + kGPTileB;  // 48 KB
 constexpr int kGPRows = 2 * kGBM;                 // weight rows of one pair item
-// epilogue: four warps per quarter of the tensor-memory lanes, each for 64
-// of the token columns (the MMAs wait while tensor memory drains, so the
-// drain gets the warps)
-constexpr int kGPEpiWarps = 16;
-constexpr int kGPThreads = (kGPEpiWarps + 2) * 32;  // 576
-// queue consumers: per CTA the epilogue warps, plus the MMA thread (CTA 0)
-// or the TMA producer (CTA 1)
-constexpr int kGPQConsumers = 2 * (kGPEpiWarps + 1);
+// gate/up: A_gate + A_up + half B per stage (48 KB), four stages
+constexpr int kGP1Stages = 4;
+constexpr int kGP1Stage = 2 * kGTileA + kGPTileB;
+constexpr int kGPMaxStages = kGP1Stages;
+// gate/up epilogue: four warps per quarter of the tensor-memory lanes, each
+// for 64 of the token columns (one accumulator set: the MMAs wait while
+// tensor memory drains, so the drain gets the warps)
+constexpr int kGP1EpiWarps = 16;
+constexpr int kGP1Threads = (kGP1EpiWarps + 2) * 32;  // 576
 
 // silu(g) * u as g * u * (1 + tanh(g / 2)) / 2 with the hardware tanh (one
 // special-function operation; relative error about 2^-11, well inside the
@@ -174,14 +173,14 @@ MOE_DEVINL void tma_load_2d_pair(void *dst, const CUtensorMap *map, int x, int y
 
 // ---------------------------------------------------------------------------
 struct GPSync {
-    uint64_t full[kGPStages];   // CTA 0: both CTAs' tiles of stage s landed
-    uint64_t empty[kGPStages];  // each CTA: the MMAs reading stage s finished
-    uint64_t acc_full;          // each CTA: the item's accumulators are complete
-    uint64_t acc_empty;         // CTA 0: both epilogues have read tensor memory
-    uint64_t q_full[kGQ];       // each CTA: CTA 0 published q_item[slot]
-    uint64_t q_empty[kGQ];      // CTA 0: every consumer of both CTAs is done with it
-    uint64_t drained;           // each CTA: every MMA has completed
-    uint64_t bye;               // each CTA: the other CTA has finished
+    uint64_t full[kGPMaxStages];   // CTA 0: both CTAs' tiles of stage s landed
+    uint64_t empty[kGPMaxStages];  // each CTA: the MMAs reading stage s finished
+    uint64_t acc_full[2];          // each CTA: accumulator set b of the item is complete
+    uint64_t acc_empty[2];         // CTA 0: both epilogues have read accumulator set b
+    uint64_t q_full[kGQ];          // each CTA: CTA 0 published q_item[slot]
+    uint64_t q_empty[kGQ];         // CTA 0: every consumer of both CTAs is done with it
+    uint64_t drained;              // each CTA: every MMA has completed
+    uint64_t bye;                  // each CTA: the other CTA has finished
     int q_item[kGQ];
     uint32_t tmem_base;
     int abort;
@@ -191,34 +190,29 @@ MOE_DEVINL bool gp_aborted(const GPSync &sy) { return *(volatile const int *)&sy
 
 inline size_t gemm1_pair_smem_bytes()
 {
-    return 1024 + (size_t)kGPStages * kGPStage + sizeof(GPSync) + sizeof(GTable);
+    return 1024 + (size_t)kGP1Stages * kGP1Stage + sizeof(GPSync) + sizeof(GTable);
 }
 
-// Work items of the pair kernel: weight-row tiles of 256 rows (I % 256 == 0).
-__global__ void __launch_bounds__(kGPThreads, 1)
-    k_gemm1_pair(const __grid_constant__ CUtensorMap tm_gate,
-                 const __grid_constant__ CUtensorMap tm_up,
-                 const __grid_constant__ CUtensorMap tm_xs, Gemm1Args a)
+// Set-up of a pair kernel: barriers (thread 0), tensor memory for the pair
+// (warp kGWarpMma of both CTAs, all 512 columns), then a cluster barrier so
+// that no remote arrival reaches a barrier before it exists.  nepi: the
+// epilogue warps of one CTA.
+MOE_DEVINL void gp_setup(GPSync &sy, int stages, int nepi, int tid, int warp)
 {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *ring = g_align1024(smem_raw);
-    GPSync &sy = *reinterpret_cast<GPSync *>(ring + (size_t)kGPStages * kGPStage);
-    GTable &tb = *reinterpret_cast<GTable *>(&sy + 1);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const uint32_t rank = cluster_rank();
-    const bool lead = rank == 0;
-    int *status = &a.hdr->status;
-
     if (tid == 0) {
-        for (int s = 0; s < kGPStages; ++s) {
+        for (int s = 0; s < stages; ++s) {
             mbar_init(&sy.full[s], 1);
             mbar_init(&sy.empty[s], 1);
         }
-        mbar_init(&sy.acc_full, 1);
-        mbar_init(&sy.acc_empty, 2 * kGPEpiWarps);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sy.acc_full[b], 1);
+            mbar_init(&sy.acc_empty[b], 2 * nepi);
+        }
+        // queue consumers: per CTA the epilogue warps, plus the MMA thread
+        // (CTA 0) or the TMA producer (CTA 1)
         for (int q = 0; q < kGQ; ++q) {
             mbar_init(&sy.q_full[q], 1);
-            mbar_init(&sy.q_empty[q], kGPQConsumers);
+            mbar_init(&sy.q_empty[q], 2 * (nepi + 1));
         }
         mbar_init(&sy.drained, 1);
         mbar_init(&sy.bye, 1);
@@ -231,8 +225,109 @@ __global__ void __launch_bounds__(kGPThreads, 1)
     }
     tc_fence_before();
     __syncthreads();
-    cluster_sync_all();  // both CTAs' barriers exist before any remote arrival
+    cluster_sync_all();
     tc_fence_after();
+}
+
+// The TMA warp's next item (lane 0): CTA 0 takes `next` (or -1 to end) and
+// publishes it to both CTAs' queues once every consumer of both CTAs is done
+// with the slot; CTA 1 takes it from its queue and hands the slot back to
+// CTA 0.  Returns the item, -1 at the end, -2 if a wait gave up.
+MOE_DEVINL int gp_producer_item(GPSync &sy, GQueue &q, bool lead, uint32_t peer, int next,
+                                int *status)
+{
+    int cur;
+    if (lead) {
+        cur = next;
+        if (!mbar_wait_cluster(&sy.q_empty[q.slot], q.ph ^ 1u, status))
+            return -2;
+        sy.q_item[q.slot] = cur;
+        st_cluster_u32(cluster_addr(&sy.q_item[q.slot], peer), cur);
+        mbar_arrive(&sy.q_full[q.slot]);
+        mbar_arrive_cluster(cluster_addr(&sy.q_full[q.slot], peer));
+    } else {
+        if (!mbar_wait_cluster(&sy.q_full[q.slot], q.ph, status))
+            return -2;
+        cur = *(volatile int *)&sy.q_item[q.slot];
+        mbar_arrive_cluster(cluster_addr(&sy.q_empty[q.slot], 0));
+    }
+    q.advance();
+    return cur;
+}
+
+// An epilogue warp's next item: lane 0 waits, the warp gets one answer (-1:
+// none left, or the wait gave up and the CTA aborts).
+MOE_DEVINL int gp_take_warp(GPSync &sy, GQueue &q, int *status, int lane)
+{
+    int cur = -1;
+    if (lane == 0) {
+        if (mbar_wait_cluster(&sy.q_full[q.slot], q.ph, status))
+            cur = *(volatile int *)&sy.q_item[q.slot];
+        else
+            sy.abort = 1;
+    }
+    return __shfl_sync(0xffffffffu, cur, 0);
+}
+
+// An epilogue warp is done with its item: accumulator set `buf` read (CTA 0's
+// barrier) and the queue slot handed back (CTA 0's barrier).
+MOE_DEVINL void gp_release_warp(GPSync &sy, GQueue &q, int buf, int lane)
+{
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) {
+        mbar_arrive_cluster(cluster_addr(&sy.acc_empty[buf], 0));
+        mbar_arrive_cluster(cluster_addr(&sy.q_empty[q.slot], 0));
+    }
+    q.advance();
+}
+
+// End of a pair kernel: free tensor memory once every MMA has completed (CTA
+// 0's MMA thread waited already), the farewell handshake -- neither CTA's
+// shared memory goes away while the other may still reach it -- and the
+// last CTA resets the item counters.
+MOE_DEVINL void gp_teardown(GPSync &sy, uint32_t tmem, GSched sc, bool lead, uint32_t peer,
+                            int tid, int warp, int lane, int *status)
+{
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kGWarpMma) {
+        if (lane == 0 && !lead)
+            mbar_wait(&sy.drained, 0, status);
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, 512);
+    }
+    if (tid == 0) {
+        mbar_arrive_cluster(cluster_addr(&sy.bye, peer));
+        mbar_wait_cluster(&sy.bye, 0, status);
+        __threadfence();
+        if (atomicAdd(sc.done, 1u) == gridDim.x - 1) {
+            *sc.next = 0u;
+            *sc.done = 0u;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Gate/up GEMM on CTA pairs with the SwiGLU epilogue (I % 256 == 0).  Tensor
+// memory of each CTA: its rows' gate accumulator in columns [0, 256), up in
+// [256, 512).
+__global__ void __launch_bounds__(kGP1Threads, 1)
+    k_gemm1_pair(const __grid_constant__ CUtensorMap tm_gate,
+                 const __grid_constant__ CUtensorMap tm_up,
+                 const __grid_constant__ CUtensorMap tm_xs, Gemm1Args a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *ring = g_align1024(smem_raw);
+    GPSync &sy = *reinterpret_cast<GPSync *>(ring + (size_t)kGP1Stages * kGP1Stage);
+    GTable &tb = *reinterpret_cast<GTable *>(&sy + 1);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = cluster_rank(), peer = rank ^ 1u;
+    const bool lead = rank == 0;
+    int *status = &a.hdr->status;
+
+    gp_setup(sy, kGP1Stages, kGP1EpiWarps, tid, warp);
     const uint32_t tmem = sy.tmem_base;
 
     pdl_wait();
@@ -243,7 +338,6 @@ __global__ void __launch_bounds__(kGPThreads, 1)
     g_build_items(a.offsets, E, nrt, tb, a.T * a.k1, status);
     const int n_items = tb.ibase[E];
     GQueue q = {0, 0u};
-    const uint32_t peer = rank ^ 1u;
 
     if (warp == kGWarpTma) {
         // -------------------------------------------------------- items (CTA 0), tiles
@@ -251,33 +345,14 @@ __global__ void __launch_bounds__(kGPThreads, 1)
             uint32_t g = 0;
             int i = lead ? (int)atomicAdd(a.sched.next, 1u) : 0;
             while (true) {
-                int cur;
-                if (lead) {
-                    cur = i < n_items && !gp_aborted(sy) ? i : -1;
-                    // publish to both queues once every consumer is done with the slot
-                    if (!mbar_wait_cluster(&sy.q_empty[q.slot], q.ph ^ 1u, status)) {
-                        sy.abort = 1;
-                        break;
-                    }
-                    sy.q_item[q.slot] = cur;
-                    st_cluster_u32(cluster_addr(&sy.q_item[q.slot], peer), cur);
-                    mbar_arrive(&sy.q_full[q.slot]);
-                    mbar_arrive_cluster(cluster_addr(&sy.q_full[q.slot], peer));
-                    q.advance();
-                    if (cur < 0)
-                        break;
+                const int cur = gp_producer_item(sy, q, lead, peer,
+                                                 i < n_items && !gp_aborted(sy) ? i : -1, status);
+                if (cur == -2)
+                    sy.abort = 1;
+                if (cur < 0)
+                    break;
+                if (lead)
                     i = (int)atomicAdd(a.sched.next, 1u);  // the next one, in flight meanwhile
-                } else {
-                    if (!mbar_wait_cluster(&sy.q_full[q.slot], q.ph, status)) {
-                        sy.abort = 1;
-                        break;
-                    }
-                    cur = *(volatile int *)&sy.q_item[q.slot];
-                    mbar_arrive_cluster(cluster_addr(&sy.q_empty[q.slot], 0));
-                    q.advance();
-                    if (cur < 0)
-                        break;
-                }
                 const GItem it = g_item(tb, E, cur);
                 const int row = it.e * I + it.rt * kGPRows + (int)rank * kGBM;
                 const int nh = pad16(it.n) / 2;         // this CTA's tokens (multiple of 8)
@@ -285,12 +360,12 @@ __global__ void __launch_bounds__(kGPThreads, 1)
                 const int nb = (nh + 63) / 64;          // 64-row boxes of them
                 const uint32_t stage_bytes = 2u * (2 * kGTileA + nb * (kGTileB / 4));
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
-                    const int s = g % kGPStages;
-                    if (!mbar_wait_cluster(&sy.empty[s], ((g / kGPStages) & 1) ^ 1, status)) {
+                    const int s = g % kGP1Stages;
+                    if (!mbar_wait_cluster(&sy.empty[s], ((g / kGP1Stages) & 1) ^ 1, status)) {
                         sy.abort = 1;
                         break;
                     }
-                    uint8_t *st = ring + (size_t)s * kGPStage;
+                    uint8_t *st = ring + (size_t)s * kGP1Stage;
                     const uint32_t fb = cluster_addr(&sy.full[s], 0);
                     if (lead)  // both CTAs' bytes of the stage
                         mbar_arrive_expect_tx(&sy.full[s], stage_bytes);
@@ -307,8 +382,9 @@ __global__ void __launch_bounds__(kGPThreads, 1)
             // CTA 1's copies complete on CTA 0's barriers, which the MMAs waited for
             if (lead) {
                 const uint32_t n_iss = g;
-                for (uint32_t r = n_iss > (uint32_t)kGPStages ? n_iss - kGPStages : 0; r < n_iss; ++r)
-                    mbar_wait(&sy.full[r % kGPStages], (r / kGPStages) & 1, status);
+                for (uint32_t r = n_iss > (uint32_t)kGP1Stages ? n_iss - kGP1Stages : 0; r < n_iss;
+                     ++r)
+                    mbar_wait(&sy.full[r % kGP1Stages], (r / kGP1Stages) & 1, status);
             }
         }
     } else if (warp == kGWarpMma) {
@@ -324,20 +400,20 @@ __global__ void __launch_bounds__(kGPThreads, 1)
                 if (cur < 0)
                     break;
                 const GItem it = g_item(tb, E, cur);
-                if (!mbar_wait_cluster(&sy.acc_empty, (itc & 1) ^ 1, status)) {
+                if (!mbar_wait_cluster(&sy.acc_empty[0], (itc & 1) ^ 1, status)) {
                     sy.abort = 1;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t idesc = umma_idesc_bf16(kGPRows, pad16(it.n));
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
-                    const int s = g % kGPStages;
-                    if (!mbar_wait(&sy.full[s], (g / kGPStages) & 1, status)) {
+                    const int s = g % kGP1Stages;
+                    if (!mbar_wait(&sy.full[s], (g / kGP1Stages) & 1, status)) {
                         sy.abort = 1;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t st = smem_addr(ring + (size_t)s * kGPStage);
+                    const uint32_t st = smem_addr(ring + (size_t)s * kGP1Stage);
 #pragma unroll
                     for (int kk = 0; kk < kGBK / 16; ++kk) {
                         const uint64_t ag = umma_desc_sw128(st + kk * 32);
@@ -351,7 +427,7 @@ __global__ void __launch_bounds__(kGPThreads, 1)
                 }
                 if (gp_aborted(sy))
                     break;
-                umma_commit_pair_both(&sy.acc_full);
+                umma_commit_pair_both(&sy.acc_full[0]);
                 mbar_arrive(&sy.q_empty[q.slot]);
                 q.advance();
                 ++itc;
@@ -362,28 +438,20 @@ __global__ void __launch_bounds__(kGPThreads, 1)
         }
     } else {
         // -------------------------------------------------------- epilogue (both CTAs)
-        const int lq = warp & 3;   // tensor-memory lane quarter
+        const int lq = warp & 3;  // tensor-memory lane quarter
         // which quarter of the token columns: warps 0-3 the first, then
         // warps 6-9, 10-13, 14-17 (each set covers the four lane quarters)
         const int eh = warp < 4 ? 0 : (warp - 6) / 4 + 1;
         uint32_t itc = 0;
         const uint32_t lane_addr = tmem + ((uint32_t)(lq * 32) << 16);
-        const uint32_t acc_empty0 = cluster_addr(&sy.acc_empty, 0);
         while (true) {
-            int cur = -1;
-            if (lane == 0) {
-                if (mbar_wait_cluster(&sy.q_full[q.slot], q.ph, status))
-                    cur = *(volatile int *)&sy.q_item[q.slot];
-                else
-                    sy.abort = 1;
-            }
-            cur = __shfl_sync(0xffffffffu, cur, 0);
+            const int cur = gp_take_warp(sy, q, status, lane);
             if (cur < 0)
                 break;
             const GItem it = g_item(tb, E, cur);
             int ok = 1;
             if (lane == 0)
-                ok = mbar_wait_cluster(&sy.acc_full, itc & 1, status);
+                ok = mbar_wait_cluster(&sy.acc_full[0], itc & 1, status);
             if (!__shfl_sync(0xffffffffu, ok, 0)) {
                 sy.abort = 1;
                 break;
@@ -408,38 +476,11 @@ __global__ void __launch_bounds__(kGPThreads, 1)
                         *reinterpret_cast<uint32_t *>(hrow + (size_t)tj * I) = pair;
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive_cluster(acc_empty0);
-                mbar_arrive_cluster(cluster_addr(&sy.q_empty[q.slot], 0));
-            }
-            q.advance();
+            gp_release_warp(sy, q, 0, lane);
             ++itc;
         }
     }
-
-    // ------------------------------------------------------------ teardown
-    tc_fence_before();
-    __syncthreads();
-    if (warp == kGWarpMma) {
-        if (lane == 0 && !lead)  // CTA 0's MMA thread waited already
-            mbar_wait(&sy.drained, 0, status);
-        __syncwarp();
-        tc_fence_after();
-        tmem_dealloc_pair(tmem, 512);
-    }
-    if (tid == 0) {
-        // farewell: neither CTA's shared memory goes away while the other may
-        // still reach it
-        mbar_arrive_cluster(cluster_addr(&sy.bye, peer));
-        mbar_wait_cluster(&sy.bye, 0, status);
-        __threadfence();
-        if (atomicAdd(a.sched.done, 1u) == gridDim.x - 1) {
-            *a.sched.next = 0u;
-            *a.sched.done = 0u;
-        }
-    }
+    gp_teardown(sy, tmem, a.sched, lead, peer, tid, warp, lane, status);
 }
 
 }  // namespace moe

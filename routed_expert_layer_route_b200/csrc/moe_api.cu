@@ -100,9 +100,33 @@ struct DevInfo {
     int gemm1_pairs = 0;  // CTA pairs of k_gemm1_pair resident at once (0: not launchable)
 };
 
-// Which gate/up GEMM kernel the grouped path uses (test hook): 0 the pair
-// kernel where the shapes allow it, 1 always the single-CTA kernel.
-static int g_gemm1_single = 0;
+// Which grouped GEMM kernels the grouped path uses (test hook): 0 the pair
+// kernel for the gate/up GEMM where the shapes allow it, 1 always the
+// single-CTA kernels.
+static int g_grouped_single = 0;
+
+// CTA pairs of a pair kernel the device holds at once (0: not launchable).
+template <typename K>
+static int pair_occupancy(K kern, int threads, size_t smem, int num_sms)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (num_sms / 2));
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute at;
+    at.id = cudaLaunchAttributeClusterDimension;
+    at.val.clusterDim.x = 2;
+    at.val.clusterDim.y = 1;
+    at.val.clusterDim.z = 1;
+    cfg.attrs = &at;
+    cfg.numAttrs = 1;
+    int nc = 0;
+    if (cudaOccupancyMaxActiveClusters(&nc, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return nc < num_sms / 2 ? nc : num_sms / 2;
+}
 static DevInfo g_dev[64];
 static std::mutex g_dev_mu;
 
@@ -140,26 +164,8 @@ static int device_info(DevInfo *&out)
             cudaFuncSetAttribute(k_gemm1_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gemm1_pair_smem_bytes()) != cudaSuccess)
             return MOE_ERR_CUDA;
-        {
-            // how many CTA pairs of the pair kernel the device holds at once
-            cudaLaunchConfig_t cfg = {};
-            cfg.gridDim = dim3(2 * (di.num_sms / 2));
-            cfg.blockDim = dim3(kGPThreads);
-            cfg.dynamicSmemBytes = gemm1_pair_smem_bytes();
-            cudaLaunchAttribute at;
-            at.id = cudaLaunchAttributeClusterDimension;
-            at.val.clusterDim.x = 2;
-            at.val.clusterDim.y = 1;
-            at.val.clusterDim.z = 1;
-            cfg.attrs = &at;
-            cfg.numAttrs = 1;
-            int nc = 0;
-            if (cudaOccupancyMaxActiveClusters(&nc, k_gemm1_pair, &cfg) != cudaSuccess) {
-                cudaGetLastError();
-                nc = 0;
-            }
-            di.gemm1_pairs = nc < di.num_sms / 2 ? nc : di.num_sms / 2;
-        }
+        di.gemm1_pairs = pair_occupancy(k_gemm1_pair, kGP1Threads, gemm1_pair_smem_bytes(),
+                                        di.num_sms);
         // scores of kCtkMaxN channels + at most 16 KiB of side-by-side row partials
         if (cudaFuncSetAttribute(k_ctk_down, dsm, kCtkMaxN * 4 + 16 * 1024) != cudaSuccess)
             return MOE_ERR_CUDA;
@@ -389,13 +395,13 @@ static int enqueue_grouped(const void *x, const void *wg, const void *wu, const 
     a1.I = I;
     a1.k1 = k1;
     a1.hdr = hdr;
+    DevInfo *di;
+    if ((rc = device_info(di)) != MOE_OK)
+        return rc;
     if (which & 1) {
         // the pair kernel when the weight rows come in whole 256-row tiles
-        DevInfo *di;
-        if ((rc = device_info(di)) != MOE_OK)
-            return rc;
-        if (I % kGPRows == 0 && di->gemm1_pairs > 0 && !g_gemm1_single)
-            rc = launch(k_gemm1_pair, dim3(2 * di->gemm1_pairs), dim3(kGPThreads),
+        if (I % kGPRows == 0 && di->gemm1_pairs > 0 && !g_grouped_single)
+            rc = launch(k_gemm1_pair, dim3(2 * di->gemm1_pairs), dim3(kGP1Threads),
                         gemm1_pair_smem_bytes(), s, (pdl ? kPdl : 0) | kPair, tg, tu, tx, a1);
         else
             rc = launch(k_gemm1, dim3(G), dim3(kG1Threads), gemm1_smem_bytes(), s, pdl, tg, tu,
@@ -1248,16 +1254,18 @@ int moe_test_wait_never_set(void *ws, size_t ws_bytes, int which, void *stream)
                   0, static_cast<WsHeader *>(ws), which);
 }
 
-int moe_test_set_gemm1_single(int single)
+int moe_test_set_grouped_single(int single)
 {
     if (single != 0 && single != 1)
         return MOE_ERR_INVALID_ARG;
-    g_gemm1_single = single;
+    g_grouped_single = single;
     return MOE_OK;
 }
 
-int moe_test_gemm1_pairs(void)
+int moe_test_grouped_pairs(int which)
 {
+    if (which != 1)
+        return -1;
     DevInfo *di;
     if (device_info(di) != MOE_OK)
         return -1;

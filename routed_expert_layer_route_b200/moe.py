@@ -73,8 +73,8 @@ SIGNATURES = {
                                     _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_test_exp_c": (_i, [_vp, _vp, ctypes.c_int64, _vp]),
     "moe_test_num_sms": (_i, []),
-    "moe_test_set_gemm1_single": (_i, [_i]),
-    "moe_test_gemm1_pairs": (_i, []),
+    "moe_test_set_grouped_single": (_i, [_i]),
+    "moe_test_grouped_pairs": (_i, [_i]),
     "moe_test_set_wait_limit_ns": (_i, [ctypes.c_uint64]),
     "moe_test_wait_never_set": (_i, [_vp, _sz, _i, _vp]),
     "moe_test_expert_stream": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _i, _i, _vp,
@@ -325,12 +325,12 @@ def moe_test_num_sms():
     return lib().moe_test_num_sms()
 
 
-def moe_test_set_gemm1_single(single):
-    _check(lib().moe_test_set_gemm1_single(int(single)), "moe_test_set_gemm1_single")
+def moe_test_set_grouped_single(single):
+    _check(lib().moe_test_set_grouped_single(int(single)), "moe_test_set_grouped_single")
 
 
-def moe_test_gemm1_pairs():
-    return lib().moe_test_gemm1_pairs()
+def moe_test_grouped_pairs(which):
+    return lib().moe_test_grouped_pairs(int(which))
 
 
 def moe_test_set_wait_limit_ns(ns):

@@ -258,28 +258,29 @@ GSMALL = [
 
 
 @pytest.fixture(params=["pair", "single"])
-def gemm1_kernel(request):
+def gemm_kernels(request):
     """Run a grouped-path test with the CTA-pair gate/up GEMM (where I allows
     it) and again with the single-CTA one."""
-    moe.moe_test_set_gemm1_single(1 if request.param == "single" else 0)
+    moe.moe_test_set_grouped_single(1 if request.param == "single" else 0)
     yield request.param
-    moe.moe_test_set_gemm1_single(0)
+    moe.moe_test_set_grouped_single(0)
 
 
-def test_gemm1_pair_kernel_launchable():
+def test_pair_kernels_launchable():
     # a B200 holds many clusters of two of these CTAs; the pair kernel is the default
-    assert moe.moe_test_gemm1_pairs() >= 1
+    assert moe.moe_test_grouped_pairs(1) >= 1
+    assert moe.moe_test_grouped_pairs(2) == -1
 
 
 @pytest.mark.parametrize("T,d,E,I,k1,k2,bias", GSMALL)
-def test_layer_grouped_all_tokens(T, d, E, I, k1, k2, bias, gemm1_kernel):
+def test_layer_grouped_all_tokens(T, d, E, I, k1, k2, bias, gemm_kernels):
     L = synth.make_layer(T, d, E, I, seed=T + d + E + 1, device=DEV, bias=bias)
     check_layer_full(L, k1, k2, flags=GROUPED, tight=False)
 
 
 @pytest.mark.parametrize("T,d,E,I,k1", [(48, 256, 8, 128, 2), (520, 128, 4, 256, 2),
                                        (300, 256, 6, 512, 3)])
-def test_expert_ffn_grouped_per_slot(T, d, E, I, k1, gemm1_kernel):
+def test_expert_ffn_grouped_per_slot(T, d, E, I, k1, gemm_kernels):
     L = synth.make_layer(T, d, E, I, seed=11, device=DEV, bias="normal")
     ws = moe.workspace(T, d, E, I, k1, device=DEV)
     idx = torch.empty(T, k1, dtype=torch.int32, device=DEV)
