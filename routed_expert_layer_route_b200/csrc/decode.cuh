@@ -14,9 +14,11 @@
 //
 // Design (one CTA per SM, cooperative launch; 12 consumer warps + 1 producer
 // warp):
-//  * router: CTA b dots x with router rows b, b+G, ... (fetched into shared
-//    memory before the programmatic-launch wait -- weights no earlier kernel
-//    writes -- with an L2 evict-last policy), writes the logits and counts
+//  * router: CTA b dots x with router rows R*b .. R*b+R-1 (R rows per
+//    router CTA, chosen on the host: fewer router CTAs each with more rows
+//    make fewer arrivals to wait for), fetched into shared memory before the
+//    programmatic-launch wait -- weights no earlier kernel writes -- with an
+//    L2 evict-last policy; it writes the logits and counts
 //    them on a release counter in the workspace header (spread over lines);
 //    warp 0 of every CTA waits for all E, reads them back, forms the float32
 //    softmax, takes the top min(k2, E) in rank order by repeated warp arg-max
@@ -83,6 +85,7 @@ struct DecodeArgs {
     int y_dtype;
     VarK vk;       // variable k: cascade or skip (kind 0 with the fixed-k kernel)
     int32_t *count;  // nullable: kt
+    int rrows;       // router rows per router CTA: decode_router_rows(d, E, G)
     WsHeader *hdr;
 };
 
@@ -277,7 +280,8 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
     int *status = &a.hdr->status;
     const int d = a.d, E = a.E, I = a.I, k1 = a.k1;
     const bool fused = a.wr != nullptr;
-    const int nr = fused && b < E ? (E - 1 - b) / G + 1 : 0;  // router rows e = b + G*i
+    const int R = max(a.rrows, (E + G - 1) / G);  // the grid covers all E rows
+    const int nr = fused && b * R < E ? min(R, E - b * R) : 0;  // router rows e = R*b + i
     const int nvec = d >> 3;                                   // 16-byte vectors per row
 
     if (tid == 0) {
@@ -301,7 +305,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
         const uint64_t keep = l2_evict_last_policy();  // the router, read by every call
         mbar_arrive_expect_tx(rbar, (uint32_t)(nr * d * 2));
         for (int i = 0; i < nr; ++i)
-            bulk_g2s(ring + (size_t)i * d * 2, a.wr + (size_t)(b + G * i) * d, (uint32_t)(d * 2),
+            bulk_g2s(ring + (size_t)i * d * 2, a.wr + (size_t)(b * R + i) * d, (uint32_t)(d * 2),
                      rbar, keep);
     }
 
@@ -354,7 +358,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
                     router_step(a0, a1, i, row[v], xg[v]);
             }
             float z = warp_sum(a0 + a1);
-            const int e = b + G * warp;
+            const int e = b * R + warp;
             if (a.bias)
                 z = z + a.bias[e];
             if (lane == 0) {
@@ -717,13 +721,23 @@ inline size_t decode_smem_bytes(int d)
 // The single-pass path serves one token per call (T == 1) whose output rows
 // fit the register partials, with the down matrix channel-major; each CTA's
 // router rows fit the ring.
+// Router rows per router CTA: about 32 KB of them (at most kDMaxRouterRows),
+// and enough for the grid to cover all E rows.
+inline int decode_router_rows(int d, int E, int G)
+{
+    int r = (32 * 1024) / (2 * d);
+    r = r < 1 ? 1 : (r > kDMaxRouterRows ? kDMaxRouterRows : r);
+    const int need = (E + G - 1) / G;
+    return r > need ? r : need;
+}
+
 inline bool decode_fits(int T, int d, int E, int I, int k1, int G)
 {
     if (T != 1 || k1 > kDMaxK1 || (d >> 3) > kWPS * 32 * kDMaxRowVec || E > kMaxExperts)
         return false;
     if (decode_smem_bytes(d) > 227 * 1024 || (size_t)kDStages * d * 4 > (size_t)kDSlots * kDStageBytes)
         return false;
-    const int rows = (E + G - 1) / G;
+    const int rows = decode_router_rows(d, E, G);
     if (rows > kDMaxRouterRows || (size_t)rows * d * 2 > (size_t)kDRouterBytes)
         return false;
     const long chmax = ((long)k1 * I + G - 1) / G;

@@ -295,6 +295,7 @@ static int enqueue_decode(const void *x, const void *wr, const float *bias, floa
     a.y_dtype = y_dtype;
     a.vk = vk;
     a.count = count;
+    a.rrows = decode_router_rows(d, E, G);
     a.hdr = static_cast<WsHeader *>(ws);
     const size_t smem = decode_smem_bytes(d);
     const dim3 grid(G), block(kSThreads);
