@@ -363,10 +363,13 @@ def time_grouped_kernels(stack, k1, ws_list, stream, reps):
     return out
 
 
-def e2e_tokens_per_s(stack, k1, k2, ws_list, steps, warmup, stream):
+def e2e_tokens_per_s(stack, k1, k2, ws_list, steps, warmup, stream, graph=True):
     """Through the public API with host buffers: per step, pinned-host ->
     device copy of every layer's tokens, every layer's moe_layer call, and a
-    device -> pinned-host copy of every layer's output."""
+    device -> pinned-host copy of every layer's output.  graph: the step (the
+    two copies and the layer calls, made through moe_layer while capturing)
+    is captured once into a CUDA graph and replayed, as a serving loop
+    would; else every step issues the calls from Python."""
     wl = stack.wl
     T, d, L_ = wl["T"], wl["d"], wl["layers"]
     host_x = torch.stack([L.x for L in stack.layers]).cpu().pin_memory()
@@ -380,18 +383,29 @@ def e2e_tokens_per_s(stack, k1, k2, ws_list, steps, warmup, stream):
             stack.call(L, k1, k2, dev_y[l], ws, stream, x=dev_x[l])
         host_y.copy_(dev_y, non_blocking=True)
 
+    run = step
+    g = None
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            step()  # one eager pass: first-use set-up stays outside capture
+            stream.synchronize()
+            with torch.cuda.graph(g, stream=stream):
+                step()
+        run = g.replay
     with torch.cuda.stream(stream):
         for _ in range(warmup):
-            step()
+            run()
         stream.synchronize()
         s = torch.cuda.Event(enable_timing=True)
         e = torch.cuda.Event(enable_timing=True)
         s.record(stream)
         for _ in range(steps):
-            step()
+            run()
         e.record(stream)
         e.synchronize()
     ms = s.elapsed_time(e) / steps
+    del g
     return T * 1000.0 / ms, host_x[0].numel() * 2 * L_, host_y[0].numel() * 2 * L_
 
 
@@ -759,10 +773,14 @@ def run_native(args, world, rank):
     k1h, k2h = head
     _, ws_list, ys = graphs[head]
 
-    # end to end through the public API with host buffers
+    # end to end through the public API with host buffers: the step captured
+    # once into a CUDA graph (as a serving loop would), and issued from Python
     e2e_val, h2d, d2h = e2e_tokens_per_s(stack, k1h, k2h, ws_list, max(3, args.steps // 4),
-                                         args.warmup, stream)
+                                         args.warmup, stream, graph=True)
     e2e_val = world * T * 1000.0 / allreduce_max(T * 1000.0 / e2e_val, world)
+    e2e_eager, _, _ = e2e_tokens_per_s(stack, k1h, k2h, ws_list, max(3, args.steps // 4),
+                                       args.warmup, stream, graph=False)
+    e2e_eager = world * T * 1000.0 / allreduce_max(T * 1000.0 / e2e_eager, world)
     ratio, ratio_pair = k1_ratio(results)
 
     cpu = None
@@ -791,7 +809,11 @@ def run_native(args, world, rank):
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_val, 3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
-                "path": "moe_layer C-ABI per layer from Python, pinned host x in, y out"},
+                "path": "per step: pinned host x -> device, moe_layer (C-ABI) per layer, y -> "
+                        "pinned host; the step captured once into a CUDA graph and replayed",
+                "eager": {"value": round(e2e_eager, 3), "unit": "tokens/s",
+                          "path": "the same step issued from Python every time (ctypes call "
+                                  "per layer)"}},
         "gpu_launches": per_step_launches * Ln * args.steps,
         "clocks": clk,
         "sweep": results,
