@@ -849,8 +849,18 @@ __global__ void __launch_bounds__(256) k_gather_rows(const uint16_t *x, const in
         const int t = slot / k1;
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * d);
         uint4 *dst = reinterpret_cast<uint4 *>(xs + (size_t)p * d);
-        for (int v = lane; v < nv; v += 32)
-            dst[v] = __ldg(&src[v]);
+        // eight 16-byte loads of the row in flight before their stores
+        for (int v0 = lane; v0 < nv; v0 += 8 * 32) {
+            uint4 r[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (v0 + 32 * u < nv)
+                    r[u] = __ldg(&src[v0 + 32 * u]);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (v0 + 32 * u < nv)
+                    dst[v0 + 32 * u] = r[u];
+        }
     }
 }
 
