@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode(DecodeArgs a)
         if (b == 0 && tid < kSpread)  // the count of the call two ahead starts at zero
             a.hdr->xcnt[(call + 2u) & 3u].c[tid][0] = 0u;
         // ------------------------------------------------------------ router logits
-        // warp i < nr: router row b + G*i in router_step's order (the order of
+        // warp i < nr: router row R*b + i in router_step's order (the order of
         // k_logits), its x vectors all in flight at once; warp 0 also keeps
         // the token's x row in shared memory for the FFN
         const uint4 *xg = reinterpret_cast<const uint4 *>(a.x);
