@@ -65,7 +65,11 @@ def test_pack_w_down_is_the_transpose(E, d, I):
 
 @pytest.mark.parametrize("d,E,I,k1,k2", [(64, 16, 32, 2, 4), (256, 64, 96, 8, 16),
                                           (1024, 40, 112, 6, 1000), (192, 20, 32, 20, 20),
-                                          (512, 128, 256, 32, 64)])
+                                          (512, 128, 256, 32, 64),
+                                          # many experts: 128 router CTAs of 8 rows, the
+                                          # widest warp router; E not a power of two
+                                          (256, 1024, 32, 8, 16), (512, 1000, 48, 6, 40),
+                                          (4096, 300, 64, 4, 12)])
 def test_decode_path_single_token(d, E, I, k1, k2):
     L = synth.make_layer(1, d, E, I, seed=d + E + k1, device=DEV, bias="normal")
     wdc = moe.moe_pack_w_down(L.w_down)
