@@ -80,7 +80,7 @@ typedef enum {
 #define MOE_EMPTY_SLOT 0x7fffffff
 
 /* moe_layer / moe_expert_ffn flags: which expert-FFN path runs.
- * AUTO: one token with the channel-major down matrix -> DECODE; two or more
+ * AUTO: up to eight tokens with the channel-major down matrix -> DECODE; two or more
  * tokens with d and I multiples of 128 -> GROUPED; otherwise STREAM. */
 #define MOE_PATH_AUTO 0
 #define MOE_PATH_STREAM 1  /* two-phase weight streaming on CUDA cores, deterministic
@@ -89,8 +89,9 @@ typedef enum {
                               of 128); h rounded to bf16 before the down projection;
                               the float32 combine runs in a timing-dependent order, so
                               y may differ between runs in the last bits              */
-#define MOE_PATH_DECODE 3  /* one token: a single pass over the routed experts with the
-                              down matrix channel-major (needs MOE_WDOWN_CHANNEL_MAJOR);
+#define MOE_PATH_DECODE 3  /* 1 <= T <= 8 tokens: a single pass over the union of the
+                              routed experts with the down matrix channel-major (needs
+                              MOE_WDOWN_CHANNEL_MAJOR);
                               the float32 sum into y runs in a timing-dependent order,
                               so y may differ between runs in the last bits           */
 #define MOE_PATH_MASK 0xff
@@ -175,8 +176,10 @@ int moe_combine(const float *expert_out, const int32_t *slot_pos, const float *t
  * topk_idx_out / topk_w_out [T x k1], logits_out [T x E] float32.
  * flags: MOE_PATH_* | MOE_WDOWN_CHANNEL_MAJOR.  With the HF down layout
  * [E x d x I] the two-phase streaming path runs (deterministic).  With
- * MOE_WDOWN_CHANNEL_MAJOR (w_down from moe_pack_w_down) and T == 1 the
- * single-pass decode path runs; other T return MOE_ERR_UNSUPPORTED_SHAPE.
+ * MOE_WDOWN_CHANNEL_MAJOR (w_down from moe_pack_w_down) and 1 <= T <= 8 the
+ * single-pass decode path runs (each routed expert's weights read once for
+ * all the tokens routed to it; for 5 <= T <= 8, d <= 3072); other shapes
+ * return MOE_ERR_UNSUPPORTED_SHAPE.
  * ws: workspace. */
 int moe_layer(const void *x_bf16, const void *w_router_bf16, const float *bias,
               const void *w_gate_bf16, const void *w_up_bf16, const void *w_down_bf16, int T, int d,
@@ -201,8 +204,8 @@ int moe_route_cascade(const void *x_bf16, const void *w_router_bf16, const float
                       size_t ws_bytes, void *stream);
 
 /* moe_layer with the variable-k route of moe_route_cascade: y[t] sums only
- * the token's k_t experts.  Runs on the one-token decode path (down matrix
- * channel-major) and on the tensor-core grouped path (d, I multiples of 128);
+ * the token's k_t experts.  Runs on the decode path (down matrix
+ * channel-major, up to eight tokens) and on the tensor-core grouped path (d, I multiples of 128);
  * other shapes return MOE_ERR_UNSUPPORTED_SHAPE.  topk_count_out [T] int32
  * (nullable) receives k_t.  Other arguments as for moe_layer. */
 int moe_layer_cascade(const void *x_bf16, const void *w_router_bf16, const float *bias,

@@ -14,6 +14,7 @@
 #include "combine.cuh"
 #include "ctopk.cuh"
 #include "decode.cuh"
+#include "decode_mt.cuh"
 #include "gemm_pair.cuh"
 #include "grouped.cuh"
 #include "route.cuh"
@@ -42,6 +43,9 @@ static WsLayout ws_layout(int T, int d, int E, int I, int k1)
     WsLayout L;
     size_t o = sizeof(WsHeader);
     const size_t n = (size_t)T * k1;
+    // the decode kernels' accumulator (kMtMaxT tokens, kept zero between
+    // calls), first after the header: the same place for every T
+    L.dyacc = o;       o = align256(o + sizeof(float) * (size_t)kMtMaxT * d);
     L.logits = o;      o = align256(o + sizeof(float) * (size_t)T * E);
     L.idx = o;         o = align256(o + sizeof(int32_t) * n);
     L.w = o;           o = align256(o + sizeof(float) * n);
@@ -55,8 +59,6 @@ static WsLayout ws_layout(int T, int d, int E, int I, int k1)
     L.y_acc = o;       o = align256(o + sizeof(float) * (size_t)T * d);
     L.hist = o;        o = align256(o + sizeof(int32_t) * (size_t)perm_chunks(T) * E);
     L.ctk = o;         o = align256(o + 2 * sizeof(float) * (size_t)k1 * I);  // one token's h, scores
-    // one token: the decode kernel's accumulator (kept zero between calls)
-    L.dyacc = o;       o = align256(o + (T == 1 ? sizeof(float) * (size_t)d : 0));
     L.total = o;
     return L;
 }
@@ -155,7 +157,12 @@ static int device_info(DevInfo *&out)
             cudaFuncSetAttribute(k_decode<16, false>, dsm, decode_smem) != cudaSuccess ||
             cudaFuncSetAttribute(k_decode<0, true>, dsm, decode_smem) != cudaSuccess ||
             cudaFuncSetAttribute(k_decode<8, true>, dsm, decode_smem) != cudaSuccess ||
-            cudaFuncSetAttribute(k_decode<16, true>, dsm, decode_smem) != cudaSuccess)
+            cudaFuncSetAttribute(k_decode<16, true>, dsm, decode_smem) != cudaSuccess ||
+            cudaFuncSetAttribute(k_decode_mt<2, 1>, dsm, decode_smem) != cudaSuccess ||
+            cudaFuncSetAttribute(k_decode_mt<4, 1>, dsm, decode_smem) != cudaSuccess ||
+            cudaFuncSetAttribute(k_decode_mt<8, 1>, dsm, decode_smem) != cudaSuccess ||
+            cudaFuncSetAttribute(k_decode_mt<2, 2>, dsm, decode_smem) != cudaSuccess ||
+            cudaFuncSetAttribute(k_decode_mt<4, 2>, dsm, decode_smem) != cudaSuccess)
             return MOE_ERR_CUDA;
         if (cudaFuncSetAttribute(k_gemm1, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gemm1_smem_bytes()) != cudaSuccess ||
@@ -313,6 +320,60 @@ static int enqueue_decode(const void *x, const void *wr, const float *bias, floa
     return launch(k_decode<0, false>, grid, block, smem, s, kPdl | kCoop, a);
 }
 
+// The few-token decode path of moe_layer (2 <= T <= 8, down matrix
+// channel-major): one kernel -- router logits, routing, the union of the
+// routed experts streamed once, per-token partials into y_acc, y written by
+// its last CTA.
+static int enqueue_decode_mt(const void *x, const void *wr, const float *bias, float *logits_out,
+                             const void *wg, const void *wu, const void *wdt, int T, int d, int E,
+                             int I, int k1, int k2, void *y, int y_dtype, int32_t *idx_copy,
+                             float *w_copy, void *ws, int G, cudaStream_t s, VarK vk,
+                             int32_t *count)
+{
+    const WsLayout L = ws_layout(T, d, E, I, k1);
+    const MtLayout ML = mt_layout(T, d);
+    MtArgs a = {};
+    a.x = static_cast<const uint16_t *>(x);
+    a.wg = static_cast<const uint16_t *>(wg);
+    a.wu = static_cast<const uint16_t *>(wu);
+    a.wdt = static_cast<const uint16_t *>(wdt);
+    a.wr = static_cast<const uint16_t *>(wr);
+    a.bias = bias;
+    a.logits = at<float>(ws, L.logits);
+    a.logits_out = logits_out;
+    a.topk_idx = at<int32_t>(ws, L.idx);
+    a.topk_w = at<float>(ws, L.w);
+    a.idx_copy = idx_copy;
+    a.w_copy = w_copy;
+    a.count = count;
+    a.yacc = at<float>(ws, L.dyacc);
+    a.y = y;
+    a.y_dtype = y_dtype;
+    a.T = T;
+    a.d = d;
+    a.E = E;
+    a.I = I;
+    a.k1 = k1;
+    a.k2 = k2;
+    a.rrows = mt_router_rows(E, G);
+    a.nslots = ML.nslots;
+    a.vk = vk;
+    a.hdr = static_cast<WsHeader *>(ws);
+    int TM, RVM;
+    mt_shape(T, d, TM, RVM);
+    const dim3 grid(G), block(kSThreads);
+    const int opts = kPdl | kCoop;
+    if (RVM == 1) {
+        if (TM == 2)
+            return launch(k_decode_mt<2, 1>, grid, block, ML.total, s, opts, a);
+        if (TM == 4)
+            return launch(k_decode_mt<4, 1>, grid, block, ML.total, s, opts, a);
+        return launch(k_decode_mt<8, 1>, grid, block, ML.total, s, opts, a);
+    }
+    if (TM == 2)
+        return launch(k_decode_mt<2, 2>, grid, block, ML.total, s, opts, a);
+    return launch(k_decode_mt<4, 2>, grid, block, ML.total, s, opts, a);
+}
 
 // ------------------------------------------------------------------ grouped GEMM path
 // cuTensorMapEncodeTiled from the driver, looked up once through the runtime
@@ -917,13 +978,14 @@ static int layer_impl(const void *x_bf16, const void *w_router_bf16, const float
 
     const int G = di->num_sms;
     const bool decode = down_cm && decode_fits(T, d, E, I, k1, G);
-    if (down_cm && !decode)
-        return MOE_ERR_UNSUPPORTED_SHAPE;  // channel-major down matrix: one-token calls only
+    const bool decode_mt = down_cm && !decode && mt_fits(T, d, E, I, k1, G);
+    if (down_cm && !decode && !decode_mt)
+        return MOE_ERR_UNSUPPORTED_SHAPE;  // channel-major down matrix: up to kMtMaxT tokens
     const bool grouped = !down_cm && (path == MOE_PATH_GROUPED ||
                                       (path == MOE_PATH_AUTO && auto_grouped(T, d, E, I, k1)));
     if (grouped && !grouped_fits(d, E, I))
         return MOE_ERR_UNSUPPORTED_SHAPE;
-    if (cascade && !decode && !grouped)
+    if (cascade && !decode && !decode_mt && !grouped)
         return MOE_ERR_UNSUPPORTED_SHAPE;  // the variable-k route runs on those two paths
     if (grouped) {
         // router logits (tensor-core GEMM when the experts fill 128-row tiles),
@@ -954,6 +1016,10 @@ static int layer_impl(const void *x_bf16, const void *w_router_bf16, const float
         return enqueue_decode(x_bf16, w_router_bf16, bias, logits_out, w_gate_bf16, w_up_bf16,
                               w_down_bf16, d, E, I, k1, k2, y, y_dtype, topk_idx_out, topk_w_out,
                               ws, G, s, vk, count_out);
+    if (decode_mt)
+        return enqueue_decode_mt(x_bf16, w_router_bf16, bias, logits_out, w_gate_bf16, w_up_bf16,
+                                 w_down_bf16, T, d, E, I, k1, k2, y, y_dtype, topk_idx_out,
+                                 topk_w_out, ws, G, s, vk, count_out);
     if ((rc = enqueue_logits(x_bf16, w_router_bf16, bias, z, logits_out, T, d, E, s)) != MOE_OK)
         return rc;
     if (T > 1) {

@@ -49,7 +49,7 @@ CM = moe.MOE_WDOWN_CHANNEL_MAJOR
 def test_layer_small_all_tokens(T, d, E, I, k1, k2, bias):
     L = synth.make_layer(T, d, E, I, seed=T + d + E, device=DEV, bias=bias)
     check_layer_full(L, k1, k2)
-    if T == 1:  # the single-pass decode path on the channel-major down matrix
+    if T <= 8:  # the single-pass decode path on the channel-major down matrix
         wdc = moe.moe_pack_w_down(L.w_down)
         check_layer_full(L, k1, k2, flags=CM, w_down=wdc)
         check_layer_full(L, k1, k2, flags=moe.MOE_PATH_DECODE | CM, w_down=wdc)
@@ -76,6 +76,52 @@ def test_decode_path_single_token(d, E, I, k1, k2):
     check_layer_full(L, k1, k2, flags=CM, w_down=wdc)
 
 
+# the few-token decode kernel: (tokens the partials cover, row vectors per lane)
+# = (2, 1), (4, 1), (8, 1), (2, 2), (4, 2); one to three channels per stage;
+# experts shared by several tokens (E small) and none shared (E large)
+FEW = [
+    # T, d, E, I, k1, k2, bias
+    (2, 256, 64, 96, 8, 16, "normal"),
+    (2, 6144, 16, 32, 2, 4, None),        # one channel per stage, two row vectors per lane
+    (3, 512, 128, 256, 4, 16, None),
+    (4, 4096, 300, 64, 4, 12, "normal"),  # E not a power of two, two row vectors per lane
+    (5, 1024, 40, 112, 6, 1000, None),    # k2 > E
+    (6, 256, 1024, 32, 8, 16, "normal"),  # seven router rows per CTA, the widest router
+    (7, 3072, 64, 128, 8, 8, None),       # the widest d with one row vector per lane
+    (8, 128, 8, 16, 8, 8, None),          # k1 = E: all eight tokens on every expert
+    (8, 2048, 128, 768, 8, 16, "zipf"),
+    (8, 512, 200, 48, 8, 1000, None),     # T*k1 = 64 slots, short experts: several per CTA
+]
+
+
+@pytest.mark.parametrize("T,d,E,I,k1,k2,bias", FEW)
+def test_decode_path_few_tokens(T, d, E, I, k1, k2, bias):
+    L = synth.make_layer(T, d, E, I, seed=T * 7 + d + E, device=DEV, bias=bias)
+    wdc = moe.moe_pack_w_down(L.w_down)
+    check_layer_full(L, k1, k2, flags=CM, w_down=wdc)
+    check_layer_full(L, k1, k2, flags=moe.MOE_PATH_DECODE | CM, w_down=wdc)
+    # bf16 output: the float32 result rounded (up to one step: the sums' order varies)
+    y32, *_ = run_layer(L, k1, k2, flags=CM, w_down=wdc)
+    y16, *_ = run_layer(L, k1, k2, flags=CM, w_down=wdc, y_dtype=torch.bfloat16)
+    assert torch.allclose(y32.to(torch.bfloat16).float(), y16.float(), rtol=2 ** -7, atol=1e-6)
+
+
+@pytest.mark.parametrize("T,E,k1,k2,group", [(4, 128, 8, 16, 2), (8, 64, 6, 20, 3),
+                                             (2, 128, 32, 127, 128), (5, 16, 4, 8, 16)])
+def test_decode_few_tokens_route_ties(T, E, k1, k2, group):
+    """Equal logits on the few-token path: repeated router rows give bit-equal
+    logits; the rank order falls back to the lower expert index."""
+    d, I = 256, 32
+    L = synth.make_layer(T, d, E, I, seed=E + k1 + group + T, device=DEV)
+    L.w_router = L.w_router[torch.arange(E, device=DEV) // group * group].contiguous()
+    wdc = moe.moe_pack_w_down(L.w_down)
+    _, idx, _, z = run_layer(L, k1, k2, flags=CM, w_down=wdc)
+    zn = z.cpu().numpy()
+    for g0 in range(0, E, group):
+        assert np.all(zn[:, g0:g0 + group] == zn[:, g0:g0 + 1])
+    check_layer_full(L, k1, k2, flags=CM, w_down=wdc)
+
+
 @pytest.mark.parametrize("E,k1,k2,group", [(128, 8, 16, 2), (128, 4, 128, 4), (128, 32, 127, 128),
                                            (64, 6, 20, 3), (16, 4, 8, 16), (100, 5, 9, 7),
                                            (512, 10, 20, 4)])
@@ -95,12 +141,16 @@ def test_decode_route_ties(E, k1, k2, group):
     check_layer_full(L, k1, k2, flags=CM, w_down=wdc)
 
 
-def test_channel_major_down_needs_one_token():
+def test_channel_major_down_token_limits():
+    # nine tokens, or eight with more than one row vector per lane per token
+    # partial (d > 3072), or more than 64 routed slots: no decode kernel
+    for T, d, k1 in ((9, 256, 2), (8, 4096, 2), (5, 256, 16)):
+        L = synth.make_layer(T, d, 16, 32, seed=7, device=DEV)
+        wdc = moe.moe_pack_w_down(L.w_down)
+        with pytest.raises(moe.MoeError) as ei:
+            run_layer(L, k1, 16, flags=CM, w_down=wdc)
+        assert ei.value.status == moe.MOE_ERR_UNSUPPORTED_SHAPE
     L = synth.make_layer(2, 256, 16, 32, seed=7, device=DEV)
-    wdc = moe.moe_pack_w_down(L.w_down)
-    with pytest.raises(moe.MoeError) as ei:
-        run_layer(L, 2, 4, flags=CM, w_down=wdc)
-    assert ei.value.status == moe.MOE_ERR_UNSUPPORTED_SHAPE
     with pytest.raises(moe.MoeError) as ei:  # the decode path needs the channel-major matrix
         run_layer(L, 2, 4, flags=moe.MOE_PATH_DECODE)
     assert ei.value.status == moe.MOE_ERR_INVALID_ARG
@@ -134,6 +184,14 @@ def test_layer_deterministic_and_workspace_reuse():
     d_y, d_i, d_w, _ = run_layer(L1, 4, 16, ws=big, flags=CM, w_down=moe.moe_pack_w_down(L1.w_down))
     assert torch.equal(d_i, s_i) and torch.equal(d_w, s_w)
     assert torch.allclose(d_y, s_y, rtol=1e-5, atol=1e-6)
+    # the few-token decode path on the same workspace after the calls above
+    # (the decode accumulator sits at one place for every batch size)
+    wdc = moe.moe_pack_w_down(L.w_down)
+    for _ in range(2):
+        m_y, m_i, m_w, _ = run_layer(L, 4, 16, ws=big, flags=CM, w_down=wdc)
+        assert torch.equal(m_i, ia) and torch.equal(m_w, wa)
+        assert torch.allclose(m_y, a, rtol=1e-5, atol=1e-6)
+        run_layer(L1, 4, 16, ws=big, flags=st)
 
 
 def test_indices_do_not_depend_on_k2():
@@ -208,6 +266,8 @@ def test_decode_small_batch_full_size(T, k1, k2):
     tokens = list(range(T)) if T == 8 else [0, 5, 17, 31]
     check_layer_sampled(L, k1, k2, tokens)  # AUTO: the tensor-core path
     check_layer_sampled(L, k1, k2, tokens, flags=moe.MOE_PATH_STREAM)
+    if T <= 8:  # the few-token decode kernel
+        check_layer_sampled(L, k1, k2, tokens, flags=CM, w_down=moe.moe_pack_w_down(L.w_down))
 
 
 @pytest.mark.parametrize("T", [1, 64])
