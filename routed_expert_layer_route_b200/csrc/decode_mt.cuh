@@ -12,7 +12,7 @@
 // for every token t routed to e, w the Eq. 2 weight ("Paper of the Week #3",
 // section "The Receipt").
 //
-// Design (one CTA per SM, cooperative launch; 12 consumer warps + 1 producer):
+// Design (one CTA per SM, cooperative launch; 11 consumer warps + 1 producer):
 //  * every CTA stages the T tokens' x rows in shared memory; router CTA b
 //    fetches router rows R*b .. R*b+R-1 (R = ceil(E / grid)) before the
 //    programmatic-launch wait, and its consumer warps share the R*T dot
@@ -25,10 +25,10 @@
 //  * the U activated experts are laid end to end as U*I channels, CTA b takes
 //    a balanced contiguous range, and the producer streams stages of up to
 //    three whole channels through the bulk-copy ring;
-//  * all 12 consumer warps serve every stage: first the gate and up dot
+//  * all 11 consumer warps serve every stage: first the gate and up dot
 //    products of the stage's (channel, token) pairs -- a job per channel and
 //    chunk of at most two of the expert's tokens (a gate/up vector read once
-//    for both), one warp each -- with w*h into shared memory (two buffers by
+//    for both), dealt over the warps -- with w*h into shared memory (two buffers by
 //    stage parity); after the consumer barrier each warp adds w*h*down_row
 //    into the register partials of its own output rows, one set per token
 //    slot of the current expert -- the warps own disjoint rows, so no partial
@@ -46,7 +46,11 @@ namespace moe {
 
 constexpr int kMtMaxT = 8;        // tokens per call
 constexpr int kMtMaxSlots = 64;   // T * k1
-constexpr int kMtMaxRowVec = 2;   // 16-byte row vectors per lane (d <= 6144)
+constexpr int kMtMaxRowVec = 2;   // 16-byte row vectors per lane (d <= 5632)
+// 11 consumer warps and the producer: 12 warps, three per scheduler, so a
+// thread may hold up to 168 registers (the per-token row partials)
+constexpr int kMtC = 11;
+constexpr int kMtThreads = (kMtC + 1) * 32;
 
 struct MtArgs {
     const uint16_t *x;    // [T x d]
@@ -137,6 +141,8 @@ __device__ void mt_segments(MtSmem *ms, int U, int I, int G, int b, int *status)
     ms->nseg = ns;
 }
 
+MOE_DEVINL void mt_sync() { named_bar_sync(kConsumerBar, kMtC * 32); }
+
 // Token position of the r-th set bit of m (r < popc(m)).
 MOE_DEVINL int nth_bit(unsigned m, int r)
 {
@@ -168,7 +174,9 @@ MOE_DEVINL float pair_total(uint64_t a, uint64_t b)
 
 // h = SiLU(gate_row . x_t) * (up_row . x_t) for NT tokens (1 or 2) of one
 // channel, the weight vectors read once for both; two partial chains per dot
-// product (vectors lane + 64i and lane + 64i + 32).
+// product (vectors lane + 64i and lane + 64i + 32).  x0, x1: the tokens' rows
+// as two planes of float32 pairs, elements 0-3 of 16-byte vector v at [v],
+// elements 4-7 at [v + nvec] (consecutive lanes read consecutive 16 bytes).
 template <int NT>
 MOE_DEVINL void mt_channel(const uint4 *grow, const uint4 *urow, const ulonglong2 *x0,
                            const ulonglong2 *x1, int nvec, int lane, float (&h)[2])
@@ -182,13 +190,13 @@ MOE_DEVINL void mt_channel(const uint4 *grow, const uint4 *urow, const ulonglong
         const uint4 z = make_uint4(0, 0, 0, 0);
         const uint4 wg0 = grow[v], wu0 = urow[v];
         const uint4 wg1 = second ? grow[v + 32] : z, wu1 = second ? urow[v + 32] : z;
-        mt_step(g[0][0], u[0][0], wg0, wu0, x0[2 * v], x0[2 * v + 1]);
+        mt_step(g[0][0], u[0][0], wg0, wu0, x0[v], x0[v + nvec]);
         if (second)
-            mt_step(g[0][1], u[0][1], wg1, wu1, x0[2 * v + 64], x0[2 * v + 65]);
+            mt_step(g[0][1], u[0][1], wg1, wu1, x0[v + 32], x0[v + 32 + nvec]);
         if constexpr (NT > 1) {
-            mt_step(g[1][0], u[1][0], wg0, wu0, x1[2 * v], x1[2 * v + 1]);
+            mt_step(g[1][0], u[1][0], wg0, wu0, x1[v], x1[v + nvec]);
             if (second)
-                mt_step(g[1][1], u[1][1], wg1, wu1, x1[2 * v + 64], x1[2 * v + 65]);
+                mt_step(g[1][1], u[1][1], wg1, wu1, x1[v + 32], x1[v + 32 + nvec]);
         }
     }
 #pragma unroll
@@ -221,9 +229,9 @@ __device__ __forceinline__ void mt_route(const MtArgs &a, int t, bool ok, int la
 }
 
 // TM: tokens the partials cover (T <= TM); RVM: 16-byte output-row vectors per
-// lane (d <= RVM * kSC * 256).
+// lane (d <= RVM * kMtC * 256).
 template <int TM, int RVM>
-__global__ void __launch_bounds__(kSThreads, 1) k_decode_mt(MtArgs a)
+__global__ void __launch_bounds__(kMtThreads, 1) k_decode_mt(MtArgs a)
 {
     static_assert(TM <= kMtMaxT && RVM <= kMtMaxRowVec, "few-token kernel: partials");
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -232,7 +240,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode_mt(MtArgs a)
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bar_off);
     uint64_t *empty = full + kDSlots;
     uint64_t *rbar = empty + kDSlots;  // the router rows' bulk copies
-    float *xs = reinterpret_cast<float *>(smem + L.x_off);  // [T][d] float32
+    float *xs = reinterpret_cast<float *>(smem + L.x_off);  // [T][2 planes][d/2] float32
     uint8_t *ring = smem + L.ring_off;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -247,7 +255,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode_mt(MtArgs a)
     if (tid == 0) {
         for (int s = 0; s < kDSlots; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kSC);
+            mbar_init(&empty[s], kMtC);
         }
         mbar_init(rbar, 1);
         ms->abort = 0;
@@ -257,7 +265,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode_mt(MtArgs a)
     __syncthreads();
     // this CTA's router rows: weights no earlier kernel writes, so they are
     // fetched before the dependency wait and overlap the previous kernel
-    if (warp == kSC && lane == 0 && nr > 0) {
+    if (warp == kMtC && lane == 0 && nr > 0) {
         const uint64_t keep = l2_evict_last_policy();  // the router, read by every call
         mbar_arrive_expect_tx(rbar, (uint32_t)(nr * d * 2));
         for (int i = 0; i < nr; ++i)
@@ -268,7 +276,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode_mt(MtArgs a)
     pdl_wait();
     pdl_trigger();
 
-    if (warp < kSC) {
+    if (warp < kMtC) {
         const unsigned call = ld_relaxed_u32(&a.hdr->decode_seq) + 1u;
         const unsigned slot = call & 3u;
         if (b == 0 && tid < kSpread)  // the count of the call two ahead starts at zero
@@ -277,21 +285,22 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode_mt(MtArgs a)
         // widened to float32 once (exact), for the router and the dot jobs
         {
             const uint4 *xg = reinterpret_cast<const uint4 *>(a.x);
-            float4 *xw = reinterpret_cast<float4 *>(xs);
-            for (int i = tid; i < T * nvec; i += kSC * 32) {
-                const uint4 v = xg[i];
-                xw[2 * i] = make_float4(bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y));
-                xw[2 * i + 1] = make_float4(bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w));
+            for (int i = tid; i < T * nvec; i += kMtC * 32) {
+                const int t = i / nvec, v = i - t * nvec;
+                const uint4 w = xg[i];
+                float4 *row = reinterpret_cast<float4 *>(xs + (size_t)t * d);
+                row[v] = make_float4(bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y));
+                row[v + nvec] = make_float4(bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w));
             }
         }
-        consumer_sync();
+        mt_sync();
         // ------------------------------------------------------------ router logits
         // dot product (row i, token t) = job i*T + t, shared by the consumer
         // warps; each in router_step's order (the order of k_logits)
         if (warp < nr * T) {
             if (!mbar_wait(rbar, 0, status))
                 ms->abort = 1;
-            for (int job = warp; job < nr * T; job += kSC) {
+            for (int job = warp; job < nr * T; job += kMtC) {
                 const int i = job / T, t = job % T;
                 const uint4 *row = reinterpret_cast<const uint4 *>(ring + (size_t)i * d * 2);
                 const float *xt = xs + (size_t)t * d;
@@ -300,9 +309,9 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode_mt(MtArgs a)
                 for (int v = lane; v < nvec; v += 32, ++q) {
                     // router_step's order (k_logits): vectors alternate between a0 and a1
                     float xf[8];
-                    *reinterpret_cast<float4 *>(xf) = *reinterpret_cast<const float4 *>(xt + 8 * v);
+                    *reinterpret_cast<float4 *>(xf) = reinterpret_cast<const float4 *>(xt)[v];
                     *reinterpret_cast<float4 *>(xf + 4) =
-                        *reinterpret_cast<const float4 *>(xt + 8 * v + 4);
+                        reinterpret_cast<const float4 *>(xt)[v + nvec];
                     if (q & 1)
                         a1 = dot8_bf16(row[v], xf, a1);
                     else
@@ -356,7 +365,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode_mt(MtArgs a)
             if (lane == 0)
                 ms->ktok[warp] = kt;
         }
-        consumer_sync();
+        mt_sync();
 
         // ------------------------------------------------------------ the union (warp 0)
         if (warp == 0) {
@@ -420,7 +429,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode_mt(MtArgs a)
     const int nseg = ms->nseg;
     const int nch = decode_channels_per_stage(d);
 
-    if (warp == kSC) {
+    if (warp == kMtC) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             const uint64_t pol = l2_evict_first_policy();
@@ -457,7 +466,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode_mt(MtArgs a)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ consumers
-        // this warp's output rows: vectors v = warp*32 + lane + kSC*32*j, j < RVM;
+        // this warp's output rows: vectors v = warp*32 + lane + kMtC*32*j, j < RVM;
         // partials as float32 pairs, per token slot k of the current expert
         // (its k-th token), added into the accumulator when the expert changes
         uint64_t yq[TM][RVM][4];
@@ -476,7 +485,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode_mt(MtArgs a)
                     const int t = ms->utok[cur_u][k];
 #pragma unroll
                     for (int j = 0; j < RVM; ++j) {
-                        const int v = warp * 32 + lane + kSC * 32 * j;
+                        const int v = warp * 32 + lane + kMtC * 32 * j;
                         if (v < nvec) {
                             float *dst = a.yacc + (size_t)t * d + (size_t)v * 8;
                             red_add_v4(dst, pair_lo(yq[k][j][0]), pair_hi(yq[k][j][0]),
@@ -520,14 +529,14 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode_mt(MtArgs a)
             const uint8_t *stg = ring + (size_t)slot * kDStageBytes;
             const size_t rb = (size_t)n * d * 2;  // bytes of one of the three row blocks
             // (1) w*h: a job per (channel c, chunk of at most two of the expert's
-            // m tokens), one warp each: chunks per channel q = kSC / n, tokens
-            // per chunk 1 (m <= q) or 2 (n * chunks <= kSC since m <= 8 <= 2q)
-            const int q = n == 3 ? 4 : (n == 2 ? 6 : 12);
+            // m tokens), job j = chunk * n + c on warp j % kMtC: chunks per
+            // channel q = kMtC / n, tokens per chunk 1 (m <= q) or 2
+            const int q = n == 3 ? 3 : (n == 2 ? 5 : 11);
             const int tpc = m > q ? 2 : 1;
             const int nq = tpc == 1 ? m : (m + 1) >> 1;
-            if (ok && warp < n * nq) {
-                const int ch = n == 3 ? warp / 3 : (n == 2 ? warp >> 1 : warp);
-                const int c = warp - ch * n;
+            for (int j = warp; ok && j < n * nq; j += kMtC) {
+                const int ch = n == 3 ? j / 3 : (n == 2 ? j >> 1 : j);
+                const int c = j - ch * n;
                 const int k0 = ch * tpc;
                 const bool two = tpc == 2 && k0 + 1 < m;
                 const int t0 = ms->utok[u][k0];
@@ -547,7 +556,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode_mt(MtArgs a)
                         ms->hs[hb][c][k0 + 1] = h[1] * ms->uw[u][k0 + 1];
                 }
             }
-            consumer_sync();  // the stage's w*h are in shared memory
+            mt_sync();  // the stage's w*h are in shared memory
             // (2) y partials += w*h * down row, for this warp's rows and the
             // expert's m token slots.  hs alternates by stage parity: a warp
             // writes the buffer again two stages later, past the next stage's
@@ -560,7 +569,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode_mt(MtArgs a)
                         const uint4 *drow = reinterpret_cast<const uint4 *>(drows + (size_t)c * d * 2);
 #pragma unroll
                         for (int j = 0; j < RVM; ++j) {
-                            const int v = warp * 32 + lane + kSC * 32 * j;
+                            const int v = warp * 32 + lane + kMtC * 32 * j;
                             if (v < nvec) {
                                 const uint4 w = drow[v];
                                 const uint64_t w0 = bf16x2_pair(w.x), w1 = bf16x2_pair(w.y);
@@ -607,7 +616,7 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode_mt(MtArgs a)
             mbar_wait(&full[s], parity, status);
         }
     }
-    if (warp == kSC)
+    if (warp == kMtC)
         return;
 
     // ------------------------------------------------------------ y (last CTA to check in)
@@ -621,10 +630,10 @@ __global__ void __launch_bounds__(kSThreads, 1) k_decode_mt(MtArgs a)
                      : "memory");
         ms->last = prev == (unsigned)G - 1;
     }
-    consumer_sync();
+    mt_sync();
     if (ms->last) {
         const int tot = T * d;
-        for (int i = tid * 4; i < tot; i += kSC * 32 * 4) {
+        for (int i = tid * 4; i < tot; i += kMtC * 32 * 4) {
             const float4 v = __ldcg(reinterpret_cast<const float4 *>(a.yacc + i));
             if (a.y_dtype == MOE_DTYPE_BF16) {
                 const uint32_t lo = f32_to_bf16_rn(v.x) | ((uint32_t)f32_to_bf16_rn(v.y) << 16);
@@ -669,7 +678,7 @@ inline void mt_shape(int T, int d, int &TM, int &RVM)
 {
     const int nvec = d >> 3;
     TM = T <= 2 ? 2 : (T <= 4 ? 4 : 8);
-    RVM = nvec <= kSC * 32 ? 1 : (nvec <= 2 * kSC * 32 ? 2 : 0);
+    RVM = nvec <= kMtC * 32 ? 1 : (nvec <= 2 * kMtC * 32 ? 2 : 0);
     if (T < 2 || T > kMtMaxT || RVM == 0 || TM * RVM > 8)
         TM = 0;
 }

@@ -361,7 +361,7 @@ static int enqueue_decode_mt(const void *x, const void *wr, const float *bias, f
     a.hdr = static_cast<WsHeader *>(ws);
     int TM, RVM;
     mt_shape(T, d, TM, RVM);
-    const dim3 grid(G), block(kSThreads);
+    const dim3 grid(G), block(kMtThreads);
     const int opts = kPdl | kCoop;
     if (RVM == 1) {
         if (TM == 2)

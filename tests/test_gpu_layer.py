@@ -82,12 +82,12 @@ def test_decode_path_single_token(d, E, I, k1, k2):
 FEW = [
     # T, d, E, I, k1, k2, bias
     (2, 256, 64, 96, 8, 16, "normal"),
-    (2, 6144, 16, 32, 2, 4, None),        # one channel per stage, two row vectors per lane
+    (2, 5632, 16, 32, 2, 4, None),        # one channel per stage, two row vectors per lane
     (3, 512, 128, 256, 4, 16, None),
     (4, 4096, 300, 64, 4, 12, "normal"),  # E not a power of two, two row vectors per lane
     (5, 1024, 40, 112, 6, 1000, None),    # k2 > E
     (6, 256, 1024, 32, 8, 16, "normal"),  # seven router rows per CTA, the widest router
-    (7, 3072, 64, 128, 8, 8, None),       # the widest d with one row vector per lane
+    (7, 2816, 64, 128, 8, 8, None),       # the widest d with one row vector per lane
     (8, 128, 8, 16, 8, 8, None),          # k1 = E: all eight tokens on every expert
     (8, 2048, 128, 768, 8, 16, "zipf"),
     (8, 512, 200, 48, 8, 1000, None),     # T*k1 = 64 slots, short experts: several per CTA
@@ -143,7 +143,7 @@ def test_decode_route_ties(E, k1, k2, group):
 
 def test_channel_major_down_token_limits():
     # nine tokens, or eight with more than one row vector per lane per token
-    # partial (d > 3072), or more than 64 routed slots: no decode kernel
+    # partial (d > 2816), or more than 64 routed slots: no decode kernel
     for T, d, k1 in ((9, 256, 2), (8, 4096, 2), (5, 256, 16)):
         L = synth.make_layer(T, d, 16, 32, seed=7, device=DEV)
         wdc = moe.moe_pack_w_down(L.w_down)
