@@ -212,10 +212,13 @@ class Stack:
         self.skip = skip  # not None: (theta_expert, theta_weight) of expert skipping
         self.keep_frac = keep_frac  # not None: channel top-k, this share of k1*I kept
         self.layers = []
-        self.channel_major = wl["T"] == 1
-        # two or more tokens: the tensor-core grouped GEMMs (what AUTO picks when d
-        # and I fill 128-row tiles), named explicitly so the timed kernels are known
-        self.grouped = wl["T"] > 1 and wl["d"] % 128 == 0 and wl["I"] % 128 == 0
+        # one token, or up to eight with "cm": the down matrix channel-major and the
+        # single-pass decode kernels (k_decode, k_decode_mt)
+        self.channel_major = wl["T"] == 1 or (wl.get("cm") == 1 and wl["T"] <= 8)
+        # otherwise two or more tokens: the tensor-core grouped GEMMs (what AUTO picks
+        # when d and I fill 128-row tiles), named explicitly so the timed kernels are known
+        self.grouped = (not self.channel_major and wl["T"] > 1 and wl["d"] % 128 == 0
+                        and wl["I"] % 128 == 0)
         self.flags = (moe.MOE_WDOWN_CHANNEL_MAJOR if self.channel_major else
                       moe.MOE_PATH_GROUPED if self.grouped else moe.MOE_PATH_STREAM)
         for l in range(wl["layers"]):
@@ -468,7 +471,7 @@ def workload_config(name, wl, head, world):
     """The line's config: what was run (both arms print this same dict)."""
     T, d, E, I, Ln = wl["T"], wl["d"], wl["E"], wl["I"], wl["layers"]
     k1, k2 = head
-    one = T == 1
+    one = T == 1 or wl.get("cm") == 1
     return {"workload": "%s: %d layers, d=%d, E=%d, I=%d, T=%d per rank, k1=%d, k2=%d"
                         % (name, Ln, d, E, I, T, k1, k2),
             "layers": Ln, "d": d, "E": E, "I": I, "T": T, "k1": k1, "k2": k2,
@@ -594,13 +597,15 @@ def roofline_record(stack, workload, head, res, graphs, stream, peaks, variant):
     if variant or stack.channel_major:
         lay_s = res["us_per_layer"] * 1e-6
         achieved = alg_bytes / lay_s / 1e9
+        dk = "k_decode" if T == 1 else "k_decode_mt"
         kname = ("whole layer (cascade route)" if stack.tau is not None else
                  "whole layer (expert skipping)" if stack.skip is not None else
                  "whole layer (channel top-k: k_logits, k_ctk_gateup, k_ctk_down)"
-                 if stack.keep_frac is not None else "moe::k_decode")
+                 if stack.keep_frac is not None else "moe::" + dk)
         return {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(achieved / hbm_peak, 4),
-                "traffic": None if variant else recorded_traffic(workload, k1, "k_decode"),
+                "traffic": None if variant else recorded_traffic(
+                    workload if T == 1 else "%s_T%d" % (workload, T), k1, dk),
                 "frac_of_nominal_8000_GBps": round(achieved / 8000.0, 4),
                 "kernel": kname, "kernel_us": round(lay_s * 1e6, 3),
                 "launches_per_layer": 1 if not variant or stack.keep_frac is None else 3,
@@ -672,7 +677,9 @@ def layer_roofline(res, peaks):
 
 # workloads timed after the headline in the default run, each a sub-record
 EXTRA_WORKLOADS = [
-    ("decode_small_batch", {"T": 8}), ("decode_small_batch", {"T": 32}),
+    ("decode_small_batch", {"T": 8}), ("decode_small_batch", {"T": 2, "cm": 1}),
+    ("decode_small_batch", {"T": 4, "cm": 1}), ("decode_small_batch", {"T": 8, "cm": 1}),
+    ("decode_small_batch", {"T": 32}),
     ("decode_small_batch", {"T": 64}), ("prefill", {}),
     ("large", {"T": 1}), ("large", {"T": 64}),
 ]

@@ -123,6 +123,20 @@ def test_layer_cascade_decode_one_token(tau):
         _check_against_oracle(L, k1, k2, tau, y, idx, w, cnt, z, [0])
 
 
+@pytest.mark.parametrize("tau", [0.3, 0.7])
+def test_layer_cascade_decode_few_tokens(tau):
+    # the few-token decode kernel: each token's k_t slots, empty slots skipped
+    # in the union of the routed experts
+    d, E, I, k1, k2 = 256, 16, 64, 6, 8
+    ks = []
+    for T, seed in ((2, 50), (5, 51), (8, 52)):
+        L = _peaky_layer(T, d, E, I, seed=seed, bias="normal")
+        wdc = moe.moe_pack_w_down(L.w_down)
+        y, idx, w, cnt, z = _run_cascade(L, k1, k2, tau, moe.MOE_WDOWN_CHANNEL_MAJOR, w_down=wdc)
+        ks.append(_check_against_oracle(L, k1, k2, tau, y, idx, w, cnt, z, list(range(T))))
+    assert np.concatenate(ks).min() < k1  # the cascade stops early for some tokens
+
+
 @pytest.mark.parametrize("tau", [0.5, 0.9])
 def test_layer_cascade_full_size_decode_and_batch(tau):
     L1 = _peaky_layer(1, 2048, 128, 768, seed=0)

@@ -113,6 +113,20 @@ def test_layer_skip_decode_one_token():
     assert hits > 0
 
 
+def test_layer_skip_decode_few_tokens():
+    # the few-token decode kernel: skipped slots between kept ones
+    d, E, I, k1, k2 = 256, 16, 64, 6, 8
+    hits = 0
+    for T, seed in ((2, 60), (4, 61), (7, 62)):
+        L = _peaky(T, d, E, I, seed=seed)
+        tab = _table(E, seed).to(DEV)
+        out = _run(L, k1, k2, tab, 0.6, 0.15, moe.MOE_WDOWN_CHANNEL_MAJOR,
+                   w_down=moe.moe_pack_w_down(L.w_down))
+        k = _check(L, k1, k2, tab, 0.6, 0.15, out, list(range(T)))
+        hits += int((k < k1).sum())
+    assert hits > 0
+
+
 def test_layer_skip_full_size_decode_and_batch():
     tab = _table(128, 11).to(DEV)
     L1 = _peaky(1, 2048, 128, 768, seed=0)
