@@ -459,6 +459,8 @@ def workload_of(args):
         wl["T"] = args.T
     if args.layers:
         wl["layers"] = args.layers
+    if args.cm:
+        wl["cm"] = 1
     sweep = list(wl["sweep"])
     if args.k1:
         sweep = [(args.k1, args.k2 or args.k1)]
@@ -676,12 +678,14 @@ def layer_roofline(res, peaks):
 
 
 # workloads timed after the headline in the default run, each a sub-record
+# the few-token channel-major runs last: timed after the long 48-layer decode stacks, the
+# power-capped prefill GEMMs ran ~10 % slower than alone
 EXTRA_WORKLOADS = [
-    ("decode_small_batch", {"T": 8}), ("decode_small_batch", {"T": 2, "cm": 1}),
-    ("decode_small_batch", {"T": 4, "cm": 1}), ("decode_small_batch", {"T": 8, "cm": 1}),
-    ("decode_small_batch", {"T": 32}),
+    ("decode_small_batch", {"T": 8}), ("decode_small_batch", {"T": 32}),
     ("decode_small_batch", {"T": 64}), ("prefill", {}),
     ("large", {"T": 1}), ("large", {"T": 64}),
+    ("decode_small_batch", {"T": 2, "cm": 1}), ("decode_small_batch", {"T": 4, "cm": 1}),
+    ("decode_small_batch", {"T": 8, "cm": 1}),
 ]
 
 
@@ -838,6 +842,7 @@ def run_native(args, world, rank):
     # the other workloads (small batches, prefill, the large model), each a
     # sub-record with its own sweep, unique experts, k1 ratio and roofline
     default = (args.workload == "decode_b1" and not args.k1 and not args.T and not args.layers
+               and not args.cm
                and not variant and not args.no_extra)
     if default:
         extra = {}
@@ -906,6 +911,9 @@ def main():
     ap.add_argument("--k2", type=int, default=0)
     ap.add_argument("--T", type=int, default=0)
     ap.add_argument("--layers", type=int, default=0)
+    ap.add_argument("--cm", action="store_true",
+                    help="2 <= T <= 8: down matrices packed channel-major at set-up, the layers "
+                         "on the few-token decode kernel")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="time only the chosen workload (the default run also times the small "
