@@ -459,7 +459,7 @@ def workload_of(args):
         wl["T"] = args.T
     if args.layers:
         wl["layers"] = args.layers
-    if args.cm:
+    if getattr(args, "cm", False):
         wl["cm"] = 1
     sweep = list(wl["sweep"])
     if args.k1:
@@ -842,7 +842,7 @@ def run_native(args, world, rank):
     # the other workloads (small batches, prefill, the large model), each a
     # sub-record with its own sweep, unique experts, k1 ratio and roofline
     default = (args.workload == "decode_b1" and not args.k1 and not args.T and not args.layers
-               and not args.cm
+               and not getattr(args, "cm", False)
                and not variant and not args.no_extra)
     if default:
         extra = {}
