@@ -23,8 +23,9 @@
 //    the union of the routed experts, ascending, each with its tokens (a bit
 //    mask) and their weights;
 //  * the U activated experts are laid end to end as U*I channels, CTA b takes
-//    a balanced contiguous range, and the producer streams stages of up to
-//    three whole channels through the bulk-copy ring;
+//    a balanced contiguous range, and the producer streams stages of whole
+//    channels (up to eight: two slots of the largest size that fits) through
+//    the bulk-copy ring;
 //  * all 11 consumer warps serve every stage: first the gate and up dot
 //    products of the stage's (channel, token) pairs -- a job per channel and
 //    chunk of at most two of the expert's tokens (a gate/up vector read once
@@ -47,6 +48,7 @@ namespace moe {
 constexpr int kMtMaxT = 8;        // tokens per call
 constexpr int kMtMaxSlots = 64;   // T * k1
 constexpr int kMtMaxRowVec = 2;   // 16-byte row vectors per lane (d <= 5632)
+constexpr int kMtMaxCh = 8;       // channels per stage
 // 11 consumer warps and the producer: 12 warps, three per scheduler, so a
 // thread may hold up to 168 registers (the per-token row partials)
 constexpr int kMtC = 11;
@@ -77,7 +79,7 @@ struct MtArgs {
 };
 
 struct __align__(16) MtSmem {
-    float hs[2][kWPS][kMtMaxT];       // w*h of the stage's channels per token slot, by stage parity
+    float hs[2][kMtMaxCh][kMtMaxT];   // w*h of the stage's channels per token slot, by stage parity
     float uw[kMtMaxSlots][kMtMaxT];   // activated expert u, token slot k: the Eq. 2 weight
     uint8_t utok[kMtMaxSlots][kMtMaxT];  //   the token (slots k < popc(tmask[u]), ascending)
     int sj[kMtMaxSlots];              // the route by slot t*k1 + s: expert (or MOE_EMPTY_SLOT),
@@ -97,11 +99,14 @@ struct __align__(16) MtSmem {
 };
 
 // Shared memory of the few-token kernel: MtSmem, the barriers, the T tokens'
-// x rows (widened to float32 once), then the ring (as many 36 KB slots as fit, at most
-// kDSlots).
+// x rows (widened to float32 once), then the ring.  A stage is nch whole
+// channels (three d-element bf16 rows each, 6d bytes): the most, up to
+// kMtMaxCh, of which two slots fit -- a stage's cost is dominated by one dot
+// job's latency and grows slowly with its channels, so two large slots move
+// more bytes per stage than more small ones (measured at T = 2, 4, 8).
 struct MtLayout {
-    size_t bar_off, x_off, ring_off, total;
-    int nslots;
+    size_t bar_off, x_off, ring_off, stage, total;
+    int nch, nslots;
 };
 __host__ __device__ inline MtLayout mt_layout(int T, int d)
 {
@@ -111,9 +116,13 @@ __host__ __device__ inline MtLayout mt_layout(int T, int d)
     L.ring_off = (L.x_off + (size_t)T * d * 4 + 127) & ~(size_t)127;  // x as float32
     const size_t cap = 227 * 1024;
     const size_t room = cap > L.ring_off ? cap - L.ring_off : 0;
-    const int ns = (int)(room / kDStageBytes);
+    const size_t ch = (size_t)6 * d;  // one channel's rows
+    const int n = (int)(room / 2 / ch);
+    L.nch = n > kMtMaxCh ? kMtMaxCh : n;
+    L.stage = (size_t)L.nch * ch;
+    const int ns = L.nch > 0 ? (int)(room / L.stage) : 0;
     L.nslots = ns > kDSlots ? kDSlots : ns;
-    L.total = L.ring_off + (size_t)L.nslots * kDStageBytes;
+    L.total = L.ring_off + (size_t)L.nslots * L.stage;
     return L;
 }
 
@@ -142,6 +151,14 @@ __device__ void mt_segments(MtSmem *ms, int U, int I, int G, int b, int *status)
 }
 
 MOE_DEVINL void mt_sync() { named_bar_sync(kConsumerBar, kMtC * 32); }
+
+// j / n for 1 <= n <= kMtMaxCh and 0 <= j < 40: (j * ceil(256 / n)) >> 8.
+MOE_DEVINL int div_small(int j, int n)
+{
+    const int mul = n == 1 ? 256 : n == 2 ? 128 : n == 3 ? 86 : n == 4 ? 64 : n == 5 ? 52
+                  : n == 6 ? 43 : n == 7 ? 37 : 32;
+    return (j * mul) >> 8;
+}
 
 // Token position of the r-th set bit of m (r < popc(m)).
 MOE_DEVINL int nth_bit(unsigned m, int r)
@@ -427,7 +444,8 @@ __global__ void __launch_bounds__(kMtThreads, 1) k_decode_mt(MtArgs a)
     }
     __syncthreads();
     const int nseg = ms->nseg;
-    const int nch = decode_channels_per_stage(d);
+    const int nch = L.nch;
+    const size_t stage_bytes = L.stage;
 
     if (warp == kMtC) {
         // ------------------------------------------------------------ producer
@@ -449,7 +467,7 @@ __global__ void __launch_bounds__(kMtThreads, 1) k_decode_mt(MtArgs a)
                 const int e = ms->ue[ms->seg[it.s].u];
                 const size_t row0 = (size_t)e * I + it.c;
                 const uint32_t bytes = (uint32_t)n * d * 2;
-                uint8_t *dst = ring + (size_t)slot_r * kDStageBytes;
+                uint8_t *dst = ring + (size_t)slot_r * stage_bytes;
                 mbar_arrive_expect_tx(&full[slot_r], 3 * bytes);
                 bulk_g2s(dst, a.wg + row0 * d, bytes, &full[slot_r], pol);
                 bulk_g2s(dst + bytes, a.wu + row0 * d, bytes, &full[slot_r], pol);
@@ -526,16 +544,16 @@ __global__ void __launch_bounds__(kMtThreads, 1) k_decode_mt(MtArgs a)
             ok = __all_sync(0xffffffffu, ok);
             if (!ok && lane == 0)
                 ms->abort = 1;
-            const uint8_t *stg = ring + (size_t)slot * kDStageBytes;
+            const uint8_t *stg = ring + (size_t)slot * stage_bytes;
             const size_t rb = (size_t)n * d * 2;  // bytes of one of the three row blocks
-            // (1) w*h: a job per (channel c, chunk of at most two of the expert's
-            // m tokens), job j = chunk * n + c on warp j % kMtC: chunks per
-            // channel q = kMtC / n, tokens per chunk 1 (m <= q) or 2
-            const int q = n == 3 ? 3 : (n == 2 ? 5 : 11);
-            const int tpc = m > q ? 2 : 1;
+            // (1) w*h: a job per (channel c, chunk of the expert's m tokens),
+            // job j = chunk * n + c on warp j % kMtC; a chunk holds one token,
+            // or two (a gate/up vector read once for both) when the n*m pairs
+            // outnumber the warps; J = n * chunks <= kMtMaxCh * 4 jobs
+            const int tpc = n * m > kMtC && m > 1 ? 2 : 1;
             const int nq = tpc == 1 ? m : (m + 1) >> 1;
             for (int j = warp; ok && j < n * nq; j += kMtC) {
-                const int ch = n == 3 ? j / 3 : (n == 2 ? j >> 1 : j);
+                const int ch = div_small(j, n);
                 const int c = j - ch * n;
                 const int k0 = ch * tpc;
                 const bool two = tpc == 2 && k0 + 1 < m;
@@ -564,7 +582,7 @@ __global__ void __launch_bounds__(kMtThreads, 1) k_decode_mt(MtArgs a)
             if (ok) {
                 const uint8_t *drows = stg + 2 * rb;
 #pragma unroll
-                for (int c = 0; c < kWPS; ++c) {
+                for (int c = 0; c < kMtMaxCh; ++c) {
                     if (c < n) {
                         const uint4 *drow = reinterpret_cast<const uint4 *>(drows + (size_t)c * d * 2);
 #pragma unroll
@@ -694,13 +712,11 @@ inline bool mt_fits(int T, int d, int E, int I, int k1, int G)
     mt_shape(T, d, TM, RVM);
     if (TM == 0 || T * k1 > kMtMaxSlots || k1 > kDMaxK1 || E > kMaxExperts)
         return false;
-    if ((size_t)6 * d > (size_t)kDStageBytes)  // one channel's three rows per slot at least
-        return false;
     const MtLayout L = mt_layout(T, d);
     if (L.nslots < 2)
         return false;
     const int rows = mt_router_rows(E, G);
-    if ((size_t)rows * d * 2 > (size_t)L.nslots * kDStageBytes)
+    if ((size_t)rows * d * 2 > (size_t)L.nslots * L.stage)
         return false;
     const int umax = T * k1 < E ? T * k1 : E;
     const long chmax = ((long)umax * I + G - 1) / G;
