@@ -511,11 +511,13 @@ __global__ void __launch_bounds__(kMtThreads, 1) k_decode_mt(MtArgs a)
                             red_add_v4(dst + 4, pair_lo(yq[k][j][2]), pair_hi(yq[k][j][2]),
                                        pair_lo(yq[k][j][3]), pair_hi(yq[k][j][3]));
                         }
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            yq[k][j][q] = 0;
                     }
                 }
+#pragma unroll
+                for (int j = 0; j < RVM; ++j)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        yq[k][j][q] = 0;  // every slot: those past cur_m held only w*0
             }
         };
 
@@ -592,16 +594,17 @@ __global__ void __launch_bounds__(kMtThreads, 1) k_decode_mt(MtArgs a)
                                 const uint4 w = drow[v];
                                 const uint64_t w0 = bf16x2_pair(w.x), w1 = bf16x2_pair(w.y);
                                 const uint64_t w2 = bf16x2_pair(w.z), w3 = bf16x2_pair(w.w);
+                                // every slot, branch-free: w*h = 0 past the
+                                // expert's m tokens (those slots are dropped,
+                                // not added, at the next flush)
 #pragma unroll
                                 for (int k = 0; k < TM; ++k) {
-                                    if (k < m) {
-                                        const float hv = ms->hs[hb][c][k];
-                                        const uint64_t h2 = f32_pair(hv, hv);
-                                        yq[k][j][0] = ffma2(w0, h2, yq[k][j][0]);
-                                        yq[k][j][1] = ffma2(w1, h2, yq[k][j][1]);
-                                        yq[k][j][2] = ffma2(w2, h2, yq[k][j][2]);
-                                        yq[k][j][3] = ffma2(w3, h2, yq[k][j][3]);
-                                    }
+                                    const float hv = k < m ? ms->hs[hb][c][k] : 0.0f;
+                                    const uint64_t h2 = f32_pair(hv, hv);
+                                    yq[k][j][0] = ffma2(w0, h2, yq[k][j][0]);
+                                    yq[k][j][1] = ffma2(w1, h2, yq[k][j][1]);
+                                    yq[k][j][2] = ffma2(w2, h2, yq[k][j][2]);
+                                    yq[k][j][3] = ffma2(w3, h2, yq[k][j][3]);
                                 }
                             }
                         }
