@@ -245,6 +245,41 @@ __device__ __forceinline__ void mt_route(const MtArgs &a, int t, bool ok, int la
     warp_route_vals<R>(p, E, a.k1, a.k2, lane, my_j, my_w, a.vk, &kt);
 }
 
+// The down phase of one stage for one warp: y partials += w*h * down row for
+// the warp's rows (vectors v = warp*32 + lane + kMtC*32*j) and token slots
+// k < MM, every slot branch-free with w*h = 0 at k >= m (those slots are
+// dropped, not added, at the next flush).  MM >= m is chosen per stage, so
+// an expert with one or two tokens costs one or two slots' FMAs, not TM's.
+template <int MM, int TM, int RVM>
+MOE_DEVINL void mt_down(uint64_t (&yq)[TM][RVM][4], const float (&hs)[kMtMaxCh][kMtMaxT],
+                        const uint8_t *drows, int n, int m, int d, int nvec, int warp, int lane)
+{
+#pragma unroll
+    for (int c = 0; c < kMtMaxCh; ++c) {
+        if (c < n) {
+            const uint4 *drow = reinterpret_cast<const uint4 *>(drows + (size_t)c * d * 2);
+#pragma unroll
+            for (int j = 0; j < RVM; ++j) {
+                const int v = warp * 32 + lane + kMtC * 32 * j;
+                if (v < nvec) {
+                    const uint4 w = drow[v];
+                    const uint64_t w0 = bf16x2_pair(w.x), w1 = bf16x2_pair(w.y);
+                    const uint64_t w2 = bf16x2_pair(w.z), w3 = bf16x2_pair(w.w);
+#pragma unroll
+                    for (int k = 0; k < MM; ++k) {
+                        const float hv = k < m ? hs[c][k] : 0.0f;
+                        const uint64_t h2 = f32_pair(hv, hv);
+                        yq[k][j][0] = ffma2(w0, h2, yq[k][j][0]);
+                        yq[k][j][1] = ffma2(w1, h2, yq[k][j][1]);
+                        yq[k][j][2] = ffma2(w2, h2, yq[k][j][2]);
+                        yq[k][j][3] = ffma2(w3, h2, yq[k][j][3]);
+                    }
+                }
+            }
+        }
+    }
+}
+
 // TM: tokens the partials cover (T <= TM); RVM: 16-byte output-row vectors per
 // lane (d <= RVM * kMtC * 256).
 template <int TM, int RVM>
@@ -577,39 +612,21 @@ __global__ void __launch_bounds__(kMtThreads, 1) k_decode_mt(MtArgs a)
                 }
             }
             mt_sync();  // the stage's w*h are in shared memory
-            // (2) y partials += w*h * down row, for this warp's rows and the
-            // expert's m token slots.  hs alternates by stage parity: a warp
+            // (2) y partials += w*h * down row (mt_down), for this warp's rows
+            // and the expert's m token slots.  hs alternates by stage parity: a warp
             // writes the buffer again two stages later, past the next stage's
             // barrier, which every warp reaches only after this read.
             if (ok) {
                 const uint8_t *drows = stg + 2 * rb;
-#pragma unroll
-                for (int c = 0; c < kMtMaxCh; ++c) {
-                    if (c < n) {
-                        const uint4 *drow = reinterpret_cast<const uint4 *>(drows + (size_t)c * d * 2);
-#pragma unroll
-                        for (int j = 0; j < RVM; ++j) {
-                            const int v = warp * 32 + lane + kMtC * 32 * j;
-                            if (v < nvec) {
-                                const uint4 w = drow[v];
-                                const uint64_t w0 = bf16x2_pair(w.x), w1 = bf16x2_pair(w.y);
-                                const uint64_t w2 = bf16x2_pair(w.z), w3 = bf16x2_pair(w.w);
-                                // every slot, branch-free: w*h = 0 past the
-                                // expert's m tokens (those slots are dropped,
-                                // not added, at the next flush)
-#pragma unroll
-                                for (int k = 0; k < TM; ++k) {
-                                    const float hv = k < m ? ms->hs[hb][c][k] : 0.0f;
-                                    const uint64_t h2 = f32_pair(hv, hv);
-                                    yq[k][j][0] = ffma2(w0, h2, yq[k][j][0]);
-                                    yq[k][j][1] = ffma2(w1, h2, yq[k][j][1]);
-                                    yq[k][j][2] = ffma2(w2, h2, yq[k][j][2]);
-                                    yq[k][j][3] = ffma2(w3, h2, yq[k][j][3]);
-                                }
-                            }
-                        }
-                    }
-                }
+                constexpr int M2 = TM < 2 ? TM : 2, M4 = TM < 4 ? TM : 4;
+                if (m <= 1)
+                    mt_down<1, TM, RVM>(yq, ms->hs[hb], drows, n, m, d, nvec, warp, lane);
+                else if (m <= M2)
+                    mt_down<M2, TM, RVM>(yq, ms->hs[hb], drows, n, m, d, nvec, warp, lane);
+                else if (m <= M4)
+                    mt_down<M4, TM, RVM>(yq, ms->hs[hb], drows, n, m, d, nvec, warp, lane);
+                else
+                    mt_down<TM, TM, RVM>(yq, ms->hs[hb], drows, n, m, d, nvec, warp, lane);
             }
             __syncwarp();
             if (ok && lane == 0)
