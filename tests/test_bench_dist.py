@@ -117,3 +117,23 @@ def test_both_arms_report_the_same_config():
     assert c["workload"].startswith("decode_b1: 48 layers, d=2048, E=128, I=768, T=1")
     assert (c["k1"], c["k2"]) == (4, 16)
     assert "us_per_layer" not in c  # measured values stay out of the shared config
+
+
+def test_few_token_workload_config():
+    # --cm: the small-batch workload on the channel-major down matrix (the few-token
+    # decode kernel); the default run times T = 2 / 4 / 8 that way after the others
+    sys.path.insert(0, ROOT)
+    import bench
+
+    class A:
+        workload, T, layers, k1, k2, cm = "decode_small_batch", 4, 0, 4, 16, True
+        cascade = channel_keep = skip = router_std = None
+    wl, sweep = bench.workload_of(A())
+    assert wl["cm"] == 1 and wl["T"] == 4 and sweep == [(4, 16)]
+    c = bench.line_config(A(), wl, sweep[0], 1)
+    assert c["w_down_layout"].startswith("channel-major")
+    keys = [name + "".join("_%s%d" % kv for kv in sorted(over.items()))
+            for name, over in bench.EXTRA_WORKLOADS]
+    assert keys[-3:] == ["decode_small_batch_T2_cm1", "decode_small_batch_T4_cm1",
+                         "decode_small_batch_T8_cm1"]
+    assert "prefill" in keys and keys.index("prefill") < keys.index("decode_small_batch_T2_cm1")
