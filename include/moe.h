@@ -177,9 +177,9 @@ int moe_combine(const float *expert_out, const int32_t *slot_pos, const float *t
  * flags: MOE_PATH_* | MOE_WDOWN_CHANNEL_MAJOR.  With the HF down layout
  * [E x d x I] the two-phase streaming path runs (deterministic).  With
  * MOE_WDOWN_CHANNEL_MAJOR (w_down from moe_pack_w_down) and 1 <= T <= 8 the
- * single-pass decode path runs (each routed expert's weights read once for
- * all the tokens routed to it; for 5 <= T <= 8, d <= 2816; for T <= 4, d <= 5632); other shapes
- * return MOE_ERR_UNSUPPORTED_SHAPE.
+ * single-pass decode path runs, each routed expert's weights read once for
+ * all the tokens routed to it (2 <= T <= 4: d <= 5632; 5 <= T <= 8:
+ * d <= 2816; T * k1 <= 64); other shapes return MOE_ERR_UNSUPPORTED_SHAPE.
  * ws: workspace. */
 int moe_layer(const void *x_bf16, const void *w_router_bf16, const float *bias,
               const void *w_gate_bf16, const void *w_up_bf16, const void *w_down_bf16, int T, int d,
