@@ -18,6 +18,7 @@ def test_small_parity_cases_pass_in_the_checked_build():
     build.build(checks=True)
     env = dict(os.environ, MOE_LIB_VARIANT="checks")
     sel = ("test_layer_small_all_tokens or test_decode_path_single_token or "
+           "test_decode_path_few_tokens or "
            "test_layer_grouped_all_tokens or test_expert_ffn_grouped_per_slot or "
            "test_expert_ffn_and_combine_steps")
     cmd = [sys.executable, "-m", "pytest", "-q", "-m", "gpu", "-p", "no:cacheprovider",
