@@ -678,11 +678,13 @@ def layer_roofline(res, peaks):
 
 
 # workloads timed after the headline in the default run, each a sub-record
-# the few-token channel-major runs last: timed after the long 48-layer decode stacks, the
-# power-capped prefill GEMMs ran ~10 % slower than alone
+# prefill first: timed after the long 48-layer decode stacks, its power-capped GEMMs ran
+# 7-10 % slower than alone
 EXTRA_WORKLOADS = [
+    ("prefill", {}),
+    ("decode_small_batch", {"T": 2}), ("decode_small_batch", {"T": 4}),
     ("decode_small_batch", {"T": 8}), ("decode_small_batch", {"T": 32}),
-    ("decode_small_batch", {"T": 64}), ("prefill", {}),
+    ("decode_small_batch", {"T": 64}),
     ("large", {"T": 1}), ("large", {"T": 64}),
     ("decode_small_batch", {"T": 2, "cm": 1}), ("decode_small_batch", {"T": 4, "cm": 1}),
     ("decode_small_batch", {"T": 8, "cm": 1}),
