@@ -678,8 +678,8 @@ def layer_roofline(res, peaks):
 
 
 # workloads timed after the headline in the default run, each a sub-record
-# prefill first: timed after the long 48-layer decode stacks, its power-capped GEMMs ran
-# 7-10 % slower than alone
+# prefill, the small batches on the grouped GEMMs, the large model, then the few-token
+# kernel on the channel-major down matrix at the small batches' sizes
 EXTRA_WORKLOADS = [
     ("prefill", {}),
     ("decode_small_batch", {"T": 2}), ("decode_small_batch", {"T": 4}),

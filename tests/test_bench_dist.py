@@ -136,6 +136,6 @@ def test_few_token_workload_config():
             for name, over in bench.EXTRA_WORKLOADS]
     assert keys[-3:] == ["decode_small_batch_T2_cm1", "decode_small_batch_T4_cm1",
                          "decode_small_batch_T8_cm1"]
-    assert keys[0] == "prefill"  # before the long decode stacks
+    assert keys[0] == "prefill"
     # the grouped GEMMs at the same batch sizes, for the comparison
     assert {"decode_small_batch_T2", "decode_small_batch_T4", "decode_small_batch_T8"} <= set(keys)
